@@ -1,0 +1,412 @@
+"""Benchmark of the hybrid-attention forward on B200 (one process per GPU).
+
+`python bench.py --gpus N --steps K --warmup W` times K steps of one workload (default: the CSA
+prefill at 8k tokens, bf16) and rank 0 prints one JSON line. A step is one csa_forward call: the
+compressor over kv and over the indexer key stream, the indexer score, top-k, and the sparse +
+sliding attention with the sink and both RoPE rotations. With N > 1 (torchrun, NCCL) every rank
+runs its own sequence (data parallel, no collective on the data path; weak scaling) and the time
+is the maximum over ranks. `--impl reference` times the fp64 CPU oracle on a bounded sample of
+the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from sparse_attention_compressor_b200 import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+FP32_LANES_PER_SM = 128
+N_SM = 148
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work (only the causal, visible work)
+# ------------------------------------------------------------------------------------------------
+def visible(wl, S=None):
+    S = wl.S if S is None else S
+    t = np.arange(S, dtype=np.int64)
+    nwin = np.minimum(t + 1, wl.W)
+    nvis = (t + 1) // wl.m if wl.m else np.zeros_like(t)
+    return nwin, nvis
+
+
+def work(wl) -> dict:
+    """Per-step algorithmic FLOPs / bytes of each kernel (summed over B sequences)."""
+    nwin, nvis = visible(wl)
+    esz = 4 if wl.dtype == "f32" else 2
+    out = {}
+    if wl.kind == "csa":
+        nsel = np.minimum(nvis, wl.k)
+        out["attention"] = ("flops", float((nwin + nsel).sum()) * 4 * wl.H * wl.D * wl.B)
+        out["indexer_score"] = ("flops", float(nvis.sum()) * 2 * wl.nI * wl.cI * wl.B)
+        out["topk"] = ("bytes", float(nvis.sum() * 4 + wl.S * wl.k * 4) * wl.B)
+        out["compress_index"] = ("bytes", float(wl.S * wl.cI + wl.N * wl.cI) * esz * wl.B)
+    elif wl.kind == "hca":
+        out["attention"] = ("flops", float((nwin + nvis).sum()) * 4 * wl.H * wl.D * wl.B)
+    else:
+        out["attention"] = ("flops", float(nwin.sum()) * 4 * wl.H * wl.D * wl.B)
+    if wl.kind in ("csa", "hca"):
+        out["compress"] = ("bytes", float(wl.S * wl.D + wl.N * wl.D) * esz * wl.B)
+    out["rotate_kv"] = ("bytes", float(2 * wl.S * wl.D) * esz * wl.B)
+    return out
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# distributed plumbing
+# ------------------------------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=120))
+
+
+def rank_workload(wl: W.Workload, rank: int) -> W.Workload:
+    """Data-parallel replica: every rank runs the same shapes on its own seeded sequence."""
+    from dataclasses import replace
+    return replace(wl, seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        if device is not None and device.type == "cuda":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+def make_step(wl, g, dev):
+    import sparse_attention_compressor_b200 as sac
+    p = sac.make_params(wl.B, wl.S, wl.H, wl.D, wl.R, wl.theta, m=wl.m, win_len=wl.L,
+                        sliding_window=wl.W, n_idx_heads=wl.nI, idx_dim=wl.cI, topk=wl.k,
+                        dtype=wl.dtype)
+    kind = {"swa": sac.SAC_KIND_SWA, "hca": sac.SAC_KIND_HCA, "csa": sac.SAC_KIND_CSA}[wl.kind]
+    ws = torch.empty(sac.sac_workspace_size(p, kind), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(g["q"])
+
+    def step():
+        if wl.kind == "csa":
+            sac.csa_forward(p, g["q"], g["kv"], g["cmp_gate"], g["cmp_bias"], g["q_idx"],
+                            g["w_idx"], g["k_idx"], g["idx_gate"], g["idx_bias"], g["sinks"], o,
+                            None, None, None, ws)
+        elif wl.kind == "hca":
+            sac.hca_forward(p, g["q"], g["kv"], g["cmp_gate"], g["cmp_bias"], g["sinks"], o, None,
+                            ws)
+        else:
+            sac.swa_forward(p, g["q"], g["kv"], g["sinks"], o, ws)
+    return step, o
+
+
+def timed(step, steps, dev):
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    return a.elapsed_time(b)
+
+
+def roofline(wl, ktimes: dict, peaks: dict, steps: int, tensor_kernels: set) -> tuple:
+    wk = work(wl)
+    total = sum(v[1] for v in ktimes.values()) or 1.0
+    rows = {}
+    for name, (launches, ms) in ktimes.items():
+        per_launch_ms = ms / max(launches, 1)
+        launches_per_step = launches / steps
+        entry = {"launches": launches, "ms_per_launch": per_launch_ms, "share": ms / total}
+        if name in wk:
+            kind, amount = wk[name]
+            amount /= launches_per_step  # per launch
+            if kind == "flops":
+                achieved = amount / (per_launch_ms * 1e-3) / 1e12
+                if name in tensor_kernels:
+                    bound, peak = "tensor", peaks["bf16_tflops"]
+                else:
+                    bound = "alu"
+                    peak = N_SM * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+                entry.update(bound=bound, achieved=achieved, peak=peak, unit="TFLOP/s",
+                             frac=achieved / peak)
+            else:
+                achieved = amount / (per_launch_ms * 1e-3) / 1e9
+                entry.update(bound="hbm", achieved=achieved, peak=peaks["hbm_gbs"], unit="GB/s",
+                             frac=achieved / peaks["hbm_gbs"])
+        rows[name] = entry
+    dom = max(ktimes, key=lambda k: ktimes[k][1])
+    d = rows[dom]
+    roof = {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
+            "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),
+            "traffic": None, "peak_source": peaks["source"]}
+    return roof, rows
+
+
+def cpu_baseline(wl, budget_s: float = 12.0) -> dict:
+    """The fp64 oracle on a bounded sample of query rows of the same workload (rank 0, N=1)."""
+    import oracle
+    t0 = time.perf_counter()
+    threads = oracle.max_threads()
+    n = max(1, threads)
+    value, sample = None, None
+    x = W.prefill_inputs(wl, with_queries=False)
+    rng = np.random.default_rng(0)
+    while True:
+        rows = np.sort(rng.choice(wl.B * wl.S, size=min(n, wl.B * wl.S), replace=False))
+        dt = oracle_rows(wl, x, rows)
+        if dt > budget_s / 3 or n >= wl.B * wl.S or time.perf_counter() - t0 > budget_s:
+            value = len(rows) / dt
+            sample = (f"{len(rows)} random query rows of {wl.name} (full path incl. compressor "
+                      f"over all {wl.S} tokens), {dt:.2f} s")
+            break
+        n = int(n * min(8.0, max(2.0, (budget_s / 3) / max(dt, 1e-3))))
+    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": sample}
+
+
+def oracle_rows(wl, x, rows) -> float:
+    import oracle
+    p = oracle.OracleParams(wl.B, wl.S, wl.H, wl.D, wl.R, wl.theta, wl.W, m=wl.m, L=wl.L,
+                            nI=wl.nI, cI=wl.cI, k=wl.k)
+    rq = W.prefill_row_inputs(wl, rows)
+    t = time.perf_counter()
+    if wl.kind == "csa":
+        oracle.csa_forward(p, rq["q"], x["kv"], x["cmp_gate"], x["cmp_bias"], rq["q_idx"],
+                           rq["w_idx"], x["k_idx"], x["idx_gate"], x["idx_bias"], x["sinks"],
+                           rows=rows)
+    elif wl.kind == "hca":
+        oracle.hca_forward(p, rq["q"], x["kv"], x["cmp_gate"], x["cmp_bias"], x["sinks"],
+                           rows=rows)
+    else:
+        oracle.swa_forward(p, rq["q"], x["kv"], x["sinks"], rows=rows)
+    return time.perf_counter() - t
+
+
+def config_of(wl, world):
+    cfg = {"workload": wl.name, "B": wl.B, "S": wl.S, "H": wl.H, "head_dim": wl.D,
+           "rope_dim": wl.R, "rope_theta": wl.theta, "sliding_window": wl.W,
+           "parallelism": f"dp{world}",
+           "l2": "inputs larger than L2 (q alone %d MiB > 126 MiB), no flush" %
+                 (wl.B * wl.S * wl.H * wl.D * (2 if wl.dtype == "bf16" else 4) // 2 ** 20)}
+    if wl.kind in ("csa", "hca"):
+        cfg.update(m=wl.m, compressor_window=wl.L)
+    if wl.kind == "csa":
+        cfg.update(index_n_heads=wl.nI, index_head_dim=wl.cI, index_topk=wl.k)
+    return cfg
+
+
+def run_ours(args, wl0):
+    import sparse_attention_compressor_b200 as sac
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    wl = rank_workload(wl0, rank)
+    host = W.prefill_inputs(wl)
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    g = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+    torch.cuda.synchronize(dev)
+    step, o = make_step(wl, g, dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    sac.sac_timing_begin()
+    with ClockSampler(dev.index) as clk:
+        ms = timed(step, args.steps, dev)
+    ktimes = sac.sac_timing_end()
+    ms = max_over_ranks(ms, dev)
+    ms_step = ms / args.steps
+    tokens = wl.B * wl.S * world
+    value = tokens / (ms_step * 1e-3)
+
+    # end to end: pinned host inputs -> device, the call, the output back to pinned host memory
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = o.numel() * o.element_size()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            g[k].copy_(v, non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(timed(e2e_step, args.steps, dev), dev) / args.steps
+
+    peaks = measured_peaks()
+    roof, krows = roofline(wl, ktimes, peaks, args.steps, tensor_kernels=set())
+    launches = sum(v[0] for v in ktimes.values())
+    line = {
+        "metric": f"{wl.kind.upper()} attention fwd tokens/s (prefill)", "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded; see DESIGN.md)",
+        "config": config_of(wl, world), "clocks": clk.summary(),
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches, "roofline": roof, "kernels": krows,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args, wl):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    x = W.prefill_inputs(wl, with_queries=False)
+    threads = oracle.max_threads()
+    n = max(32, 32 * threads)
+    rng = np.random.default_rng(1)
+    samples = [np.sort(rng.choice(wl.B * wl.S, size=n, replace=False))
+               for _ in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        oracle_rows(wl, x, samples[i])
+    t = [oracle_rows(wl, x, samples[args.warmup + i]) for i in range(args.steps)]
+    ms_step = 1e3 * sum(t) / len(t)
+    value = n / (ms_step * 1e-3)
+    sample = (f"each step: {n} random query rows of {wl.name} through the full oracle path "
+              f"(compressor over all {wl.S} tokens, indexer, top-k, attention)")
+    line = {
+        "impl": "reference", "metric": f"{wl.kind.upper()} attention fwd tokens/s (prefill)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="csa_8k_bf16",
+                    choices=[k for k, v in W.WORKLOADS.items() if v.kind != "decode"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    wl = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

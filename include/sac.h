@@ -1,0 +1,199 @@
+/*
+ * sac.h -- C ABI of the B200 (sm_100a) hybrid long-range attention forward of DeepSeek-V4:
+ * compressor, Lightning Indexer + top-k, shared K=V sparse / sliding-window multi-query attention
+ * with a per-head sink, and partial interleaved RoPE with the inverse rotation of the output.
+ *
+ * Source of the operations: the "DeepSeek-V4" model documentation page (Hugging Face
+ * Transformers), sections "Hybrid attention (section 2.3)" (three layer types; shared K=V MQA;
+ * partial RoPE and the -i output rotation, eq. 26; per-head sink, eq. 27; sliding-window branch),
+ * "Attention mask layout" (sliding mask, CSA slots with the -1 sentinel, HCA visibility
+ * w < (t+1)//m), "Cache layers" (compressor / indexer buffer, pool, count, overlap) and
+ * "DeepseekV4Config" (head_dim, sliding_window, compress_rates, index_* fields, rope bases).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are caller-owned DEVICE pointers, dense row-major, 16-byte aligned. The library
+ *    never allocates device memory; scratch space is a caller-provided workspace of at least
+ *    sac_workspace_size() / sac_decode_workspace_size() bytes (256-byte aligned).
+ *  - Element type of q, kv, k_idx, q_idx, gates, pools and o is params.dtype (SAC_F32 or
+ *    SAC_BF16). Biases, sinks and indexer head weights are always fp32; indices are int32.
+ *  - Every call enqueues kernels on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream) and returns without synchronising. Host-visible errors come back as a
+ *    status code; sac_last_error() gives a message for the calling thread's last failure.
+ *  - Prefill inputs are un-rotated; the library applies RoPE itself. The softmax scale is
+ *    params.softmax_scale (> 0).
+ *  - Thread safety: calls on different streams may run concurrently as long as they do not share
+ *    a workspace or an output.
+ */
+#ifndef SAC_H
+#define SAC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAC_API __attribute__((visibility("default")))
+#else
+#define SAC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types */
+#define SAC_F32 0
+#define SAC_BF16 1
+
+/* status codes */
+#define SAC_OK 0
+#define SAC_ERR_ARG (-1)          /* null pointer, non-positive or inconsistent size, misalignment */
+#define SAC_ERR_UNSUPPORTED (-2)  /* a shape or dtype outside the supported envelope              */
+#define SAC_ERR_WORKSPACE (-3)    /* workspace missing or smaller than required                    */
+#define SAC_ERR_LAUNCH (-4)       /* a CUDA launch or attribute call failed                        */
+
+/* layer kinds for the workspace queries */
+#define SAC_KIND_SWA 0
+#define SAC_KIND_HCA 1
+#define SAC_KIND_CSA 2
+
+/*
+ * Attention hyper-parameters of one layer ("DeepseekV4Config" names in brackets).
+ *   B, S            batch and tokens per sequence (prefill). For decode, S is an upper bound on
+ *                   every context length and B is ignored.
+ *   H, D            query heads [num_attention_heads], head_dim [head_dim]; one shared K=V head
+ *                   [num_key_value_heads = 1].
+ *   R               rope channels [head_dim * partial_rotary_factor]: the trailing R channels of
+ *                   each head rotate in interleaved pairs (D-R+2i, D-R+2i+1) by pos*theta^(-2i/R).
+ *   rope_theta      base for q, window keys and pool entries of this layer [rope_theta for
+ *                   sliding layers, compress_rope_theta for compressed layers].
+ *   m, win_len      compression rate and compressor window [compress_rates]: CSA m=4, win_len=8
+ *                   (overlapping); HCA m=128, win_len=128; sliding layers m=0.
+ *   sliding_window  W [sliding_window]: query t attends tokens (t-W, t].
+ *   n_idx_heads, idx_dim, topk   [index_n_heads, index_head_dim, index_topk], CSA only.
+ *   softmax_scale   logit scale (e.g. 1/sqrt(D)).
+ *   pos0            absolute position of token 0 (prefill); added to every decode position.
+ *   dtype           SAC_F32 or SAC_BF16.
+ */
+typedef struct {
+  int B, S, H, D, R;
+  double rope_theta;
+  int m, win_len;
+  int sliding_window;
+  int n_idx_heads, idx_dim, topk;
+  float softmax_scale;
+  int64_t pos0;
+  int dtype;
+} sac_params;
+
+/* Message of the calling thread's last failed call ("" if none). Static storage. */
+SAC_API const char* sac_last_error(void);
+
+/* ABI version (major*100 + minor). */
+SAC_API int sac_version(void);
+
+/*
+ * Workspace bytes a prefill call of `kind` (SAC_KIND_*) needs for `p`, assuming every nullable
+ * output is NULL (a call that passes those outputs never needs more). 0 on invalid params.
+ */
+SAC_API size_t sac_workspace_size(const sac_params* p, int kind);
+
+/*
+ * Sliding-window layer forward ("Hybrid attention": sliding_attention layers; "Attention mask
+ * layout": plain causal sliding-window mask).
+ *   q      [B,S,H,D]   un-rotated queries
+ *   kv     [B,S,D]     un-rotated shared key/value head
+ *   sinks  [H] fp32    per-head sink logits (eq. 27)
+ *   o      [B,S,H,D]   output; its rope slice is rotated back by -P_t (eq. 26)
+ * o[b,t,h] = sum_x p_x v_x with p over {kv_j rotated at P_j : t-W < j <= t} and the sink:
+ * p_x = exp(l_x) / (exp(sink_h) + sum_y exp(l_y)), l_x = scale <q~_t,h, k~_x>, q~ rotated at P_t.
+ */
+SAC_API int swa_forward(const sac_params* p, const void* q, const void* kv, const float* sinks, void* o,
+                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Heavily compressed attention forward ("Hybrid attention": HCA, m'=128, non-overlapping
+ * windows, no indexer; "Attention mask layout": entry w visible to t iff w < (t+1)//m).
+ *   cmp_gate [D] (dtype), cmp_bias [win_len] fp32: compressor gate. Entry w pools the window
+ *            [(w+1)m - win_len, (w+1)m) clipped at 0 by a softmax over g_j = <kv_j, u> + b[o_j],
+ *            o_j = j - (w+1)m + win_len; N = floor(S/m) entries per sequence.
+ *   pool_out [B,N,D] nullable: the pool as attended, rotated at p_w = pos0 + w*m.
+ * The key set of query t is the sliding window plus every visible entry.
+ */
+SAC_API int hca_forward(const sac_params* p, const void* q, const void* kv, const void* cmp_gate,
+                const float* cmp_bias, const float* sinks, void* o, void* pool_out, void* ws,
+                size_t ws_bytes, void* stream);
+
+/*
+ * Compressed sparse attention forward ("Hybrid attention": CSA, m=4, overlapping windows, plus
+ * the Lightning Indexer, eq. 13-17, keeping index_topk entries per query).
+ *   cmp_gate, cmp_bias   main compressor gate (as in hca_forward), over kv
+ *   q_idx [B,S,nI,cI]    indexer queries; w_idx [B,S,nI] fp32 indexer head weights
+ *   k_idx [B,S,cI]       indexer key stream; idx_gate [cI], idx_bias [win_len] fp32: its gate
+ *   topk_out [B,S,k]     nullable int32: the selected entries of each query in ascending entry
+ *                        order, then -1 for empty slots (queries with fewer than k visible)
+ *   pool_out [B,N,D]     nullable: rotated main pool; idx_pool_out [B,N,cI] nullable: indexer pool
+ * Score I[t,w] = sum_h w_idx[t,h] * max(0, <q_idx[t,h], KI_w>) over visible w; the k largest win,
+ * ties to the lower w. The key set of query t is the sliding window plus its selected entries.
+ */
+SAC_API int csa_forward(const sac_params* p, const void* q, const void* kv, const void* cmp_gate,
+                const float* cmp_bias, const void* q_idx, const float* w_idx, const void* k_idx,
+                const void* idx_gate, const float* idx_bias, const float* sinks, void* o,
+                int32_t* topk_out, void* pool_out, void* idx_pool_out, void* ws, size_t ws_bytes,
+                void* stream);
+
+/*
+ * Decode: nseq sequences, one new token each, over paged caches ("Cache layers").
+ * Cache contract:
+ *   - kv_pages [num_pages, page_size, D] hold kv already rotated at each token's position
+ *     (pos0 + j); row j of sequence s is kv_pages[kv_block_table[s*kv_max_pages + j/page_size]]
+ *     [j % page_size]. The new token's row is already written.
+ *   - pool_pages [.., page_size, D] hold pool entries already rotated at pos0 + w*m;
+ *     idx_pool_pages [.., page_size, cI] hold un-rotated indexer entries; both use
+ *     pool_block_table [nseq, pool_max_pages] with entry w at page w/page_size, row w%page_size.
+ *   - ctx_lens [nseq] int32 (device) counts the new token: the query is token t = ctx-1 at
+ *     position pos0 + t, it sees the last min(ctx, W) tokens and floor(ctx/m) entries.
+ *     Every ctx must satisfy 1 <= ctx <= p->S.
+ *   q [nseq,H,D] un-rotated; o [nseq,H,D]; q_idx [nseq,nI,cI], w_idx [nseq,nI] fp32 (CSA);
+ *   topk_out [nseq,k] nullable (ascending entries, -1 fill).
+ */
+SAC_API size_t sac_decode_workspace_size(const sac_params* p, int kind, int nseq);
+
+SAC_API int swa_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
+               const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+               int page_size, const float* sinks, void* o, void* ws, size_t ws_bytes,
+               void* stream);
+
+SAC_API int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
+               const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+               int page_size, const void* pool_pages, const int32_t* pool_block_table,
+               int pool_max_pages, const float* sinks, void* o, void* ws, size_t ws_bytes,
+               void* stream);
+
+SAC_API int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
+               const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+               int page_size, const void* pool_pages, const void* idx_pool_pages,
+               const int32_t* pool_block_table, int pool_max_pages, const void* q_idx,
+               const float* w_idx, const float* sinks, void* o, int32_t* topk_out, void* ws,
+               size_t ws_bytes, void* stream);
+
+/*
+ * Optional per-kernel timing (no counterpart on the page: a measurement aid). Between
+ * sac_timing_begin() and sac_timing_end() every kernel the library launches is bracketed by a
+ * pair of CUDA events recorded on the launch's own stream. sac_timing_end() waits for those
+ * events, fills up to max_entries records (one per kernel name: launches and summed device time)
+ * and returns the number of distinct kernels (which may exceed max_entries), or SAC_ERR_LAUNCH.
+ */
+typedef struct {
+  char name[32];
+  int launches;
+  double total_ms;
+} sac_kernel_time;
+
+SAC_API int sac_timing_begin(void);
+SAC_API int sac_timing_end(sac_kernel_time* out, int max_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAC_H */

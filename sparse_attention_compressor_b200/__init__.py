@@ -1,0 +1,201 @@
+"""B200 (sm_100a) hybrid long-range attention forward of DeepSeek-V4 (CSA / HCA / sliding).
+
+Thin Python binding of the C ABI in ``include/sac.h``: every function here marshals torch CUDA
+tensors into pointers and calls the function of the same name in ``libsac.so``; all computation
+runs in that library's CUDA kernels. There is no CPU path: calling into a missing or unbuilt
+library raises.
+
+Source: the "DeepSeek-V4" model documentation page (Hugging Face Transformers), sections "Hybrid
+attention (section 2.3)", "Attention mask layout", "Cache layers", "DeepseekV4Config".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsac.so")
+
+SAC_F32, SAC_BF16 = 0, 1
+SAC_KIND_SWA, SAC_KIND_HCA, SAC_KIND_CSA = 0, 1, 2
+ABI_SYMBOLS = ("sac_last_error", "sac_version", "sac_workspace_size", "swa_forward",
+               "hca_forward", "csa_forward", "sac_decode_workspace_size", "swa_decode",
+               "hca_decode", "csa_decode", "sac_timing_begin", "sac_timing_end")
+
+
+class SacError(RuntimeError):
+    """A non-zero status returned by the library, with its message."""
+
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+class sac_params(ctypes.Structure):
+    """Mirror of ``sac_params`` in include/sac.h."""
+    _fields_ = [("B", ctypes.c_int), ("S", ctypes.c_int), ("H", ctypes.c_int),
+                ("D", ctypes.c_int), ("R", ctypes.c_int), ("rope_theta", ctypes.c_double),
+                ("m", ctypes.c_int), ("win_len", ctypes.c_int), ("sliding_window", ctypes.c_int),
+                ("n_idx_heads", ctypes.c_int), ("idx_dim", ctypes.c_int), ("topk", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float), ("pos0", ctypes.c_int64),
+                ("dtype", ctypes.c_int)]
+
+
+def make_params(B: int, S: int, H: int, D: int, R: int, rope_theta: float, *, m: int = 0,
+                win_len: int = 0, sliding_window: int = 128, n_idx_heads: int = 0,
+                idx_dim: int = 0, topk: int = 0, softmax_scale: Optional[float] = None,
+                pos0: int = 0, dtype: str = "bf16") -> sac_params:
+    scale = softmax_scale if softmax_scale is not None else D ** -0.5
+    return sac_params(B, S, H, D, R, float(rope_theta), m, win_len, sliding_window, n_idx_heads,
+                      idx_dim, topk, float(scale), int(pos0),
+                      SAC_F32 if dtype in ("f32", "float32") else SAC_BF16)
+
+
+class sac_kernel_time(ctypes.Structure):
+    """Mirror of ``sac_kernel_time`` in include/sac.h."""
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int),
+                ("total_ms", ctypes.c_double)]
+
+
+_lib_handle = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libsac.so (raises if it is missing: build it with ``python -m
+    sparse_attention_compressor_b200.build`` or ``__graft_entry__.build()``)."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(path):
+        raise RuntimeError(f"libsac.so not found at {path}; the CUDA library must be built")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(sac_params)
+    vp, sz, i32p, fp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
+    ci = ctypes.c_int
+    lib.sac_last_error.restype = ctypes.c_char_p
+    lib.sac_version.restype = ci
+    lib.sac_workspace_size.restype = sz
+    lib.sac_workspace_size.argtypes = [P, ci]
+    lib.sac_decode_workspace_size.restype = sz
+    lib.sac_decode_workspace_size.argtypes = [P, ci, ci]
+    lib.swa_forward.argtypes = [P, vp, vp, fp, vp, vp, sz, vp]
+    lib.hca_forward.argtypes = [P, vp, vp, vp, fp, fp, vp, vp, vp, sz, vp]
+    lib.csa_forward.argtypes = [P, vp, vp, vp, fp, vp, fp, vp, vp, fp, fp, vp, i32p, vp, vp, vp,
+                                sz, vp]
+    lib.swa_decode.argtypes = [P, ci, vp, vp, i32p, ci, i32p, ci, fp, vp, vp, sz, vp]
+    lib.hca_decode.argtypes = [P, ci, vp, vp, i32p, ci, i32p, ci, vp, i32p, ci, fp, vp, vp, sz,
+                               vp]
+    lib.csa_decode.argtypes = [P, ci, vp, vp, i32p, ci, i32p, ci, vp, vp, i32p, ci, vp, fp, fp,
+                               vp, i32p, vp, sz, vp]
+    lib.sac_timing_begin.restype = ci
+    lib.sac_timing_end.restype = ci
+    lib.sac_timing_end.argtypes = [ctypes.POINTER(sac_kernel_time), ci]
+    for name in ("swa_forward", "hca_forward", "csa_forward", "swa_decode", "hca_decode",
+                 "csa_decode"):
+        getattr(lib, name).restype = ci
+    _lib_handle = lib
+    return lib
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a CUDA tensor (None passes NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("the library takes CUDA tensors (device pointers)")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise SacError(fn, rc, load_library().sac_last_error().decode())
+
+
+def _nbytes(ws) -> int:
+    return 0 if ws is None else ws.numel() * ws.element_size()
+
+
+def sac_version() -> int:
+    return int(load_library().sac_version())
+
+
+def sac_workspace_size(p: sac_params, kind: int) -> int:
+    return int(load_library().sac_workspace_size(ctypes.byref(p), kind))
+
+
+def sac_decode_workspace_size(p: sac_params, kind: int, nseq: int) -> int:
+    return int(load_library().sac_decode_workspace_size(ctypes.byref(p), kind, nseq))
+
+
+def sac_timing_begin() -> None:
+    _check("sac_timing_begin", load_library().sac_timing_begin())
+
+
+def sac_timing_end(max_entries: int = 32) -> dict:
+    """{kernel name: (launches, total device ms)} since sac_timing_begin()."""
+    buf = (sac_kernel_time * max_entries)()
+    n = load_library().sac_timing_end(buf, max_entries)
+    if n < 0:
+        _check("sac_timing_end", n)
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms)
+            for i in range(min(n, max_entries))}
+
+
+def swa_forward(p, q, kv, sinks, o, ws, stream=None) -> None:
+    _check("swa_forward", load_library().swa_forward(
+        ctypes.byref(p), _ptr(q), _ptr(kv), _ptr(sinks), _ptr(o), _ptr(ws), _nbytes(ws),
+        _stream(stream)))
+
+
+def hca_forward(p, q, kv, cmp_gate, cmp_bias, sinks, o, pool_out, ws, stream=None) -> None:
+    _check("hca_forward", load_library().hca_forward(
+        ctypes.byref(p), _ptr(q), _ptr(kv), _ptr(cmp_gate), _ptr(cmp_bias), _ptr(sinks), _ptr(o),
+        _ptr(pool_out), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def csa_forward(p, q, kv, cmp_gate, cmp_bias, q_idx, w_idx, k_idx, idx_gate, idx_bias, sinks, o,
+                topk_out, pool_out, idx_pool_out, ws, stream=None) -> None:
+    _check("csa_forward", load_library().csa_forward(
+        ctypes.byref(p), _ptr(q), _ptr(kv), _ptr(cmp_gate), _ptr(cmp_bias), _ptr(q_idx),
+        _ptr(w_idx), _ptr(k_idx), _ptr(idx_gate), _ptr(idx_bias), _ptr(sinks), _ptr(o),
+        _ptr(topk_out), _ptr(pool_out), _ptr(idx_pool_out), _ptr(ws), _nbytes(ws),
+        _stream(stream)))
+
+
+def swa_decode(p, nseq, q, kv_pages, kv_block_table, ctx_lens, page_size, sinks, o, ws=None,
+               stream=None) -> None:
+    _check("swa_decode", load_library().swa_decode(
+        ctypes.byref(p), nseq, _ptr(q), _ptr(kv_pages), _ptr(kv_block_table),
+        kv_block_table.shape[1], _ptr(ctx_lens), page_size, _ptr(sinks), _ptr(o), _ptr(ws),
+        _nbytes(ws), _stream(stream)))
+
+
+def hca_decode(p, nseq, q, kv_pages, kv_block_table, ctx_lens, page_size, pool_pages,
+               pool_block_table, sinks, o, ws=None, stream=None) -> None:
+    _check("hca_decode", load_library().hca_decode(
+        ctypes.byref(p), nseq, _ptr(q), _ptr(kv_pages), _ptr(kv_block_table),
+        kv_block_table.shape[1], _ptr(ctx_lens), page_size, _ptr(pool_pages),
+        _ptr(pool_block_table), pool_block_table.shape[1], _ptr(sinks), _ptr(o), _ptr(ws),
+        _nbytes(ws), _stream(stream)))
+
+
+def csa_decode(p, nseq, q, kv_pages, kv_block_table, ctx_lens, page_size, pool_pages,
+               idx_pool_pages, pool_block_table, q_idx, w_idx, sinks, o, topk_out, ws,
+               stream=None) -> None:
+    _check("csa_decode", load_library().csa_decode(
+        ctypes.byref(p), nseq, _ptr(q), _ptr(kv_pages), _ptr(kv_block_table),
+        kv_block_table.shape[1], _ptr(ctx_lens), page_size, _ptr(pool_pages),
+        _ptr(idx_pool_pages), _ptr(pool_block_table), pool_block_table.shape[1], _ptr(q_idx),
+        _ptr(w_idx), _ptr(sinks), _ptr(o), _ptr(topk_out), _ptr(ws), _nbytes(ws),
+        _stream(stream)))

@@ -1,0 +1,466 @@
+// C ABI of the hybrid-attention library (declared in include/sac.h): argument validation,
+// workspace carving and the launch sequence of each layer type.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "sac.h"
+#include "sac_kernels.h"
+#include "sac_timing.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SAC_ERR_LAUNCH, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 256;
+constexpr size_t kScoresBudget = size_t(1) << 30;  // bytes of indexer scores per prefill chunk
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+size_t esize(int dtype) { return dtype == SAC_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+#define REQUIRE(cond, code, ...) \
+  do {                           \
+    if (!(cond)) return fail(code, __VA_ARGS__); \
+  } while (0)
+
+#define REQUIRE_PTR(ptr)                                                               \
+  do {                                                                                 \
+    if ((ptr) == nullptr) return fail(SAC_ERR_ARG, "%s must not be NULL", #ptr);       \
+    if (!aligned16(ptr)) return fail(SAC_ERR_ARG, "%s must be 16-byte aligned", #ptr); \
+  } while (0)
+
+#define OPTIONAL_PTR(ptr)                                                               \
+  do {                                                                                  \
+    if ((ptr) != nullptr && !aligned16(ptr))                                            \
+      return fail(SAC_ERR_ARG, "%s must be 16-byte aligned", #ptr);                     \
+  } while (0)
+
+bool pow2_between(int x, int lo, int hi) {
+  return x >= lo && x <= hi && (x & (x - 1)) == 0;
+}
+
+// Shape checks shared by every layer kind. kind: SAC_KIND_*; decode: p->S bounds the contexts.
+int check_params(const sac_params* p, int kind, bool decode) {
+  REQUIRE(p != nullptr, SAC_ERR_ARG, "params must not be NULL");
+  REQUIRE(p->dtype == SAC_F32 || p->dtype == SAC_BF16, SAC_ERR_UNSUPPORTED, "dtype %d", p->dtype);
+  REQUIRE(decode || p->B >= 1, SAC_ERR_ARG, "B must be >= 1 (got %d)", p->B);
+  REQUIRE(p->S >= 1, SAC_ERR_ARG, "S must be >= 1 (got %d)", p->S);
+  REQUIRE(p->H >= 1, SAC_ERR_ARG, "H must be >= 1 (got %d)", p->H);
+  REQUIRE(pow2_between(p->D, 64, 512), SAC_ERR_UNSUPPORTED,
+          "head_dim must be 64, 128, 256 or 512 (got %d)", p->D);
+  REQUIRE(p->R >= 0 && p->R <= p->D && p->R % 2 == 0 && p->R / 2 <= sac::kMaxRopePairs,
+          SAC_ERR_UNSUPPORTED, "rope dim must be even, <= head_dim and <= 128 (got %d)", p->R);
+  REQUIRE(p->rope_theta > 0 && std::isfinite(p->rope_theta), SAC_ERR_ARG, "rope_theta must be > 0");
+  REQUIRE(p->sliding_window >= 1, SAC_ERR_ARG, "sliding_window must be >= 1");
+  REQUIRE(p->softmax_scale > 0 && std::isfinite(p->softmax_scale), SAC_ERR_ARG,
+          "softmax_scale must be > 0");
+  if (kind == SAC_KIND_HCA || kind == SAC_KIND_CSA) {
+    REQUIRE(p->m >= 1, SAC_ERR_ARG, "compression rate m must be >= 1 (got %d)", p->m);
+    REQUIRE(p->win_len >= 1 && p->win_len <= 4096, SAC_ERR_UNSUPPORTED,
+            "compressor window must be in [1, 4096] (got %d)", p->win_len);
+  }
+  if (kind == SAC_KIND_CSA) {
+    REQUIRE(p->n_idx_heads >= 1 && p->n_idx_heads <= 128, SAC_ERR_UNSUPPORTED,
+            "index_n_heads must be in [1, 128] (got %d)", p->n_idx_heads);
+    REQUIRE(pow2_between(p->idx_dim, 32, 256), SAC_ERR_UNSUPPORTED,
+            "index_head_dim must be 32, 64, 128 or 256 (got %d)", p->idx_dim);
+    REQUIRE(p->topk >= 1, SAC_ERR_ARG, "index_topk must be >= 1 (got %d)", p->topk);
+    REQUIRE(p->S / p->m <= sac::topk_max_entries(), SAC_ERR_UNSUPPORTED,
+            "at most %d pool entries per sequence (S/m = %d)", sac::topk_max_entries(),
+            p->S / p->m);
+    size_t smem = 4 * ((size_t)p->n_idx_heads * p->idx_dim + p->n_idx_heads +
+                       64 * (size_t)(p->idx_dim + 1) + 512);
+    REQUIRE(smem <= 200 * 1024, SAC_ERR_UNSUPPORTED, "indexer heads x dim too large");
+  }
+  return SAC_OK;
+}
+
+sac::RopeFreqs rope_freqs(const sac_params* p) {
+  sac::RopeFreqs rf;
+  std::memset(&rf, 0, sizeof(rf));
+  rf.R = p->R;
+  for (int i = 0; i < p->R / 2; ++i) rf.inv_freq[i] = std::pow(p->rope_theta, -2.0 * i / p->R);
+  return rf;
+}
+
+int64_t csa_chunk_rows(const sac_params* p) {
+  int64_t rows = (int64_t)p->B * p->S;
+  int64_t n = p->S / p->m;
+  if (n == 0) return rows;
+  int64_t per = (int64_t)(kScoresBudget / ((size_t)n * 4));
+  if (per < 1) per = 1;
+  return per < rows ? per : rows;
+}
+
+// Bump allocator over the caller's workspace.
+struct Carve {
+  char* base;
+  size_t used = 0;
+  explicit Carve(void* ws) : base(static_cast<char*>(ws)) {}
+  void* take(size_t bytes) {
+    void* ptr = base ? base + used : nullptr;
+    used += align_up(bytes);
+    return ptr;
+  }
+};
+
+struct Sizes {
+  size_t kv_rot = 0, pool = 0, idx_pool = 0, scores = 0, topk = 0;
+  size_t total() const {
+    return align_up(kv_rot) + align_up(pool) + align_up(idx_pool) + align_up(scores) +
+           align_up(topk);
+  }
+};
+
+Sizes prefill_sizes(const sac_params* p, int kind) {
+  Sizes s;
+  const size_t rows = (size_t)p->B * p->S;
+  s.kv_rot = rows * p->D * esize(p->dtype);
+  if (kind == SAC_KIND_HCA || kind == SAC_KIND_CSA)
+    s.pool = (size_t)p->B * (p->S / p->m) * p->D * esize(p->dtype);
+  if (kind == SAC_KIND_CSA) {
+    s.idx_pool = (size_t)p->B * (p->S / p->m) * p->idx_dim * esize(p->dtype);
+    s.scores = (size_t)csa_chunk_rows(p) * (p->S / p->m) * 4;
+    s.topk = rows * p->topk * 4;
+  }
+  return s;
+}
+
+sac::RowAddr contiguous(const void* base, int64_t seq_stride, int width) {
+  return sac::RowAddr{base, nullptr, seq_stride, 0, 1, width};
+}
+
+sac::RowAddr paged(const void* base, const int32_t* bt, int max_pages, int page_size, int width) {
+  return sac::RowAddr{base, bt, 0, max_pages, page_size, width};
+}
+
+sac::AttnArgs attn_common(const sac_params* p, const void* q, void* o, const float* sinks) {
+  sac::AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.o = o;
+  a.sinks = sinks;
+  a.H = p->H;
+  a.D = p->D;
+  a.W = p->sliding_window;
+  a.scale = p->softmax_scale;
+  a.pos0 = p->pos0;
+  a.m = p->m;
+  a.k = p->topk;
+  a.rf = rope_freqs(p);
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sac_last_error(void) { return g_err; }
+
+int sac_version(void) { return 100; }
+
+size_t sac_workspace_size(const sac_params* p, int kind) {
+  if (kind < SAC_KIND_SWA || kind > SAC_KIND_CSA || check_params(p, kind, false) != SAC_OK)
+    return 0;
+  return prefill_sizes(p, kind).total();
+}
+
+int swa_forward(const sac_params* p, const void* q, const void* kv, const float* sinks, void* o,
+                void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_params(p, SAC_KIND_SWA, false);
+  if (rc) return rc;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kv);
+  REQUIRE_PTR(sinks);
+  REQUIRE_PTR(o);
+  Sizes sz = prefill_sizes(p, SAC_KIND_SWA);
+  REQUIRE(ws != nullptr && ws_bytes >= sz.total(), SAC_ERR_WORKSPACE,
+          "workspace of %zu bytes needed (got %zu)", sz.total(), ws_bytes);
+  REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carve cv(ws);
+  void* kv_rot = cv.take(sz.kv_rot);
+  sac::RopeFreqs rf = rope_freqs(p);
+  const int64_t rows = (int64_t)p->B * p->S;
+  cudaError_t e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
+  sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.qr = sac::QueryRows{p->S, nullptr, 0};
+  a.nrows = rows;
+  a.win = contiguous(kv_rot, p->S, p->D);
+  a.pool_mode = 0;
+  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+int hca_forward(const sac_params* p, const void* q, const void* kv, const void* cmp_gate,
+                const float* cmp_bias, const float* sinks, void* o, void* pool_out, void* ws,
+                size_t ws_bytes, void* stream) {
+  int rc = check_params(p, SAC_KIND_HCA, false);
+  if (rc) return rc;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kv);
+  REQUIRE_PTR(cmp_gate);
+  REQUIRE(cmp_bias != nullptr, SAC_ERR_ARG, "cmp_bias must not be NULL");
+  REQUIRE_PTR(sinks);
+  REQUIRE_PTR(o);
+  OPTIONAL_PTR(pool_out);
+  Sizes sz = prefill_sizes(p, SAC_KIND_HCA);
+  if (pool_out) sz.pool = 0;
+  REQUIRE(ws != nullptr && ws_bytes >= sz.total(), SAC_ERR_WORKSPACE,
+          "workspace of %zu bytes needed (got %zu)", sz.total(), ws_bytes);
+  REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carve cv(ws);
+  void* kv_rot = cv.take(sz.kv_rot);
+  void* pool = pool_out ? pool_out : cv.take(sz.pool);
+  sac::RopeFreqs rf = rope_freqs(p);
+  const int64_t rows = (int64_t)p->B * p->S;
+  cudaError_t e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
+  e = sac::timed("compress", st, [&] { return sac::launch_compress(p->dtype, kv, cmp_gate, cmp_bias, p->B, p->S, p->D, p->m, p->win_len,
+                           true, rf, p->pos0, pool, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "compress");
+  sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.qr = sac::QueryRows{p->S, nullptr, 0};
+  a.nrows = rows;
+  a.win = contiguous(kv_rot, p->S, p->D);
+  a.pool_mode = 1;
+  a.pool = contiguous(pool, p->S / p->m, p->D);
+  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+int csa_forward(const sac_params* p, const void* q, const void* kv, const void* cmp_gate,
+                const float* cmp_bias, const void* q_idx, const float* w_idx, const void* k_idx,
+                const void* idx_gate, const float* idx_bias, const float* sinks, void* o,
+                int32_t* topk_out, void* pool_out, void* idx_pool_out, void* ws, size_t ws_bytes,
+                void* stream) {
+  int rc = check_params(p, SAC_KIND_CSA, false);
+  if (rc) return rc;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kv);
+  REQUIRE_PTR(cmp_gate);
+  REQUIRE(cmp_bias != nullptr, SAC_ERR_ARG, "cmp_bias must not be NULL");
+  REQUIRE_PTR(q_idx);
+  REQUIRE_PTR(w_idx);
+  REQUIRE_PTR(k_idx);
+  REQUIRE_PTR(idx_gate);
+  REQUIRE(idx_bias != nullptr, SAC_ERR_ARG, "idx_bias must not be NULL");
+  REQUIRE_PTR(sinks);
+  REQUIRE_PTR(o);
+  OPTIONAL_PTR(topk_out);
+  OPTIONAL_PTR(pool_out);
+  OPTIONAL_PTR(idx_pool_out);
+  Sizes sz = prefill_sizes(p, SAC_KIND_CSA);
+  if (pool_out) sz.pool = 0;
+  if (idx_pool_out) sz.idx_pool = 0;
+  if (topk_out) sz.topk = 0;
+  REQUIRE(ws != nullptr && ws_bytes >= sz.total(), SAC_ERR_WORKSPACE,
+          "workspace of %zu bytes needed (got %zu)", sz.total(), ws_bytes);
+  REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carve cv(ws);
+  void* kv_rot = cv.take(sz.kv_rot);
+  void* pool = pool_out ? pool_out : cv.take(sz.pool);
+  void* ipool = idx_pool_out ? idx_pool_out : cv.take(sz.idx_pool);
+  float* scores = static_cast<float*>(cv.take(sz.scores));
+  int32_t* sel = topk_out ? topk_out : static_cast<int32_t*>(cv.take(sz.topk));
+
+  sac::RopeFreqs rf = rope_freqs(p);
+  const int64_t rows = (int64_t)p->B * p->S;
+  const int N = p->S / p->m;
+  cudaError_t e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
+  e = sac::timed("compress", st, [&] { return sac::launch_compress(p->dtype, kv, cmp_gate, cmp_bias, p->B, p->S, p->D, p->m, p->win_len,
+                           true, rf, p->pos0, pool, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "compress");
+  e = sac::timed("compress_index", st, [&] { return sac::launch_compress(p->dtype, k_idx, idx_gate, idx_bias, p->B, p->S, p->idx_dim, p->m,
+                           p->win_len, false, rf, p->pos0, ipool, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "compress indexer stream");
+
+  const int64_t chunk = csa_chunk_rows(p);
+  const size_t qi_row = (size_t)p->n_idx_heads * p->idx_dim * esize(p->dtype);
+  for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
+    const int64_t nr = chunk < rows - r0 ? chunk : rows - r0;
+    sac::QueryRows qr{p->S, nullptr, r0};
+    // largest visible count in the chunk (a chunk may span sequences)
+    int64_t t_last = (r0 + nr - 1) % p->S;
+    int max_vis = (nr >= p->S || (r0 % p->S) > t_last) ? N : (int)((t_last + 1) / p->m);
+    sac::IndexerArgs ia;
+    ia.q_idx = static_cast<const char*>(q_idx) + (size_t)r0 * qi_row;
+    ia.w_idx = w_idx + (size_t)r0 * p->n_idx_heads;
+    ia.kpool = contiguous(ipool, N, p->idx_dim);
+    ia.qr = qr;
+    ia.nI = p->n_idx_heads;
+    ia.cI = p->idx_dim;
+    ia.m = p->m;
+    ia.nrows = nr;
+    ia.n_stride = N;
+    ia.scores = scores;
+    e = sac::timed("indexer_score", st, [&] { return sac::launch_indexer(p->dtype, ia, max_vis, st); });
+    if (e != cudaSuccess) return cuda_fail(e, "indexer");
+    e = sac::timed("topk", st, [&] { return sac::launch_topk(scores, N, qr, p->m, nr, p->topk, sel + r0 * p->topk, st); });
+    if (e != cudaSuccess) return cuda_fail(e, "top-k");
+  }
+
+  sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.qr = sac::QueryRows{p->S, nullptr, 0};
+  a.nrows = rows;
+  a.win = contiguous(kv_rot, p->S, p->D);
+  a.pool_mode = 2;
+  a.pool = contiguous(pool, N, p->D);
+  a.sel = sel;
+  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// decode
+// ---------------------------------------------------------------------------------------------
+size_t sac_decode_workspace_size(const sac_params* p, int kind, int nseq) {
+  if (kind < SAC_KIND_SWA || kind > SAC_KIND_CSA || nseq < 1 ||
+      check_params(p, kind, true) != SAC_OK)
+    return 0;
+  if (kind != SAC_KIND_CSA) return 0;
+  const size_t n = (size_t)(p->S / p->m);
+  return align_up((size_t)nseq * n * 4) + align_up((size_t)nseq * p->topk * 4);
+}
+
+static int check_decode_common(const sac_params* p, int kind, int nseq, const void* q,
+                               const void* kv_pages, const int32_t* kv_block_table,
+                               int kv_max_pages, const int32_t* ctx_lens, int page_size,
+                               const float* sinks, void* o) {
+  int rc = check_params(p, kind, true);
+  if (rc) return rc;
+  REQUIRE(nseq >= 1, SAC_ERR_ARG, "nseq must be >= 1 (got %d)", nseq);
+  REQUIRE(page_size >= 1, SAC_ERR_ARG, "page_size must be >= 1 (got %d)", page_size);
+  REQUIRE(kv_max_pages >= 1, SAC_ERR_ARG, "kv_max_pages must be >= 1");
+  REQUIRE((int64_t)kv_max_pages * page_size >= p->S, SAC_ERR_ARG,
+          "kv block table too short for contexts up to S=%d", p->S);
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kv_pages);
+  REQUIRE(kv_block_table != nullptr, SAC_ERR_ARG, "kv_block_table must not be NULL");
+  REQUIRE(ctx_lens != nullptr, SAC_ERR_ARG, "ctx_lens must not be NULL");
+  REQUIRE_PTR(sinks);
+  REQUIRE_PTR(o);
+  return SAC_OK;
+}
+
+int swa_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
+               const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+               int page_size, const float* sinks, void* o, void* ws, size_t ws_bytes,
+               void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  int rc = check_decode_common(p, SAC_KIND_SWA, nseq, q, kv_pages, kv_block_table, kv_max_pages,
+                               ctx_lens, page_size, sinks, o);
+  if (rc) return rc;
+  sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.qr = sac::QueryRows{0, ctx_lens, 0};
+  a.nrows = nseq;
+  a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
+  a.pool_mode = 0;
+  cudaError_t e = sac::timed("attention", static_cast<cudaStream_t>(stream), [&] { return sac::launch_attention_simt(p->dtype, a, static_cast<cudaStream_t>(stream)); });
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
+               const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+               int page_size, const void* pool_pages, const int32_t* pool_block_table,
+               int pool_max_pages, const float* sinks, void* o, void* ws, size_t ws_bytes,
+               void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  int rc = check_decode_common(p, SAC_KIND_HCA, nseq, q, kv_pages, kv_block_table, kv_max_pages,
+                               ctx_lens, page_size, sinks, o);
+  if (rc) return rc;
+  REQUIRE_PTR(pool_pages);
+  REQUIRE(pool_block_table != nullptr, SAC_ERR_ARG, "pool_block_table must not be NULL");
+  REQUIRE((int64_t)pool_max_pages * page_size >= p->S / p->m, SAC_ERR_ARG,
+          "pool block table too short for S/m entries");
+  sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.qr = sac::QueryRows{0, ctx_lens, 0};
+  a.nrows = nseq;
+  a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
+  a.pool_mode = 1;
+  a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
+  cudaError_t e = sac::timed("attention", static_cast<cudaStream_t>(stream), [&] { return sac::launch_attention_simt(p->dtype, a, static_cast<cudaStream_t>(stream)); });
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
+               const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+               int page_size, const void* pool_pages, const void* idx_pool_pages,
+               const int32_t* pool_block_table, int pool_max_pages, const void* q_idx,
+               const float* w_idx, const float* sinks, void* o, int32_t* topk_out, void* ws,
+               size_t ws_bytes, void* stream) {
+  int rc = check_decode_common(p, SAC_KIND_CSA, nseq, q, kv_pages, kv_block_table, kv_max_pages,
+                               ctx_lens, page_size, sinks, o);
+  if (rc) return rc;
+  REQUIRE_PTR(pool_pages);
+  REQUIRE_PTR(idx_pool_pages);
+  REQUIRE(pool_block_table != nullptr, SAC_ERR_ARG, "pool_block_table must not be NULL");
+  REQUIRE((int64_t)pool_max_pages * page_size >= p->S / p->m, SAC_ERR_ARG,
+          "pool block table too short for S/m entries");
+  REQUIRE_PTR(q_idx);
+  REQUIRE_PTR(w_idx);
+  OPTIONAL_PTR(topk_out);
+  const int N = p->S / p->m;
+  size_t need = align_up((size_t)nseq * N * 4) + (topk_out ? 0 : align_up((size_t)nseq * p->topk * 4));
+  REQUIRE(ws != nullptr && ws_bytes >= need, SAC_ERR_WORKSPACE,
+          "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carve cv(ws);
+  float* scores = static_cast<float*>(cv.take((size_t)nseq * N * 4));
+  int32_t* sel = topk_out ? topk_out : static_cast<int32_t*>(cv.take((size_t)nseq * p->topk * 4));
+  sac::QueryRows qr{0, ctx_lens, 0};
+  sac::IndexerArgs ia;
+  ia.q_idx = q_idx;
+  ia.w_idx = w_idx;
+  ia.kpool = paged(idx_pool_pages, pool_block_table, pool_max_pages, page_size, p->idx_dim);
+  ia.qr = qr;
+  ia.nI = p->n_idx_heads;
+  ia.cI = p->idx_dim;
+  ia.m = p->m;
+  ia.nrows = nseq;
+  ia.n_stride = N;
+  ia.scores = scores;
+  cudaError_t e = sac::timed("indexer_score", st, [&] { return sac::launch_indexer(p->dtype, ia, N, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "indexer");
+  e = sac::timed("topk", st, [&] { return sac::launch_topk(scores, N, qr, p->m, nseq, p->topk, sel, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "top-k");
+  sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.qr = qr;
+  a.nrows = nseq;
+  a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
+  a.pool_mode = 2;
+  a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
+  a.sel = sel;
+  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+}  // extern "C"

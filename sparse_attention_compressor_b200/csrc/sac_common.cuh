@@ -1,0 +1,89 @@
+// Shared device helpers of the sm_100a hybrid-attention library: element conversion, the RoPE
+// angle table, key-row addressing for contiguous and paged caches, and warp reductions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sac {
+
+constexpr int kMaxRopePairs = 64;  // R <= 128
+
+// Per-call RoPE frequencies theta^(-2i/R), computed once on the host in double precision.
+struct RopeFreqs {
+  double inv_freq[kMaxRopePairs];
+  int R;
+};
+
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// cos/sin of pair i at absolute position pos. The angle is formed and reduced in fp64 so that
+// positions up to 2^20 keep full fp32 accuracy after the rotation.
+__device__ __forceinline__ void rope_cos_sin(const RopeFreqs& rf, int i, int64_t pos, float& c,
+                                             float& s) {
+  double phi = (double)pos * rf.inv_freq[i];
+  double sd, cd;
+  sincos(phi, &sd, &cd);
+  c = (float)cd;
+  s = (float)sd;
+}
+
+// Rows of a key stream: contiguous [seqs, seq_stride, width], or pages [*, page_size, width]
+// reached through a block table [seqs, max_pages].
+struct RowAddr {
+  const void* base;
+  const int32_t* block_table;  // nullptr: contiguous
+  int64_t seq_stride;          // rows per sequence (contiguous layout)
+  int max_pages;
+  int page_size;
+  int width;                   // elements per row
+
+  template <typename T>
+  __device__ __forceinline__ const T* row(int seq, int64_t j) const {
+    const T* b = reinterpret_cast<const T*>(base);
+    if (block_table == nullptr) return b + ((int64_t)seq * seq_stride + j) * width;
+    int page = __ldg(block_table + (int64_t)seq * max_pages + j / page_size);
+    if (page < 0) return nullptr;  // unallocated page: read as an empty key
+    return b + ((int64_t)page * page_size + (j % page_size)) * width;
+  }
+};
+
+// Query rows: prefill row r = seq*S + t; decode row r = seq with t = ctx_lens[seq] - 1.
+struct QueryRows {
+  int S;                     // prefill tokens per sequence (0 for decode)
+  const int32_t* ctx_lens;   // decode only
+  int64_t row0;              // first flat row of this launch (prefill chunking)
+
+  __device__ __forceinline__ void locate(int64_t r, int& seq, int64_t& t) const {
+    if (ctx_lens != nullptr) {
+      seq = (int)r;
+      t = (int64_t)__ldg(ctx_lens + r) - 1;
+    } else {
+      seq = (int)(r / S);
+      t = r % S;
+    }
+  }
+};
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace sac

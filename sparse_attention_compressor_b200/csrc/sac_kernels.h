@@ -1,0 +1,61 @@
+// Host-side launch interface of the library's kernels (internal; the public ABI is include/sac.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sac_common.cuh"
+
+namespace sac {
+
+// ---- compressor + rotations (compress.cu) --------------------------------------------------
+// Pool of x [B,S,C]: entry w pools the window [(w+1)m - L, (w+1)m) (clipped at 0) with a softmax
+// gate; with rotate != 0 the entry is then rotated at pos0 + w*m. out [B,N,C].
+cudaError_t launch_compress(int dtype, const void* x, const void* gate, const float* bias, int B,
+                            int S, int C, int m, int L, bool rotate, const RopeFreqs& rf,
+                            int64_t pos0, void* out, cudaStream_t st);
+// out[b,t] = x[b,t] with its trailing R channels rotated at pos0 + t. x, out [B*S, C].
+cudaError_t launch_rotate_rows(int dtype, const void* x, int64_t rows, int S, int C,
+                               const RopeFreqs& rf, int64_t pos0, void* out, cudaStream_t st);
+
+// ---- indexer (indexer.cu) -----------------------------------------------------------------
+struct IndexerArgs {
+  const void* q_idx;     // [rows, nI, cI] (flat query rows starting at qr.row0)
+  const float* w_idx;    // [rows, nI]
+  RowAddr kpool;         // indexer pool rows (width cI)
+  QueryRows qr;
+  int nI, cI, m;
+  int64_t nrows;         // rows in this launch
+  int n_stride;          // scores row stride (>= largest visible count)
+  float* scores;         // [nrows, n_stride]; entries w < (t+1)//m written
+};
+cudaError_t launch_indexer(int dtype, const IndexerArgs& a, int max_visible, cudaStream_t st);
+
+// ---- top-k (topk.cu) ----------------------------------------------------------------------
+// Per row: the k largest of the first (t+1)//m scores, ties to the lower index, written in
+// ascending entry order followed by -1.
+cudaError_t launch_topk(const float* scores, int n_stride, QueryRows qr, int m, int64_t nrows,
+                        int k, int32_t* out, cudaStream_t st);
+int topk_max_entries();
+
+// ---- attention (attention_simt.cu) --------------------------------------------------------
+struct AttnArgs {
+  const void* q;         // [rows, H, D] un-rotated
+  void* o;               // [rows, H, D]
+  const float* sinks;    // [H]
+  QueryRows qr;
+  int64_t nrows;
+  int H, D, W;
+  float scale;
+  int64_t pos0;
+  RowAddr win;           // rotated kv rows
+  int pool_mode;         // 0: none, 1: all visible entries (t+1)//m, 2: selection list
+  RowAddr pool;          // rotated pool rows
+  int m;
+  const int32_t* sel;    // [rows, k] for pool_mode 2
+  int k;
+  RopeFreqs rf;
+};
+cudaError_t launch_attention_simt(int dtype, const AttnArgs& a, cudaStream_t st);
+
+}  // namespace sac

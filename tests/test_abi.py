@@ -1,0 +1,125 @@
+"""The C-ABI library loads, exports every entry point include/sac.h declares, and rejects bad
+arguments on the host with the documented status codes (no GPU needed: validation runs before any
+CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_compressor_b200 as sac
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sac.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"SAC_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return sac.load_library()
+
+
+def test_header_declares_the_abi():
+    assert set(declared_symbols()) == set(sac.ABI_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert sac.sac_version() == 100
+
+
+def test_params_struct_layout_matches_header():
+    # B,S,H,D,R ints (20) + pad (4) + double (8) + 6 ints (24) + float (4) + pad (4) + int64 (8)
+    # + int (4) + pad (4)
+    assert ctypes.sizeof(sac.sac_params) == 80
+    assert sac.sac_params.rope_theta.offset == 24
+    assert sac.sac_params.pos0.offset == 64
+
+
+def p_csa(**kw):
+    base = dict(B=1, S=8192, H=64, D=512, R=64, rope_theta=160000.0, m=4, win_len=8,
+                sliding_window=128, n_idx_heads=64, idx_dim=128, topk=512)
+    base.update(kw)
+    return sac.make_params(**base)
+
+
+def test_workspace_sizes():
+    p = p_csa()
+    n = 8192 // 4
+    ws = sac.sac_workspace_size(p, sac.SAC_KIND_CSA)
+    # rotated kv + pool + indexer pool + scores + top-k, each 256-byte aligned
+    expect = 8192 * 512 * 2 + n * 512 * 2 + n * 128 * 2 + 8192 * n * 4 + 8192 * 512 * 4
+    assert ws == expect
+    assert sac.sac_workspace_size(p, sac.SAC_KIND_SWA) == 8192 * 512 * 2
+    assert sac.sac_workspace_size(p_csa(m=128, win_len=128), sac.SAC_KIND_HCA) == \
+        8192 * 512 * 2 + 64 * 512 * 2
+    assert sac.sac_decode_workspace_size(p_csa(S=65536), sac.SAC_KIND_CSA, 64) == \
+        64 * 16384 * 4 + 64 * 512 * 4
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_HCA, 64) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(D=96), -2), (dict(D=1024), -2), (dict(R=63), -2), (dict(R=66 * 2), -2),
+    (dict(dtype="f16"), None), (dict(S=0), -1), (dict(H=0), -1), (dict(sliding_window=0), -1),
+    (dict(idx_dim=48), -2), (dict(topk=0), -1), (dict(m=0), -1), (dict(S=4 * 60000), -2),
+    (dict(softmax_scale=-1.0), -1), (dict(rope_theta=0.0), -1),
+])
+def test_invalid_params_rejected_on_host(bad, code):
+    kw = dict(bad)
+    if kw.get("dtype") == "f16":
+        p = p_csa()
+        p.dtype = 7
+        code = -2
+    else:
+        p = p_csa(**kw)
+    assert sac.sac_workspace_size(p, sac.SAC_KIND_CSA) == 0
+    lib = sac.load_library()
+    fake = 1 << 20  # never dereferenced: validation fails first
+    rc = lib.csa_forward(ctypes.byref(p), *([fake] * 11), None, None, None, fake, 1 << 40, None)
+    assert rc == code
+    assert lib.sac_last_error().decode() != ""
+
+
+def test_null_and_misaligned_pointers_rejected():
+    lib = sac.load_library()
+    p = p_csa()
+    fake = 1 << 20
+    args = [fake] * 11
+    args[0] = None
+    rc = lib.csa_forward(ctypes.byref(p), *args, None, None, None, fake, 1 << 40, None)
+    assert rc == -1
+    assert "q must not be NULL" in lib.sac_last_error().decode()
+    args = [fake] * 11
+    args[1] = fake + 2
+    rc = lib.csa_forward(ctypes.byref(p), *args, None, None, None, fake, 1 << 40, None)
+    assert rc == -1 and "aligned" in lib.sac_last_error().decode()
+
+
+def test_small_workspace_rejected():
+    lib = sac.load_library()
+    p = p_csa()
+    fake = 1 << 20
+    need = sac.sac_workspace_size(p, sac.SAC_KIND_CSA)
+    rc = lib.csa_forward(ctypes.byref(p), *([fake] * 11), None, None, None, fake, need - 1, None)
+    assert rc == -3 and "workspace" in lib.sac_last_error().decode()
+    p2 = sac.make_params(1, 1024, 8, 128, 32, 1e4, sliding_window=16)
+    rc = lib.swa_forward(ctypes.byref(p2), fake, fake, fake, fake, None, 0, None)
+    assert rc == -3
+
+
+def test_decode_validation():
+    lib = sac.load_library()
+    p = p_csa(S=65536, m=128, win_len=128)
+    fake = 1 << 20
+    # kv block table too short for contexts up to S
+    rc = lib.hca_decode(ctypes.byref(p), 4, fake, fake, fake, 10, fake, 64, fake, fake, 8, fake,
+                        fake, None, 0, None)
+    assert rc == -1 and "block table" in lib.sac_last_error().decode()
+    rc = lib.hca_decode(ctypes.byref(p), 0, fake, fake, fake, 1024, fake, 64, fake, fake, 8, fake,
+                        fake, None, 0, None)
+    assert rc == -1 and "nseq" in lib.sac_last_error().decode()
