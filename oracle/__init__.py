@@ -34,6 +34,7 @@ class _Params(ctypes.Structure):
         ("R", ctypes.c_int), ("theta", ctypes.c_double), ("m", ctypes.c_int),
         ("L", ctypes.c_int), ("W", ctypes.c_int), ("nI", ctypes.c_int), ("cI", ctypes.c_int),
         ("k", ctypes.c_int), ("scale", ctypes.c_double), ("pos0", ctypes.c_int64),
+        ("bf16_pools", ctypes.c_int),
     ]
 
 
@@ -54,11 +55,13 @@ class OracleParams:
     k: int = 0
     scale: float = 0.0
     pos0: int = 0
+    bf16_pools: bool = False  # pools cached in bf16 (the layer's working dtype)
 
     def c(self) -> _Params:
         scale = self.scale if self.scale > 0 else 1.0 / np.sqrt(self.D)
         return _Params(self.B, self.S, self.H, self.D, self.R, float(self.theta), self.m,
-                       self.L, self.W, self.nI, self.cI, self.k, float(scale), int(self.pos0))
+                       self.L, self.W, self.nI, self.cI, self.k, float(scale), int(self.pos0),
+                       int(self.bf16_pools))
 
 
 def build(force: bool = False) -> str:
@@ -95,6 +98,8 @@ def _lib():
         lib.orc_csa_index_scores.argtypes = [P, _dp, _dp, _dp, _dp, _dp, _lp, ctypes.c_long, _dp]
         lib.orc_decode.argtypes = [P, ctypes.c_int, _dp, _dp, _ip, ctypes.c_int, _ip, ctypes.c_int,
                                    _dp, _dp, _ip, ctypes.c_int, _dp, _dp, _dp, _dp, _ip, _ip]
+        lib.orc_round_bf16.restype = ctypes.c_double
+        lib.orc_round_bf16.argtypes = [ctypes.c_double]
         lib.orc_max_threads.restype = ctypes.c_int
         lib.orc_set_threads.argtypes = [ctypes.c_int]
         _lib_handle = lib
@@ -120,6 +125,11 @@ def _i32(x) -> np.ndarray:
 
 def _ptr(a, kind=_dp):
     return None if a is None else a.ctypes.data_as(kind)
+
+
+def round_bf16(x: float) -> float:
+    """A pool value as cached in bf16 (nearest, ties to even, from its fp32 value)."""
+    return float(_lib().orc_round_bf16(float(x)))
 
 
 def max_threads() -> int:

@@ -36,6 +36,7 @@ typedef struct {
   int nI, cI, k;       /* index_n_heads, index_head_dim, index_topk (CSA only)                */
   double scale;        /* softmax scale tau                                                   */
   int64_t pos0;        /* absolute position of token 0                                        */
+  int bf16_pools;      /* 1: pools are cached in bf16 (see orc_round_bf16)                     */
 } orc_params;
 
 int orc_max_threads(void) {
@@ -52,6 +53,25 @@ void orc_set_threads(int n) {
 #else
   (void)n;
 #endif
+}
+
+/* [reading] The compressor's pools are cached tensors ("Cache layers": compressor / indexer
+ * pool) held in the layer's working dtype. For a bf16 layer each stored pool entry is the fp32
+ * value rounded to the nearest bf16, ties to even. The top-k is an integer decision taken from
+ * scores of the stored indexer pool, so the oracle scores the same stored values. */
+double orc_round_bf16(double x) {
+  float f = (float)x;
+  uint32_t u;
+  memcpy(&u, &f, sizeof(u));
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  u &= 0xFFFF0000u;
+  memcpy(&f, &u, sizeof(f));
+  return (double)f;
+}
+
+static void round_pool(const orc_params *p, double *x, size_t n) {
+  if (!p->bf16_pools) return;
+  for (size_t i = 0; i < n; ++i) x[i] = orc_round_bf16(x[i]);
 }
 
 /* ---------------------------------------------------------------------------------------------
@@ -265,6 +285,7 @@ static long rotated_pool(const orc_params *p, const double *kv, const double *u,
   for (int b = 0; b < p->B; ++b)
     for (long w = 0; w < N; ++w)
       orc_rope(pool + ((size_t)b * N + w) * p->D, p->D, p->R, p->theta, entry_pos(p, w));
+  round_pool(p, pool, (size_t)p->B * N * p->D);
   return N;
 }
 
@@ -310,6 +331,7 @@ int orc_csa_forward(const orc_params *p, const double *q, const double *kv, cons
   /* the indexer pool: same windows over the indexer key stream, its own gate, no rotation
    * ("Cache layers": parallel indexer buffer / pool / count / overlap at index_head_dim) */
   orc_compress(p->B, p->S, p->cI, p->m, p->L, kI, uI, bI, kpool);
+  round_pool(p, kpool, (size_t)p->B * N * p->cI);
   if (pool_out) memcpy(pool_out, pool, sizeof(double) * (size_t)p->B * N * p->D);
   if (idx_pool_out) memcpy(idx_pool_out, kpool, sizeof(double) * (size_t)p->B * N * p->cI);
   long total = rows ? nrows : (long)p->B * p->S;
@@ -362,6 +384,7 @@ int orc_csa_index_scores(const orc_params *p, const double *qI, const double *wI
   long N = p->S / p->m;
   double *kpool = (double *)malloc(sizeof(double) * ((size_t)p->B * N * p->cI + 1));
   orc_compress(p->B, p->S, p->cI, p->m, p->L, kI, uI, bI, kpool);
+  round_pool(p, kpool, (size_t)p->B * N * p->cI);
 #pragma omp parallel for schedule(dynamic, 1)
   for (long i = 0; i < nrows; ++i) {
     long r = (long)rows[i];

@@ -18,7 +18,8 @@ TIE_REL = 1e-3
 
 def oracle_params(wl: W.Workload, pos0: int = 0) -> oracle.OracleParams:
     return oracle.OracleParams(wl.B, wl.S, wl.H, wl.D, wl.R, wl.theta, wl.W, m=wl.m, L=wl.L,
-                               nI=wl.nI, cI=wl.cI, k=wl.k, pos0=pos0)
+                               nI=wl.nI, cI=wl.cI, k=wl.k, pos0=pos0,
+                               bf16_pools=wl.dtype == "bf16")
 
 
 def sac_params(wl: W.Workload, pos0: int = 0):

@@ -552,3 +552,28 @@ def test_decode_equals_prefill_row(kind):
         q_idx=None if kind != "csa" else d["q_idx"][0, ts],
         w_idx=None if kind != "csa" else d["w_idx"][0, ts], sinks=d["sinks"])
     np.testing.assert_allclose(o, full[ts], atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------------------
+# bf16 storage of the pools
+# ------------------------------------------------------------------------------------------------
+def test_round_bf16_matches_torch_conversion():
+    r = rng(50)
+    vals = np.concatenate([r.standard_normal(20000) * 10.0 ** r.integers(-6, 6, 20000),
+                           [0.0, -0.0, 1.0, -1.0, 3.0e38, 1e-40]])
+    # torch converts float32 -> bfloat16 with round-to-nearest-even
+    ref = torch.from_numpy(vals.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    got = np.array([oracle.round_bf16(v) for v in vals])
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_bf16_pools_round_the_stored_entries():
+    p = _tiny("csa")
+    d = _inputs(p, 51)
+    args = (d["q"], d["kv"], d["cmp_gate"], d["cmp_bias"], d["q_idx"], d["w_idx"], d["k_idx"],
+            d["idx_gate"], d["idx_bias"], d["sinks"])
+    _, _, pool, kpool = oracle.csa_forward(p, *args)
+    p.bf16_pools = True
+    _, _, pool_r, kpool_r = oracle.csa_forward(p, *args)
+    np.testing.assert_array_equal(pool_r, np.vectorize(oracle.round_bf16)(pool))
+    np.testing.assert_array_equal(kpool_r, np.vectorize(oracle.round_bf16)(kpool))
