@@ -111,6 +111,27 @@ SAC_API int swa_forward(const sac_params* p, const void* q, const void* kv, cons
                 void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * swa_forward without any device allocation by the caller: the same computation and kernels as
+ * swa_forward, with the scratch that swa_forward takes from `ws` (the rotated kv stream,
+ * B*S*D elements of dtype) held instead in a fixed 16 MiB array inside this library (a static
+ * __device__ array present on every GPU that loads the library, until the process exits).
+ * The page has no counterpart of this entry point; it exists for callers that cannot call
+ * cudaMalloc: code that runs inside a host framework whose caching allocator owns all device
+ * memory and does not lend it to plug-ins, and serving loops that forbid any allocation after
+ * start-up so that memory use stays fixed.
+ *   - Returns SAC_ERR_UNSUPPORTED when B*S*D*sizeof(dtype) exceeds sac_static_scratch_bytes().
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents; every byte a call
+ *     reads is first written by the same call. Calls that overlap on the GPU (concurrent streams
+ *     or devices sharing nothing but this array per device) race on it: serialise them.
+ *   - Allocates nothing: no cudaMalloc / cudaFree and no allocating library routine.
+ */
+SAC_API size_t sac_static_scratch_bytes(void);
+SAC_API int swa_forward_static(const sac_params* p, const void* q, const void* kv,
+                               const float* sinks, void* o, void* stream);
+
+/*
  * Heavily compressed attention forward ("Hybrid attention": HCA, m'=128, non-overlapping
  * windows, no indexer; "Attention mask layout": entry w visible to t iff w < (t+1)//m).
  *   cmp_gate [D] (dtype), cmp_bias [win_len] fp32: compressor gate. Entry w pools the window

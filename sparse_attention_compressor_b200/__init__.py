@@ -20,7 +20,8 @@ SAC_F32, SAC_BF16 = 0, 1
 SAC_KIND_SWA, SAC_KIND_HCA, SAC_KIND_CSA = 0, 1, 2
 ABI_SYMBOLS = ("sac_last_error", "sac_version", "sac_workspace_size", "swa_forward",
                "hca_forward", "csa_forward", "sac_decode_workspace_size", "swa_decode",
-               "hca_decode", "csa_decode", "sac_timing_begin", "sac_timing_end")
+               "hca_decode", "csa_decode", "sac_timing_begin", "sac_timing_end",
+               "sac_static_scratch_bytes", "swa_forward_static")
 
 
 class SacError(RuntimeError):
@@ -87,6 +88,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                vp]
     lib.csa_decode.argtypes = [P, ci, vp, vp, i32p, ci, i32p, ci, vp, vp, i32p, ci, vp, fp, fp,
                                vp, i32p, vp, sz, vp]
+    lib.sac_static_scratch_bytes.restype = sz
+    lib.swa_forward_static.restype = ci
+    lib.swa_forward_static.argtypes = [P, vp, vp, fp, vp, vp]
     lib.sac_timing_begin.restype = ci
     lib.sac_timing_end.restype = ci
     lib.sac_timing_end.argtypes = [ctypes.POINTER(sac_kernel_time), ci]
@@ -156,6 +160,17 @@ def swa_forward(p, q, kv, sinks, o, ws, stream=None) -> None:
     _check("swa_forward", load_library().swa_forward(
         ctypes.byref(p), _ptr(q), _ptr(kv), _ptr(sinks), _ptr(o), _ptr(ws), _nbytes(ws),
         _stream(stream)))
+
+
+def sac_static_scratch_bytes() -> int:
+    return int(load_library().sac_static_scratch_bytes())
+
+
+def swa_forward_static(p, q, kv, sinks, o, stream=None) -> None:
+    """swa_forward with the library's fixed scratch array instead of a caller workspace: for
+    callers that cannot allocate device memory (see include/sac.h)."""
+    _check("swa_forward_static", load_library().swa_forward_static(
+        ctypes.byref(p), _ptr(q), _ptr(kv), _ptr(sinks), _ptr(o), _stream(stream)))
 
 
 def hca_forward(p, q, kv, cmp_gate, cmp_bias, sinks, o, pool_out, ws, stream=None) -> None:

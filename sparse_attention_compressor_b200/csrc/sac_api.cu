@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "sac.h"
 #include "sac_kernels.h"
@@ -198,6 +199,78 @@ int swa_forward(const sac_params* p, const void* q, const void* kv, const float*
   sac::RopeFreqs rf = rope_freqs(p);
   const int64_t rows = (int64_t)p->B * p->S;
   cudaError_t e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
+  sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.qr = sac::QueryRows{p->S, nullptr, 0};
+  a.nrows = rows;
+  a.win = contiguous(kv_rot, p->S, p->D);
+  a.pool_mode = 0;
+  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// swa_forward_static: the sliding-window forward with its scratch (the rotated kv stream) in a
+// fixed device array owned by this library, for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------------------------
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB on every device that loads us
+constexpr int kMaxDevices = 64;
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device, looked up once per device (the host
+// symbol is only a stand-in: kernels must be given this address).
+int static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  REQUIRE(dev >= 0 && dev < kMaxDevices, SAC_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_static_scratch_mu);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_scratch_addr[dev] = ptr;
+  }
+  *out = g_static_scratch_addr[dev];
+  return SAC_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t sac_static_scratch_bytes(void) { return kStaticScratchBytes; }
+
+int swa_forward_static(const sac_params* p, const void* q, const void* kv, const float* sinks,
+                       void* o, void* stream) {
+  int rc = check_params(p, SAC_KIND_SWA, false);
+  if (rc) return rc;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kv);
+  REQUIRE_PTR(sinks);
+  REQUIRE_PTR(o);
+  const size_t need = (size_t)p->B * p->S * p->D * esize(p->dtype);
+  REQUIRE(need <= kStaticScratchBytes, SAC_ERR_UNSUPPORTED,
+          "B*S*head_dim needs %zu bytes of scratch; the static scratch holds %zu", need,
+          kStaticScratchBytes);
+  void* kv_rot = nullptr;
+  rc = static_scratch_address(&kv_rot);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  sac::RopeFreqs rf = rope_freqs(p);
+  const int64_t rows = (int64_t)p->B * p->S;
+  cudaError_t e = sac::timed("rotate_kv", st, [&] {
+    return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st);
+  });
   if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
   sac::AttnArgs a = attn_common(p, q, o, sinks);
   a.qr = sac::QueryRows{p->S, nullptr, 0};
