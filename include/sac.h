@@ -198,6 +198,15 @@ SAC_API int csa_decode(const sac_params* p, int nseq, const void* q, const void*
                size_t ws_bytes, void* stream);
 
 /*
+ * Device status of the last prefill call that used workspace `ws` (no counterpart on the page:
+ * failure reporting). Every prefill call clears the first word of its workspace; a tensor-core
+ * kernel that gives up a bounded wait (2 s) writes a nonzero code there and returns instead of
+ * hanging. This call waits for `stream`, copies the word to *status (0 = ok, 1 = a wait timed
+ * out, 2 = misaligned shared memory) and returns SAC_OK, or SAC_ERR_LAUNCH if the copy fails.
+ */
+SAC_API int sac_device_status(const void* ws, int* status, void* stream);
+
+/*
  * Optional per-kernel timing (no counterpart on the page: a measurement aid). Between
  * sac_timing_begin() and sac_timing_end() every kernel the library launches is bracketed by a
  * pair of CUDA events recorded on the launch's own stream. sac_timing_end() waits for those

@@ -21,7 +21,7 @@ SAC_KIND_SWA, SAC_KIND_HCA, SAC_KIND_CSA = 0, 1, 2
 ABI_SYMBOLS = ("sac_last_error", "sac_version", "sac_workspace_size", "swa_forward",
                "hca_forward", "csa_forward", "sac_decode_workspace_size", "swa_decode",
                "hca_decode", "csa_decode", "sac_timing_begin", "sac_timing_end",
-               "sac_static_scratch_bytes", "swa_forward_static")
+               "sac_static_scratch_bytes", "swa_forward_static", "sac_device_status")
 
 
 class SacError(RuntimeError):
@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                vp]
     lib.csa_decode.argtypes = [P, ci, vp, vp, i32p, ci, i32p, ci, vp, vp, i32p, ci, vp, fp, fp,
                                vp, i32p, vp, sz, vp]
+    lib.sac_device_status.restype = ci
+    lib.sac_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
     lib.sac_static_scratch_bytes.restype = sz
     lib.swa_forward_static.restype = ci
     lib.swa_forward_static.argtypes = [P, vp, vp, fp, vp, vp]
@@ -160,6 +162,14 @@ def swa_forward(p, q, kv, sinks, o, ws, stream=None) -> None:
     _check("swa_forward", load_library().swa_forward(
         ctypes.byref(p), _ptr(q), _ptr(kv), _ptr(sinks), _ptr(o), _ptr(ws), _nbytes(ws),
         _stream(stream)))
+
+
+def sac_device_status(ws, stream=None) -> int:
+    """Status word of the last prefill call on workspace ws (0 = ok); waits for the stream."""
+    out = ctypes.c_int(-1)
+    _check("sac_device_status", load_library().sac_device_status(_ptr(ws), ctypes.byref(out),
+                                                                 _stream(stream)))
+    return out.value
 
 
 def sac_static_scratch_bytes() -> int:

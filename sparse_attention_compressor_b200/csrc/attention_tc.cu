@@ -1,0 +1,378 @@
+// Tensor-core (tcgen05) version of the shared K=V multi-query attention for bf16 layers with
+// 64 query heads and head_dim 512 ("Hybrid attention": shared K=V MQA; per-head sink, eq. 27;
+// partial RoPE with the -i output rotation, eq. 26; sliding-window branch + compressor entries).
+//
+// One query row at a time per CTA (persistent over rows). Its 64 heads are the M = 64 rows of
+// both contractions:  S = Q K^T  (M=64, N=64 keys, K=512)  and  O += P V  (M=64, N=256 x 2, K=64).
+// Because K = V, one shared-memory key tile serves as the K-major B operand of QK^T and as the
+// MN-major B operand of PV. Key rows are gathered with TMA tile::gather4 (four rows per copy) into
+// 128-byte-swizzled tiles: window rows from the rotated kv stream, entries from the rotated pool
+// (all visible ones, or the query's selection list). Tiles never mix the two sources.
+//
+// Tensor memory (512 columns, fp32): O[:, 0:256] in lanes 0-15 of each sub-partition and
+// O[:, 256:512] in lanes 16-31 (the M = 64 layout leaves half the lanes free, so the two output
+// halves share columns 0..255); two S buffers in columns 256..319 and 320..383.
+//
+// Warps: 0 = TMA producer, 1 = MMA issuer (one thread) and TMEM owner, 4..7 = softmax + output.
+// The softmax keeps the running max in log2 units and only moves it (and rescales O) when a tile's
+// max exceeds it by more than 8, so P <= 2^8 stays exact enough in bf16 and O is rarely touched.
+#include <cuda_bf16.h>
+
+#include "sac_kernels.h"
+#include "tc_ptx.cuh"
+#include "tma_host.h"
+
+namespace sac {
+namespace {
+
+constexpr int kHeads = 64;
+constexpr int kDim = 512;
+constexpr int kNK = 64;                          // keys per tile
+constexpr int kRegion = 64 * 128;                // [64 rows x 128 B]: one swizzle column
+constexpr int kQBytes = 8 * kRegion;             // 64 KB
+constexpr int kTileBytes = 8 * kRegion;          // 64 KB
+constexpr int kPBytes = kHeads * kNK * 2;        // 8 KB
+
+constexpr int kOffQ = 0;
+constexpr int kOffTile = kOffQ + kQBytes;                 // 2 tiles
+constexpr int kOffP = kOffTile + 2 * kTileBytes;          // 2 P buffers
+constexpr int kOffBar = kOffP + 2 * kPBytes;
+enum Bar { kQFull, kQEmpty, kKvFull0, kKvFull1, kKvEmpty0, kKvEmpty1, kSFull0, kSFull1, kPFull0,
+           kPFull1, kPvDone0, kPvDone1, kOFull, kOEmpty, kNumBars };
+constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffTmemPtr + 16 + 1024;       // + alignment slack
+
+constexpr uint32_t kColS0 = 256, kColS1 = 320;
+constexpr uint32_t kIdescQK = tc::idesc_bf16(64, kNK, false, false);
+constexpr uint32_t kIdescPV = tc::idesc_bf16(64, 256, false, true);
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazy = 8.0f;  // move the running max only when a tile exceeds it by 2^8
+
+struct Row {
+  int seq;
+  int64_t t, lo;
+  int nwin, npool, twin, tiles;
+};
+
+__device__ __forceinline__ Row locate_row(const AttnArgs& a, int64_t r) {
+  Row w;
+  a.qr.locate(a.qr.row0 + r, w.seq, w.t);
+  w.lo = w.t - a.W + 1 < 0 ? 0 : w.t - a.W + 1;
+  w.nwin = (int)(w.t - w.lo + 1);
+  const int nvis = a.pool_mode ? (int)((w.t + 1) / a.m) : 0;
+  w.npool = a.pool_mode == 2 ? (nvis < a.k ? nvis : a.k) : nvis;
+  w.twin = (w.nwin + kNK - 1) / kNK;
+  w.tiles = w.twin + (w.npool + kNK - 1) / kNK;
+  return w;
+}
+
+// Physical row (in the tensor map) of key c of tile j; keys past the tile's count reuse a valid
+// row (their logits are masked).
+__device__ __forceinline__ int32_t key_row(const AttnArgs& a, const Row& w, int64_t row, int j,
+                                           int c) {
+  if (j < w.twin) {
+    int x = j * kNK + c;
+    if (x >= w.nwin) x = 0;
+    return (int32_t)a.win.row_index(w.seq, w.lo + x);
+  }
+  int i = (j - w.twin) * kNK + c;
+  if (i >= w.npool) i = 0;
+  int64_t e = a.pool_mode == 2 ? (int64_t)__ldg(a.sel + row * a.k + i) : i;
+  return (int32_t)a.pool.row_index(w.seq, e < 0 ? 0 : e);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(256, 1)
+    attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_win,
+                        const __grid_constant__ CUtensorMap tm_pool, AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar[kQFull], 1);
+    tc::mbar_init(&bar[kQEmpty], 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bar[kKvFull0 + i], 1);
+      tc::mbar_init(&bar[kKvEmpty0 + i], 1);
+      tc::mbar_init(&bar[kSFull0 + i], 1);
+      tc::mbar_init(&bar[kPFull0 + i], 128);
+      tc::mbar_init(&bar[kPvDone0 + i], 1);
+    }
+    tc::mbar_init(&bar[kOFull], 1);
+    tc::mbar_init(&bar[kOEmpty], 128);
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_ptr, 512);
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tm_q);
+    tc::tma_prefetch_desc(&tm_win);
+    tc::tma_prefetch_desc(&tm_pool);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  int* status = a.status;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    uint32_t g = 0, qi = 0;
+    bool ok = true;
+    for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
+      const Row w = locate_row(a, r);
+      if (qi > 0) ok = __all_sync(~0u, tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status));
+      if (!ok) break;
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&bar[kQFull], kQBytes);
+        for (int c = 0; c < 8; ++c)
+          tc::tma_load_2d(smem + kOffQ + c * kRegion, &tm_q, &bar[kQFull], 64 * c,
+                          (int32_t)(r * kHeads));
+      }
+      for (int j = 0; j < w.tiles && ok; ++j, ++g) {
+        const uint32_t b = g & 1;
+        if (g >= 2)
+          ok = __all_sync(~0u, tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - 2) >> 1) & 1, status));
+        if (!ok) break;
+        if (lane == 0) tc::mbar_arrive_expect_tx(&bar[kKvFull0 + b], kTileBytes);
+        __syncwarp();
+        if (lane < kNK / 4) {
+          int32_t y[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) y[u] = key_row(a, w, r, j, lane * 4 + u);
+          const CUtensorMap* map = j < w.twin ? &tm_win : &tm_pool;
+          uint8_t* dst = smem + kOffTile + b * kTileBytes + lane * 4 * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            tc::tma_gather4(dst + c * kRegion, map, &bar[kKvFull0 + b], 64 * c, y[0], y[1], y[2],
+                            y[3]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t g0 = 0, qi = 0;
+      bool ok = true;
+      const uint32_t q_base = tc::smem_u32(smem + kOffQ);
+      for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
+        const Row w = locate_row(a, r);
+        ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
+        for (int j = 0; j <= w.tiles && ok; ++j) {
+          if (j < w.tiles) {  // S(g) = Q K^T
+            const uint32_t g = g0 + j, b = g & 1;
+            ok = tc::mbar_wait(&bar[kKvFull0 + b], (g >> 1) & 1, status);
+            if (ok && g >= 2) ok = tc::mbar_wait(&bar[kPFull0 + b], ((g - 2) >> 1) & 1, status);
+            if (!ok) break;
+            tc::tc_fence_after();
+            const uint32_t k_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
+            const uint32_t d = tmem + (b ? kColS1 : kColS0);
+#pragma unroll 4
+            for (int kk = 0; kk < kDim / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
+              tc::mma_bf16_ss(d, tc::desc_sw128(q_base + off, 0, 1024),
+                              tc::desc_sw128(k_base + off, 0, 1024), kIdescQK, kk > 0);
+            }
+            tc::mma_commit(&bar[kSFull0 + b]);
+            if (j == w.tiles - 1) tc::mma_commit(&bar[kQEmpty]);
+          }
+          if (j >= 1) {  // O += P(g) V(g)
+            const uint32_t g = g0 + j - 1, b = g & 1;
+            ok = tc::mbar_wait(&bar[kPFull0 + b], (g >> 1) & 1, status);
+            if (ok && j == 1 && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
+            if (!ok) break;
+            tc::tc_fence_after();
+            const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
+            const uint32_t p_base = tc::smem_u32(smem + kOffP + b * kPBytes);
+#pragma unroll
+            for (int kk = 0; kk < kNK / 16; ++kk) {
+              const uint64_t pd = tc::desc_sw128(p_base + kk * 32, 0, 1024);
+              const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
+              tc::mma_bf16_ss(tmem, pd,
+                              tc::desc_sw128(v_base + kk * 2048, kRegion, 1024), kIdescPV, acc);
+              tc::mma_bf16_ss(tmem + (16u << 16), pd,
+                              tc::desc_sw128(v_base + 4 * kRegion + kk * 2048, kRegion, 1024),
+                              kIdescPV, acc);
+            }
+            tc::mma_commit(&bar[kKvEmpty0 + b]);
+            tc::mma_commit(&bar[kPvDone0 + b]);
+            if (j == w.tiles) tc::mma_commit(&bar[kOFull]);
+          }
+        }
+        g0 += w.tiles;
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax + output
+    const int sp = warp & 3;                 // TMEM sub-partition of this warp
+    const int half = lane >> 4;              // 0: lanes 0-15 (S rows, O[:,0:256]); 1: O[:,256:512]
+    const int h = 16 * sp + (lane & 15);     // head of this thread's row
+    const uint32_t t_row = tmem + ((uint32_t)(32 * sp) << 16);
+    const float scale_log2 = a.scale * kLog2e;
+    const float sink_log2 = __ldg(a.sinks + h) * kLog2e;
+    uint32_t g0 = 0, qi = 0;
+    bool ok = true;
+    for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
+      const Row w = locate_row(a, r);
+      float m_run = sink_log2, l_run = 1.f;
+      for (int j = 0; j < w.tiles && ok; ++j) {
+        const uint32_t g = g0 + j, b = g & 1;
+        ok = __all_sync(~0u, tc::mbar_wait(&bar[kSFull0 + b], (g >> 1) & 1, status));
+        if (!ok) break;
+        tc::tc_fence_after();
+        float s[kNK];
+#pragma unroll
+        for (int c = 0; c < kNK; c += 16) {
+          uint32_t v[16];
+          tc::tmem_ld16(t_row + (b ? kColS1 : kColS0) + c, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 16; ++u) s[c + u] = __uint_as_float(v[u]);
+        }
+        const int nk = j < w.twin ? min(kNK, w.nwin - j * kNK)
+                                  : min(kNK, w.npool - (j - w.twin) * kNK);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kNK; ++c) {
+          s[c] = c < nk ? s[c] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, s[c]);
+        }
+        const bool move = half == 0 && mx > m_run + kLazy;
+        const float m_new = move ? mx : m_run;
+        const float alpha = exp2f(m_run - m_new);
+        // rescale the rows of O this warp owns (rare: only when some row's max moved)
+        if (__any_sync(0xffffffffu, move) && j > 0) {
+          const uint32_t gp = g - 1;
+          ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + (gp & 1)], (gp >> 1) & 1, status));
+          if (!ok) break;
+          tc::tc_fence_after();
+          const float al = __shfl_sync(0xffffffffu, alpha, lane & 15);
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 16) {
+            uint32_t v[16];
+            tc::tmem_ld16(t_row + c, v);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * al);
+            tc::tmem_st16(t_row + c, v);
+          }
+          tc::tmem_wait_st();
+        }
+        float sum = 0.f;
+        uint32_t pk[kNK / 2];
+#pragma unroll
+        for (int c = 0; c < kNK; c += 2) {
+          const float p0 = exp2f(s[c] - m_new), p1 = exp2f(s[c + 1] - m_new);
+          sum += p0 + p1;
+          pk[c / 2] = pack_bf16(p0, p1);
+        }
+        l_run = l_run * alpha + sum;
+        m_run = m_new;
+        // P buffer b is free once PV(g-2) completed
+        if (g >= 2)
+          ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + b], ((g - 2) >> 1) & 1, status));
+        if (!ok) break;
+        if (half == 0) {
+          uint8_t* prow = smem + kOffP + b * kPBytes + h * 128;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(prow + ((ch ^ (h & 7)) << 4)) =
+                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        }
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&bar[kPFull0 + b]);
+      }
+      if (!ok) break;
+      // ---- output: O / l, the rope slice turned by -P_t, bf16 store. Lane p holds the cos/sin
+      // of rope pair p; the rotation reads them with warp shuffles.
+      const int64_t P = a.pos0 + w.t;
+      float my_c = 1.f, my_s = 0.f;
+      if (lane < a.rf.R / 2) rope_cos_sin(a.rf, lane, -P, my_c, my_s);
+      ok = __all_sync(~0u, tc::mbar_wait(&bar[kOFull], qi & 1, status));
+      if (!ok) break;
+      tc::tc_fence_after();
+      const float inv_l = 1.f / __shfl_sync(0xffffffffu, l_run, lane & 15);
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + ((int64_t)r * kHeads + h) * kDim + half * 256;
+      const int rope_lo = kDim - a.rf.R;  // first rotated channel (always in the upper half)
+#pragma unroll 1
+      for (int c = 0; c < 256; c += 16) {
+        uint32_t v[16];
+        tc::tmem_ld16(t_row + c, v);
+        tc::tmem_wait_ld();
+        float x[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) x[u] = __uint_as_float(v[u]) * inv_l;
+        if (256 + c + 16 > rope_lo) {  // warp-uniform: some upper-half lane rotates here
+#pragma unroll
+          for (int u = 0; u < 16; u += 2) {
+            const int ch = half * 256 + c + u;
+            const int p = ch >= rope_lo ? (ch - rope_lo) >> 1 : 0;
+            const float cc = __shfl_sync(0xffffffffu, my_c, p);
+            const float ss = __shfl_sync(0xffffffffu, my_s, p);
+            if (ch >= rope_lo) {
+              const float x0 = x[u], x1 = x[u + 1];
+              x[u] = x0 * cc - x1 * ss;
+              x[u + 1] = x0 * ss + x1 * cc;
+            }
+          }
+        }
+        uint4 o0 = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                              pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+        uint4 o1 = make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]),
+                              pack_bf16(x[12], x[13]), pack_bf16(x[14], x[15]));
+        reinterpret_cast<uint4*>(orow + c)[0] = o0;
+        reinterpret_cast<uint4*>(orow + c)[1] = o1;
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bar[kOEmpty]);
+      g0 += w.tiles;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool attention_tc_supported(const AttnArgs& a, int dtype) {
+  return dtype == 1 && a.H == kHeads && a.D == kDim && a.rf.R <= 64 && a.rf.R % 2 == 0;
+}
+
+cudaError_t launch_attention_tc(const AttnArgs& a, const void* q_rot, int64_t win_rows,
+                                int64_t pool_rows, cudaStream_t st) {
+  if (a.nrows == 0) return cudaSuccess;
+  CUtensorMap tq, tw, tp;
+  cudaError_t e = make_tmap_bf16_2d(&tq, q_rot, (uint64_t)a.nrows * kHeads, kDim, kDim * 2, 64, 64);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16_2d(&tw, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, 1, 64);
+  if (e != cudaSuccess) return e;
+  const bool has_pool = a.pool_mode != 0 && pool_rows > 0;
+  e = make_tmap_bf16_2d(&tp, has_pool ? a.pool.base : a.win.base,
+                        (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, 1, 64);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = (int)(a.nrows < sms ? a.nrows : sms);
+  attention_tc_kernel<<<grid, 256, kSmemBytes, st>>>(tq, tw, tp, a);
+  return cudaGetLastError();
+}
+
+}  // namespace sac

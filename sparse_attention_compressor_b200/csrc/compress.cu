@@ -146,14 +146,14 @@ __global__ void __launch_bounds__(256) compress_kernel(const T* __restrict__ x,
 template <typename T, int V>
 __global__ void __launch_bounds__(256) rotate_rows_kernel(const T* __restrict__ x, int64_t rows,
                                                           int S, RopeFreqs rf, int64_t pos0,
-                                                          T* __restrict__ out) {
+                                                          T* __restrict__ out, int rows_per_pos) {
   constexpr int C = 32 * V;
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (r >= rows) return;
   float v[V];
   load_lane<T, V>(x + r * C, lane, v);
-  rotate_lane<V>(v, lane, C, rf, pos0 + r % S);
+  rotate_lane<V>(v, lane, C, rf, pos0 + (r / rows_per_pos) % S);
   store_lane<T, V>(out + r * C, lane, v);
 }
 
@@ -177,10 +177,11 @@ cudaError_t compress_t(const void* x, const void* gate, const float* bias, int B
 
 template <typename T, int V>
 cudaError_t rotate_t(const void* x, int64_t rows, int S, const RopeFreqs& rf, int64_t pos0,
-                     void* out, cudaStream_t st) {
+                     void* out, cudaStream_t st, int rows_per_pos) {
   if (rows == 0) return cudaSuccess;
   rotate_rows_kernel<T, V><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)x, rows, S, rf,
-                                                                        pos0, (T*)out);
+                                                                        pos0, (T*)out,
+                                                                        rows_per_pos);
   return cudaGetLastError();
 }
 
@@ -206,8 +207,8 @@ static cudaError_t compress_dispatch(const void* x, const void* gate, const floa
 
 template <typename T>
 static cudaError_t rotate_dispatch(const void* x, int64_t rows, int S, int C, const RopeFreqs& rf,
-                                   int64_t pos0, void* out, cudaStream_t st) {
-  SAC_DISPATCH_C(C, rotate_t, x, rows, S, rf, pos0, out, st)
+                                   int64_t pos0, void* out, cudaStream_t st, int rows_per_pos) {
+  SAC_DISPATCH_C(C, rotate_t, x, rows, S, rf, pos0, out, st, rows_per_pos)
 }
 
 cudaError_t launch_compress(int dtype, const void* x, const void* gate, const float* bias, int B,
@@ -220,9 +221,10 @@ cudaError_t launch_compress(int dtype, const void* x, const void* gate, const fl
 }
 
 cudaError_t launch_rotate_rows(int dtype, const void* x, int64_t rows, int S, int C,
-                               const RopeFreqs& rf, int64_t pos0, void* out, cudaStream_t st) {
-  if (dtype == 0) return rotate_dispatch<float>(x, rows, S, C, rf, pos0, out, st);
-  return rotate_dispatch<__nv_bfloat16>(x, rows, S, C, rf, pos0, out, st);
+                               const RopeFreqs& rf, int64_t pos0, void* out, cudaStream_t st,
+                               int rows_per_pos) {
+  if (dtype == 0) return rotate_dispatch<float>(x, rows, S, C, rf, pos0, out, st, rows_per_pos);
+  return rotate_dispatch<__nv_bfloat16>(x, rows, S, C, rf, pos0, out, st, rows_per_pos);
 }
 
 }  // namespace sac

@@ -120,11 +120,19 @@ struct Carve {
   }
 };
 
+// bf16 layers with 64 heads of 512 run the attention on tcgen05 (attention_tc.cu).
+bool use_tc_attention(const sac_params* p) {
+  return p->dtype == SAC_BF16 && p->H == 64 && p->D == 512 && p->R <= 64;
+}
+
+constexpr size_t kStatusBytes = 256;  // device status word at the start of every workspace
+
 struct Sizes {
-  size_t kv_rot = 0, pool = 0, idx_pool = 0, scores = 0, topk = 0;
+  size_t status = kStatusBytes, kv_rot = 0, q_rot = 0, pool = 0, idx_pool = 0, scores = 0,
+         topk = 0;
   size_t total() const {
-    return align_up(kv_rot) + align_up(pool) + align_up(idx_pool) + align_up(scores) +
-           align_up(topk);
+    return align_up(status) + align_up(kv_rot) + align_up(q_rot) + align_up(pool) +
+           align_up(idx_pool) + align_up(scores) + align_up(topk);
   }
 };
 
@@ -132,6 +140,7 @@ Sizes prefill_sizes(const sac_params* p, int kind) {
   Sizes s;
   const size_t rows = (size_t)p->B * p->S;
   s.kv_rot = rows * p->D * esize(p->dtype);
+  if (use_tc_attention(p)) s.q_rot = rows * p->H * p->D * esize(p->dtype);
   if (kind == SAC_KIND_HCA || kind == SAC_KIND_CSA)
     s.pool = (size_t)p->B * (p->S / p->m) * p->D * esize(p->dtype);
   if (kind == SAC_KIND_CSA) {
@@ -148,6 +157,24 @@ sac::RowAddr contiguous(const void* base, int64_t seq_stride, int width) {
 
 sac::RowAddr paged(const void* base, const int32_t* bt, int max_pages, int page_size, int width) {
   return sac::RowAddr{base, bt, 0, max_pages, page_size, width};
+}
+
+// The attention step of a prefill call: the tensor-core kernel (after rotating q once into
+// q_rot) for bf16 64 x 512 layers, the CUDA-core kernel otherwise.
+cudaError_t run_attention(const sac_params* p, const sac::AttnArgs& a, void* q_rot,
+                          int64_t win_rows, int64_t pool_rows, cudaStream_t st) {
+  if (use_tc_attention(p)) {
+    const int64_t qrows = (int64_t)p->B * p->S * p->H;
+    cudaError_t e = sac::timed("rotate_q", st, [&] {
+      return sac::launch_rotate_rows(p->dtype, a.q, qrows, p->S, p->D, a.rf, p->pos0, q_rot, st,
+                                     p->H);
+    });
+    if (e != cudaSuccess) return e;
+    return sac::timed("attention", st, [&] {
+      return sac::launch_attention_tc(a, q_rot, win_rows, pool_rows, st);
+    });
+  }
+  return sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
 }
 
 sac::AttnArgs attn_common(const sac_params* p, const void* q, void* o, const float* sinks) {
@@ -195,17 +222,22 @@ int swa_forward(const sac_params* p, const void* q, const void* kv, const float*
   REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carve cv(ws);
+  int* status = static_cast<int*>(cv.take(sz.status));
   void* kv_rot = cv.take(sz.kv_rot);
+  void* q_rot = cv.take(sz.q_rot);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
   sac::RopeFreqs rf = rope_freqs(p);
   const int64_t rows = (int64_t)p->B * p->S;
-  cudaError_t e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
+  e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
   if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
   sac::AttnArgs a = attn_common(p, q, o, sinks);
   a.qr = sac::QueryRows{p->S, nullptr, 0};
   a.nrows = rows;
   a.win = contiguous(kv_rot, p->S, p->D);
   a.pool_mode = 0;
-  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  a.status = status;
+  e = run_attention(p, a, q_rot, rows, 0, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -301,11 +333,15 @@ int hca_forward(const sac_params* p, const void* q, const void* kv, const void* 
   REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carve cv(ws);
+  int* status = static_cast<int*>(cv.take(sz.status));
   void* kv_rot = cv.take(sz.kv_rot);
+  void* q_rot = cv.take(sz.q_rot);
   void* pool = pool_out ? pool_out : cv.take(sz.pool);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
   sac::RopeFreqs rf = rope_freqs(p);
   const int64_t rows = (int64_t)p->B * p->S;
-  cudaError_t e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
+  e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
   if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
   e = sac::timed("compress", st, [&] { return sac::launch_compress(p->dtype, kv, cmp_gate, cmp_bias, p->B, p->S, p->D, p->m, p->win_len,
                            true, rf, p->pos0, pool, st); });
@@ -316,7 +352,8 @@ int hca_forward(const sac_params* p, const void* q, const void* kv, const void* 
   a.win = contiguous(kv_rot, p->S, p->D);
   a.pool_mode = 1;
   a.pool = contiguous(pool, p->S / p->m, p->D);
-  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  a.status = status;
+  e = run_attention(p, a, q_rot, rows, (int64_t)p->B * (p->S / p->m), st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -351,7 +388,9 @@ int csa_forward(const sac_params* p, const void* q, const void* kv, const void* 
   REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carve cv(ws);
+  int* status = static_cast<int*>(cv.take(sz.status));
   void* kv_rot = cv.take(sz.kv_rot);
+  void* q_rot = cv.take(sz.q_rot);
   void* pool = pool_out ? pool_out : cv.take(sz.pool);
   void* ipool = idx_pool_out ? idx_pool_out : cv.take(sz.idx_pool);
   float* scores = static_cast<float*>(cv.take(sz.scores));
@@ -360,7 +399,9 @@ int csa_forward(const sac_params* p, const void* q, const void* kv, const void* 
   sac::RopeFreqs rf = rope_freqs(p);
   const int64_t rows = (int64_t)p->B * p->S;
   const int N = p->S / p->m;
-  cudaError_t e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
   if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
   e = sac::timed("compress", st, [&] { return sac::launch_compress(p->dtype, kv, cmp_gate, cmp_bias, p->B, p->S, p->D, p->m, p->win_len,
                            true, rf, p->pos0, pool, st); });
@@ -401,8 +442,18 @@ int csa_forward(const sac_params* p, const void* q, const void* kv, const void* 
   a.pool_mode = 2;
   a.pool = contiguous(pool, N, p->D);
   a.sel = sel;
-  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  a.status = status;
+  e = run_attention(p, a, q_rot, rows, (int64_t)p->B * N, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+int sac_device_status(const void* ws, int* status, void* stream) {
+  REQUIRE(ws != nullptr && status != nullptr, SAC_ERR_ARG, "ws and status must not be NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(status, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
   return SAC_OK;
 }
 

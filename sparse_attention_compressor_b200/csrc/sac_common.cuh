@@ -56,6 +56,15 @@ struct RowAddr {
     if (page < 0) return nullptr;  // unallocated page: read as an empty key
     return b + ((int64_t)page * page_size + (j % page_size)) * width;
   }
+
+  // Row number of row j of sequence seq in the flat [rows, width] view of the base buffer (TMA
+  // coordinates). An unallocated page maps to row 0.
+  __device__ __forceinline__ int64_t row_index(int seq, int64_t j) const {
+    if (block_table == nullptr) return (int64_t)seq * seq_stride + j;
+    int page = __ldg(block_table + (int64_t)seq * max_pages + j / page_size);
+    if (page < 0) page = 0;
+    return (int64_t)page * page_size + (j % page_size);
+  }
 };
 
 // Query rows: prefill row r = seq*S + t; decode row r = seq with t = ctx_lens[seq] - 1.

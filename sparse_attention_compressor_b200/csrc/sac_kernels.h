@@ -14,9 +14,11 @@ namespace sac {
 cudaError_t launch_compress(int dtype, const void* x, const void* gate, const float* bias, int B,
                             int S, int C, int m, int L, bool rotate, const RopeFreqs& rf,
                             int64_t pos0, void* out, cudaStream_t st);
-// out[b,t] = x[b,t] with its trailing R channels rotated at pos0 + t. x, out [B*S, C].
+// out[r] = x[r] with its trailing R channels rotated at pos0 + (r / rows_per_pos) % S.
+// x, out [rows, C] (kv: rows_per_pos = 1; q viewed as [B*S*H, D]: rows_per_pos = H).
 cudaError_t launch_rotate_rows(int dtype, const void* x, int64_t rows, int S, int C,
-                               const RopeFreqs& rf, int64_t pos0, void* out, cudaStream_t st);
+                               const RopeFreqs& rf, int64_t pos0, void* out, cudaStream_t st,
+                               int rows_per_pos = 1);
 
 // ---- indexer (indexer.cu) -----------------------------------------------------------------
 struct IndexerArgs {
@@ -55,7 +57,15 @@ struct AttnArgs {
   const int32_t* sel;    // [rows, k] for pool_mode 2
   int k;
   RopeFreqs rf;
+  int* status;           // device status word (tensor-core kernels record wait timeouts)
 };
 cudaError_t launch_attention_simt(int dtype, const AttnArgs& a, cudaStream_t st);
+
+// ---- attention on tcgen05 (attention_tc.cu): bf16, 64 heads, head_dim 512 ------------------
+// q_rot: [nrows, 64, 512] already rotated; win/pool bases are [rows, 512] buffers whose row
+// counts (win_rows, pool_rows) bound the TMA coordinates.
+bool attention_tc_supported(const AttnArgs& a, int dtype);
+cudaError_t launch_attention_tc(const AttnArgs& a, const void* q_rot, int64_t win_rows,
+                                int64_t pool_rows, cudaStream_t st);
 
 }  // namespace sac

@@ -57,6 +57,7 @@ def gpu_prefill(wl: W.Workload, x: dict, pos0: int = 0, with_aux: bool = True) -
                         ws)
         out.update(topk=tk, pool=pool, idx_pool=ipool)
     torch.cuda.synchronize()
+    assert sac.sac_device_status(ws) == 0, "a kernel reported a device-side wait timeout"
     out["o"] = o
     return {k: (v.cpu() if v is not None else None) for k, v in out.items()}
 
