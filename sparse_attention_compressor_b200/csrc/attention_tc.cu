@@ -89,7 +89,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
 __global__ void __launch_bounds__(256, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_win,
-                        const __grid_constant__ CUtensorMap tm_pool, AttnArgs a) {
+                        const __grid_constant__ CUtensorMap tm_pool,
+                        const __grid_constant__ CUtensorMap tm_win_box,
+                        const __grid_constant__ CUtensorMap tm_pool_box, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -116,7 +118,13 @@ __global__ void __launch_bounds__(256, 1)
     tc::tma_prefetch_desc(&tm_q);
     tc::tma_prefetch_desc(&tm_win);
     tc::tma_prefetch_desc(&tm_pool);
+    tc::tma_prefetch_desc(&tm_win_box);
+    tc::tma_prefetch_desc(&tm_pool_box);
   }
+  // window rows of a prefill are consecutive rows of the rotated kv stream, and so are the
+  // entries of an HCA prefill: such tiles load as 8 boxes of [64 rows x 64 columns]
+  const bool win_contig = a.win.block_table == nullptr;
+  const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -144,7 +152,18 @@ __global__ void __launch_bounds__(256, 1)
         if (!ok) break;
         if (lane == 0) tc::mbar_arrive_expect_tx(&bar[kKvFull0 + b], kTileBytes);
         __syncwarp();
-        if (lane < kNK / 4) {
+        const bool is_win = j < w.twin;
+        if (is_win ? win_contig : pool_contig) {
+          if (lane == 0) {
+            const int64_t y0 = is_win ? a.win.row_index(w.seq, w.lo + (int64_t)j * kNK)
+                                      : a.pool.row_index(w.seq, (int64_t)(j - w.twin) * kNK);
+            const CUtensorMap* map = is_win ? &tm_win_box : &tm_pool_box;
+            uint8_t* dst = smem + kOffTile + b * kTileBytes;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              tc::tma_load_2d(dst + c * kRegion, map, &bar[kKvFull0 + b], 64 * c, (int32_t)y0);
+          }
+        } else if (lane < kNK / 4) {
           int32_t y[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) y[u] = key_row(a, w, r, j, lane * 4 + u);
@@ -355,7 +374,7 @@ bool attention_tc_supported(const AttnArgs& a, int dtype) {
 cudaError_t launch_attention_tc(const AttnArgs& a, const void* q_rot, int64_t win_rows,
                                 int64_t pool_rows, cudaStream_t st) {
   if (a.nrows == 0) return cudaSuccess;
-  CUtensorMap tq, tw, tp;
+  CUtensorMap tq, tw, tp, twb, tpb;
   cudaError_t e = make_tmap_bf16_2d(&tq, q_rot, (uint64_t)a.nrows * kHeads, kDim, kDim * 2, 64, 64);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16_2d(&tw, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, 1, 64);
@@ -364,6 +383,11 @@ cudaError_t launch_attention_tc(const AttnArgs& a, const void* q_rot, int64_t wi
   e = make_tmap_bf16_2d(&tp, has_pool ? a.pool.base : a.win.base,
                         (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, 1, 64);
   if (e != cudaSuccess) return e;
+  e = make_tmap_bf16_2d(&twb, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, kNK, 64);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16_2d(&tpb, has_pool ? a.pool.base : a.win.base,
+                        (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, kNK, 64);
+  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -371,7 +395,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, const void* q_rot, int64_t wi
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = (int)(a.nrows < sms ? a.nrows : sms);
-  attention_tc_kernel<<<grid, 256, kSmemBytes, st>>>(tq, tw, tp, a);
+  attention_tc_kernel<<<grid, 256, kSmemBytes, st>>>(tq, tw, tp, twb, tpb, a);
   return cudaGetLastError();
 }
 

@@ -410,29 +410,52 @@ int csa_forward(const sac_params* p, const void* q, const void* kv, const void* 
                            p->win_len, false, rf, p->pos0, ipool, st); });
   if (e != cudaSuccess) return cuda_fail(e, "compress indexer stream");
 
+  // indexer + top-k in chunks of query rows of one sequence (bounded scores buffer)
   const int64_t chunk = csa_chunk_rows(p);
   const size_t qi_row = (size_t)p->n_idx_heads * p->idx_dim * esize(p->dtype);
-  for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
-    const int64_t nr = chunk < rows - r0 ? chunk : rows - r0;
-    sac::QueryRows qr{p->S, nullptr, r0};
-    // largest visible count in the chunk (a chunk may span sequences)
-    int64_t t_last = (r0 + nr - 1) % p->S;
-    int max_vis = (nr >= p->S || (r0 % p->S) > t_last) ? N : (int)((t_last + 1) / p->m);
-    sac::IndexerArgs ia;
-    ia.q_idx = static_cast<const char*>(q_idx) + (size_t)r0 * qi_row;
-    ia.w_idx = w_idx + (size_t)r0 * p->n_idx_heads;
-    ia.kpool = contiguous(ipool, N, p->idx_dim);
-    ia.qr = qr;
-    ia.nI = p->n_idx_heads;
-    ia.cI = p->idx_dim;
-    ia.m = p->m;
-    ia.nrows = nr;
-    ia.n_stride = N;
-    ia.scores = scores;
-    e = sac::timed("indexer_score", st, [&] { return sac::launch_indexer(p->dtype, ia, max_vis, st); });
-    if (e != cudaSuccess) return cuda_fail(e, "indexer");
-    e = sac::timed("topk", st, [&] { return sac::launch_topk(scores, N, qr, p->m, nr, p->topk, sel + r0 * p->topk, st); });
-    if (e != cudaSuccess) return cuda_fail(e, "top-k");
+  const bool idx_tc = sac::indexer_tc_supported(p->dtype, p->n_idx_heads, p->idx_dim);
+  for (int b = 0; b < p->B; ++b) {
+    for (int64_t t0 = 0; t0 < p->S; t0 += chunk) {
+      const int64_t t1 = t0 + chunk < p->S ? t0 + chunk : p->S;
+      const int64_t r0 = (int64_t)b * p->S + t0, nr = t1 - t0;
+      sac::QueryRows qr{p->S, nullptr, r0};
+      if (idx_tc) {
+        sac::IndexerTcArgs ta;
+        ta.w_idx = w_idx;
+        ta.scores = scores;
+        ta.status = status;
+        ta.t0 = t0;
+        ta.t1 = t1;
+        ta.seq = b;
+        ta.S = p->S;
+        ta.N = N;
+        ta.m = p->m;
+        ta.n_stride = N;
+        e = sac::timed("indexer_score", st, [&] {
+          return sac::launch_indexer_tc(ta, q_idx, rows, ipool, (int64_t)p->B * N, st);
+        });
+      } else {
+        sac::IndexerArgs ia;
+        ia.q_idx = static_cast<const char*>(q_idx) + (size_t)r0 * qi_row;
+        ia.w_idx = w_idx + (size_t)r0 * p->n_idx_heads;
+        ia.kpool = contiguous(ipool, N, p->idx_dim);
+        ia.qr = qr;
+        ia.nI = p->n_idx_heads;
+        ia.cI = p->idx_dim;
+        ia.m = p->m;
+        ia.nrows = nr;
+        ia.n_stride = N;
+        ia.scores = scores;
+        const int max_vis = (int)(t1 / p->m);
+        e = sac::timed("indexer_score", st,
+                       [&] { return sac::launch_indexer(p->dtype, ia, max_vis, st); });
+      }
+      if (e != cudaSuccess) return cuda_fail(e, "indexer");
+      e = sac::timed("topk", st, [&] {
+        return sac::launch_topk(scores, N, qr, p->m, nr, p->topk, sel + r0 * p->topk, st);
+      });
+      if (e != cudaSuccess) return cuda_fail(e, "top-k");
+    }
   }
 
   sac::AttnArgs a = attn_common(p, q, o, sinks);

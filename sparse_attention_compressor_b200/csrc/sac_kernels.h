@@ -33,6 +33,19 @@ struct IndexerArgs {
 };
 cudaError_t launch_indexer(int dtype, const IndexerArgs& a, int max_visible, cudaStream_t st);
 
+// ---- indexer on tcgen05 (indexer_tc.cu): bf16, 64 heads x 128 ---------------------------
+struct IndexerTcArgs {
+  const float* w_idx;    // [B*S, nI] head weights of all query rows
+  float* scores;         // [t1 - t0, n_stride] scores of query positions t0..t1-1
+  int* status;           // device status word
+  int64_t t0, t1;        // query positions of sequence `seq` handled by this launch
+  int seq, S, N, m, n_stride;
+};
+bool indexer_tc_supported(int dtype, int nI, int cI);
+// q_idx: [q_rows_total, 64, 128] (all query rows); kpool: [kpool_rows, 128] (all sequences).
+cudaError_t launch_indexer_tc(const IndexerTcArgs& a, const void* q_idx, int64_t q_rows_total,
+                              const void* kpool, int64_t kpool_rows, cudaStream_t st);
+
 // ---- top-k (topk.cu) ----------------------------------------------------------------------
 // Per row: the k largest of the first (t+1)//m scores, ties to the lower index, written in
 // ascending entry order followed by -1.
