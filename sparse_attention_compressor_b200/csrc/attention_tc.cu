@@ -3,19 +3,25 @@
 // partial RoPE with the -i output rotation, eq. 26; sliding-window branch + compressor entries).
 //
 // One query row at a time per CTA (persistent over rows). Its 64 heads are the M = 64 rows of
-// both contractions:  S = Q K^T  (M=64, N=64 keys, K=512)  and  O += P V  (M=64, N=256 x 2, K=64).
+// both contractions:  S = Q K^T  (M=64, N=48 keys, K=512)  and  O += P V  (M=64, N=256 x 2, K=48).
 // Because K = V, one shared-memory key tile serves as the K-major B operand of QK^T and as the
-// MN-major B operand of PV. Key rows are gathered with TMA tile::gather4 (four rows per copy) into
-// 128-byte-swizzled tiles: window rows from the rotated kv stream, entries from the rotated pool
-// (all visible ones, or the query's selection list). Tiles never mix the two sources.
+// MN-major B operand of PV. Tiles of 48 keys keep three tile buffers resident next to the 64 KB
+// query tile, so the next tiles load while the tensor core works. Window rows and HCA entries are
+// consecutive rows and load as 8 TMA boxes per tile; CSA selections are gathered with TMA
+// tile::gather4 (four rows per copy) from indices staged in shared memory. Tiles never mix the
+// two sources.
+//
+// The query tile arrives un-rotated; two warps turn its rope slice (channels 448..511) in shared
+// memory before the first QK^T of the row, so no rotated copy of q is ever written to HBM.
 //
 // Tensor memory (512 columns, fp32): O[:, 0:256] in lanes 0-15 of each sub-partition and
 // O[:, 256:512] in lanes 16-31 (the M = 64 layout leaves half the lanes free, so the two output
-// halves share columns 0..255); two S buffers in columns 256..319 and 320..383.
+// halves share columns 0..255); two S buffers in columns 256..303 and 304..351.
 //
-// Warps: 0 = TMA producer, 1 = MMA issuer (one thread) and TMEM owner, 4..7 = softmax + output.
-// The softmax keeps the running max in log2 units and only moves it (and rescales O) when a tile's
-// max exceeds it by more than 8, so P <= 2^8 stays exact enough in bf16 and O is rarely touched.
+// Warps: 0 = TMA producer, 1 = MMA issuer (one thread) and TMEM owner, 2-3 = query rotation,
+// 4..7 = softmax + output. The softmax keeps the running max in log2 units and only moves it (and
+// rescales O) when a tile's max exceeds it by more than 8, so P <= 2^8 stays exact enough in bf16
+// and O is rarely touched.
 #include <cuda_bf16.h>
 
 #include "sac_kernels.h"
@@ -27,22 +33,27 @@ namespace {
 
 constexpr int kHeads = 64;
 constexpr int kDim = 512;
-constexpr int kNK = 64;                          // keys per tile
-constexpr int kRegion = 64 * 128;                // [64 rows x 128 B]: one swizzle column
-constexpr int kQBytes = 8 * kRegion;             // 64 KB
-constexpr int kTileBytes = 8 * kRegion;          // 64 KB
-constexpr int kPBytes = kHeads * kNK * 2;        // 8 KB
+constexpr int kNK = 48;                          // keys per tile
+constexpr int kStages = 3;                       // key tiles in flight
+constexpr int kMaxSel = 512;                     // selection entries staged per row
+constexpr int kQRegion = 64 * 128;               // [64 rows x 128 B]: one swizzle column of Q
+constexpr int kKRegion = kNK * 128;              // [48 rows x 128 B]
+constexpr int kQBytes = 8 * kQRegion;            // 64 KB
+constexpr int kTileBytes = 8 * kKRegion;         // 48 KB
+constexpr int kPBytes = kHeads * 128;            // 64 rows x 128 B (48 keys used)
 
 constexpr int kOffQ = 0;
-constexpr int kOffTile = kOffQ + kQBytes;                 // 2 tiles
-constexpr int kOffP = kOffTile + 2 * kTileBytes;          // 2 P buffers
-constexpr int kOffBar = kOffP + 2 * kPBytes;
-enum Bar { kQFull, kQEmpty, kKvFull0, kKvFull1, kKvEmpty0, kKvEmpty1, kSFull0, kSFull1, kPFull0,
-           kPFull1, kPvDone0, kPvDone1, kOFull, kOEmpty, kNumBars };
+constexpr int kOffTile = kOffQ + kQBytes;
+constexpr int kOffP = kOffTile + kStages * kTileBytes;
+constexpr int kOffSel = kOffP + 2 * kPBytes;
+constexpr int kOffBar = kOffSel + kMaxSel * 4;
+enum Bar { kQFull, kQReady, kQEmpty, kKvFull0, kKvEmpty0 = kKvFull0 + kStages,
+           kSFull0 = kKvEmpty0 + kStages, kPFull0 = kSFull0 + 2, kPvDone0 = kPFull0 + 2,
+           kOFull = kPvDone0 + 2, kOEmpty, kNumBars };
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffTmemPtr + 16 + 1024;       // + alignment slack
+constexpr int kSmemBytes = kOffTmemPtr + 16;
 
-constexpr uint32_t kColS0 = 256, kColS1 = 320;
+constexpr uint32_t kColS0 = 256, kColS1 = 256 + kNK;
 constexpr uint32_t kIdescQK = tc::idesc_bf16(64, kNK, false, false);
 constexpr uint32_t kIdescPV = tc::idesc_bf16(64, 256, false, true);
 constexpr float kLog2e = 1.4426950408889634f;
@@ -66,24 +77,13 @@ __device__ __forceinline__ Row locate_row(const AttnArgs& a, int64_t r) {
   return w;
 }
 
-// Physical row (in the tensor map) of key c of tile j; keys past the tile's count reuse a valid
-// row (their logits are masked).
-__device__ __forceinline__ int32_t key_row(const AttnArgs& a, const Row& w, int64_t row, int j,
-                                           int c) {
-  if (j < w.twin) {
-    int x = j * kNK + c;
-    if (x >= w.nwin) x = 0;
-    return (int32_t)a.win.row_index(w.seq, w.lo + x);
-  }
-  int i = (j - w.twin) * kNK + c;
-  if (i >= w.npool) i = 0;
-  int64_t e = a.pool_mode == 2 ? (int64_t)__ldg(a.sel + row * a.k + i) : i;
-  return (int32_t)a.pool.row_index(w.seq, e < 0 ? 0 : e);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
   __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(v);
 }
 
 __global__ void __launch_bounds__(256, 1)
@@ -92,19 +92,27 @@ __global__ void __launch_bounds__(256, 1)
                         const __grid_constant__ CUtensorMap tm_pool,
                         const __grid_constant__ CUtensorMap tm_win_box,
                         const __grid_constant__ CUtensorMap tm_pool_box, AttnArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = tc::smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
+  int32_t* sel_s = reinterpret_cast<int32_t*>(smem + kOffSel);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* status = a.status;
+  // the 128-byte swizzle needs 1024-byte aligned tiles; the dynamic window starts aligned
+  if ((tc::smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicExch(status, tc::kStatusMisaligned);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bar[kQFull], 1);
+    tc::mbar_init(&bar[kQReady], 64);
     tc::mbar_init(&bar[kQEmpty], 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&bar[kKvFull0 + i], 1);
       tc::mbar_init(&bar[kKvEmpty0 + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&bar[kSFull0 + i], 1);
       tc::mbar_init(&bar[kPFull0 + i], 128);
       tc::mbar_init(&bar[kPvDone0 + i], 1);
@@ -121,15 +129,14 @@ __global__ void __launch_bounds__(256, 1)
     tc::tma_prefetch_desc(&tm_win_box);
     tc::tma_prefetch_desc(&tm_pool_box);
   }
-  // window rows of a prefill are consecutive rows of the rotated kv stream, and so are the
-  // entries of an HCA prefill: such tiles load as 8 boxes of [64 rows x 64 columns]
-  const bool win_contig = a.win.block_table == nullptr;
-  const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  int* status = a.status;
+  // window rows of a prefill are consecutive rows of the rotated kv stream, and so are the
+  // entries of an HCA prefill
+  const bool win_contig = a.win.block_table == nullptr;
+  const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -142,37 +149,55 @@ __global__ void __launch_bounds__(256, 1)
       if (lane == 0) {
         tc::mbar_arrive_expect_tx(&bar[kQFull], kQBytes);
         for (int c = 0; c < 8; ++c)
-          tc::tma_load_2d(smem + kOffQ + c * kRegion, &tm_q, &bar[kQFull], 64 * c,
+          tc::tma_load_2d(smem + kOffQ + c * kQRegion, &tm_q, &bar[kQFull], 64 * c,
                           (int32_t)(r * kHeads));
       }
+      // stage this row's selections (only this warp reads them)
+      if (a.pool_mode == 2) {
+        __syncwarp();
+        for (int i = lane; i < w.npool; i += 32) sel_s[i] = __ldg(a.sel + r * a.k + i);
+        __syncwarp();
+      }
       for (int j = 0; j < w.tiles && ok; ++j, ++g) {
-        const uint32_t b = g & 1;
-        if (g >= 2)
-          ok = __all_sync(~0u, tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - 2) >> 1) & 1, status));
+        const uint32_t b = g % kStages;
+        if (g >= kStages)
+          ok = __all_sync(~0u, tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - kStages) / kStages) & 1,
+                                             status));
         if (!ok) break;
         if (lane == 0) tc::mbar_arrive_expect_tx(&bar[kKvFull0 + b], kTileBytes);
         __syncwarp();
+        uint8_t* tile = smem + kOffTile + b * kTileBytes;
         const bool is_win = j < w.twin;
         if (is_win ? win_contig : pool_contig) {
           if (lane == 0) {
             const int64_t y0 = is_win ? a.win.row_index(w.seq, w.lo + (int64_t)j * kNK)
                                       : a.pool.row_index(w.seq, (int64_t)(j - w.twin) * kNK);
             const CUtensorMap* map = is_win ? &tm_win_box : &tm_pool_box;
-            uint8_t* dst = smem + kOffTile + b * kTileBytes;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              tc::tma_load_2d(dst + c * kRegion, map, &bar[kKvFull0 + b], 64 * c, (int32_t)y0);
+              tc::tma_load_2d(tile + c * kKRegion, map, &bar[kKvFull0 + b], 64 * c, (int32_t)y0);
           }
         } else if (lane < kNK / 4) {
           int32_t y[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) y[u] = key_row(a, w, r, j, lane * 4 + u);
-          const CUtensorMap* map = j < w.twin ? &tm_win : &tm_pool;
-          uint8_t* dst = smem + kOffTile + b * kTileBytes + lane * 4 * 128;
+          for (int u = 0; u < 4; ++u) {
+            const int c = lane * 4 + u;
+            if (is_win) {
+              int x = j * kNK + c;
+              if (x >= w.nwin) x = 0;  // past the tile's keys: any valid row (masked)
+              y[u] = (int32_t)a.win.row_index(w.seq, w.lo + x);
+            } else {
+              int i = (j - w.twin) * kNK + c;
+              if (i >= w.npool) i = 0;
+              int64_t e = a.pool_mode == 2 ? (int64_t)sel_s[i] : i;
+              y[u] = (int32_t)a.pool.row_index(w.seq, e < 0 ? 0 : e);
+            }
+          }
+          const CUtensorMap* map = is_win ? &tm_win : &tm_pool;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            tc::tma_gather4(dst + c * kRegion, map, &bar[kKvFull0 + b], 64 * c, y[0], y[1], y[2],
-                            y[3]);
+            tc::tma_gather4(tile + c * kKRegion + lane * 512, map, &bar[kKvFull0 + b], 64 * c,
+                            y[0], y[1], y[2], y[3]);
         }
       }
     }
@@ -184,45 +209,46 @@ __global__ void __launch_bounds__(256, 1)
       const uint32_t q_base = tc::smem_u32(smem + kOffQ);
       for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
         const Row w = locate_row(a, r);
-        ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
+        ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
         for (int j = 0; j <= w.tiles && ok; ++j) {
           if (j < w.tiles) {  // S(g) = Q K^T
-            const uint32_t g = g0 + j, b = g & 1;
-            ok = tc::mbar_wait(&bar[kKvFull0 + b], (g >> 1) & 1, status);
-            if (ok && g >= 2) ok = tc::mbar_wait(&bar[kPFull0 + b], ((g - 2) >> 1) & 1, status);
+            const uint32_t g = g0 + j, b = g % kStages, s = g & 1;
+            ok = tc::mbar_wait(&bar[kKvFull0 + b], (g / kStages) & 1, status);
+            if (ok && g >= 2) ok = tc::mbar_wait(&bar[kPFull0 + s], ((g - 2) >> 1) & 1, status);
             if (!ok) break;
             tc::tc_fence_after();
             const uint32_t k_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
-            const uint32_t d = tmem + (b ? kColS1 : kColS0);
+            const uint32_t d = tmem + (s ? kColS1 : kColS0);
 #pragma unroll 4
             for (int kk = 0; kk < kDim / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-              tc::mma_bf16_ss(d, tc::desc_sw128(q_base + off, 0, 1024),
-                              tc::desc_sw128(k_base + off, 0, 1024), kIdescQK, kk > 0);
+              const uint32_t qo = (kk >> 2) * kQRegion + (kk & 3) * 32;
+              const uint32_t ko = (kk >> 2) * kKRegion + (kk & 3) * 32;
+              tc::mma_bf16_ss(d, tc::desc_sw128(q_base + qo, 0, 1024),
+                              tc::desc_sw128(k_base + ko, 0, 1024), kIdescQK, kk > 0);
             }
-            tc::mma_commit(&bar[kSFull0 + b]);
+            tc::mma_commit(&bar[kSFull0 + s]);
             if (j == w.tiles - 1) tc::mma_commit(&bar[kQEmpty]);
           }
           if (j >= 1) {  // O += P(g) V(g)
-            const uint32_t g = g0 + j - 1, b = g & 1;
-            ok = tc::mbar_wait(&bar[kPFull0 + b], (g >> 1) & 1, status);
+            const uint32_t g = g0 + j - 1, b = g % kStages, s = g & 1;
+            ok = tc::mbar_wait(&bar[kPFull0 + s], (g >> 1) & 1, status);
             if (ok && j == 1 && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
             if (!ok) break;
             tc::tc_fence_after();
             const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
-            const uint32_t p_base = tc::smem_u32(smem + kOffP + b * kPBytes);
+            const uint32_t p_base = tc::smem_u32(smem + kOffP + s * kPBytes);
 #pragma unroll
             for (int kk = 0; kk < kNK / 16; ++kk) {
               const uint64_t pd = tc::desc_sw128(p_base + kk * 32, 0, 1024);
               const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
-              tc::mma_bf16_ss(tmem, pd,
-                              tc::desc_sw128(v_base + kk * 2048, kRegion, 1024), kIdescPV, acc);
+              tc::mma_bf16_ss(tmem, pd, tc::desc_sw128(v_base + kk * 2048, kKRegion, 1024),
+                              kIdescPV, acc);
               tc::mma_bf16_ss(tmem + (16u << 16), pd,
-                              tc::desc_sw128(v_base + 4 * kRegion + kk * 2048, kRegion, 1024),
+                              tc::desc_sw128(v_base + 4 * kKRegion + kk * 2048, kKRegion, 1024),
                               kIdescPV, acc);
             }
             tc::mma_commit(&bar[kKvEmpty0 + b]);
-            tc::mma_commit(&bar[kPvDone0 + b]);
+            tc::mma_commit(&bar[kPvDone0 + s]);
             if (j == w.tiles) tc::mma_commit(&bar[kOFull]);
           }
         }
@@ -230,7 +256,38 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------------ query rotation
+    // thread i turns the rope pairs of head row i of the staged query tile (row h's 16-byte
+    // chunk c of a 128-byte region sits at chunk c ^ (h & 7)).
+    const int h = (warp - 2) * 32 + lane;
+    const int R = a.rf.R;
+    const int p0 = (kDim - R) >> 1;  // first rotated pair among the 256 channel pairs
+    uint32_t qi = 0;
+    bool ok = true;
+    for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
+      int seq;
+      int64_t t;
+      a.qr.locate(a.qr.row0 + r, seq, t);
+      float my_c = 1.f, my_s = 0.f;
+      if (lane < R / 2) rope_cos_sin(a.rf, lane, a.pos0 + t, my_c, my_s);
+      ok = __all_sync(~0u, tc::mbar_wait(&bar[kQFull], qi & 1, status));
+      if (!ok) break;
+      uint8_t* row = smem + kOffQ + h * 128;
+      for (int p = 0; p < R / 2; ++p) {
+        const float cc = __shfl_sync(~0u, my_c, p), ss = __shfl_sync(~0u, my_s, p);
+        const int pp = p0 + p;                  // channels 2pp, 2pp+1
+        const int region = pp >> 5;             // 32 pairs per 128-byte region
+        const int chunk = (pp & 31) >> 2;       // 4 pairs per 16-byte chunk
+        uint32_t* word = reinterpret_cast<uint32_t*>(row + region * kQRegion +
+                                                     ((chunk ^ (h & 7)) << 4) + (pp & 3) * 4);
+        const float2 x = unpack_bf16(*word);
+        *word = pack_bf16(x.x * cc - x.y * ss, x.x * ss + x.y * cc);
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[kQReady]);
+    }
+  } else {
     // ------------------------------------------------------------------ softmax + output
     const int sp = warp & 3;                 // TMEM sub-partition of this warp
     const int half = lane >> 4;              // 0: lanes 0-15 (S rows, O[:,0:256]); 1: O[:,256:512]
@@ -244,37 +301,37 @@ __global__ void __launch_bounds__(256, 1)
       const Row w = locate_row(a, r);
       float m_run = sink_log2, l_run = 1.f;
       for (int j = 0; j < w.tiles && ok; ++j) {
-        const uint32_t g = g0 + j, b = g & 1;
-        ok = __all_sync(~0u, tc::mbar_wait(&bar[kSFull0 + b], (g >> 1) & 1, status));
+        const uint32_t g = g0 + j, s = g & 1;
+        ok = __all_sync(~0u, tc::mbar_wait(&bar[kSFull0 + s], (g >> 1) & 1, status));
         if (!ok) break;
         tc::tc_fence_after();
-        float s[kNK];
+        float sv[kNK];
 #pragma unroll
         for (int c = 0; c < kNK; c += 16) {
           uint32_t v[16];
-          tc::tmem_ld16(t_row + (b ? kColS1 : kColS0) + c, v);
+          tc::tmem_ld16(t_row + (s ? kColS1 : kColS0) + c, v);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 16; ++u) s[c + u] = __uint_as_float(v[u]);
+          for (int u = 0; u < 16; ++u) sv[c + u] = __uint_as_float(v[u]);
         }
         const int nk = j < w.twin ? min(kNK, w.nwin - j * kNK)
                                   : min(kNK, w.npool - (j - w.twin) * kNK);
         float mx = -INFINITY;
 #pragma unroll
         for (int c = 0; c < kNK; ++c) {
-          s[c] = c < nk ? s[c] * scale_log2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+          sv[c] = c < nk ? sv[c] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sv[c]);
         }
         const bool move = half == 0 && mx > m_run + kLazy;
         const float m_new = move ? mx : m_run;
         const float alpha = exp2f(m_run - m_new);
         // rescale the rows of O this warp owns (rare: only when some row's max moved)
-        if (__any_sync(0xffffffffu, move) && j > 0) {
+        if (__any_sync(~0u, move) && j > 0) {
           const uint32_t gp = g - 1;
           ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + (gp & 1)], (gp >> 1) & 1, status));
           if (!ok) break;
           tc::tc_fence_after();
-          const float al = __shfl_sync(0xffffffffu, alpha, lane & 15);
+          const float al = __shfl_sync(~0u, alpha, lane & 15);
 #pragma unroll 1
           for (int c = 0; c < 256; c += 16) {
             uint32_t v[16];
@@ -290,26 +347,26 @@ __global__ void __launch_bounds__(256, 1)
         uint32_t pk[kNK / 2];
 #pragma unroll
         for (int c = 0; c < kNK; c += 2) {
-          const float p0 = exp2f(s[c] - m_new), p1 = exp2f(s[c + 1] - m_new);
-          sum += p0 + p1;
-          pk[c / 2] = pack_bf16(p0, p1);
+          const float e0 = exp2f(sv[c] - m_new), e1 = exp2f(sv[c + 1] - m_new);
+          sum += e0 + e1;
+          pk[c / 2] = pack_bf16(e0, e1);
         }
         l_run = l_run * alpha + sum;
         m_run = m_new;
-        // P buffer b is free once PV(g-2) completed
+        // P buffer s is free once PV(g-2) completed
         if (g >= 2)
-          ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + b], ((g - 2) >> 1) & 1, status));
+          ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + s], ((g - 2) >> 1) & 1, status));
         if (!ok) break;
         if (half == 0) {
-          uint8_t* prow = smem + kOffP + b * kPBytes + h * 128;
+          uint8_t* prow = smem + kOffP + s * kPBytes + h * 128;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
+          for (int ch = 0; ch < kNK / 8; ++ch)
             *reinterpret_cast<uint4*>(prow + ((ch ^ (h & 7)) << 4)) =
                 make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
-        tc::mbar_arrive(&bar[kPFull0 + b]);
+        tc::mbar_arrive(&bar[kPFull0 + s]);
       }
       if (!ok) break;
       // ---- output: O / l, the rope slice turned by -P_t, bf16 store. Lane p holds the cos/sin
@@ -320,8 +377,9 @@ __global__ void __launch_bounds__(256, 1)
       ok = __all_sync(~0u, tc::mbar_wait(&bar[kOFull], qi & 1, status));
       if (!ok) break;
       tc::tc_fence_after();
-      const float inv_l = 1.f / __shfl_sync(0xffffffffu, l_run, lane & 15);
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + ((int64_t)r * kHeads + h) * kDim + half * 256;
+      const float inv_l = 1.f / __shfl_sync(~0u, l_run, lane & 15);
+      __nv_bfloat16* orow =
+          reinterpret_cast<__nv_bfloat16*>(a.o) + ((int64_t)r * kHeads + h) * kDim + half * 256;
       const int rope_lo = kDim - a.rf.R;  // first rotated channel (always in the upper half)
 #pragma unroll 1
       for (int c = 0; c < 256; c += 16) {
@@ -336,8 +394,8 @@ __global__ void __launch_bounds__(256, 1)
           for (int u = 0; u < 16; u += 2) {
             const int ch = half * 256 + c + u;
             const int p = ch >= rope_lo ? (ch - rope_lo) >> 1 : 0;
-            const float cc = __shfl_sync(0xffffffffu, my_c, p);
-            const float ss = __shfl_sync(0xffffffffu, my_s, p);
+            const float cc = __shfl_sync(~0u, my_c, p);
+            const float ss = __shfl_sync(~0u, my_s, p);
             if (ch >= rope_lo) {
               const float x0 = x[u], x1 = x[u + 1];
               x[u] = x0 * cc - x1 * ss;
@@ -368,25 +426,26 @@ __global__ void __launch_bounds__(256, 1)
 }  // namespace
 
 bool attention_tc_supported(const AttnArgs& a, int dtype) {
-  return dtype == 1 && a.H == kHeads && a.D == kDim && a.rf.R <= 64 && a.rf.R % 2 == 0;
+  return dtype == 1 && a.H == kHeads && a.D == kDim && a.rf.R <= 64 && a.rf.R % 2 == 0 &&
+         (a.pool_mode != 2 || a.k <= kMaxSel);
 }
 
-cudaError_t launch_attention_tc(const AttnArgs& a, const void* q_rot, int64_t win_rows,
-                                int64_t pool_rows, cudaStream_t st) {
+cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t pool_rows,
+                                cudaStream_t st) {
   if (a.nrows == 0) return cudaSuccess;
   CUtensorMap tq, tw, tp, twb, tpb;
-  cudaError_t e = make_tmap_bf16_2d(&tq, q_rot, (uint64_t)a.nrows * kHeads, kDim, kDim * 2, 64, 64);
+  cudaError_t e = make_tmap_bf16_2d(&tq, a.q, (uint64_t)a.nrows * kHeads, kDim, kDim * 2, 64, 64);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16_2d(&tw, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, 1, 64);
   if (e != cudaSuccess) return e;
   const bool has_pool = a.pool_mode != 0 && pool_rows > 0;
-  e = make_tmap_bf16_2d(&tp, has_pool ? a.pool.base : a.win.base,
-                        (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, 1, 64);
+  const void* pb = has_pool ? a.pool.base : a.win.base;
+  const uint64_t pr = (uint64_t)(has_pool ? pool_rows : win_rows);
+  e = make_tmap_bf16_2d(&tp, pb, pr, kDim, kDim * 2, 1, 64);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16_2d(&twb, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
-  e = make_tmap_bf16_2d(&tpb, has_pool ? a.pool.base : a.win.base,
-                        (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, kNK, 64);
+  e = make_tmap_bf16_2d(&tpb, pb, pr, kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes);

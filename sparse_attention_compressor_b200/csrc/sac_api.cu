@@ -128,11 +128,10 @@ bool use_tc_attention(const sac_params* p) {
 constexpr size_t kStatusBytes = 256;  // device status word at the start of every workspace
 
 struct Sizes {
-  size_t status = kStatusBytes, kv_rot = 0, q_rot = 0, pool = 0, idx_pool = 0, scores = 0,
-         topk = 0;
+  size_t status = kStatusBytes, kv_rot = 0, pool = 0, idx_pool = 0, scores = 0, topk = 0;
   size_t total() const {
-    return align_up(status) + align_up(kv_rot) + align_up(q_rot) + align_up(pool) +
-           align_up(idx_pool) + align_up(scores) + align_up(topk);
+    return align_up(status) + align_up(kv_rot) + align_up(pool) + align_up(idx_pool) +
+           align_up(scores) + align_up(topk);
   }
 };
 
@@ -140,7 +139,6 @@ Sizes prefill_sizes(const sac_params* p, int kind) {
   Sizes s;
   const size_t rows = (size_t)p->B * p->S;
   s.kv_rot = rows * p->D * esize(p->dtype);
-  if (use_tc_attention(p)) s.q_rot = rows * p->H * p->D * esize(p->dtype);
   if (kind == SAC_KIND_HCA || kind == SAC_KIND_CSA)
     s.pool = (size_t)p->B * (p->S / p->m) * p->D * esize(p->dtype);
   if (kind == SAC_KIND_CSA) {
@@ -159,19 +157,13 @@ sac::RowAddr paged(const void* base, const int32_t* bt, int max_pages, int page_
   return sac::RowAddr{base, bt, 0, max_pages, page_size, width};
 }
 
-// The attention step of a prefill call: the tensor-core kernel (after rotating q once into
-// q_rot) for bf16 64 x 512 layers, the CUDA-core kernel otherwise.
-cudaError_t run_attention(const sac_params* p, const sac::AttnArgs& a, void* q_rot,
-                          int64_t win_rows, int64_t pool_rows, cudaStream_t st) {
-  if (use_tc_attention(p)) {
-    const int64_t qrows = (int64_t)p->B * p->S * p->H;
-    cudaError_t e = sac::timed("rotate_q", st, [&] {
-      return sac::launch_rotate_rows(p->dtype, a.q, qrows, p->S, p->D, a.rf, p->pos0, q_rot, st,
-                                     p->H);
-    });
-    if (e != cudaSuccess) return e;
+// The attention step of a call: the tensor-core kernel for bf16 layers with 64 heads of 512 (it
+// rotates q itself), the CUDA-core kernel otherwise.
+cudaError_t run_attention(const sac_params* p, const sac::AttnArgs& a, int64_t win_rows,
+                          int64_t pool_rows, cudaStream_t st) {
+  if (use_tc_attention(p) && sac::attention_tc_supported(a, p->dtype)) {
     return sac::timed("attention", st, [&] {
-      return sac::launch_attention_tc(a, q_rot, win_rows, pool_rows, st);
+      return sac::launch_attention_tc(a, win_rows, pool_rows, st);
     });
   }
   return sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
@@ -224,7 +216,6 @@ int swa_forward(const sac_params* p, const void* q, const void* kv, const float*
   Carve cv(ws);
   int* status = static_cast<int*>(cv.take(sz.status));
   void* kv_rot = cv.take(sz.kv_rot);
-  void* q_rot = cv.take(sz.q_rot);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
   if (e != cudaSuccess) return cuda_fail(e, "clear status");
   sac::RopeFreqs rf = rope_freqs(p);
@@ -237,7 +228,7 @@ int swa_forward(const sac_params* p, const void* q, const void* kv, const float*
   a.win = contiguous(kv_rot, p->S, p->D);
   a.pool_mode = 0;
   a.status = status;
-  e = run_attention(p, a, q_rot, rows, 0, st);
+  e = run_attention(p, a, rows, 0, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -335,7 +326,6 @@ int hca_forward(const sac_params* p, const void* q, const void* kv, const void* 
   Carve cv(ws);
   int* status = static_cast<int*>(cv.take(sz.status));
   void* kv_rot = cv.take(sz.kv_rot);
-  void* q_rot = cv.take(sz.q_rot);
   void* pool = pool_out ? pool_out : cv.take(sz.pool);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
   if (e != cudaSuccess) return cuda_fail(e, "clear status");
@@ -353,7 +343,7 @@ int hca_forward(const sac_params* p, const void* q, const void* kv, const void* 
   a.pool_mode = 1;
   a.pool = contiguous(pool, p->S / p->m, p->D);
   a.status = status;
-  e = run_attention(p, a, q_rot, rows, (int64_t)p->B * (p->S / p->m), st);
+  e = run_attention(p, a, rows, (int64_t)p->B * (p->S / p->m), st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -390,7 +380,6 @@ int csa_forward(const sac_params* p, const void* q, const void* kv, const void* 
   Carve cv(ws);
   int* status = static_cast<int*>(cv.take(sz.status));
   void* kv_rot = cv.take(sz.kv_rot);
-  void* q_rot = cv.take(sz.q_rot);
   void* pool = pool_out ? pool_out : cv.take(sz.pool);
   void* ipool = idx_pool_out ? idx_pool_out : cv.take(sz.idx_pool);
   float* scores = static_cast<float*>(cv.take(sz.scores));
@@ -466,7 +455,7 @@ int csa_forward(const sac_params* p, const void* q, const void* kv, const void* 
   a.pool = contiguous(pool, N, p->D);
   a.sel = sel;
   a.status = status;
-  e = run_attention(p, a, q_rot, rows, (int64_t)p->B * N, st);
+  e = run_attention(p, a, rows, (int64_t)p->B * N, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }

@@ -75,10 +75,10 @@ struct AttnArgs {
 cudaError_t launch_attention_simt(int dtype, const AttnArgs& a, cudaStream_t st);
 
 // ---- attention on tcgen05 (attention_tc.cu): bf16, 64 heads, head_dim 512 ------------------
-// q_rot: [nrows, 64, 512] already rotated; win/pool bases are [rows, 512] buffers whose row
-// counts (win_rows, pool_rows) bound the TMA coordinates.
+// a.q: [nrows, 64, 512] un-rotated (rotated in the kernel); win/pool bases are [rows, 512]
+// buffers whose row counts (win_rows, pool_rows) bound the TMA coordinates.
 bool attention_tc_supported(const AttnArgs& a, int dtype);
-cudaError_t launch_attention_tc(const AttnArgs& a, const void* q_rot, int64_t win_rows,
-                                int64_t pool_rows, cudaStream_t st);
+cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t pool_rows,
+                                cudaStream_t st);
 
 }  // namespace sac

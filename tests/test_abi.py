@@ -52,16 +52,12 @@ def test_workspace_sizes():
     p = p_csa()
     n = 8192 // 4
     ws = sac.sac_workspace_size(p, sac.SAC_KIND_CSA)
-    # status word + rotated kv + rotated q (tensor-core attention) + pool + indexer pool +
-    # scores + top-k, each 256-byte aligned
-    qrot = 8192 * 64 * 512 * 2
-    expect = 256 + 8192 * 512 * 2 + qrot + n * 512 * 2 + n * 128 * 2 + 8192 * n * 4 + \
-        8192 * 512 * 4
+    # status word + rotated kv + pool + indexer pool + scores + top-k, each 256-byte aligned
+    expect = 256 + 8192 * 512 * 2 + n * 512 * 2 + n * 128 * 2 + 8192 * n * 4 + 8192 * 512 * 4
     assert ws == expect
-    assert sac.sac_workspace_size(p, sac.SAC_KIND_SWA) == 256 + 8192 * 512 * 2 + qrot
+    assert sac.sac_workspace_size(p, sac.SAC_KIND_SWA) == 256 + 8192 * 512 * 2
     assert sac.sac_workspace_size(p_csa(m=128, win_len=128), sac.SAC_KIND_HCA) == \
-        256 + 8192 * 512 * 2 + qrot + 64 * 512 * 2
-    # the CUDA-core path (fp32) needs no rotated q
+        256 + 8192 * 512 * 2 + 64 * 512 * 2
     assert sac.sac_workspace_size(p_csa(dtype="f32"), sac.SAC_KIND_SWA) == 256 + 8192 * 512 * 4
     assert sac.sac_decode_workspace_size(p_csa(S=65536), sac.SAC_KIND_CSA, 64) == \
         64 * 16384 * 4 + 64 * 512 * 4
