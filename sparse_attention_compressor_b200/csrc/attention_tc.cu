@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) {
       uint32_t g0 = 0, qi = 0;
       bool ok = true;
-      const uint32_t q_base = tc::smem_u32(smem + kOffQ);
+      const uint64_t qd = tc::desc_sw128(tc::smem_u32(smem + kOffQ), 0, 1024);
       for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
         const Row w = locate_row(a, r);
         ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
@@ -217,14 +217,16 @@ __global__ void __launch_bounds__(256, 1)
             if (ok && g >= 2) ok = tc::mbar_wait(&bar[kPFull0 + s], ((g - 2) >> 1) & 1, status);
             if (!ok) break;
             tc::tc_fence_after();
-            const uint32_t k_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
+            const uint64_t kd = tc::desc_sw128(tc::smem_u32(smem + kOffTile + b * kTileBytes), 0,
+                                               1024);
             const uint32_t d = tmem + (s ? kColS1 : kColS0);
-#pragma unroll 4
+            // the descriptor's start-address field counts 16-byte units: advancing along K adds
+            // the byte offset >> 4 to the base descriptor
+#pragma unroll
             for (int kk = 0; kk < kDim / 16; ++kk) {
-              const uint32_t qo = (kk >> 2) * kQRegion + (kk & 3) * 32;
-              const uint32_t ko = (kk >> 2) * kKRegion + (kk & 3) * 32;
-              tc::mma_bf16_ss(d, tc::desc_sw128(q_base + qo, 0, 1024),
-                              tc::desc_sw128(k_base + ko, 0, 1024), kIdescQK, kk > 0);
+              const uint32_t qo = ((kk >> 2) * kQRegion + (kk & 3) * 32) >> 4;
+              const uint32_t ko = ((kk >> 2) * kKRegion + (kk & 3) * 32) >> 4;
+              tc::mma_bf16_ss(d, qd + qo, kd + ko, kIdescQK, kk > 0);
             }
             tc::mma_commit(&bar[kSFull0 + s]);
             if (j == w.tiles - 1) tc::mma_commit(&bar[kQEmpty]);
@@ -236,16 +238,14 @@ __global__ void __launch_bounds__(256, 1)
             if (!ok) break;
             tc::tc_fence_after();
             const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
-            const uint32_t p_base = tc::smem_u32(smem + kOffP + s * kPBytes);
+            const uint64_t pd = tc::desc_sw128(tc::smem_u32(smem + kOffP + s * kPBytes), 0, 1024);
+            const uint64_t vlo = tc::desc_sw128(v_base, kKRegion, 1024);
+            const uint64_t vhi = tc::desc_sw128(v_base + 4 * kKRegion, kKRegion, 1024);
 #pragma unroll
             for (int kk = 0; kk < kNK / 16; ++kk) {
-              const uint64_t pd = tc::desc_sw128(p_base + kk * 32, 0, 1024);
               const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
-              tc::mma_bf16_ss(tmem, pd, tc::desc_sw128(v_base + kk * 2048, kKRegion, 1024),
-                              kIdescPV, acc);
-              tc::mma_bf16_ss(tmem + (16u << 16), pd,
-                              tc::desc_sw128(v_base + 4 * kKRegion + kk * 2048, kKRegion, 1024),
-                              kIdescPV, acc);
+              tc::mma_bf16_ss(tmem, pd + kk * 2, vlo + kk * 128, kIdescPV, acc);
+              tc::mma_bf16_ss(tmem + (16u << 16), pd + kk * 2, vhi + kk * 128, kIdescPV, acc);
             }
             tc::mma_commit(&bar[kKvEmpty0 + b]);
             tc::mma_commit(&bar[kPvDone0 + s]);
@@ -274,15 +274,35 @@ __global__ void __launch_bounds__(256, 1)
       ok = __all_sync(~0u, tc::mbar_wait(&bar[kQFull], qi & 1, status));
       if (!ok) break;
       uint8_t* row = smem + kOffQ + h * 128;
-      for (int p = 0; p < R / 2; ++p) {
-        const float cc = __shfl_sync(~0u, my_c, p), ss = __shfl_sync(~0u, my_s, p);
+      // four pairs per 16-byte chunk (R is even and the rope slice starts on a chunk boundary
+      // whenever R is a multiple of 8; other R take the per-pair path)
+      for (int p = 0; p < R / 2; p += 4) {
         const int pp = p0 + p;                  // channels 2pp, 2pp+1
         const int region = pp >> 5;             // 32 pairs per 128-byte region
         const int chunk = (pp & 31) >> 2;       // 4 pairs per 16-byte chunk
-        uint32_t* word = reinterpret_cast<uint32_t*>(row + region * kQRegion +
-                                                     ((chunk ^ (h & 7)) << 4) + (pp & 3) * 4);
-        const float2 x = unpack_bf16(*word);
-        *word = pack_bf16(x.x * cc - x.y * ss, x.x * ss + x.y * cc);
+        uint8_t* cptr = row + region * kQRegion + ((chunk ^ (h & 7)) << 4);
+        if ((pp & 3) == 0 && p + 4 <= R / 2) {
+          uint4 v = *reinterpret_cast<uint4*>(cptr);
+          uint32_t* w4 = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float cc = __shfl_sync(~0u, my_c, p + u), ss = __shfl_sync(~0u, my_s, p + u);
+            const float2 x = unpack_bf16(w4[u]);
+            w4[u] = pack_bf16(x.x * cc - x.y * ss, x.x * ss + x.y * cc);
+          }
+          *reinterpret_cast<uint4*>(cptr) = v;
+        } else {
+          for (int u = 0; u < 4; ++u) {
+            const int pu = p + u < R / 2 ? p + u : R / 2 - 1;
+            const float cc = __shfl_sync(~0u, my_c, pu), ss = __shfl_sync(~0u, my_s, pu);
+            if (p + u >= R / 2) continue;
+            const int q = p0 + p + u;
+            uint32_t* word = reinterpret_cast<uint32_t*>(
+                row + (q >> 5) * kQRegion + ((((q & 31) >> 2) ^ (h & 7)) << 4) + (q & 3) * 4);
+            const float2 x = unpack_bf16(*word);
+            *word = pack_bf16(x.x * cc - x.y * ss, x.x * ss + x.y * cc);
+          }
+        }
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bar[kQReady]);
