@@ -6,22 +6,29 @@
 // both contractions:  S = Q K^T  (M=64, N=48 keys, K=512)  and  O += P V  (M=64, N=256 x 2, K=48).
 // Because K = V, one shared-memory key tile serves as the K-major B operand of QK^T and as the
 // MN-major B operand of PV. Tiles of 48 keys keep three tile buffers resident next to the 64 KB
-// query tile, so the next tiles load while the tensor core works. Window rows and HCA entries are
-// consecutive rows and load as 8 TMA boxes per tile; CSA selections are gathered with TMA
-// tile::gather4 (four rows per copy) from indices staged in shared memory. Tiles never mix the
-// two sources.
+// query tile. Window rows and HCA entries are consecutive rows and load as 8 TMA boxes per tile;
+// CSA selections (and paged rows) are gathered with 16-byte cp.async copies by two producer
+// groups that take alternate tiles. Tiles never mix window rows and entries.
 //
-// The query tile arrives un-rotated; two warps turn its rope slice (channels 448..511) in shared
-// memory before the first QK^T of the row, so no rotated copy of q is ever written to HBM.
+// QK^T of a tile is 32 MMAs of K=16. Accumulating them into one TMEM tile would chain each MMA
+// on its predecessor, so they rotate over four partial accumulators and the softmax adds the
+// four partials.
+//
+// The query tile arrives un-rotated; one warp turns its rope slice in shared memory before the
+// first QK^T of the row, so no rotated copy of q is written to HBM.
 //
 // Tensor memory (512 columns, fp32): O[:, 0:256] in lanes 0-15 of each sub-partition and
-// O[:, 256:512] in lanes 16-31 (the M = 64 layout leaves half the lanes free, so the two output
-// halves share columns 0..255); two S buffers in columns 256..303 and 304..351.
+// O[:, 256:512] in lanes 16-31 (the M = 64 layout leaves half the lanes free); for each of the two
+// S buffers, partials 0/2 in lanes 0-15 and partials 1/3 in lanes 16-31 of 96 columns at 256
+// (buffer 0) and 352 (buffer 1). A softmax thread of lane i < 16 and its partner i + 16 own the
+// same head: they add their partials, exchange halves, and each finishes 24 of the 48 keys.
 //
-// Warps: 0 = TMA producer, 1 = MMA issuer (one thread) and TMEM owner, 2-3 = query rotation,
-// 4..7 = softmax + output. The softmax keeps the running max in log2 units and only moves it (and
-// rescales O) when a tile's max exceeds it by more than 8, so P <= 2^8 stays exact enough in bf16
-// and O is rarely touched.
+// Warps: 0 = TMA thread, 1-2 = MMA issuers (warp 1 also owns TMEM), 3 = query rotation, 4-5 / 6-7 =
+// gather groups (even / odd tiles), 8-11 = softmax + output. Each tcgen05.mma costs its issuing
+// thread a fixed time, so two threads issue: warp 1 the even partials of QK^T and PV of
+// O[:, 0:256], warp 2 the odd partials and PV of O[:, 256:512]; every barrier the MMAs signal
+// counts both. The softmax keeps the running max in log2 units and moves it (rescaling O) only
+// when a tile's max exceeds it by more than 8.
 #include <cuda_bf16.h>
 
 #include "sac_kernels.h"
@@ -34,26 +41,27 @@ namespace {
 constexpr int kHeads = 64;
 constexpr int kDim = 512;
 constexpr int kNK = 48;                          // keys per tile
+constexpr int kHalfNK = kNK / 2;
 constexpr int kStages = 3;                       // key tiles in flight
-constexpr int kMaxSel = 512;                     // selection entries staged per row
 constexpr int kQRegion = 64 * 128;               // [64 rows x 128 B]: one swizzle column of Q
 constexpr int kKRegion = kNK * 128;              // [48 rows x 128 B]
 constexpr int kQBytes = 8 * kQRegion;            // 64 KB
 constexpr int kTileBytes = 8 * kKRegion;         // 48 KB
 constexpr int kPBytes = kHeads * 128;            // 64 rows x 128 B (48 keys used)
+constexpr int kGroupThreads = 64;                // threads of one gather group
+constexpr int kThreads = 384;
 
 constexpr int kOffQ = 0;
 constexpr int kOffTile = kOffQ + kQBytes;
 constexpr int kOffP = kOffTile + kStages * kTileBytes;
-constexpr int kOffSel = kOffP + 2 * kPBytes;
-constexpr int kOffBar = kOffSel + kMaxSel * 4;
+constexpr int kOffBar = kOffP + 2 * kPBytes;
 enum Bar { kQFull, kQReady, kQEmpty, kKvFull0, kKvEmpty0 = kKvFull0 + kStages,
            kSFull0 = kKvEmpty0 + kStages, kPFull0 = kSFull0 + 2, kPvDone0 = kPFull0 + 2,
            kOFull = kPvDone0 + 2, kOEmpty, kNumBars };
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemPtr + 16;
 
-constexpr uint32_t kColS0 = 256, kColS1 = 256 + kNK;
+constexpr uint32_t kColS = 256, kSStride = 2 * kNK;  // S buffer s at kColS + s * kSStride
 constexpr uint32_t kIdescQK = tc::idesc_bf16(64, kNK, false, false);
 constexpr uint32_t kIdescPV = tc::idesc_bf16(64, 256, false, true);
 constexpr float kLog2e = 1.4426950408889634f;
@@ -86,16 +94,29 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return __bfloat1622float2(v);
 }
 
-__global__ void __launch_bounds__(256, 1)
+// Global address of key c of tile j (keys past the tile's count reuse a valid row: masked).
+__device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const Row& w,
+                                                        int64_t r, int j, int c) {
+  if (j < w.twin) {
+    int x = j * kNK + c;
+    if (x >= w.nwin) x = 0;
+    const __nv_bfloat16* p = a.win.row<__nv_bfloat16>(w.seq, w.lo + x);
+    return p ? p : a.win.row<__nv_bfloat16>(w.seq, w.lo);
+  }
+  int i = (j - w.twin) * kNK + c;
+  if (i >= w.npool) i = 0;
+  int64_t e = a.pool_mode == 2 ? (int64_t)__ldg(a.sel + r * a.k + i) : i;
+  const __nv_bfloat16* p = a.pool.row<__nv_bfloat16>(w.seq, e < 0 ? 0 : e);
+  return p ? p : reinterpret_cast<const __nv_bfloat16*>(a.pool.base);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                        const __grid_constant__ CUtensorMap tm_win,
-                        const __grid_constant__ CUtensorMap tm_pool,
                         const __grid_constant__ CUtensorMap tm_win_box,
                         const __grid_constant__ CUtensorMap tm_pool_box, AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
-  int32_t* sel_s = reinterpret_cast<int32_t*>(smem + kOffSel);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* status = a.status;
   // the 128-byte swizzle needs 1024-byte aligned tiles; the dynamic window starts aligned
@@ -106,26 +127,24 @@ __global__ void __launch_bounds__(256, 1)
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bar[kQFull], 1);
-    tc::mbar_init(&bar[kQReady], 64);
-    tc::mbar_init(&bar[kQEmpty], 1);
+    tc::mbar_init(&bar[kQReady], 32);
+    tc::mbar_init(&bar[kQEmpty], 2);
     for (int i = 0; i < kStages; ++i) {
-      tc::mbar_init(&bar[kKvFull0 + i], 1);
-      tc::mbar_init(&bar[kKvEmpty0 + i], 1);
+      tc::mbar_init(&bar[kKvFull0 + i], 1 + kGroupThreads);  // TMA thread + one gather group
+      tc::mbar_init(&bar[kKvEmpty0 + i], 2);
     }
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bar[kSFull0 + i], 1);
+      tc::mbar_init(&bar[kSFull0 + i], 2);
       tc::mbar_init(&bar[kPFull0 + i], 128);
-      tc::mbar_init(&bar[kPvDone0 + i], 1);
+      tc::mbar_init(&bar[kPvDone0 + i], 2);
     }
-    tc::mbar_init(&bar[kOFull], 1);
+    tc::mbar_init(&bar[kOFull], 2);
     tc::mbar_init(&bar[kOEmpty], 128);
     tc::fence_barrier_init();
   }
   if (warp == 1) tc::tmem_alloc(tmem_ptr, 512);
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tm_q);
-    tc::tma_prefetch_desc(&tm_win);
-    tc::tma_prefetch_desc(&tm_pool);
     tc::tma_prefetch_desc(&tm_win_box);
     tc::tma_prefetch_desc(&tm_pool_box);
   }
@@ -134,75 +153,48 @@ __global__ void __launch_bounds__(256, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
   // window rows of a prefill are consecutive rows of the rotated kv stream, and so are the
-  // entries of an HCA prefill
+  // entries of an HCA prefill: those tiles load as TMA boxes; the rest are gathered
   const bool win_contig = a.win.block_table == nullptr;
   const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    uint32_t g = 0, qi = 0;
-    bool ok = true;
-    for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
-      const Row w = locate_row(a, r);
-      if (qi > 0) ok = __all_sync(~0u, tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status));
-      if (!ok) break;
-      if (lane == 0) {
+    // ------------------------------------------------------------------ TMA thread
+    if (lane == 0) {
+      uint32_t g = 0, qi = 0;
+      bool ok = true;
+      for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
+        const Row w = locate_row(a, r);
+        if (qi > 0) ok = tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status);
+        if (!ok) break;
         tc::mbar_arrive_expect_tx(&bar[kQFull], kQBytes);
         for (int c = 0; c < 8; ++c)
           tc::tma_load_2d(smem + kOffQ + c * kQRegion, &tm_q, &bar[kQFull], 64 * c,
                           (int32_t)(r * kHeads));
-      }
-      // stage this row's selections (only this warp reads them)
-      if (a.pool_mode == 2) {
-        __syncwarp();
-        for (int i = lane; i < w.npool; i += 32) sel_s[i] = __ldg(a.sel + r * a.k + i);
-        __syncwarp();
-      }
-      for (int j = 0; j < w.tiles && ok; ++j, ++g) {
-        const uint32_t b = g % kStages;
-        if (g >= kStages)
-          ok = __all_sync(~0u, tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - kStages) / kStages) & 1,
-                                             status));
-        if (!ok) break;
-        if (lane == 0) tc::mbar_arrive_expect_tx(&bar[kKvFull0 + b], kTileBytes);
-        __syncwarp();
-        uint8_t* tile = smem + kOffTile + b * kTileBytes;
-        const bool is_win = j < w.twin;
-        if (is_win ? win_contig : pool_contig) {
-          if (lane == 0) {
+        for (int j = 0; j < w.tiles && ok; ++j, ++g) {
+          const uint32_t b = g % kStages;
+          if (g >= kStages) ok = tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - kStages) / kStages) & 1,
+                                               status);
+          if (!ok) break;
+          const bool is_win = j < w.twin;
+          if (is_win ? win_contig : pool_contig) {
+            tc::mbar_arrive_expect_tx(&bar[kKvFull0 + b], kTileBytes);
             const int64_t y0 = is_win ? a.win.row_index(w.seq, w.lo + (int64_t)j * kNK)
                                       : a.pool.row_index(w.seq, (int64_t)(j - w.twin) * kNK);
             const CUtensorMap* map = is_win ? &tm_win_box : &tm_pool_box;
+            uint8_t* tile = smem + kOffTile + b * kTileBytes;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
               tc::tma_load_2d(tile + c * kKRegion, map, &bar[kKvFull0 + b], 64 * c, (int32_t)y0);
+          } else {
+            tc::mbar_arrive(&bar[kKvFull0 + b]);
           }
-        } else if (lane < kNK / 4) {
-          int32_t y[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = lane * 4 + u;
-            if (is_win) {
-              int x = j * kNK + c;
-              if (x >= w.nwin) x = 0;  // past the tile's keys: any valid row (masked)
-              y[u] = (int32_t)a.win.row_index(w.seq, w.lo + x);
-            } else {
-              int i = (j - w.twin) * kNK + c;
-              if (i >= w.npool) i = 0;
-              int64_t e = a.pool_mode == 2 ? (int64_t)sel_s[i] : i;
-              y[u] = (int32_t)a.pool.row_index(w.seq, e < 0 ? 0 : e);
-            }
-          }
-          const CUtensorMap* map = is_win ? &tm_win : &tm_pool;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            tc::tma_gather4(tile + c * kKRegion + lane * 512, map, &bar[kKvFull0 + b], 64 * c,
-                            y[0], y[1], y[2], y[3]);
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+    __syncwarp();
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------------ MMA issuers
+    const uint32_t me = warp - 1;  // 0: even partials + O[:,0:256]; 1: odd partials + O[:,256:]
     if (lane == 0) {
       uint32_t g0 = 0, qi = 0;
       bool ok = true;
@@ -211,22 +203,27 @@ __global__ void __launch_bounds__(256, 1)
         const Row w = locate_row(a, r);
         ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
         for (int j = 0; j <= w.tiles && ok; ++j) {
-          if (j < w.tiles) {  // S(g) = Q K^T
+          if (j < w.tiles) {  // S(g) = Q K^T over four partial accumulators
             const uint32_t g = g0 + j, b = g % kStages, s = g & 1;
             ok = tc::mbar_wait(&bar[kKvFull0 + b], (g / kStages) & 1, status);
             if (ok && g >= 2) ok = tc::mbar_wait(&bar[kPFull0 + s], ((g - 2) >> 1) & 1, status);
             if (!ok) break;
             tc::tc_fence_after();
-            const uint64_t kd = tc::desc_sw128(tc::smem_u32(smem + kOffTile + b * kTileBytes), 0,
-                                               1024);
-            const uint32_t d = tmem + (s ? kColS1 : kColS0);
+            const uint64_t kd =
+                tc::desc_sw128(tc::smem_u32(smem + kOffTile + b * kTileBytes), 0, 1024);
+            const uint32_t d0 = tmem + kColS + s * kSStride;
             // the descriptor's start-address field counts 16-byte units: advancing along K adds
             // the byte offset >> 4 to the base descriptor
+            // partial p = kk & 3 lives in lanes 16*(p&1), columns + (p>>1)*48; this issuer owns
+            // the partials with (p & 1) == me
+            const uint32_t dme = d0 + (me ? (16u << 16) : 0u);
 #pragma unroll
-            for (int kk = 0; kk < kDim / 16; ++kk) {
-              const uint32_t qo = ((kk >> 2) * kQRegion + (kk & 3) * 32) >> 4;
-              const uint32_t ko = ((kk >> 2) * kKRegion + (kk & 3) * 32) >> 4;
-              tc::mma_bf16_ss(d, qd + qo, kd + ko, kIdescQK, kk > 0);
+            for (int k2 = 0; k2 < kDim / 32; ++k2) {
+              const int kk0 = 2 * k2 + (int)me;  // kk0 & 1 == me
+              const uint32_t qo = ((kk0 >> 2) * kQRegion + (kk0 & 3) * 32) >> 4;
+              const uint32_t ko = ((kk0 >> 2) * kKRegion + (kk0 & 3) * 32) >> 4;
+              tc::mma_bf16_ss(dme + ((kk0 & 2) ? (uint32_t)kNK : 0u), qd + qo, kd + ko, kIdescQK,
+                              kk0 >= 4);
             }
             tc::mma_commit(&bar[kSFull0 + s]);
             if (j == w.tiles - 1) tc::mma_commit(&bar[kQEmpty]);
@@ -239,13 +236,12 @@ __global__ void __launch_bounds__(256, 1)
             tc::tc_fence_after();
             const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
             const uint64_t pd = tc::desc_sw128(tc::smem_u32(smem + kOffP + s * kPBytes), 0, 1024);
-            const uint64_t vlo = tc::desc_sw128(v_base, kKRegion, 1024);
-            const uint64_t vhi = tc::desc_sw128(v_base + 4 * kKRegion, kKRegion, 1024);
+            const uint64_t vd = tc::desc_sw128(v_base + me * 4 * kKRegion, kKRegion, 1024);
+            const uint32_t od = tmem + (me ? (16u << 16) : 0u);
 #pragma unroll
             for (int kk = 0; kk < kNK / 16; ++kk) {
               const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
-              tc::mma_bf16_ss(tmem, pd + kk * 2, vlo + kk * 128, kIdescPV, acc);
-              tc::mma_bf16_ss(tmem + (16u << 16), pd + kk * 2, vhi + kk * 128, kIdescPV, acc);
+              tc::mma_bf16_ss(od, pd + kk * 2, vd + kk * 128, kIdescPV, acc);
             }
             tc::mma_commit(&bar[kKvEmpty0 + b]);
             tc::mma_commit(&bar[kPvDone0 + s]);
@@ -256,11 +252,10 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp == 3) {
     // ------------------------------------------------------------------ query rotation
-    // thread i turns the rope pairs of head row i of the staged query tile (row h's 16-byte
-    // chunk c of a 128-byte region sits at chunk c ^ (h & 7)).
-    const int h = (warp - 2) * 32 + lane;
+    // thread i turns the rope pairs of head rows i and i+32 of the staged query tile (row h's
+    // 16-byte chunk c of a 128-byte region sits at chunk c ^ (h & 7)).
     const int R = a.rf.R;
     const int p0 = (kDim - R) >> 1;  // first rotated pair among the 256 channel pairs
     uint32_t qi = 0;
@@ -273,9 +268,9 @@ __global__ void __launch_bounds__(256, 1)
       if (lane < R / 2) rope_cos_sin(a.rf, lane, a.pos0 + t, my_c, my_s);
       ok = __all_sync(~0u, tc::mbar_wait(&bar[kQFull], qi & 1, status));
       if (!ok) break;
+      for (int hh = 0; hh < 2; ++hh) {
+      const int h = hh * 32 + lane;
       uint8_t* row = smem + kOffQ + h * 128;
-      // four pairs per 16-byte chunk (R is even and the rope slice starts on a chunk boundary
-      // whenever R is a multiple of 8; other R take the per-pair path)
       for (int p = 0; p < R / 2; p += 4) {
         const int pp = p0 + p;                  // channels 2pp, 2pp+1
         const int region = pp >> 5;             // 32 pairs per 128-byte region
@@ -304,13 +299,55 @@ __global__ void __launch_bounds__(256, 1)
           }
         }
       }
+      }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bar[kQReady]);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ gather groups
+    // group 0 (warps 4-5) fills even tiles, group 1 (warps 6-7) odd tiles. Thread t copies rows
+    // t/8, t/8 + 8, ..., t/8 + 40 of the tile; for each it copies 16-byte slot t%8 of all 8
+    // regions, so a warp instruction reads four whole 128-byte row segments and a thread needs
+    // only six row addresses. Once its copies landed it makes them visible to the tensor core
+    // and arrives on the tile's barrier.
+    const int grp = (warp - 4) >> 1;
+    const int gt = (warp & 1) * 32 + lane;    // 0..63
+    const int row0 = gt >> 3, slot = gt & 7;
+    constexpr int kRowsPer = kNK / 8;         // 6
+    uint32_t g = 0;
+    bool ok = true;
+    for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x) {
+      const Row w = locate_row(a, r);
+      for (int j = 0; j < w.tiles && ok; ++j, ++g) {
+        if ((int)(g & 1) != grp) continue;
+        const uint32_t b = g % kStages;
+        if (g >= kStages)
+          ok = __all_sync(~0u, tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - kStages) / kStages) & 1,
+                                             status));
+        if (!ok) break;
+        const bool is_win = j < w.twin;
+        if (!(is_win ? win_contig : pool_contig)) {
+          uint8_t* tile = smem + kOffTile + b * kTileBytes;
+          const __nv_bfloat16* src[kRowsPer];
+#pragma unroll
+          for (int i = 0; i < kRowsPer; ++i) src[i] = key_ptr(a, w, r, j, row0 + 8 * i);
+#pragma unroll
+          for (int i = 0; i < kRowsPer; ++i) {
+            const int row = row0 + 8 * i;
+            uint8_t* d = tile + row * 128 + ((slot ^ (row & 7)) << 4);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) tc::cp_async16(d + q * kKRegion, src[i] + q * 64 + slot * 8);
+          }
+          tc::cp_async_wait_all();
+          tc::fence_proxy_async_smem();
+        }
+        tc::mbar_arrive(&bar[kKvFull0 + b]);
+      }
     }
   } else {
     // ------------------------------------------------------------------ softmax + output
     const int sp = warp & 3;                 // TMEM sub-partition of this warp
-    const int half = lane >> 4;              // 0: lanes 0-15 (S rows, O[:,0:256]); 1: O[:,256:512]
+    const int half = lane >> 4;              // 0: keys 0..23, O[:,0:256]; 1: keys 24..47, O[:,256:]
     const int h = 16 * sp + (lane & 15);     // head of this thread's row
     const uint32_t t_row = tmem + ((uint32_t)(32 * sp) << 16);
     const float scale_log2 = a.scale * kLog2e;
@@ -325,24 +362,38 @@ __global__ void __launch_bounds__(256, 1)
         ok = __all_sync(~0u, tc::mbar_wait(&bar[kSFull0 + s], (g >> 1) & 1, status));
         if (!ok) break;
         tc::tc_fence_after();
-        float sv[kNK];
-#pragma unroll
-        for (int c = 0; c < kNK; c += 16) {
+        // own partials: columns [0,48) and [48,96) of this S buffer in this thread's lane
+        float own[kNK];
+        {
           uint32_t v[16];
-          tc::tmem_ld16(t_row + (s ? kColS1 : kColS0) + c, v);
-          tc::tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 16; ++u) sv[c + u] = __uint_as_float(v[u]);
+          for (int c = 0; c < kNK; c += 16) {
+            uint32_t u[16];
+            tc::tmem_ld16(t_row + kColS + s * kSStride + c, v);
+            tc::tmem_ld16(t_row + kColS + s * kSStride + kNK + c, u);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) own[c + e] = __uint_as_float(v[e]) + __uint_as_float(u[e]);
+          }
+        }
+        // exchange: this thread finishes keys [half*24, half*24+24) of the row
+        float sv[kHalfNK];
+#pragma unroll
+        for (int k = 0; k < kHalfNK; ++k) {
+          const float send = half ? own[k] : own[kHalfNK + k];
+          const float recv = __shfl_xor_sync(~0u, send, 16);
+          sv[k] = (half ? own[kHalfNK + k] : own[k]) + recv;
         }
         const int nk = j < w.twin ? min(kNK, w.nwin - j * kNK)
                                   : min(kNK, w.npool - (j - w.twin) * kNK);
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kNK; ++c) {
-          sv[c] = c < nk ? sv[c] * scale_log2 : -INFINITY;
-          mx = fmaxf(mx, sv[c]);
+        for (int k = 0; k < kHalfNK; ++k) {
+          sv[k] = half * kHalfNK + k < nk ? sv[k] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sv[k]);
         }
-        const bool move = half == 0 && mx > m_run + kLazy;
+        mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, 16));
+        const bool move = mx > m_run + kLazy;
         const float m_new = move ? mx : m_run;
         const float alpha = exp2f(m_run - m_new);
         // rescale the rows of O this warp owns (rare: only when some row's max moved)
@@ -351,38 +402,38 @@ __global__ void __launch_bounds__(256, 1)
           ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + (gp & 1)], (gp >> 1) & 1, status));
           if (!ok) break;
           tc::tc_fence_after();
-          const float al = __shfl_sync(~0u, alpha, lane & 15);
 #pragma unroll 1
           for (int c = 0; c < 256; c += 16) {
             uint32_t v[16];
             tc::tmem_ld16(t_row + c, v);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 16; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * al);
+            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
             tc::tmem_st16(t_row + c, v);
           }
           tc::tmem_wait_st();
         }
         float sum = 0.f;
-        uint32_t pk[kNK / 2];
+        uint32_t pk[kHalfNK / 2];
 #pragma unroll
-        for (int c = 0; c < kNK; c += 2) {
-          const float e0 = exp2f(sv[c] - m_new), e1 = exp2f(sv[c + 1] - m_new);
+        for (int k = 0; k < kHalfNK; k += 2) {
+          const float e0 = exp2f(sv[k] - m_new), e1 = exp2f(sv[k + 1] - m_new);
           sum += e0 + e1;
-          pk[c / 2] = pack_bf16(e0, e1);
+          pk[k / 2] = pack_bf16(e0, e1);
         }
+        sum += __shfl_xor_sync(~0u, sum, 16);
         l_run = l_run * alpha + sum;
         m_run = m_new;
         // P buffer s is free once PV(g-2) completed
         if (g >= 2)
           ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + s], ((g - 2) >> 1) & 1, status));
         if (!ok) break;
-        if (half == 0) {
-          uint8_t* prow = smem + kOffP + s * kPBytes + h * 128;
+        uint8_t* prow = smem + kOffP + s * kPBytes + h * 128;
 #pragma unroll
-          for (int ch = 0; ch < kNK / 8; ++ch)
-            *reinterpret_cast<uint4*>(prow + ((ch ^ (h & 7)) << 4)) =
-                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        for (int ch = 0; ch < kHalfNK / 8; ++ch) {
+          const int cg = half * (kHalfNK / 8) + ch;  // 16-byte chunk of keys 8cg..8cg+7
+          *reinterpret_cast<uint4*>(prow + ((cg ^ (h & 7)) << 4)) =
+              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -397,41 +448,48 @@ __global__ void __launch_bounds__(256, 1)
       ok = __all_sync(~0u, tc::mbar_wait(&bar[kOFull], qi & 1, status));
       if (!ok) break;
       tc::tc_fence_after();
-      const float inv_l = 1.f / __shfl_sync(~0u, l_run, lane & 15);
+      const float inv_l = 1.f / l_run;
       __nv_bfloat16* orow =
           reinterpret_cast<__nv_bfloat16*>(a.o) + ((int64_t)r * kHeads + h) * kDim + half * 256;
       const int rope_lo = kDim - a.rf.R;  // first rotated channel (always in the upper half)
 #pragma unroll 1
-      for (int c = 0; c < 256; c += 16) {
-        uint32_t v[16];
-        tc::tmem_ld16(t_row + c, v);
+      for (int c0 = 0; c0 < 256; c0 += 64) {
+        uint32_t v[4][16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tc::tmem_ld16(t_row + c0 + 16 * q, v[q]);
         tc::tmem_wait_ld();
-        float x[16];
+        if (c0 + 64 == 256) {  // last chunk: every upper-half lane holds rope channels here
+          tc::tc_fence_before();
+          tc::mbar_arrive(&bar[kOEmpty]);
+        }
 #pragma unroll
-        for (int u = 0; u < 16; ++u) x[u] = __uint_as_float(v[u]) * inv_l;
-        if (256 + c + 16 > rope_lo) {  // warp-uniform: some upper-half lane rotates here
+        for (int q = 0; q < 4; ++q) {
+          const int c = c0 + 16 * q;
+          float x[16];
 #pragma unroll
-          for (int u = 0; u < 16; u += 2) {
-            const int ch = half * 256 + c + u;
-            const int p = ch >= rope_lo ? (ch - rope_lo) >> 1 : 0;
-            const float cc = __shfl_sync(~0u, my_c, p);
-            const float ss = __shfl_sync(~0u, my_s, p);
-            if (ch >= rope_lo) {
-              const float x0 = x[u], x1 = x[u + 1];
-              x[u] = x0 * cc - x1 * ss;
-              x[u + 1] = x0 * ss + x1 * cc;
+          for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[q][e]) * inv_l;
+          if (256 + c + 16 > rope_lo) {  // warp-uniform: some upper-half lane rotates here
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const int ch = half * 256 + c + e;
+              const int p = ch >= rope_lo ? (ch - rope_lo) >> 1 : 0;
+              const float cc = __shfl_sync(~0u, my_c, p);
+              const float ss = __shfl_sync(~0u, my_s, p);
+              if (ch >= rope_lo) {
+                const float x0 = x[e], x1 = x[e + 1];
+                x[e] = x0 * cc - x1 * ss;
+                x[e + 1] = x0 * ss + x1 * cc;
+              }
             }
           }
+          uint4 o0 = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+          uint4 o1 = make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]),
+                                pack_bf16(x[12], x[13]), pack_bf16(x[14], x[15]));
+          reinterpret_cast<uint4*>(orow + c)[0] = o0;
+          reinterpret_cast<uint4*>(orow + c)[1] = o1;
         }
-        uint4 o0 = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                              pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-        uint4 o1 = make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]),
-                              pack_bf16(x[12], x[13]), pack_bf16(x[14], x[15]));
-        reinterpret_cast<uint4*>(orow + c)[0] = o0;
-        reinterpret_cast<uint4*>(orow + c)[1] = o1;
       }
-      tc::tc_fence_before();
-      tc::mbar_arrive(&bar[kOEmpty]);
       g0 += w.tiles;
     }
   }
@@ -446,26 +504,20 @@ __global__ void __launch_bounds__(256, 1)
 }  // namespace
 
 bool attention_tc_supported(const AttnArgs& a, int dtype) {
-  return dtype == 1 && a.H == kHeads && a.D == kDim && a.rf.R <= 64 && a.rf.R % 2 == 0 &&
-         (a.pool_mode != 2 || a.k <= kMaxSel);
+  return dtype == 1 && a.H == kHeads && a.D == kDim && a.rf.R <= 64 && a.rf.R % 2 == 0;
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t pool_rows,
                                 cudaStream_t st) {
   if (a.nrows == 0) return cudaSuccess;
-  CUtensorMap tq, tw, tp, twb, tpb;
+  CUtensorMap tq, twb, tpb;
   cudaError_t e = make_tmap_bf16_2d(&tq, a.q, (uint64_t)a.nrows * kHeads, kDim, kDim * 2, 64, 64);
-  if (e != cudaSuccess) return e;
-  e = make_tmap_bf16_2d(&tw, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, 1, 64);
-  if (e != cudaSuccess) return e;
-  const bool has_pool = a.pool_mode != 0 && pool_rows > 0;
-  const void* pb = has_pool ? a.pool.base : a.win.base;
-  const uint64_t pr = (uint64_t)(has_pool ? pool_rows : win_rows);
-  e = make_tmap_bf16_2d(&tp, pb, pr, kDim, kDim * 2, 1, 64);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16_2d(&twb, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
-  e = make_tmap_bf16_2d(&tpb, pb, pr, kDim, kDim * 2, kNK, 64);
+  const bool has_pool = a.pool_mode != 0 && pool_rows > 0;
+  e = make_tmap_bf16_2d(&tpb, has_pool ? a.pool.base : a.win.base,
+                        (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes);
@@ -474,7 +526,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = (int)(a.nrows < sms ? a.nrows : sms);
-  attention_tc_kernel<<<grid, 256, kSmemBytes, st>>>(tq, tw, tp, twb, tpb, a);
+  attention_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
   return cudaGetLastError();
 }
 
