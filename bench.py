@@ -212,6 +212,17 @@ def timed(step, steps, dev):
     return a.elapsed_time(b)
 
 
+def tensor_kernels(wl) -> set:
+    """Kernels that run on tcgen05 for this workload (bf16 layers with 64 heads of 512; the
+    indexer with 64 heads of 128); the rest run on CUDA cores."""
+    out = set()
+    if wl.dtype == "bf16" and wl.H == 64 and wl.D == 512 and wl.R <= 64:
+        out.add("attention")
+    if wl.kind == "csa" and wl.dtype == "bf16" and wl.nI == 64 and wl.cI == 128:
+        out.add("indexer_score")
+    return out
+
+
 def roofline(wl, ktimes: dict, peaks: dict, steps: int, tensor_kernels: set) -> tuple:
     wk = work(wl)
     total = sum(v[1] for v in ktimes.values()) or 1.0
@@ -338,7 +349,7 @@ def run_ours(args, wl0):
     e2e_ms = max_over_ranks(timed(e2e_step, args.steps, dev), dev) / args.steps
 
     peaks = measured_peaks()
-    roof, krows = roofline(wl, ktimes, peaks, args.steps, tensor_kernels=set())
+    roof, krows = roofline(wl, ktimes, peaks, args.steps, tensor_kernels=tensor_kernels(wl))
     launches = sum(v[0] for v in ktimes.values())
     line = {
         "metric": f"{wl.kind.upper()} attention fwd tokens/s (prefill)", "value": value,
@@ -352,6 +363,124 @@ def run_ours(args, wl0):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------------------------
+# decode: one step = the CSA layer and the HCA layer, each over its paged cache
+# ------------------------------------------------------------------------------------------------
+def decode_bytes(wl, d_csa, d_hca) -> dict:
+    """Algorithmic HBM bytes per decode step (what must be read / written once)."""
+    esz = 2
+    out = {}
+    ctx = d_csa["ctx_lens"].numpy().astype(np.int64)
+    nv = ctx // wl.m
+    win = np.minimum(ctx, wl.W)
+    qb = wl.nseq * wl.H * wl.D * esz
+    out["indexer_score"] = float((nv * wl.cI * esz).sum() + wl.nseq * wl.nI * (wl.cI * esz + 4)
+                                 + (nv * 4).sum())
+    out["topk"] = float((nv * 4).sum() + wl.nseq * wl.k * 4)
+    att_csa = float(((np.minimum(nv, wl.k) + win) * wl.D * esz).sum() + 2 * qb)
+    ctx_h = d_hca["ctx_lens"].numpy().astype(np.int64)
+    att_hca = float(((ctx_h // d_hca["m"] + np.minimum(ctx_h, wl.W)) * wl.D * esz).sum() + 2 * qb)
+    out["attention"] = att_csa + att_hca
+    return out
+
+
+def run_decode(args, wl0):
+    import sparse_attention_compressor_b200 as sac
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    wl = rank_workload(wl0, rank)
+    dc = W.decode_inputs(wl, "csa")
+    dh = W.decode_inputs(wl, "hca")
+    gc = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in dc.items()}
+    gh = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in dh.items()}
+    max_ctx = int(max(dc["ctx_lens"].max(), dh["ctx_lens"].max()))
+    pc = sac.make_params(1, max_ctx, wl.H, wl.D, wl.R, wl.theta, m=wl.m, win_len=wl.L,
+                         sliding_window=wl.W, n_idx_heads=wl.nI, idx_dim=wl.cI, topk=wl.k,
+                         dtype=wl.dtype)
+    ph = sac.make_params(1, max_ctx, wl.H, wl.D, wl.R, wl.theta, m=dh["m"], win_len=dh["m"],
+                         sliding_window=wl.W, dtype=wl.dtype)
+    ws = torch.empty(sac.sac_decode_workspace_size(pc, sac.SAC_KIND_CSA, wl.nseq),
+                     dtype=torch.uint8, device=dev)
+    oc = torch.empty_like(gc["q"])
+    oh = torch.empty_like(gh["q"])
+    ps = wl.page_size
+
+    def step():
+        sac.csa_decode(pc, wl.nseq, gc["q"], gc["kv_pages"], gc["kv_block_table"], gc["ctx_lens"],
+                       ps, gc["pool_pages"], gc["idx_pool_pages"], gc["pool_block_table"],
+                       gc["q_idx"], gc["w_idx"], gc["sinks"], oc, None, ws)
+        sac.hca_decode(ph, wl.nseq, gh["q"], gh["kv_pages"], gh["kv_block_table"], gh["ctx_lens"],
+                       ps, gh["pool_pages"], gh["pool_block_table"], gh["sinks"], oh)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sac.sac_timing_begin()
+    with ClockSampler(dev.index) as clk:
+        ms = timed(step, args.steps, dev)
+    ktimes = sac.sac_timing_end()
+    ms = max_over_ranks(ms, dev)
+    us_step = 1e3 * ms / args.steps
+    # end to end: the step's new-token inputs from pinned host memory, outputs back
+    pin = {k: dc[k].pin_memory() for k in ("q", "q_idx", "w_idx")}
+    pin["q_h"] = dh["q"].pin_memory()
+    oc_h = torch.empty(oc.shape, dtype=oc.dtype, pin_memory=True)
+    oh_h = torch.empty(oh.shape, dtype=oh.dtype, pin_memory=True)
+
+    def e2e_step():
+        gc["q"].copy_(pin["q"], non_blocking=True)
+        gc["q_idx"].copy_(pin["q_idx"], non_blocking=True)
+        gc["w_idx"].copy_(pin["w_idx"], non_blocking=True)
+        gh["q"].copy_(pin["q_h"], non_blocking=True)
+        step()
+        oc_h.copy_(oc, non_blocking=True)
+        oh_h.copy_(oh, non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_us = 1e3 * max_over_ranks(timed(e2e_step, args.steps, dev), dev) / args.steps
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = (oc.numel() + oh.numel()) * oc.element_size()
+    peaks = measured_peaks()
+    wb = decode_bytes(wl, dc, dh)
+    krows = {}
+    total = sum(v[1] for v in ktimes.values()) or 1.0
+    for name, (launches, kms) in ktimes.items():
+        per = kms / max(launches, 1)
+        row = {"launches": launches, "ms_per_launch": per, "share": kms / total}
+        if name in wb:
+            per_launch_bytes = wb[name] / (launches / args.steps)
+            ach = per_launch_bytes / (per * 1e-3) / 1e9
+            row.update(bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
+                       frac=ach / peaks["hbm_gbs"])
+        krows[name] = row
+    dom = max(ktimes, key=lambda k: ktimes[k][1])
+    d = krows[dom]
+    line = {
+        "metric": "decode us/step (CSA + HCA layer, 64 sequences)", "value": us_step,
+        "unit": "us/step", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us_step / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded; see DESIGN.md)",
+        "config": {"workload": wl.name, "nseq": wl.nseq, "ctx": f"U[{wl.ctx_lo},{wl.ctx_hi}]",
+                   "page_size": wl.page_size, "H": wl.H, "head_dim": wl.D, "csa_m": wl.m,
+                   "hca_m": dh["m"], "index_topk": wl.k, "sliding_window": wl.W,
+                   "parallelism": f"dp{world}", "l2": "paged caches of several GB, no flush"},
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": sum(v[0] for v in ktimes.values()),
+        "roofline": {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
+                     "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),
+                     "traffic": None, "peak_source": peaks["source"]},
+        "kernels": krows,
+    }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -397,13 +526,14 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="csa_8k_bf16",
-                    choices=[k for k, v in W.WORKLOADS.items() if v.kind != "decode"])
+    ap.add_argument("--workload", default="csa_8k_bf16", choices=list(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     wl = W.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)
+    elif wl.kind == "decode":
+        run_decode(args, wl)
     else:
         run_ours(args, wl)
 

@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* status = a.status;
   // the 128-byte swizzle needs 1024-byte aligned tiles; the dynamic window starts aligned
   if ((tc::smem_u32(smem) & 1023u) != 0) {
-    if (threadIdx.x == 0) atomicExch(status, tc::kStatusMisaligned);
+    if (threadIdx.x == 0 && status) atomicExch(status, tc::kStatusMisaligned);
     return;
   }
 

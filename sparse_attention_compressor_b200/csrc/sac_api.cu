@@ -515,7 +515,7 @@ int swa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.nrows = nseq;
   a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
   a.pool_mode = 0;
-  cudaError_t e = sac::timed("attention", static_cast<cudaStream_t>(stream), [&] { return sac::launch_attention_simt(p->dtype, a, static_cast<cudaStream_t>(stream)); });
+  cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -540,7 +540,7 @@ int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
   a.pool_mode = 1;
   a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
-  cudaError_t e = sac::timed("attention", static_cast<cudaStream_t>(stream), [&] { return sac::launch_attention_simt(p->dtype, a, static_cast<cudaStream_t>(stream)); });
+  cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -594,7 +594,7 @@ int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.pool_mode = 2;
   a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
   a.sel = sel;
-  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  e = run_attention(p, a, 1, 1, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
