@@ -212,6 +212,24 @@ def timed(step, steps, dev):
     return a.elapsed_time(b)
 
 
+def timed_flushed(step, steps, dev):
+    """Like timed(), but L2 is flushed (a write of twice its size) before every step; each step
+    is bracketed by its own events and only the steps are summed."""
+    junk = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    for a, b in evs:
+        junk.fill_(0)
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    return sum(a.elapsed_time(b) for a, b in evs)
+
+
 def tensor_kernels(wl) -> set:
     """Kernels that run on tcgen05 for this workload (bf16 layers with 64 heads of 512; the
     indexer with 64 heads of 128); the rest run on CUDA cores."""
@@ -387,6 +405,14 @@ def decode_bytes(wl, d_csa, d_hca) -> dict:
     ctx_h = d_hca["ctx_lens"].numpy().astype(np.int64)
     att_hca = float(((ctx_h // d_hca["m"] + np.minimum(ctx_h, wl.W)) * wl.D * esz).sum() + 2 * qb)
     out["attention"] = att_csa + att_hca
+    # cache append: the new row read, written rotated to its page and un-rotated to the ring; a
+    # closing window (ctx % m == 0) reads its L ring rows and writes one entry
+    app = 0.0
+    for d, m, L, cI in ((d_csa, wl.m, wl.L, wl.cI), (d_hca, d_hca["m"], d_hca["m"], 0)):
+        c = d["ctx_lens"].numpy().astype(np.int64)
+        closing = int((c % m == 0).sum())
+        app += wl.nseq * (3 * wl.D + 2 * cI) * esz + closing * (L + 1) * (wl.D + cI) * esz
+    out["decode_append"] = app
     return out
 
 
@@ -414,9 +440,21 @@ def run_decode(args, wl0):
     ps = wl.page_size
 
     def step():
+        # each layer: append the new token to its caches, then attend
+        sac.decode_append(pc, sac.SAC_KIND_CSA, wl.nseq, gc["ctx_lens"], gc["kv_new"],
+                          gc["kv_pages"], gc["kv_block_table"], ps, cmp_state=gc["cmp_state"],
+                          cmp_gate=gc["cmp_gate"], cmp_bias=gc["cmp_bias"],
+                          pool_pages=gc["pool_pages"], pool_block_table=gc["pool_block_table"],
+                          k_idx_new=gc["k_idx_new"], idx_state=gc["idx_state"],
+                          idx_gate=gc["idx_gate"], idx_bias=gc["idx_bias"],
+                          idx_pool_pages=gc["idx_pool_pages"])
         sac.csa_decode(pc, wl.nseq, gc["q"], gc["kv_pages"], gc["kv_block_table"], gc["ctx_lens"],
                        ps, gc["pool_pages"], gc["idx_pool_pages"], gc["pool_block_table"],
                        gc["q_idx"], gc["w_idx"], gc["sinks"], oc, None, ws)
+        sac.decode_append(ph, sac.SAC_KIND_HCA, wl.nseq, gh["ctx_lens"], gh["kv_new"],
+                          gh["kv_pages"], gh["kv_block_table"], ps, cmp_state=gh["cmp_state"],
+                          cmp_gate=gh["cmp_gate"], cmp_bias=gh["cmp_bias"],
+                          pool_pages=gh["pool_pages"], pool_block_table=gh["pool_block_table"])
         sac.hca_decode(ph, wl.nseq, gh["q"], gh["kv_pages"], gh["kv_block_table"], gh["ctx_lens"],
                        ps, gh["pool_pages"], gh["pool_block_table"], gh["sinks"], oh)
 
@@ -425,13 +463,14 @@ def run_decode(args, wl0):
     torch.cuda.synchronize(dev)
     sac.sac_timing_begin()
     with ClockSampler(dev.index) as clk:
-        ms = timed(step, args.steps, dev)
+        ms = timed_flushed(step, args.steps, dev)
     ktimes = sac.sac_timing_end()
     ms = max_over_ranks(ms, dev)
     us_step = 1e3 * ms / args.steps
     # end to end: the step's new-token inputs from pinned host memory, outputs back
-    pin = {k: dc[k].pin_memory() for k in ("q", "q_idx", "w_idx")}
+    pin = {k: dc[k].pin_memory() for k in ("q", "q_idx", "w_idx", "kv_new", "k_idx_new")}
     pin["q_h"] = dh["q"].pin_memory()
+    pin["kv_new_h"] = dh["kv_new"].pin_memory()
     oc_h = torch.empty(oc.shape, dtype=oc.dtype, pin_memory=True)
     oh_h = torch.empty(oh.shape, dtype=oh.dtype, pin_memory=True)
 
@@ -439,13 +478,16 @@ def run_decode(args, wl0):
         gc["q"].copy_(pin["q"], non_blocking=True)
         gc["q_idx"].copy_(pin["q_idx"], non_blocking=True)
         gc["w_idx"].copy_(pin["w_idx"], non_blocking=True)
+        gc["kv_new"].copy_(pin["kv_new"], non_blocking=True)
+        gc["k_idx_new"].copy_(pin["k_idx_new"], non_blocking=True)
         gh["q"].copy_(pin["q_h"], non_blocking=True)
+        gh["kv_new"].copy_(pin["kv_new_h"], non_blocking=True)
         step()
         oc_h.copy_(oc, non_blocking=True)
         oh_h.copy_(oh, non_blocking=True)
     e2e_step()
     torch.cuda.synchronize(dev)
-    e2e_us = 1e3 * max_over_ranks(timed(e2e_step, args.steps, dev), dev) / args.steps
+    e2e_us = 1e3 * max_over_ranks(timed_flushed(e2e_step, args.steps, dev), dev) / args.steps
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
     d2h = (oc.numel() + oh.numel()) * oc.element_size()
     peaks = measured_peaks()
@@ -471,7 +513,7 @@ def run_decode(args, wl0):
         "config": {"workload": wl.name, "nseq": wl.nseq, "ctx": f"U[{wl.ctx_lo},{wl.ctx_hi}]",
                    "page_size": wl.page_size, "H": wl.H, "head_dim": wl.D, "csa_m": wl.m,
                    "hca_m": dh["m"], "index_topk": wl.k, "sliding_window": wl.W,
-                   "parallelism": f"dp{world}", "l2": "paged caches of several GB, no flush"},
+                   "parallelism": f"dp{world}", "l2": "flushed before every step (write of 252 MiB)"},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

@@ -176,6 +176,10 @@ SAC_API int csa_forward(const sac_params* p, const void* q, const void* kv, cons
  *     Every ctx must satisfy 1 <= ctx <= p->S.
  *   q [nseq,H,D] un-rotated; o [nseq,H,D]; q_idx [nseq,nI,cI], w_idx [nseq,nI] fp32 (CSA);
  *   topk_out [nseq,k] nullable (ascending entries, -1 fill).
+ * Workspace: sac_decode_workspace_size() bytes, 16-byte aligned: a 256-byte status word (see
+ * sac_device_status) and, for CSA, the scores [nseq, S/m] fp32 and the selection [nseq, k]. ws is
+ * required by csa_decode; swa_decode / hca_decode accept NULL (no status word is then kept) or at
+ * least 256 bytes. Entries on an unallocated page (block table entry < 0) read as zero keys.
  */
 SAC_API size_t sac_decode_workspace_size(const sac_params* p, int kind, int nseq);
 
@@ -198,8 +202,38 @@ SAC_API int csa_decode(const sac_params* p, int nseq, const void* q, const void*
                size_t ws_bytes, void* stream);
 
 /*
- * Device status of the last prefill call that used workspace `ws` (no counterpart on the page:
- * failure reporting). Every prefill call clears the first word of its workspace; a tensor-core
+ * Decode cache append ("Cache layers": the sliding K=V window plus the compressor buffer / pool /
+ * count / overlap state and the indexer's copy of it at index_head_dim; "Hybrid attention": an
+ * entry exists once its source window has closed). Call it once per decode step, before
+ * *_decode, for the new token of each of nseq sequences; ctx_lens [nseq] (device, int32) already
+ * counts that token, which sits at t = ctx - 1 (position pos0 + t). kind: SAC_KIND_*.
+ *   kv_new [nseq, D]          the new token's un-rotated kv row; written rotated at pos0 + t to row
+ *                             t of kv_pages (same paging as *_decode)
+ *   cmp_state [nseq, win_len, D]   HCA / CSA: compressor buffer, a ring of the last win_len
+ *                             un-rotated kv rows (row j in slot j mod win_len; for CSA the older
+ *                             half is the overlap with the previous window). Caller-owned; after a
+ *                             prefill of P tokens seed it with rows P - win_len .. P - 1.
+ *   cmp_gate [D], cmp_bias [win_len] fp32   the compressor gate, as in hca_forward
+ *   pool_pages, pool_block_table, pool_max_pages   as in hca_decode / csa_decode
+ * When t + 1 is a multiple of m, entry w = (t+1)/m - 1 closes: it is pooled over the ring rows of
+ * its window [(w+1)m - win_len, (w+1)m) (clipped at 0) with the compressor's softmax gate, exactly
+ * as the prefill compressor does, rotated at pos0 + w*m and written to row w of pool_pages.
+ * CSA also takes k_idx_new [nseq, cI], idx_state [nseq, win_len, cI], idx_gate [cI], idx_bias
+ * [win_len] fp32 and idx_pool_pages, and closes the indexer entry the same way without rotation.
+ * SWA uses only kv_new and the kv pages (the other pointers may be NULL). Rows on unallocated
+ * pages (block table entry < 0) are skipped. No workspace; returns before the kernel runs.
+ */
+SAC_API int decode_append(const sac_params* p, int kind, int nseq, const int32_t* ctx_lens,
+               const void* kv_new, const void* k_idx_new, const void* cmp_gate,
+               const float* cmp_bias, const void* idx_gate, const float* idx_bias,
+               void* kv_pages, const int32_t* kv_block_table, int kv_max_pages, int page_size,
+               void* cmp_state, void* idx_state, void* pool_pages, void* idx_pool_pages,
+               const int32_t* pool_block_table, int pool_max_pages, void* stream);
+
+/*
+ * Device status of the last call that used workspace `ws` (no counterpart on the page: failure
+ * reporting). Every prefill call, and every decode call given a workspace, clears the first word
+ * of its workspace; a tensor-core
  * kernel that gives up a bounded wait (2 s) writes a nonzero code there and returns instead of
  * hanging. This call waits for `stream`, copies the word to *status (0 = ok, 1 = a wait timed
  * out, 2 = misaligned shared memory) and returns SAC_OK, or SAC_ERR_LAUNCH if the copy fails.

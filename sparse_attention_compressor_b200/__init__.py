@@ -21,7 +21,8 @@ SAC_KIND_SWA, SAC_KIND_HCA, SAC_KIND_CSA = 0, 1, 2
 ABI_SYMBOLS = ("sac_last_error", "sac_version", "sac_workspace_size", "swa_forward",
                "hca_forward", "csa_forward", "sac_decode_workspace_size", "swa_decode",
                "hca_decode", "csa_decode", "sac_timing_begin", "sac_timing_end",
-               "sac_static_scratch_bytes", "swa_forward_static", "sac_device_status")
+               "sac_static_scratch_bytes", "swa_forward_static", "sac_device_status",
+               "decode_append")
 
 
 class SacError(RuntimeError):
@@ -88,6 +89,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                vp]
     lib.csa_decode.argtypes = [P, ci, vp, vp, i32p, ci, i32p, ci, vp, vp, i32p, ci, vp, fp, fp,
                                vp, i32p, vp, sz, vp]
+    lib.decode_append.argtypes = [P, ci, ci, i32p, vp, vp, vp, fp, vp, fp, vp, i32p, ci, ci, vp,
+                                  vp, vp, vp, i32p, ci, vp]
     lib.sac_device_status.restype = ci
     lib.sac_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
     lib.sac_static_scratch_bytes.restype = sz
@@ -97,7 +100,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sac_timing_end.restype = ci
     lib.sac_timing_end.argtypes = [ctypes.POINTER(sac_kernel_time), ci]
     for name in ("swa_forward", "hca_forward", "csa_forward", "swa_decode", "hca_decode",
-                 "csa_decode"):
+                 "csa_decode", "decode_append"):
         getattr(lib, name).restype = ci
     _lib_handle = lib
     return lib
@@ -223,4 +226,20 @@ def csa_decode(p, nseq, q, kv_pages, kv_block_table, ctx_lens, page_size, pool_p
         kv_block_table.shape[1], _ptr(ctx_lens), page_size, _ptr(pool_pages),
         _ptr(idx_pool_pages), _ptr(pool_block_table), pool_block_table.shape[1], _ptr(q_idx),
         _ptr(w_idx), _ptr(sinks), _ptr(o), _ptr(topk_out), _ptr(ws), _nbytes(ws),
+        _stream(stream)))
+
+
+def decode_append(p, kind, nseq, ctx_lens, kv_new, kv_pages, kv_block_table, page_size,
+                  cmp_state=None, cmp_gate=None, cmp_bias=None, pool_pages=None,
+                  pool_block_table=None, k_idx_new=None, idx_state=None, idx_gate=None,
+                  idx_bias=None, idx_pool_pages=None, stream=None) -> None:
+    """Append each sequence's new token (at ctx - 1) to the decode caches: the rotated kv row to
+    the window pages and, for HCA / CSA, the compressor ring(s), closing a pool entry whenever
+    ctx is a multiple of m."""
+    pmax = pool_block_table.shape[1] if pool_block_table is not None else 0
+    _check("decode_append", load_library().decode_append(
+        ctypes.byref(p), kind, nseq, _ptr(ctx_lens), _ptr(kv_new), _ptr(k_idx_new),
+        _ptr(cmp_gate), _ptr(cmp_bias), _ptr(idx_gate), _ptr(idx_bias), _ptr(kv_pages),
+        _ptr(kv_block_table), kv_block_table.shape[1], page_size, _ptr(cmp_state),
+        _ptr(idx_state), _ptr(pool_pages), _ptr(idx_pool_pages), _ptr(pool_block_table), pmax,
         _stream(stream)))

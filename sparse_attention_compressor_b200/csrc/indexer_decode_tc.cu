@@ -1,0 +1,253 @@
+// Tensor-core (tcgen05) Lightning Indexer score of a decode step ("Hybrid attention", CSA bullet,
+// eq. 13-17; "Cache layers": paged indexer pool): for each sequence's single new query at
+// t = ctx - 1, I[w] = sum_h w_idx[h] * max(0, <q_idx[h], KI_w>) over the visible entries
+// w < ctx // m, bf16 layers with 64 indexer heads of dim 128.
+//
+// The step reads every visible indexer-pool entry once (256 bytes each) and does 64 x 128 MACs per
+// entry, so it is bound by HBM. One MMA per 128 entries puts all 64 head dot products of each
+// entry into tensor memory: D[entry, head] = KI[128 x 128] * q_idx[64 x 128]^T (M = 128, N = 64,
+// K = 128). In the drain each thread owns one entry (one TMEM lane), so the head reduction needs
+// no cross-thread traffic and the score stores are coalesced.
+//
+// Pool pages may have any size, so entries are gathered with 16-byte cp.async copies: sixteen
+// threads per 256-byte entry row (one fully used 512-byte span per warp instruction), three
+// 32 KB stages in flight per CTA and two CTAs per SM. Each CTA takes one (sequence, 1024-entry
+// chunk) pair; chunks past a sequence's visible entries exit at once.
+//
+// Warps: 0..3 gather (q_idx once, then entry blocks), 4..7 drain, 8 issues the MMAs and owns TMEM.
+#include <cuda_bf16.h>
+
+#include "sac_kernels.h"
+#include "tc_ptx.cuh"
+
+namespace sac {
+namespace {
+
+constexpr int kNI = 64;                   // indexer heads (MMA N)
+constexpr int kCI = 128;                  // indexer head dim (MMA K)
+constexpr int kBE = 128;                  // entries per block (MMA M)
+constexpr int kChunkBlocks = 8;           // blocks per CTA
+constexpr int kStages = 3;
+constexpr int kGatherThreads = 128;
+constexpr int kThreads = 288;
+constexpr int kRegion = kBE * 128;        // one 64-dim half of a block: [128 rows x 128 B]
+constexpr int kBlockBytes = 2 * kRegion;  // 32 KB
+constexpr int kQRegion = kNI * 128;       // [64 rows x 128 B]
+constexpr int kQBytes = 2 * kQRegion;     // 16 KB
+
+constexpr int kOffKv = 0;
+constexpr int kOffQ = kOffKv + kStages * kBlockBytes;
+constexpr int kOffW = kOffQ + kQBytes;
+constexpr int kOffBar = kOffW + kNI * 4;
+enum Bar { kFull0, kEmpty0 = kFull0 + kStages, kAccFull0 = kEmpty0 + kStages, kAccEmpty0 = kAccFull0 + 2,
+           kNumBars = kAccEmpty0 + 2 };
+constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffTmemPtr + 16;  // two CTAs per SM fit in 228 KB
+constexpr uint32_t kIdesc = tc::idesc_bf16(kBE, kNI, false, false);
+
+// cp.async.wait_group with the stage depth as its immediate.
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Swizzled shared-memory offset of 16-byte chunk c (0..15) of row r in a two-region K-major tile
+// whose regions hold `rows` rows of 128 bytes (the TMA / MMA 128-byte swizzle pattern).
+__device__ __forceinline__ uint32_t sw_off(int r, int c, int region_bytes) {
+  return (uint32_t)((c >> 3) * region_bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerArgs a, int* status) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int seq = blockIdx.y;
+  const int64_t t = (int64_t)__ldg(a.qr.ctx_lens + seq) - 1;
+  const int64_t nvis = (t + 1) / a.m;
+  const int64_t e_begin = (int64_t)blockIdx.x * kChunkBlocks * kBE;
+  if (t < 0 || e_begin >= nvis) return;
+  const int64_t e_end = nvis < e_begin + kChunkBlocks * kBE ? nvis : e_begin + kChunkBlocks * kBE;
+  const int nkb = (int)((e_end - e_begin + kBE - 1) / kBE);
+
+  // The 128-byte swizzle needs 1024-byte aligned tiles; the dynamic window starts aligned.
+  if ((tc::smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0 && status) atomicExch(status, tc::kStatusMisaligned);
+    return;
+  }
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const __nv_bfloat16* pool = reinterpret_cast<const __nv_bfloat16*>(a.kpool.base);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&bar[kFull0 + i], kGatherThreads);
+      tc::mbar_init(&bar[kEmpty0 + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bar[kAccFull0 + i], 1);
+      tc::mbar_init(&bar[kAccEmpty0 + i], 128);
+    }
+    tc::fence_barrier_init();
+  }
+  if (warp == 8) tc::tmem_alloc(tmem_ptr, 128);
+  // head weights: plain loads before the start barrier (the drain reads them from shared memory)
+  if (threadIdx.x >= 128 && threadIdx.x < 128 + kNI)
+    reinterpret_cast<float*>(smem + kOffW)[threadIdx.x - 128] =
+        __ldg(a.w_idx + (int64_t)seq * kNI + (threadIdx.x - 128));
+
+  // Gather thread g copies 16-byte chunk (g & 15) of rows (g >> 4) + 8j; its rows share r & 7, so
+  // the swizzle term is fixed per thread. Lane l of gather warp w resolves the address of row
+  // (2w + (l & 1)) + 8 (l >> 1), and the copies take it by shuffle.
+  const int g = threadIdx.x;
+  const int gc = g & 15, gr = g >> 4;
+  auto row_ptr = [&](int64_t e) -> const __nv_bfloat16* {
+    if (e >= e_end) return nullptr;
+    const int64_t page = __ldg(a.kpool.block_table + (int64_t)seq * a.kpool.max_pages +
+                               e / a.kpool.page_size);
+    if (page < 0) return nullptr;
+    return pool + (page * a.kpool.page_size + e % a.kpool.page_size) * kCI;
+  };
+  auto issue_block = [&](int kb, const __nv_bfloat16* my_row) {
+    uint8_t* dst = smem + kOffKv + (kb % kStages) * kBlockBytes;
+    const int src_base = gr & 1;  // lane parity of the resolving lanes of my rows
+#pragma unroll
+    for (int j = 0; j < kBE / 8; ++j) {
+      const __nv_bfloat16* rp = reinterpret_cast<const __nv_bfloat16*>(
+          __shfl_sync(~0u, reinterpret_cast<uintptr_t>(my_row), src_base + 2 * j));
+      const int r = gr + 8 * j;
+      uint8_t* d = dst + sw_off(r, gc, kRegion);
+      if (rp != nullptr) {
+        tc::cp_async16(d, rp + gc * 8);
+      } else if (kb * kBE + r < e_end - e_begin) {
+        *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);  // unallocated page: empty key
+      }
+    }
+    cp_async_commit();
+  };
+
+  if (warp < 4) {
+    // q_idx [64 heads x 128] of this sequence, then the first blocks, before the start barrier
+    const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q_idx) + (int64_t)seq * kNI * kCI;
+#pragma unroll
+    for (int j = 0; j < kNI / 8; ++j) {
+      const int r = gr + 8 * j;
+      tc::cp_async16(smem + kOffQ + sw_off(r, gc, kQRegion), q + r * kCI + gc * 8);
+    }
+    const int res_row = 2 * warp + (lane & 1) + 8 * (lane >> 1);
+    for (int kb = 0; kb < kStages && kb < nkb; ++kb)
+      issue_block(kb, row_ptr(e_begin + (int64_t)kb * kBE + res_row));
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------------ gather
+    const int res_row = 2 * warp + (lane & 1) + 8 * (lane >> 1);
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      // block kb was issued kStages-1 groups ago at most: wait until it has landed
+      const int ahead = (nkb - 1 - kb) < (kStages - 1) ? (nkb - 1 - kb) : (kStages - 1);
+      if (ahead >= 2) cp_async_wait_group<2>();
+      else if (ahead == 1) cp_async_wait_group<1>();
+      else cp_async_wait_group<0>();
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[kFull0 + kb % kStages]);
+      const int nb = kb + kStages;
+      if (nb < nkb) {
+        const __nv_bfloat16* rp = row_ptr(e_begin + (int64_t)nb * kBE + res_row);
+        // stage nb % kStages was last used by block nb - kStages
+        ok = __all_sync(~0u, tc::mbar_wait(&bar[kEmpty0 + nb % kStages],
+                                           ((nb - kStages) / kStages) & 1, status));
+        if (!ok) break;
+        issue_block(nb, rp);
+      }
+    }
+    tc::cp_async_wait_all();
+  } else if (warp == 8) {
+    if (lane == 0) {
+      // ------------------------------------------------------------------ MMA issuer
+      const uint32_t q_base = tc::smem_u32(smem + kOffQ);
+      bool ok = true;
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int s = kb % kStages, acc = kb & 1;
+        ok = tc::mbar_wait(&bar[kFull0 + s], (kb / kStages) & 1, status);
+        if (ok && kb >= 2) ok = tc::mbar_wait(&bar[kAccEmpty0 + acc], ((kb - 2) >> 1) & 1, status);
+        if (!ok) break;
+        tc::tc_fence_after();
+        const uint32_t kv_base = tc::smem_u32(smem + kOffKv + s * kBlockBytes);
+#pragma unroll
+        for (int kk = 0; kk < kCI / 16; ++kk)
+          tc::mma_bf16_ss(tmem + acc * kNI,
+                          tc::desc_sw128(kv_base + (kk >> 2) * kRegion + (kk & 3) * 32, 0, 1024),
+                          tc::desc_sw128(q_base + (kk >> 2) * kQRegion + (kk & 3) * 32, 0, 1024),
+                          kIdesc, kk > 0);
+        tc::mma_commit(&bar[kEmpty0 + s]);
+        tc::mma_commit(&bar[kAccFull0 + acc]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ drain
+    const int sp = warp & 3;
+    const uint32_t t_lane = tmem + ((uint32_t)(sp * 32) << 16);
+    const float4* w4 = reinterpret_cast<const float4*>(smem + kOffW);
+    bool ok = true;
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int acc = kb & 1;
+      ok = __all_sync(~0u, tc::mbar_wait(&bar[kAccFull0 + acc], (kb >> 1) & 1, status));
+      if (!ok) break;
+      tc::tc_fence_after();
+      float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < kNI; c += 16) {
+        uint32_t v[16];
+        tc::tmem_ld16(t_lane + acc * kNI + c, v);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; u += 4) {
+          const float4 wv = w4[(c + u) / 4];
+          const float2 x0 = make_float2(fmaxf(__uint_as_float(v[u]), 0.f),
+                                        fmaxf(__uint_as_float(v[u + 1]), 0.f));
+          const float2 x1 = make_float2(fmaxf(__uint_as_float(v[u + 2]), 0.f),
+                                        fmaxf(__uint_as_float(v[u + 3]), 0.f));
+          s0 = __ffma2_rn(x0, make_float2(wv.x, wv.y), s0);
+          s1 = __ffma2_rn(x1, make_float2(wv.z, wv.w), s1);
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bar[kAccEmpty0 + acc]);
+      const int64_t e = e_begin + (int64_t)kb * kBE + sp * 32 + lane;
+      if (e < e_end) a.scores[(int64_t)seq * a.n_stride + e] = (s0.x + s0.y) + (s1.x + s1.y);
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace
+
+bool indexer_decode_tc_supported(int dtype, int nI, int cI) {
+  return dtype == 1 && nI == kNI && cI == kCI;
+}
+
+cudaError_t launch_indexer_decode_tc(const IndexerArgs& a, int max_visible, int* status,
+                                     cudaStream_t st) {
+  if (a.nrows == 0 || max_visible == 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(indexer_decode_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int chunk = kChunkBlocks * kBE;
+  dim3 grid((unsigned)((max_visible + chunk - 1) / chunk), (unsigned)a.nrows);
+  indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, status);
+  return cudaGetLastError();
+}
+
+}  // namespace sac

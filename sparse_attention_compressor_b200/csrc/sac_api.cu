@@ -476,9 +476,24 @@ size_t sac_decode_workspace_size(const sac_params* p, int kind, int nseq) {
   if (kind < SAC_KIND_SWA || kind > SAC_KIND_CSA || nseq < 1 ||
       check_params(p, kind, true) != SAC_OK)
     return 0;
-  if (kind != SAC_KIND_CSA) return 0;
+  if (kind != SAC_KIND_CSA) return kStatusBytes;
   const size_t n = (size_t)(p->S / p->m);
-  return align_up((size_t)nseq * n * 4) + align_up((size_t)nseq * p->topk * 4);
+  return kStatusBytes + align_up((size_t)nseq * n * 4) + align_up((size_t)nseq * p->topk * 4);
+}
+
+// Status word of a decode call: the first word of ws when one is given (cleared here), else none
+// (the tensor-core kernels then give up timed-out waits silently).
+static int decode_status(void* ws, size_t ws_bytes, cudaStream_t st, int** status) {
+  *status = nullptr;
+  if (ws == nullptr) return SAC_OK;
+  REQUIRE(ws_bytes >= kStatusBytes, SAC_ERR_WORKSPACE,
+          "a decode workspace holds at least the %zu-byte status word (got %zu)", kStatusBytes,
+          ws_bytes);
+  REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  *status = static_cast<int*>(ws);
+  return SAC_OK;
 }
 
 static int check_decode_common(const sac_params* p, int kind, int nseq, const void* q,
@@ -505,12 +520,14 @@ int swa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
                const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
                int page_size, const float* sinks, void* o, void* ws, size_t ws_bytes,
                void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   int rc = check_decode_common(p, SAC_KIND_SWA, nseq, q, kv_pages, kv_block_table, kv_max_pages,
                                ctx_lens, page_size, sinks, o);
   if (rc) return rc;
+  int* status = nullptr;
+  rc = decode_status(ws, ws_bytes, static_cast<cudaStream_t>(stream), &status);
+  if (rc) return rc;
   sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.status = status;
   a.qr = sac::QueryRows{0, ctx_lens, 0};
   a.nrows = nseq;
   a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
@@ -525,8 +542,6 @@ int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
                int page_size, const void* pool_pages, const int32_t* pool_block_table,
                int pool_max_pages, const float* sinks, void* o, void* ws, size_t ws_bytes,
                void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   int rc = check_decode_common(p, SAC_KIND_HCA, nseq, q, kv_pages, kv_block_table, kv_max_pages,
                                ctx_lens, page_size, sinks, o);
   if (rc) return rc;
@@ -534,7 +549,11 @@ int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   REQUIRE(pool_block_table != nullptr, SAC_ERR_ARG, "pool_block_table must not be NULL");
   REQUIRE((int64_t)pool_max_pages * page_size >= p->S / p->m, SAC_ERR_ARG,
           "pool block table too short for S/m entries");
+  int* status = nullptr;
+  rc = decode_status(ws, ws_bytes, static_cast<cudaStream_t>(stream), &status);
+  if (rc) return rc;
   sac::AttnArgs a = attn_common(p, q, o, sinks);
+  a.status = status;
   a.qr = sac::QueryRows{0, ctx_lens, 0};
   a.nrows = nseq;
   a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
@@ -563,12 +582,16 @@ int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   REQUIRE_PTR(w_idx);
   OPTIONAL_PTR(topk_out);
   const int N = p->S / p->m;
-  size_t need = align_up((size_t)nseq * N * 4) + (topk_out ? 0 : align_up((size_t)nseq * p->topk * 4));
+  size_t need = kStatusBytes + align_up((size_t)nseq * N * 4) +
+                (topk_out ? 0 : align_up((size_t)nseq * p->topk * 4));
   REQUIRE(ws != nullptr && ws_bytes >= need, SAC_ERR_WORKSPACE,
           "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
-  REQUIRE(aligned16(ws), SAC_ERR_ARG, "ws must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  rc = decode_status(ws, ws_bytes, st, &status);
+  if (rc) return rc;
   Carve cv(ws);
+  cv.take(kStatusBytes);
   float* scores = static_cast<float*>(cv.take((size_t)nseq * N * 4));
   int32_t* sel = topk_out ? topk_out : static_cast<int32_t*>(cv.take((size_t)nseq * p->topk * 4));
   sac::QueryRows qr{0, ctx_lens, 0};
@@ -583,7 +606,11 @@ int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   ia.nrows = nseq;
   ia.n_stride = N;
   ia.scores = scores;
-  cudaError_t e = sac::timed("indexer_score", st, [&] { return sac::launch_indexer(p->dtype, ia, N, st); });
+  cudaError_t e = sac::timed("indexer_score", st, [&] {
+    if (sac::indexer_decode_tc_supported(p->dtype, p->n_idx_heads, p->idx_dim))
+      return sac::launch_indexer_decode_tc(ia, N, status, st);
+    return sac::launch_indexer(p->dtype, ia, N, st);
+  });
   if (e != cudaSuccess) return cuda_fail(e, "indexer");
   e = sac::timed("topk", st, [&] { return sac::launch_topk(scores, N, qr, p->m, nseq, p->topk, sel, st); });
   if (e != cudaSuccess) return cuda_fail(e, "top-k");
@@ -594,8 +621,76 @@ int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.pool_mode = 2;
   a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
   a.sel = sel;
+  a.status = status;
   e = run_attention(p, a, 1, 1, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+int decode_append(const sac_params* p, int kind, int nseq, const int32_t* ctx_lens,
+                  const void* kv_new, const void* k_idx_new, const void* cmp_gate,
+                  const float* cmp_bias, const void* idx_gate, const float* idx_bias,
+                  void* kv_pages, const int32_t* kv_block_table, int kv_max_pages, int page_size,
+                  void* cmp_state, void* idx_state, void* pool_pages, void* idx_pool_pages,
+                  const int32_t* pool_block_table, int pool_max_pages, void* stream) {
+  REQUIRE(kind >= SAC_KIND_SWA && kind <= SAC_KIND_CSA, SAC_ERR_ARG, "unknown layer kind %d", kind);
+  int rc = check_params(p, kind, true);
+  if (rc) return rc;
+  REQUIRE(nseq >= 1, SAC_ERR_ARG, "nseq must be >= 1 (got %d)", nseq);
+  REQUIRE(page_size >= 1, SAC_ERR_ARG, "page_size must be >= 1 (got %d)", page_size);
+  REQUIRE(ctx_lens != nullptr, SAC_ERR_ARG, "ctx_lens must not be NULL");
+  REQUIRE_PTR(kv_new);
+  REQUIRE_PTR(kv_pages);
+  REQUIRE(kv_block_table != nullptr, SAC_ERR_ARG, "kv_block_table must not be NULL");
+  REQUIRE(kv_max_pages >= 1 && (int64_t)kv_max_pages * page_size >= p->S, SAC_ERR_ARG,
+          "kv block table too short for contexts up to S=%d", p->S);
+  sac::DecodeAppendArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.nseq = nseq;
+  a.ctx_lens = ctx_lens;
+  a.D = p->D;
+  a.pos0 = p->pos0;
+  a.rf = rope_freqs(p);
+  a.kv_new = kv_new;
+  a.kv_pages = kv_pages;
+  a.kv_block_table = kv_block_table;
+  a.kv_max_pages = kv_max_pages;
+  a.page_size = page_size;
+  if (kind != SAC_KIND_SWA) {
+    REQUIRE_PTR(cmp_state);
+    REQUIRE_PTR(cmp_gate);
+    REQUIRE(cmp_bias != nullptr, SAC_ERR_ARG, "cmp_bias must not be NULL");
+    REQUIRE_PTR(pool_pages);
+    REQUIRE(pool_block_table != nullptr, SAC_ERR_ARG, "pool_block_table must not be NULL");
+    REQUIRE((int64_t)pool_max_pages * page_size >= p->S / p->m, SAC_ERR_ARG,
+            "pool block table too short for S/m entries");
+    a.m = p->m;
+    a.L = p->win_len;
+    a.cmp_gate = cmp_gate;
+    a.cmp_bias = cmp_bias;
+    a.cmp_state = cmp_state;
+    a.pool_pages = pool_pages;
+    a.pool_block_table = pool_block_table;
+    a.pool_max_pages = pool_max_pages;
+  }
+  if (kind == SAC_KIND_CSA) {
+    REQUIRE_PTR(k_idx_new);
+    REQUIRE_PTR(idx_state);
+    REQUIRE_PTR(idx_gate);
+    REQUIRE(idx_bias != nullptr, SAC_ERR_ARG, "idx_bias must not be NULL");
+    REQUIRE_PTR(idx_pool_pages);
+    a.cI = p->idx_dim;
+    a.k_idx_new = k_idx_new;
+    a.idx_gate = idx_gate;
+    a.idx_bias = idx_bias;
+    a.idx_state = idx_state;
+    a.idx_pool_pages = idx_pool_pages;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = sac::timed("decode_append", st, [&] {
+    return sac::launch_decode_append(p->dtype, a, st);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "decode append");
   return SAC_OK;
 }
 

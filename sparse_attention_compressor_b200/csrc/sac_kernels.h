@@ -20,6 +20,35 @@ cudaError_t launch_rotate_rows(int dtype, const void* x, int64_t rows, int S, in
                                const RopeFreqs& rf, int64_t pos0, void* out, cudaStream_t st,
                                int rows_per_pos = 1);
 
+// ---- decode cache append (decode_append.cu) -------------------------------------------------
+// One new token per sequence at t = ctx_lens[seq] - 1: kv_new rotated into the window pages; for
+// m > 0 the un-rotated row into the ring cmp_state [nseq, L, D] (slot t % L) and, when t + 1 is a
+// multiple of m, entry (t+1)/m - 1 pooled from the ring into the pool pages (rotated). With
+// idx_state set (CSA) the indexer key row follows the same path at width cI (no rotation).
+struct DecodeAppendArgs {
+  int nseq;
+  const int32_t* ctx_lens;
+  int D, cI, m, L;
+  int64_t pos0;
+  RopeFreqs rf;
+  const void* kv_new;         // [nseq, D] un-rotated
+  const void* k_idx_new;      // [nseq, cI] (CSA)
+  const void* cmp_gate;       // [D]
+  const float* cmp_bias;      // [L]
+  const void* idx_gate;       // [cI] (CSA)
+  const float* idx_bias;      // [L] (CSA)
+  void* kv_pages;
+  const int32_t* kv_block_table;
+  int kv_max_pages, page_size;
+  void* cmp_state;            // [nseq, L, D] (m > 0)
+  void* idx_state;            // [nseq, L, cI] (CSA) or nullptr
+  void* pool_pages;
+  void* idx_pool_pages;
+  const int32_t* pool_block_table;
+  int pool_max_pages;
+};
+cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, cudaStream_t st);
+
 // ---- indexer (indexer.cu) -----------------------------------------------------------------
 struct IndexerArgs {
   const void* q_idx;     // [rows, nI, cI] (flat query rows starting at qr.row0)
@@ -45,6 +74,13 @@ bool indexer_tc_supported(int dtype, int nI, int cI);
 // q_idx: [q_rows_total, 64, 128] (all query rows); kpool: [kpool_rows, 128] (all sequences).
 cudaError_t launch_indexer_tc(const IndexerTcArgs& a, const void* q_idx, int64_t q_rows_total,
                               const void* kpool, int64_t kpool_rows, cudaStream_t st);
+
+// ---- decode indexer on tcgen05 (indexer_decode_tc.cu): bf16, 64 heads x 128 -------------
+// One query per sequence (a.qr.ctx_lens set, a.nrows sequences), paged or contiguous pool rows of
+// width 128; scores [nrows, n_stride]; entries w < ctx // m written. status: nullable.
+bool indexer_decode_tc_supported(int dtype, int nI, int cI);
+cudaError_t launch_indexer_decode_tc(const IndexerArgs& a, int max_visible, int* status,
+                                     cudaStream_t st);
 
 // ---- top-k (topk.cu) ----------------------------------------------------------------------
 // Per row: the k largest of the first (t+1)//m scores, ties to the lower index, written in

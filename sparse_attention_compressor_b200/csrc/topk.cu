@@ -2,33 +2,102 @@
 // paragraph): per query row, the k largest of the (t+1)//m visible scores, ties going to the
 // lower entry index; empty slots (fewer than k visible) hold -1.
 //
-// One block per row. Scores become order-preserving uint32 keys in shared memory; a 4-pass 8-bit
-// radix select finds the exact k-th key T; then a block scan keeps every key > T plus the first
-// (k - #{key > T}) keys == T in index order, and writes the chosen entries in ascending order.
-#include <cub/block/block_scan.cuh>
-
+// One block of 512 threads per row; scores become order-preserving uint32 keys in shared memory.
+// The exact k-th largest key T is found by a radix select on digits of 12, 12 and 8 bits. The
+// first digit (sign, exponent and 3 mantissa bits) spreads real score distributions over many
+// bins, so the histogram atomics rarely collide; the keys in the bin that holds T (usually a few
+// hundred) are compacted and the two finer digits only visit them. Every digit is located with a
+// block-wide scan of the histogram rather than a serial walk. The final pass gives each warp a
+// contiguous segment of the row and keeps every key > T plus the first (k - #{key > T}) keys == T in
+// index order, using ballots for the in-warp order and per-warp counts for the rest, so the chosen
+// entries come out in ascending order with conflict-free shared-memory reads.
 #include "sac_kernels.h"
 
 namespace sac {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kMaxEntries = 49152;  // 192 KB of keys in shared memory
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxEntries = 49152;   // keys in shared memory: 192 KB
+constexpr int kBins = 4096;          // 12-bit digits
+constexpr int kCandCap = 2048;       // compacted keys of the threshold bin
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t u = __float_as_uint(s + 0.0f);  // -0 and +0 compare equal
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+struct Shared {
+  int hist[kBins];
+  uint32_t cand[kCandCap];
+  int warp_tot[kWarps];
+  int warp_gt[kWarps], warp_eq[kWarps];
+  int n_cand;
+  int digit, rem;
+};
+
+// Exclusive prefix sum over the block (thread order); also returns the block total.
+__device__ __forceinline__ int block_exclusive_sum(int v, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(~0u, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  int before = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const int t = warp_tot[w];
+    before += w < warp ? t : 0;
+    total += t;
+  }
+  __syncthreads();  // warp_tot may be reused right after
+  return before + x - v;
+}
+
+// Given hist[0..nbins) (nbins = 8 * kThreads or fewer), find the digit d holding the rem-th
+// largest counted key: sum(hist[d+1..]) < rem <= sum(hist[d..]). Writes sh.digit and sh.rem (the
+// rank of T among the keys of digit d).
+__device__ __forceinline__ void find_digit(Shared& sh, int nbins, int rem) {
+  const int per = nbins / kThreads;  // 8 for 12-bit digits; 0 for 8-bit (threads < 256 own one)
+  const int rt = kThreads - 1 - threadIdx.x;  // thread blocks of bins counted from the top
+  int lo, cnt;
+  if (per > 0) {
+    lo = rt * per;
+    cnt = per;
+  } else {
+    lo = rt - (kThreads - nbins);
+    cnt = lo >= 0 ? 1 : 0;
+  }
+  int s = 0;
+  for (int i = 0; i < cnt; ++i) s += sh.hist[lo + i];
+  int total;
+  const int above = block_exclusive_sum(s, sh.warp_tot, total);
+  if (cnt > 0 && above < rem && rem <= above + s) {
+    int acc = above;
+    for (int d = lo + cnt - 1; d >= lo; --d) {
+      const int h = sh.hist[d];
+      if (acc + h >= rem) {
+        sh.digit = d;
+        sh.rem = rem - acc;
+        break;
+      }
+      acc += h;
+    }
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict__ scores,
                                                         int n_stride, QueryRows qr, int m, int k,
                                                         int32_t* __restrict__ out) {
-  extern __shared__ uint32_t keys[];
-  __shared__ int hist[256];
-  __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_remaining;
-  using Scan = cub::BlockScan<int, kThreads>;
-  __shared__ typename Scan::TempStorage scan_tmp;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Shared& sh = *reinterpret_cast<Shared*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(Shared));
 
   const int64_t r = blockIdx.x;
   int seq;
@@ -36,68 +105,108 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
   qr.locate(qr.row0 + r, seq, t);
   const int n = (int)((t + 1) / m);
   int32_t* orow = out + r * k;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (n <= k) {
     for (int i = tid; i < k; i += kThreads) orow[i] = i < n ? i : -1;
     return;
   }
   const float* srow = scores + r * n_stride;
-  for (int i = tid; i < n; i += kThreads) keys[i] = order_key(__ldg(srow + i));
-  if (tid == 0) { s_prefix = 0; s_mask = 0; s_remaining = k; }
-  __syncthreads();
 
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
-    __syncthreads();
-    const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int i = tid; i < n; i += kThreads) {
-      uint32_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      int rem = s_remaining, d = 255;
-      for (; d > 0; --d) {
-        if (hist[d] >= rem) break;
-        rem -= hist[d];
+  // ---- digit 1: bits 31..20
+  for (int i = tid; i < kBins; i += kThreads) sh.hist[i] = 0;
+  if (tid == 0) sh.n_cand = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += kThreads) {
+    const uint32_t key = order_key(__ldg(srow + i));
+    keys[i] = key;
+    atomicAdd(&sh.hist[key >> 20], 1);
+  }
+  __syncthreads();
+  find_digit(sh, kBins, k);
+  const uint32_t d1 = (uint32_t)sh.digit;
+  int rem = sh.rem;
+  const int c1 = sh.hist[d1];
+  __syncthreads();  // everyone has read hist before it is cleared
+
+  // ---- compact the keys of digit d1 when they fit; otherwise scan the whole row with a mask
+  const bool compact = c1 <= kCandCap;
+  if (compact) {
+    for (int i0 = warp * 32; i0 < n; i0 += kThreads) {
+      const int i = i0 + lane;
+      const uint32_t key = i < n ? keys[i] : 0u;
+      const bool hit = i < n && (key >> 20) == d1;
+      const uint32_t mask = __ballot_sync(~0u, hit);
+      if (mask) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&sh.n_cand, __popc(mask));
+        base = __shfl_sync(~0u, base, 0);
+        if (hit) sh.cand[base + __popc(mask & ((1u << lane) - 1u))] = key;
       }
-      s_prefix = prefix | ((uint32_t)d << shift);
-      s_mask = mask | (255u << shift);
-      s_remaining = rem;
     }
-    __syncthreads();
   }
-  const uint32_t T = s_prefix;
-  const int take_eq = s_remaining;  // keys equal to T to keep, lowest indices first
+  const uint32_t* ck = compact ? sh.cand : keys;
+  const int nc = compact ? c1 : n;
 
-  const int seg = (n + kThreads - 1) / kThreads;
-  const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
-  int eq = 0;
-  for (int i = i0; i < i1; ++i) eq += keys[i] == T;
-  int eq_before;
-  Scan(scan_tmp).ExclusiveSum(eq, eq_before);
+  // ---- digit 2: bits 19..8 among keys with digit 1 == d1
+  for (int i = tid; i < kBins; i += kThreads) sh.hist[i] = 0;
   __syncthreads();
-  int nsel = 0, e = eq_before;
-  for (int i = i0; i < i1; ++i) {
-    uint32_t key = keys[i];
-    if (key > T) {
-      ++nsel;
-    } else if (key == T) {
-      nsel += e < take_eq;
-      ++e;
-    }
+  for (int i = tid; i < nc; i += kThreads) {
+    const uint32_t key = ck[i];
+    if ((key >> 20) == d1) atomicAdd(&sh.hist[(key >> 8) & 0xFFFu], 1);
   }
-  int pos;
-  Scan(scan_tmp).ExclusiveSum(nsel, pos);
-  e = eq_before;
-  for (int i = i0; i < i1; ++i) {
-    uint32_t key = keys[i];
-    bool sel = key > T;
-    if (key == T) {
-      sel = e < take_eq;
-      ++e;
-    }
-    if (sel) orow[pos++] = i;
+  __syncthreads();
+  find_digit(sh, kBins, rem);
+  const uint32_t d2 = (uint32_t)sh.digit;
+  rem = sh.rem;
+  __syncthreads();
+
+  // ---- digit 3: bits 7..0 among keys with bits 31..8 == (d1, d2)
+  const uint32_t hi24 = (d1 << 12) | d2;
+  for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < nc; i += kThreads) {
+    const uint32_t key = ck[i];
+    if ((key >> 8) == hi24) atomicAdd(&sh.hist[key & 0xFFu], 1);
+  }
+  __syncthreads();
+  find_digit(sh, 256, rem);
+  const uint32_t T = (hi24 << 8) | (uint32_t)sh.digit;
+  const int take_eq = sh.rem;  // keys equal to T to keep, lowest indices first
+
+  // ---- selection: warp w owns the contiguous segment [w*seg, (w+1)*seg)
+  const int seg = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int s0 = warp * seg, s1 = min(n, s0 + seg);
+  int gt = 0, eq = 0;
+  for (int i0 = s0; i0 < s1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < s1 ? keys[i] : 0u;
+    gt += __popc(__ballot_sync(~0u, i < s1 && key > T));
+    eq += __popc(__ballot_sync(~0u, i < s1 && key == T));
+  }
+  if (lane == 0) {
+    sh.warp_gt[warp] = gt;
+    sh.warp_eq[warp] = eq;
+  }
+  __syncthreads();
+  int eq_before = 0, sel_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    const int e = sh.warp_eq[w];
+    const int take = min(max(take_eq - eq_before, 0), e);
+    sel_before += sh.warp_gt[w] + take;
+    eq_before += e;
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int i0 = s0; i0 < s1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < s1 ? keys[i] : 0u;
+    const bool is_gt = i < s1 && key > T;
+    const bool is_eq = i < s1 && key == T;
+    const uint32_t eq_mask = __ballot_sync(~0u, is_eq);
+    const bool sel = is_gt || (is_eq && eq_before + __popc(eq_mask & lt) < take_eq);
+    const uint32_t sel_mask = __ballot_sync(~0u, sel);
+    if (sel) orow[sel_before + __popc(sel_mask & lt)] = i;
+    eq_before += __popc(eq_mask);
+    sel_before += __popc(sel_mask);
   }
 }
 
@@ -108,7 +217,8 @@ int topk_max_entries() { return kMaxEntries; }
 cudaError_t launch_topk(const float* scores, int n_stride, QueryRows qr, int m, int64_t nrows,
                         int k, int32_t* out, cudaStream_t st) {
   if (nrows == 0) return cudaSuccess;
-  size_t smem = sizeof(uint32_t) * (size_t)(n_stride > 0 ? n_stride : 1);
+  if (n_stride > kMaxEntries) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Shared) + sizeof(uint32_t) * (size_t)(n_stride > 0 ? n_stride : 1);
   cudaError_t err = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;

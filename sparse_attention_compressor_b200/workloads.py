@@ -23,7 +23,9 @@ import torch
 _TENSOR_IDS = {"q": 1, "kv": 2, "cmp_gate": 3, "cmp_bias": 4, "q_idx": 5, "w_idx": 6,
                "k_idx": 7, "idx_gate": 8, "idx_bias": 9, "sinks": 10, "spike": 11,
                "ctx": 12, "pages": 13, "kv_pages": 14, "pool_pages": 15, "idx_pool_pages": 16,
-               "hca_kv_pages": 17, "hca_pool_pages": 18, "hca_page_perm": 19, "hca_sinks": 20}
+               "hca_kv_pages": 17, "hca_pool_pages": 18, "hca_page_perm": 19, "hca_sinks": 20,
+               "kv_new": 21, "k_idx_new": 22, "cmp_state": 23, "idx_state": 24,
+               "hca_cmp_gate": 25, "hca_cmp_bias": 26}
 
 ROW_CHUNK = 64  # rows per independently seeded chunk of a per-token tensor
 
@@ -253,7 +255,20 @@ def decode_inputs(wl: Workload, layer: str) -> Dict[str, object]:
            "q": _normal((wl.nseq, wl.H, wl.D), 1.0, wl.seed, "q", 10 ** 6 + (layer == "hca"))
            .to(dt),
            "sinks": _normal((wl.H,), 1.0, wl.seed, "sinks" if layer == "csa" else "hca_sinks")}
+    # the step's cache append: the new token's un-rotated kv row, the compressor gate and ring
+    L = wl.L if layer == "csa" else m
+    out["kv_new"] = _normal((wl.nseq, wl.D), 1.0, wl.seed, "kv_new", layer == "hca").to(dt)
+    out["cmp_gate"] = _normal((wl.D,), 1.0 / math.sqrt(wl.D), wl.seed,
+                              "cmp_gate" if layer == "csa" else "hca_cmp_gate").to(dt)
+    out["cmp_bias"] = _normal((L,), 1.0 / math.sqrt(L), wl.seed,
+                              "cmp_bias" if layer == "csa" else "hca_cmp_bias")
+    out["cmp_state"] = _normal((wl.nseq, L, wl.D), 1.0, wl.seed, "cmp_state",
+                               layer == "hca").to(dt)
     if layer == "csa":
+        out["k_idx_new"] = _normal((wl.nseq, wl.cI), 1.0, wl.seed, "k_idx_new").to(dt)
+        out["idx_gate"] = _normal((wl.cI,), 1.0 / math.sqrt(wl.cI), wl.seed, "idx_gate").to(dt)
+        out["idx_bias"] = _normal((L,), 1.0 / math.sqrt(L), wl.seed, "idx_bias")
+        out["idx_state"] = _normal((wl.nseq, L, wl.cI), 1.0, wl.seed, "idx_state").to(dt)
         ipool = _paged(wl, "idx_pool_pages", "pages", np.maximum(npool, 1), wl.cI, None, dt)
         assert torch.equal(ipool.block_table, pool.block_table)
         out["idx_pool_pages"] = ipool.pages

@@ -60,8 +60,9 @@ def test_workspace_sizes():
         256 + 8192 * 512 * 2 + 64 * 512 * 2
     assert sac.sac_workspace_size(p_csa(dtype="f32"), sac.SAC_KIND_SWA) == 256 + 8192 * 512 * 4
     assert sac.sac_decode_workspace_size(p_csa(S=65536), sac.SAC_KIND_CSA, 64) == \
-        64 * 16384 * 4 + 64 * 512 * 4
-    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_HCA, 64) == 0
+        256 + 64 * 16384 * 4 + 64 * 512 * 4
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_HCA, 64) == 256
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 64) == 256
 
 
 @pytest.mark.parametrize("bad,code", [
@@ -124,3 +125,34 @@ def test_decode_validation():
     rc = lib.hca_decode(ctypes.byref(p), 0, fake, fake, fake, 1024, fake, 64, fake, fake, 8, fake,
                         fake, None, 0, None)
     assert rc == -1 and "nseq" in lib.sac_last_error().decode()
+
+
+def test_decode_append_validation():
+    lib = sac.load_library()
+    fake = 1 << 20
+    p = p_csa(S=4096)
+    args = dict(kind=sac.SAC_KIND_CSA, nseq=2, ctx=fake, kv_new=fake, k_idx_new=fake,
+                cmp_gate=fake, cmp_bias=fake, idx_gate=fake, idx_bias=fake, kv_pages=fake,
+                kv_bt=fake, kv_max_pages=64, page_size=64, cmp_state=fake, idx_state=fake,
+                pool_pages=fake, idx_pool_pages=fake, pool_bt=fake, pool_max_pages=16)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.decode_append(ctypes.byref(p), a["kind"], a["nseq"], a["ctx"], a["kv_new"],
+                                 a["k_idx_new"], a["cmp_gate"], a["cmp_bias"], a["idx_gate"],
+                                 a["idx_bias"], a["kv_pages"], a["kv_bt"], a["kv_max_pages"],
+                                 a["page_size"], a["cmp_state"], a["idx_state"],
+                                 a["pool_pages"], a["idx_pool_pages"], a["pool_bt"],
+                                 a["pool_max_pages"], None)
+
+    assert call(kind=7) == -1
+    assert call(nseq=0) == -1
+    assert call(kv_max_pages=63) == -1 and "block table" in lib.sac_last_error().decode()
+    assert call(pool_max_pages=15) == -1 and "pool block table" in lib.sac_last_error().decode()
+    assert call(idx_state=None) == -1 and "idx_state" in lib.sac_last_error().decode()
+    assert call(cmp_state=fake + 8) == -1 and "aligned" in lib.sac_last_error().decode()
+    # SWA needs no compressor state
+    p_swa = sac.make_params(1, 4096, 64, 512, 64, 1e4, sliding_window=128)
+    rc = lib.decode_append(ctypes.byref(p_swa), sac.SAC_KIND_SWA, 2, fake, fake, None, None, None,
+                           None, None, fake, fake, 63, 64, None, None, None, None, None, 0, None)
+    assert rc == -1 and "block table" in lib.sac_last_error().decode()

@@ -112,6 +112,20 @@ def test_tiny_topk_matches_oracle_exactly():
         assert sorted(gs[gs >= 0].tolist()) == sorted(os_[os_ >= 0].tolist()), t
 
 
+def test_topk_all_scores_equal():
+    # With q_idx = 0 every indexer score of a row is 0: ties are decided by the entry index alone,
+    # so each row keeps its k lowest visible entries (then -1 fill).
+    wl = SMALL[2][1]  # bf16, 64 indexer heads of 128: the tensor-core indexer
+    x = W.prefill_inputs(wl)
+    x["q_idx"] = torch.zeros_like(x["q_idx"])
+    g = gpu_prefill(wl, x)
+    for t in range(wl.S):
+        nvis = (t + 1) // wl.m
+        expect = np.arange(wl.k) if nvis >= wl.k else np.concatenate(
+            [np.arange(nvis), -np.ones(wl.k - nvis, dtype=np.int64)])
+        assert np.array_equal(g["topk"][0, t].numpy(), expect), t
+
+
 def test_relative_position_invariance_on_gpu():
     wl = SMALL[1][1]
     x = W.prefill_inputs(wl)
@@ -234,18 +248,18 @@ def gpu_decode(wl, d, layer, max_ctx):
     nseq = g["q"].shape[0]
     o = torch.empty_like(g["q"])
     ps = wl.page_size
+    kind = sac.SAC_KIND_HCA if layer == "hca" else sac.SAC_KIND_CSA
+    ws = torch.empty(sac.sac_decode_workspace_size(p, kind, nseq), dtype=torch.uint8, device=dev)
     if layer == "hca":
         sac.hca_decode(p, nseq, g["q"], g["kv_pages"], g["kv_block_table"], g["ctx_lens"], ps,
-                       g["pool_pages"], g["pool_block_table"], g["sinks"], o)
-        torch.cuda.synchronize()
+                       g["pool_pages"], g["pool_block_table"], g["sinks"], o, ws)
+        assert sac.sac_device_status(ws) == 0, "a kernel reported a device-side wait timeout"
         return o.cpu(), None
-    ws = torch.empty(sac.sac_decode_workspace_size(p, sac.SAC_KIND_CSA, nseq), dtype=torch.uint8,
-                     device=dev)
     tk = torch.empty((nseq, wl.k), dtype=torch.int32, device=dev)
     sac.csa_decode(p, nseq, g["q"], g["kv_pages"], g["kv_block_table"], g["ctx_lens"], ps,
                    g["pool_pages"], g["idx_pool_pages"], g["pool_block_table"], g["q_idx"],
                    g["w_idx"], g["sinks"], o, tk, ws)
-    torch.cuda.synchronize()
+    assert sac.sac_device_status(ws) == 0, "a kernel reported a device-side wait timeout"
     return o.cpu(), tk.cpu()
 
 
