@@ -199,6 +199,15 @@ def make_step(wl, g, dev):
     return step, o
 
 
+def capture(fn):
+    """fn (which has already run eagerly) captured once into a CUDA graph; a step is then one
+    replay, so the timed region holds no host launch gaps."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        fn()
+    return g
+
+
 def timed(step, steps, dev):
     barrier(dev)
     torch.cuda.synchronize(dev)
@@ -213,15 +222,19 @@ def timed(step, steps, dev):
 
 
 def timed_flushed(step, steps, dev):
-    """Like timed(), but L2 is flushed (a write of twice its size) before every step; each step
-    is bracketed by its own events and only the steps are summed."""
+    """Like timed(), but L2 is flushed before every step: a write of twice its size, then a read
+    of another buffer of that size, so that the dirty lines of the write are evicted before the
+    step starts (their write-back would otherwise be charged to the step). Each step is bracketed
+    by its own events and only the steps are summed."""
     junk = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    junk_r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
     barrier(dev)
     torch.cuda.synchronize(dev)
     for a, b in evs:
         junk.fill_(0)
+        junk_r.sum()
         a.record()
         step()
         b.record()
@@ -239,6 +252,16 @@ def tensor_kernels(wl) -> set:
     if wl.kind == "csa" and wl.dtype == "bf16" and wl.nI == 64 and wl.cI == 128:
         out.add("indexer_score")
     return out
+
+
+# DRAM bytes (read + write) per launch from one ncu capture of the kernel as it stands, keyed by
+# (workload, kernel); the summary with its command is the named file under profiles/. An entry is
+# removed whenever its kernel changes, and the roofline then reports traffic null.
+NCU_TRAFFIC = {
+    ("csa_8k_bf16", "attention"): (563.197696e6 + 491.843584e6, "attention_tc_csa_8k_bf16.md"),
+    ("csa_8k_bf16", "indexer_score"): (136.957696e6 + 25.005312e6, "indexer_tc_csa_8k_bf16.md"),
+    ("csa_8k_bf16", "topk"): (31.865088e6 + 7.68e3, "topk_csa_8k_bf16.md"),
+}
 
 
 def roofline(wl, ktimes: dict, peaks: dict, steps: int, tensor_kernels: set) -> tuple:
@@ -268,9 +291,12 @@ def roofline(wl, ktimes: dict, peaks: dict, steps: int, tensor_kernels: set) -> 
         rows[name] = entry
     dom = max(ktimes, key=lambda k: ktimes[k][1])
     d = rows[dom]
+    tr = NCU_TRAFFIC.get((wl.name, dom))
     roof = {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
             "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),
-            "traffic": None, "peak_source": peaks["source"]}
+            "traffic": tr[0] if tr else None, "peak_source": peaks["source"]}
+    if tr:
+        roof["traffic_source"] = "profiles/" + tr[1]
     return roof, rows
 
 
@@ -319,7 +345,8 @@ def config_of(wl, world):
            "rope_dim": wl.R, "rope_theta": wl.theta, "sliding_window": wl.W,
            "parallelism": f"dp{world}",
            "l2": "inputs larger than L2 (q alone %d MiB > 126 MiB), no flush" %
-                 (wl.B * wl.S * wl.H * wl.D * (2 if wl.dtype == "bf16" else 4) // 2 ** 20)}
+                 (wl.B * wl.S * wl.H * wl.D * (2 if wl.dtype == "bf16" else 4) // 2 ** 20),
+           "launch": "one CUDA graph replay per step"}
     if wl.kind in ("csa", "hca"):
         cfg.update(m=wl.m, compressor_window=wl.L)
     if wl.kind == "csa":
@@ -343,10 +370,14 @@ def run_ours(args, wl0):
         step()
     torch.cuda.synchronize(dev)
 
+    # one step captured as a CUDA graph (with the per-kernel timing events inside it)
     sac.sac_timing_begin()
+    graph = capture(step)
+    graph.replay()
+    torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clk:
-        ms = timed(step, args.steps, dev)
-    ktimes = sac.sac_timing_end()
+        ms = timed(graph.replay, args.steps, dev)
+    ktimes = sac.sac_timing_end()  # per kernel: the last replay, i.e. one step
     ms = max_over_ranks(ms, dev)
     ms_step = ms / args.steps
     tokens = wl.B * wl.S * world
@@ -364,11 +395,12 @@ def run_ours(args, wl0):
         o_host.copy_(o, non_blocking=True)
     e2e_step()
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(timed(e2e_step, args.steps, dev), dev) / args.steps
+    e2e_graph = capture(e2e_step)
+    e2e_ms = max_over_ranks(timed(e2e_graph.replay, args.steps, dev), dev) / args.steps
 
     peaks = measured_peaks()
-    roof, krows = roofline(wl, ktimes, peaks, args.steps, tensor_kernels=tensor_kernels(wl))
-    launches = sum(v[0] for v in ktimes.values())
+    roof, krows = roofline(wl, ktimes, peaks, 1, tensor_kernels=tensor_kernels(wl))
+    launches = sum(v[0] for v in ktimes.values()) * args.steps
     line = {
         "metric": f"{wl.kind.upper()} attention fwd tokens/s (prefill)", "value": value,
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -408,11 +440,12 @@ def decode_bytes(wl, d_csa, d_hca) -> dict:
     # cache append: the new row read, written rotated to its page and un-rotated to the ring; a
     # closing window (ctx % m == 0) reads its L ring rows and writes one entry
     app = 0.0
-    for d, m, L, cI in ((d_csa, wl.m, wl.L, wl.cI), (d_hca, d_hca["m"], d_hca["m"], 0)):
-        c = d["ctx_lens"].numpy().astype(np.int64)
-        closing = int((c % m == 0).sum())
-        app += wl.nseq * (3 * wl.D + 2 * cI) * esz + closing * (L + 1) * (wl.D + cI) * esz
+    for d, m, L in ((d_csa, wl.m, wl.L), (d_hca, d_hca["m"], d_hca["m"])):
+        closing = int((d["ctx_lens"].numpy() % m == 0).sum())
+        app += wl.nseq * 3 * wl.D * esz + closing * (L + 1) * wl.D * esz
     out["decode_append"] = app
+    closing = int((d_csa["ctx_lens"].numpy() % wl.m == 0).sum())
+    out["decode_append_index"] = float(wl.nseq * 2 * wl.cI * esz + closing * (wl.L + 1) * wl.cI * esz)
     return out
 
 
@@ -462,9 +495,12 @@ def run_decode(args, wl0):
         step()
     torch.cuda.synchronize(dev)
     sac.sac_timing_begin()
+    graph = capture(step)
+    graph.replay()
+    torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clk:
-        ms = timed_flushed(step, args.steps, dev)
-    ktimes = sac.sac_timing_end()
+        ms = timed_flushed(graph.replay, args.steps, dev)
+    ktimes = sac.sac_timing_end()  # per kernel: the last replay, i.e. one step
     ms = max_over_ranks(ms, dev)
     us_step = 1e3 * ms / args.steps
     # end to end: the step's new-token inputs from pinned host memory, outputs back
@@ -487,7 +523,9 @@ def run_decode(args, wl0):
         oh_h.copy_(oh, non_blocking=True)
     e2e_step()
     torch.cuda.synchronize(dev)
-    e2e_us = 1e3 * max_over_ranks(timed_flushed(e2e_step, args.steps, dev), dev) / args.steps
+    e2e_graph = capture(e2e_step)
+    e2e_us = 1e3 * max_over_ranks(timed_flushed(e2e_graph.replay, args.steps, dev),
+                                  dev) / args.steps
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
     d2h = (oc.numel() + oh.numel()) * oc.element_size()
     peaks = measured_peaks()
@@ -498,7 +536,7 @@ def run_decode(args, wl0):
         per = kms / max(launches, 1)
         row = {"launches": launches, "ms_per_launch": per, "share": kms / total}
         if name in wb:
-            per_launch_bytes = wb[name] / (launches / args.steps)
+            per_launch_bytes = wb[name] / launches
             ach = per_launch_bytes / (per * 1e-3) / 1e9
             row.update(bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
                        frac=ach / peaks["hbm_gbs"])
@@ -513,11 +551,12 @@ def run_decode(args, wl0):
         "config": {"workload": wl.name, "nseq": wl.nseq, "ctx": f"U[{wl.ctx_lo},{wl.ctx_hi}]",
                    "page_size": wl.page_size, "H": wl.H, "head_dim": wl.D, "csa_m": wl.m,
                    "hca_m": dh["m"], "index_topk": wl.k, "sliding_window": wl.W,
-                   "parallelism": f"dp{world}", "l2": "flushed before every step (write of 252 MiB)"},
+                   "parallelism": f"dp{world}", "l2": "flushed before every step (252 MiB written, then another 252 MiB read)",
+                   "launch": "one CUDA graph replay per step (cache append + both layers)"},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": sum(v[0] for v in ktimes.values()),
+        "gpu_launches": sum(v[0] for v in ktimes.values()) * args.steps,
         "roofline": {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
                      "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),
                      "traffic": None, "peak_source": peaks["source"]},

@@ -246,6 +246,12 @@ SAC_API int sac_device_status(const void* ws, int* status, void* stream);
  * pair of CUDA events recorded on the launch's own stream. sac_timing_end() waits for those
  * events, fills up to max_entries records (one per kernel name: launches and summed device time)
  * and returns the number of distinct kernels (which may exceed max_entries), or SAC_ERR_LAUNCH.
+ * Calls captured into a CUDA graph while timing is on put their event pairs into the graph; the
+ * records then hold the times of the graph's most recent replay.
+ *
+ * CUDA graphs: after one eager call with the same shapes (which performs the one-time per-device
+ * setup), every entry point except sac_device_status and swa_forward_static's first call may be
+ * captured into a CUDA graph; nothing they enqueue synchronises or allocates.
  */
 typedef struct {
   char name[32];

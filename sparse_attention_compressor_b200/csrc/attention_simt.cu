@@ -11,6 +11,7 @@
 // CUDA-core version: fp32 math for both element types. Block = one query row and HG heads (one
 // warp per head); keys stream through shared memory 32 at a time (one per lane for the logits,
 // then every lane accumulates its D/32 output channels).
+#include "launch_util.h"
 #include "sac_kernels.h"
 
 namespace sac {
@@ -143,8 +144,7 @@ cudaError_t attention_t(const AttnArgs& a, cudaStream_t st) {
   if (a.nrows == 0) return cudaSuccess;
   const int HG = a.H < 16 ? a.H : 16;
   size_t smem = sizeof(float) * ((size_t)HG * a.D + 32 * (size_t)(a.D + 1));
-  cudaError_t err = cudaFuncSetAttribute(attention_simt_kernel<T>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t err = ensure_smem_limit((const void*)attention_simt_kernel<T>, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)a.nrows, (unsigned)((a.H + HG - 1) / HG));
   attention_simt_kernel<T><<<grid, 32 * HG, smem, st>>>(a, HG);

@@ -31,6 +31,7 @@
 // when a tile's max exceeds it by more than 8.
 #include <cuda_bf16.h>
 
+#include "launch_util.h"
 #include "sac_kernels.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
@@ -64,6 +65,7 @@ constexpr int kSmemBytes = kOffTmemPtr + 16;
 constexpr uint32_t kColS = 256, kSStride = 2 * kNK;  // S buffer s at kColS + s * kSStride
 constexpr uint32_t kIdescQK = tc::idesc_bf16(64, kNK, false, false);
 constexpr uint32_t kIdescPV = tc::idesc_bf16(64, 256, false, true);
+constexpr int kRopeK2 = 14;  // K-step pairs 14,15 (K-steps 28..31) read the last region of Q
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;  // move the running max only when a tile exceeds it by 2^8
 
@@ -201,7 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qd = tc::desc_sw128(tc::smem_u32(smem + kOffQ), 0, 1024);
       for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
         const Row w = locate_row(a, r);
-        ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
+        // the query tile has landed; its rope region (the last 128-byte column, K-steps 28..31)
+        // is still being rotated, so the first QK^T waits for kQReady only before those steps
+        ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
         for (int j = 0; j <= w.tiles && ok; ++j) {
           if (j < w.tiles) {  // S(g) = Q K^T over four partial accumulators
             const uint32_t g = g0 + j, b = g % kStages, s = g & 1;
@@ -220,11 +224,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k2 = 0; k2 < kDim / 32; ++k2) {
               const int kk0 = 2 * k2 + (int)me;  // kk0 & 1 == me
+              if (k2 == kRopeK2 && j == 0) {
+                ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
+                if (!ok) break;
+                tc::tc_fence_after();
+              }
               const uint32_t qo = ((kk0 >> 2) * kQRegion + (kk0 & 3) * 32) >> 4;
               const uint32_t ko = ((kk0 >> 2) * kKRegion + (kk0 & 3) * 32) >> 4;
               tc::mma_bf16_ss(dme + ((kk0 & 2) ? (uint32_t)kNK : 0u), qd + qo, kd + ko, kIdescQK,
                               kk0 >= 4);
             }
+            if (!ok) break;
             tc::mma_commit(&bar[kSFull0 + s]);
             if (j == w.tiles - 1) tc::mma_commit(&bar[kQEmpty]);
           }
@@ -314,35 +324,71 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gt = (warp & 1) * 32 + lane;    // 0..63
     const int row0 = gt >> 3, slot = gt & 7;
     constexpr int kRowsPer = kNK / 8;         // 6
-    uint32_t g = 0;
-    bool ok = true;
-    for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x) {
-      const Row w = locate_row(a, r);
-      for (int j = 0; j < w.tiles && ok; ++j, ++g) {
-        if ((int)(g & 1) != grp) continue;
-        const uint32_t b = g % kStages;
-        if (g >= kStages)
-          ok = __all_sync(~0u, tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - kStages) / kStages) & 1,
-                                             status));
-        if (!ok) break;
-        const bool is_win = j < w.twin;
-        if (!(is_win ? win_contig : pool_contig)) {
-          uint8_t* tile = smem + kOffTile + b * kTileBytes;
-          const __nv_bfloat16* src[kRowsPer];
-#pragma unroll
-          for (int i = 0; i < kRowsPer; ++i) src[i] = key_ptr(a, w, r, j, row0 + 8 * i);
-#pragma unroll
-          for (int i = 0; i < kRowsPer; ++i) {
-            const int row = row0 + 8 * i;
-            uint8_t* d = tile + row * 128 + ((slot ^ (row & 7)) << 4);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) tc::cp_async16(d + q * kKRegion, src[i] + q * 64 + slot * 8);
-          }
-          tc::cp_async_wait_all();
-          tc::fence_proxy_async_smem();
+    // Walk this group's tiles in order across the CTA's query rows. The source rows of the next
+    // tile are resolved while the current tile's copies are in flight, so the selection-index
+    // loads do not add to each tile's latency.
+    struct Cursor {
+      int64_t r;
+      Row w;
+      int j;
+      uint32_t g;
+    };
+    auto valid = [&](const Cursor& c) { return c.r < a.nrows; };
+    auto gathered = [&](const Cursor& c) {
+      return !(c.j < c.w.twin ? win_contig : pool_contig);
+    };
+    auto advance = [&](Cursor c) {  // next tile of this group after c
+      do {
+        ++c.g;
+        if (++c.j >= c.w.tiles) {
+          c.r += gridDim.x;
+          c.j = 0;
+          if (c.r >= a.nrows) return c;
+          c.w = locate_row(a, c.r);
         }
-        tc::mbar_arrive(&bar[kKvFull0 + b]);
+      } while ((int)(c.g & 1) != grp);
+      return c;
+    };
+    auto resolve = [&](const Cursor& c, const __nv_bfloat16* (&src)[kRowsPer]) {
+#pragma unroll
+      for (int i = 0; i < kRowsPer; ++i) src[i] = key_ptr(a, c.w, c.r, c.j, row0 + 8 * i);
+    };
+    Cursor c;
+    c.r = blockIdx.x;
+    c.j = 0;
+    c.g = 0;
+    if (valid(c)) {
+      c.w = locate_row(a, c.r);
+      if (grp == 1) c = advance(c);
+    }
+    const __nv_bfloat16* src[kRowsPer];
+    if (valid(c) && gathered(c)) resolve(c, src);
+    bool ok = true;
+    while (valid(c) && ok) {
+      const uint32_t b = c.g % kStages;
+      if (c.g >= kStages)
+        ok = __all_sync(~0u, tc::mbar_wait(&bar[kKvEmpty0 + b], ((c.g - kStages) / kStages) & 1,
+                                           status));
+      if (!ok) break;
+      const bool gath = gathered(c);
+      if (gath) {
+        uint8_t* tile = smem + kOffTile + b * kTileBytes;
+#pragma unroll
+        for (int i = 0; i < kRowsPer; ++i) {
+          const int row = row0 + 8 * i;
+          uint8_t* d = tile + row * 128 + ((slot ^ (row & 7)) << 4);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) tc::cp_async16(d + q * kKRegion, src[i] + q * 64 + slot * 8);
+        }
       }
+      const Cursor n = advance(c);
+      if (valid(n) && gathered(n)) resolve(n, src);  // overlaps the copies in flight
+      if (gath) {
+        tc::cp_async_wait_all();
+        tc::fence_proxy_async_smem();
+      }
+      tc::mbar_arrive(&bar[kKvFull0 + b]);
+      c = n;
     }
   } else {
     // ------------------------------------------------------------------ softmax + output
@@ -519,8 +565,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
   e = make_tmap_bf16_2d(&tpb, has_pool ? a.pool.base : a.win.base,
                         (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmemBytes);
+  e = ensure_smem_limit((const void*)attention_tc_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);

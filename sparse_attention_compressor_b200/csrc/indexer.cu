@@ -2,6 +2,7 @@
 // index_n_heads, index_head_dim): I[t,w] = sum_h w_idx[t,h] * max(0, <q_idx[t,h], KI_w>) for the
 // visible entries w < (t+1)//m. CUDA-core version (fp32 math): one block per (query row, 64
 // entries); warps split the heads, lanes the entries, and a shared-memory reduction sums heads.
+#include "launch_util.h"
 #include "sac_kernels.h"
 
 namespace sac {
@@ -65,8 +66,7 @@ cudaError_t indexer_t(const IndexerArgs& a, int max_visible, cudaStream_t st) {
   if (a.nrows == 0 || max_visible == 0) return cudaSuccess;
   size_t smem = sizeof(float) * ((size_t)a.nI * a.cI + a.nI +
                                  (size_t)kEntriesPerBlock * (a.cI + 1) + 8 * 64);
-  cudaError_t err = cudaFuncSetAttribute(indexer_simt_kernel<T>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t err = ensure_smem_limit((const void*)indexer_simt_kernel<T>, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)a.nrows, (unsigned)((max_visible + kEntriesPerBlock - 1) / kEntriesPerBlock));
   indexer_simt_kernel<T><<<grid, 256, smem, st>>>(a);

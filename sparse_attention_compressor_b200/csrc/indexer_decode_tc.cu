@@ -17,6 +17,7 @@
 // Warps: 0..3 gather (q_idx once, then entry blocks), 4..7 drain, 8 issues the MMAs and owns TMEM.
 #include <cuda_bf16.h>
 
+#include "launch_util.h"
 #include "sac_kernels.h"
 #include "tc_ptx.cuh"
 
@@ -241,8 +242,7 @@ bool indexer_decode_tc_supported(int dtype, int nI, int cI) {
 cudaError_t launch_indexer_decode_tc(const IndexerArgs& a, int max_visible, int* status,
                                      cudaStream_t st) {
   if (a.nrows == 0 || max_visible == 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(indexer_decode_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = ensure_smem_limit((const void*)indexer_decode_tc_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int chunk = kChunkBlocks * kBE;
   dim3 grid((unsigned)((max_visible + chunk - 1) / chunk), (unsigned)a.nrows);

@@ -14,6 +14,7 @@
 // persistent CTAs; only the causal part (entries < (t_last+1)//m) is streamed.
 #include <cuda_bf16.h>
 
+#include "launch_util.h"
 #include "sac_kernels.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
@@ -250,8 +251,7 @@ cudaError_t launch_indexer_tc(const IndexerTcArgs& a, const void* q_idx_seq_base
   e = make_tmap_bf16_2d(&tk, kpool, (uint64_t)(kpool_rows > 0 ? kpool_rows : 1), kCI, kCI * 2,
                         kBE, 64);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmemBytes);
+  e = ensure_smem_limit((const void*)indexer_tc_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);

@@ -1,0 +1,157 @@
+// The compressor's pooling of one window ("Hybrid attention": CSA / HCA compressors; "Cache
+// layers": compressor buffer), shared by the prefill compressor (compress.cu) and the decode cache
+// append (decode_append.cu): entry w pools rows j in [lo, hi) = [(w+1)m - L, (w+1)m) clipped at 0
+// with softmax weights over g_j = <x_j, u> + bias[j - hi + L], in one streaming pass with an
+// online softmax. Lane l of a warp owns channels [l*V, l*V + V) of a C = 32*V row; WPE warps
+// split the rows of one entry and merge their partial (max, sum, accumulator) in shared memory.
+#pragma once
+
+#include "sac_common.cuh"
+
+namespace sac {
+
+// kCoherent: read through L2 (rows written earlier by the same kernel), else the read-only path.
+template <typename T, int V, bool kCoherent = false>
+__device__ __forceinline__ void load_lane(const T* row, int lane, float (&v)[V]) {
+  const T* p = row + lane * V;
+  if constexpr (V * sizeof(T) % 16 == 0) {
+#pragma unroll
+    for (int i = 0; i < V * (int)sizeof(T) / 16; ++i) {
+      uint4 u = kCoherent ? __ldcg(reinterpret_cast<const uint4*>(p) + i)
+                          : __ldg(reinterpret_cast<const uint4*>(p) + i);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int k = 0; k < 16 / (int)sizeof(T); ++k) v[i * (16 / sizeof(T)) + k] = to_f<T>(e[k]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i) v[i] = to_f<T>(kCoherent ? __ldcg(p + i) : p[i]);
+  }
+}
+
+template <typename T, int V>
+__device__ __forceinline__ void store_lane(T* row, int lane, const float (&v)[V]) {
+  T* p = row + lane * V;
+  if constexpr (V * sizeof(T) % 16 == 0) {
+#pragma unroll
+    for (int i = 0; i < V * (int)sizeof(T) / 16; ++i) {
+      uint4 u;
+      T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+      for (int k = 0; k < 16 / (int)sizeof(T); ++k) e[k] = from_f<T>(v[i * (16 / sizeof(T)) + k]);
+      reinterpret_cast<uint4*>(p)[i] = u;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i) p[i] = from_f<T>(v[i]);
+  }
+}
+
+// Rotate the lane's channels that fall in the trailing R (pairs never straddle lanes: V even).
+template <int V>
+__device__ __forceinline__ void rotate_lane(float (&v)[V], int lane, int C, const RopeFreqs& rf,
+                                            int64_t pos) {
+  const int R = rf.R;
+#pragma unroll
+  for (int i = 0; i + 1 < V; i += 2) {
+    int c = lane * V + i;
+    if (c >= C - R) {
+      float cs, sn;
+      rope_cos_sin(rf, (c - (C - R)) >> 1, pos, cs, sn);
+      float a = v[i], b = v[i + 1];
+      v[i] = a * cs - b * sn;
+      v[i + 1] = a * sn + b * cs;
+    }
+  }
+}
+
+// Shared memory of pool_window for a block of 8 warps.
+template <int V, int WPE>
+struct PoolShared {
+  float acc[WPE > 1 ? 8 : 1][WPE > 1 ? 32 * V : 1];
+  float mz[8][2];
+};
+
+// One entry per group of WPE warps (warp = the calling warp's index in the 8-warp block, sub =
+// warp % WPE). row(j) gives row j's pointer. On return the group's first warp (sub == 0) holds
+// the normalised pooled row in acc; with WPE > 1 every warp of the block must call (it contains
+// __syncthreads). Rows whose gate logit is -inf get weight 0.
+template <typename T, int V, int WPE, bool kCoherent = false, typename RowFn>
+__device__ __forceinline__ void pool_window(RowFn row, const float (&u)[V], const float* bias,
+                                            int64_t lo, int64_t hi, int L, bool active, int warp,
+                                            int lane, PoolShared<V, WPE>& sh, float (&acc)[V]) {
+  const int sub = warp % WPE;
+#pragma unroll
+  for (int i = 0; i < V; ++i) acc[i] = 0.f;
+  float M = -INFINITY, Z = 0.f;
+  if (active) {
+    // rows in batches of kBatch: all loads of a batch are issued before any is used, so a
+    // window costs ceil(rows / kBatch) memory latencies instead of one per row
+    constexpr int kBatch = 4;
+    for (int64_t j0 = lo + sub; j0 < hi; j0 += kBatch * WPE) {
+      float xv[kBatch][V];
+      float bb[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int64_t j = j0 + (int64_t)k * WPE;
+        if (j < hi) {
+          load_lane<T, V, kCoherent>(row(j), lane, xv[k]);
+          bb[k] = __ldg(bias + (j - hi + L));
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        if (j0 + (int64_t)k * WPE >= hi) break;
+        float d = 0.f;
+#pragma unroll
+        for (int i = 0; i < V; ++i) d = fmaf(xv[k][i], u[i], d);
+        const float g = warp_sum(d) + bb[k];
+        if (g == -INFINITY) continue;
+        if (g > M) {
+          const float sc = __expf(M - g);  // 0 when M = -inf
+          Z *= sc;
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[i] *= sc;
+          M = g;
+        }
+        const float p = __expf(g - M);
+        Z += p;
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(p, xv[k][i], acc[i]);
+      }
+    }
+  }
+  if constexpr (WPE > 1) {
+#pragma unroll
+    for (int i = 0; i < V; ++i) sh.acc[warp][lane * V + i] = acc[i];
+    if (lane == 0) {
+      sh.mz[warp][0] = M;
+      sh.mz[warp][1] = Z;
+    }
+    __syncthreads();
+    if (sub == 0) {
+      float Mt = -INFINITY;
+      for (int s = 0; s < WPE; ++s) Mt = fmaxf(Mt, sh.mz[warp + s][0]);
+      float Zt = 0.f;
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] = 0.f;
+      for (int s = 0; s < WPE; ++s) {
+        float Ms = sh.mz[warp + s][0];
+        if (Ms == -INFINITY) continue;
+        float sc = __expf(Ms - Mt);
+        Zt = fmaf(sh.mz[warp + s][1], sc, Zt);
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(sh.acc[warp + s][lane * V + i], sc, acc[i]);
+      }
+      Z = Zt;
+    }
+    __syncthreads();  // sh is reused by a following call
+  }
+  if (sub == 0 && active) {
+    const float inv = 1.f / Z;
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] *= inv;
+  }
+}
+
+}  // namespace sac

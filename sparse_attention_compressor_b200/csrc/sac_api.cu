@@ -688,8 +688,12 @@ int decode_append(const sac_params* p, int kind, int nseq, const int32_t* ctx_le
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = sac::timed("decode_append", st, [&] {
-    return sac::launch_decode_append(p->dtype, a, st);
+    return sac::launch_decode_append(p->dtype, a, false, st);
   });
+  if (e == cudaSuccess && kind == SAC_KIND_CSA)
+    e = sac::timed("decode_append_index", st, [&] {
+      return sac::launch_decode_append(p->dtype, a, true, st);
+    });
   if (e != cudaSuccess) return cuda_fail(e, "decode append");
   return SAC_OK;
 }

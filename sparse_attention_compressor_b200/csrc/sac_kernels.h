@@ -23,8 +23,8 @@ cudaError_t launch_rotate_rows(int dtype, const void* x, int64_t rows, int S, in
 // ---- decode cache append (decode_append.cu) -------------------------------------------------
 // One new token per sequence at t = ctx_lens[seq] - 1: kv_new rotated into the window pages; for
 // m > 0 the un-rotated row into the ring cmp_state [nseq, L, D] (slot t % L) and, when t + 1 is a
-// multiple of m, entry (t+1)/m - 1 pooled from the ring into the pool pages (rotated). With
-// idx_state set (CSA) the indexer key row follows the same path at width cI (no rotation).
+// multiple of m, entry (t+1)/m - 1 pooled from the ring into the pool pages (rotated). The
+// indexer part (CSA) takes the indexer key row through the same path at width cI (no rotation).
 struct DecodeAppendArgs {
   int nseq;
   const int32_t* ctx_lens;
@@ -47,7 +47,9 @@ struct DecodeAppendArgs {
   const int32_t* pool_block_table;
   int pool_max_pages;
 };
-cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, cudaStream_t st);
+// index_part = false: the kv row and the main pool; true: the indexer ring and pool (CSA).
+cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, bool index_part,
+                                 cudaStream_t st);
 
 // ---- indexer (indexer.cu) -----------------------------------------------------------------
 struct IndexerArgs {

@@ -1,6 +1,7 @@
 // Optional per-kernel timing: while enabled, every kernel launch of the library is bracketed by a
 // pair of CUDA events recorded on the launch's own stream; sac_timing_end() waits for them and
-// returns launches and total device time per kernel name.
+// returns launches and total device time per kernel name. Launches captured into a CUDA graph
+// carry their events into the graph, and sac_timing_end() then reports the graph's latest replay.
 #include <mutex>
 #include <string>
 #include <vector>
@@ -40,6 +41,16 @@ cudaEvent_t take_event(TimerState& s) {
   return e;
 }
 
+// Inside a CUDA-graph capture an ordinary event record only marks a dependency; an external
+// record becomes an event node of the graph, timestamped on every replay.
+void record(cudaEvent_t e, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, st);
+}
+
 }  // namespace
 
 int timer_start(const char* name, cudaStream_t st, cudaEvent_t* stop_out) {
@@ -54,7 +65,7 @@ int timer_start(const char* name, cudaStream_t st, cudaEvent_t* stop_out) {
     slot = (int)s.names.size() - 1;
   }
   Pending p{slot, take_event(s), take_event(s)};
-  cudaEventRecord(p.start, st);
+  record(p.start, st);
   *stop_out = p.stop;
   s.pending.push_back(p);
   return slot;
@@ -62,7 +73,7 @@ int timer_start(const char* name, cudaStream_t st, cudaEvent_t* stop_out) {
 
 void timer_stop(int slot, cudaEvent_t stop, cudaStream_t st) {
   if (slot < 0) return;
-  cudaEventRecord(stop, st);
+  record(stop, st);
 }
 
 }  // namespace sac

@@ -2,7 +2,9 @@
 // paragraph): per query row, the k largest of the (t+1)//m visible scores, ties going to the
 // lower entry index; empty slots (fewer than k visible) hold -1.
 //
-// One block of 512 threads per row; scores become order-preserving uint32 keys in shared memory.
+// One block per row; scores become order-preserving uint32 keys, held in registers for rows of up
+// to 32768 entries (block size and keys per thread picked by the longest row) and in shared memory
+// beyond that.
 // The exact k-th largest key T is found by a radix select on digits of 12, 12 and 8 bits. The
 // first digit (sign, exponent and 3 mantissa bits) spreads real score distributions over many
 // bins, so the histogram atomics rarely collide; the keys in the bin that holds T (usually a few
@@ -11,6 +13,7 @@
 // contiguous segment of the row and keeps every key > T plus the first (k - #{key > T}) keys == T in
 // index order, using ballots for the in-warp order and per-warp counts for the rest, so the chosen
 // entries come out in ascending order with conflict-free shared-memory reads.
+#include "launch_util.h"
 #include "sac_kernels.h"
 
 namespace sac {
@@ -30,13 +33,14 @@ __device__ __forceinline__ uint32_t order_key(float s) {
 struct Shared {
   int hist[kBins];
   uint32_t cand[kCandCap];
-  int warp_tot[kWarps];
-  int warp_gt[kWarps], warp_eq[kWarps];
+  int warp_tot[32];  // up to 1024 threads
+  int warp_gt[32], warp_eq[32];
   int n_cand;
   int digit, rem;
 };
 
-// Exclusive prefix sum over the block (thread order); also returns the block total.
+// Exclusive prefix sum over the block of NT threads (thread order); also returns the total.
+template <int NT>
 __device__ __forceinline__ int block_exclusive_sum(int v, int* warp_tot, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
@@ -50,7 +54,7 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* warp_tot, int& to
   int before = 0;
   total = 0;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     const int t = warp_tot[w];
     before += w < warp ? t : 0;
     total += t;
@@ -62,21 +66,22 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* warp_tot, int& to
 // Given hist[0..nbins) (nbins = 8 * kThreads or fewer), find the digit d holding the rem-th
 // largest counted key: sum(hist[d+1..]) < rem <= sum(hist[d..]). Writes sh.digit and sh.rem (the
 // rank of T among the keys of digit d).
+template <int NT>
 __device__ __forceinline__ void find_digit(Shared& sh, int nbins, int rem) {
-  const int per = nbins / kThreads;  // 8 for 12-bit digits; 0 for 8-bit (threads < 256 own one)
-  const int rt = kThreads - 1 - threadIdx.x;  // thread blocks of bins counted from the top
+  const int per = nbins / NT;  // bins per thread; 0 when there are fewer bins than threads
+  const int rt = NT - 1 - threadIdx.x;  // thread blocks of bins counted from the top
   int lo, cnt;
   if (per > 0) {
     lo = rt * per;
     cnt = per;
   } else {
-    lo = rt - (kThreads - nbins);
+    lo = rt - (NT - nbins);
     cnt = lo >= 0 ? 1 : 0;
   }
   int s = 0;
   for (int i = 0; i < cnt; ++i) s += sh.hist[lo + i];
   int total;
-  const int above = block_exclusive_sum(s, sh.warp_tot, total);
+  const int above = block_exclusive_sum<NT>(s, sh.warp_tot, total);
   if (cnt > 0 && above < rem && rem <= above + s) {
     int acc = above;
     for (int d = lo + cnt - 1; d >= lo; --d) {
@@ -92,7 +97,7 @@ __device__ __forceinline__ void find_digit(Shared& sh, int nbins, int rem) {
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict__ scores,
+__global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __restrict__ scores,
                                                         int n_stride, QueryRows qr, int m, int k,
                                                         int32_t* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -122,7 +127,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
     atomicAdd(&sh.hist[key >> 20], 1);
   }
   __syncthreads();
-  find_digit(sh, kBins, k);
+  find_digit<kThreads>(sh, kBins, k);
   const uint32_t d1 = (uint32_t)sh.digit;
   int rem = sh.rem;
   const int c1 = sh.hist[d1];
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
     if ((key >> 20) == d1) atomicAdd(&sh.hist[(key >> 8) & 0xFFFu], 1);
   }
   __syncthreads();
-  find_digit(sh, kBins, rem);
+  find_digit<kThreads>(sh, kBins, rem);
   const uint32_t d2 = (uint32_t)sh.digit;
   rem = sh.rem;
   __syncthreads();
@@ -169,7 +174,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
     if ((key >> 8) == hi24) atomicAdd(&sh.hist[key & 0xFFu], 1);
   }
   __syncthreads();
-  find_digit(sh, 256, rem);
+  find_digit<kThreads>(sh, 256, rem);
   const uint32_t T = (hi24 << 8) | (uint32_t)sh.digit;
   const int take_eq = sh.rem;  // keys equal to T to keep, lowest indices first
 
@@ -210,6 +215,142 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
   }
 }
 
+// Rows of at most NT * KPT scores: the keys stay in registers. Warp w owns the contiguous segment
+// [w * seg, w * seg + seg) (seg a multiple of 32, the same for every warp) and its lane l holds
+// entries w * seg + 32 j + l, j < KPT: the loads are coalesced and the selection output keeps the
+// in-warp ballot order, exactly as in the shared-memory kernel; the same three digits are used.
+template <int NT, int KPT>
+__global__ void __launch_bounds__(NT, 1) topk_reg_kernel(const float* __restrict__ scores,
+                                                      int n_stride, QueryRows qr, int m, int k,
+                                                      int32_t* __restrict__ out) {
+  constexpr int NW = NT / 32;
+  __shared__ Shared sh;
+  const int64_t r = blockIdx.x;
+  int seq;
+  int64_t t;
+  qr.locate(qr.row0 + r, seq, t);
+  const int n = (int)((t + 1) / m);
+  int32_t* orow = out + r * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (n <= k) {
+    for (int i = tid; i < k; i += NT) orow[i] = i < n ? i : -1;
+    return;
+  }
+  const float* srow = scores + r * n_stride;
+  const int seg = ((n + NW * 32 - 1) / (NW * 32)) * 32;
+  const int s0 = warp * seg, s1 = min(n, s0 + seg);
+
+  for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0;
+  if (tid == 0) sh.n_cand = 0;
+  __syncthreads();
+  uint32_t key[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int i = s0 + 32 * j + lane;
+    key[j] = 0u;
+    if (i < s1) {
+      key[j] = order_key(__ldg(srow + i));
+      atomicAdd(&sh.hist[key[j] >> 20], 1);
+    }
+  }
+  __syncthreads();
+  find_digit<NT>(sh, kBins, k);
+  const uint32_t d1 = (uint32_t)sh.digit;
+  int rem = sh.rem;
+  const int c1 = sh.hist[d1];
+  __syncthreads();
+
+  const bool compact = c1 <= kCandCap;
+  if (compact) {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int i = s0 + 32 * j + lane;
+      const bool hit = i < s1 && (key[j] >> 20) == d1;
+      const uint32_t mask = __ballot_sync(~0u, hit);
+      if (mask) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&sh.n_cand, __popc(mask));
+        base = __shfl_sync(~0u, base, 0);
+        if (hit) sh.cand[base + __popc(mask & ((1u << lane) - 1u))] = key[j];
+      }
+    }
+  }
+  // digit 2 (bits 19..8) among keys with digit 1 == d1
+  for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0;
+  __syncthreads();
+  if (compact) {
+    for (int i = tid; i < c1; i += NT) atomicAdd(&sh.hist[(sh.cand[i] >> 8) & 0xFFFu], 1);
+  } else {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (s0 + 32 * j + lane < s1 && (key[j] >> 20) == d1)
+        atomicAdd(&sh.hist[(key[j] >> 8) & 0xFFFu], 1);
+  }
+  __syncthreads();
+  find_digit<NT>(sh, kBins, rem);
+  const uint32_t d2 = (uint32_t)sh.digit;
+  rem = sh.rem;
+  __syncthreads();
+  // digit 3 (bits 7..0) among keys with bits 31..8 == (d1, d2)
+  const uint32_t hi24 = (d1 << 12) | d2;
+  for (int i = tid; i < 256; i += NT) sh.hist[i] = 0;
+  __syncthreads();
+  if (compact) {
+    for (int i = tid; i < c1; i += NT)
+      if ((sh.cand[i] >> 8) == hi24) atomicAdd(&sh.hist[sh.cand[i] & 0xFFu], 1);
+  } else {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (s0 + 32 * j + lane < s1 && (key[j] >> 8) == hi24)
+        atomicAdd(&sh.hist[key[j] & 0xFFu], 1);
+  }
+  __syncthreads();
+  find_digit<NT>(sh, 256, rem);
+  const uint32_t T = (hi24 << 8) | (uint32_t)sh.digit;
+  const int take_eq = sh.rem;
+
+  int gt = 0, eq = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const bool in = s0 + 32 * j + lane < s1;
+    gt += __popc(__ballot_sync(~0u, in && key[j] > T));
+    eq += __popc(__ballot_sync(~0u, in && key[j] == T));
+  }
+  if (lane == 0) {
+    sh.warp_gt[warp] = gt;
+    sh.warp_eq[warp] = eq;
+  }
+  __syncthreads();
+  int eq_before = 0, sel_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    const int e = sh.warp_eq[w];
+    const int take = min(max(take_eq - eq_before, 0), e);
+    sel_before += sh.warp_gt[w] + take;
+    eq_before += e;
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int i = s0 + 32 * j + lane;
+    const bool in = i < s1;
+    const bool is_gt = in && key[j] > T;
+    const bool is_eq = in && key[j] == T;
+    const uint32_t eq_mask = __ballot_sync(~0u, is_eq);
+    const bool sel = is_gt || (is_eq && eq_before + __popc(eq_mask & lt) < take_eq);
+    const uint32_t sel_mask = __ballot_sync(~0u, sel);
+    if (sel) orow[sel_before + __popc(sel_mask & lt)] = i;
+    eq_before += __popc(eq_mask);
+    sel_before += __popc(sel_mask);
+  }
+}
+
+template <int NT, int KPT>
+cudaError_t topk_reg(const float* scores, int n_stride, QueryRows qr, int m, int64_t nrows, int k,
+                     int32_t* out, cudaStream_t st) {
+  topk_reg_kernel<NT, KPT><<<(unsigned)nrows, NT, 0, st>>>(scores, n_stride, qr, m, k, out);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int topk_max_entries() { return kMaxEntries; }
@@ -218,11 +359,15 @@ cudaError_t launch_topk(const float* scores, int n_stride, QueryRows qr, int m, 
                         int k, int32_t* out, cudaStream_t st) {
   if (nrows == 0) return cudaSuccess;
   if (n_stride > kMaxEntries) return cudaErrorInvalidValue;
+  // rows that fit in registers: block size and keys per thread by the longest row
+  if (n_stride <= 2048) return topk_reg<256, 8>(scores, n_stride, qr, m, nrows, k, out, st);
+  if (n_stride <= 8192) return topk_reg<512, 16>(scores, n_stride, qr, m, nrows, k, out, st);
+  if (n_stride <= 16384) return topk_reg<512, 32>(scores, n_stride, qr, m, nrows, k, out, st);
+  if (n_stride <= 32768) return topk_reg<1024, 32>(scores, n_stride, qr, m, nrows, k, out, st);
   const size_t smem = sizeof(Shared) + sizeof(uint32_t) * (size_t)(n_stride > 0 ? n_stride : 1);
-  cudaError_t err = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  cudaError_t err = ensure_smem_limit((const void*)topk_smem_kernel, (int)smem);
   if (err != cudaSuccess) return err;
-  topk_kernel<<<(unsigned)nrows, kThreads, smem, st>>>(scores, n_stride, qr, m, k, out);
+  topk_smem_kernel<<<(unsigned)nrows, kThreads, smem, st>>>(scores, n_stride, qr, m, k, out);
   return cudaGetLastError();
 }
 
