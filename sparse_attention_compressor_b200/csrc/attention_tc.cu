@@ -23,12 +23,14 @@
 // (buffer 0) and 352 (buffer 1). A softmax thread of lane i < 16 and its partner i + 16 own the
 // same head: they add their partials, exchange halves, and each finishes 24 of the 48 keys.
 //
-// Warps: 0 = TMA thread, 1-2 = MMA issuers (warp 1 also owns TMEM), 3 = query rotation, 4-5 / 6-7 =
-// gather groups (even / odd tiles), 8-11 = softmax + output. Each tcgen05.mma costs its issuing
-// thread a fixed time, so two threads issue: warp 1 the even partials of QK^T and PV of
-// O[:, 0:256], warp 2 the odd partials and PV of O[:, 256:512]; every barrier the MMAs signal
-// counts both. The softmax keeps the running max in log2 units and moves it (rescaling O) only
-// when a tile's max exceeds it by more than 8.
+// Warps: 0 = TMA thread, 1-2 = QK^T issuers (warp 1 also owns TMEM), 3 = query rotation, 4-5 / 6-7
+// = gather groups (even / odd tiles), 8-11 = softmax + output, 12 = PV issuer. Each tcgen05.mma
+// costs its issuing thread a fixed time, so two threads issue QK^T (warp 1 the even partials,
+// warp 2 the odd ones) and a third issues PV the moment P is written, instead of after the next
+// tile's QK^T. An M = 64 MMA occupies one 16-lane half of each TMEM sub-partition, and MMAs into
+// opposite halves run side by side: the two QK^T issuers' partials, and the two halves of O, sit
+// in opposite lane halves. The softmax keeps the running max in log2 units and moves it
+// (rescaling O) only when a tile's max exceeds it by more than 8.
 #include <cuda_bf16.h>
 
 #include "launch_util.h"
@@ -50,12 +52,13 @@ constexpr int kQBytes = 8 * kQRegion;            // 64 KB
 constexpr int kTileBytes = 8 * kKRegion;         // 48 KB
 constexpr int kPBytes = kHeads * 128;            // 64 rows x 128 B (48 keys used)
 constexpr int kGroupThreads = 64;                // threads of one gather group
-constexpr int kThreads = 384;
+constexpr int kThreads = 416;
 
 constexpr int kOffQ = 0;
 constexpr int kOffTile = kOffQ + kQBytes;
 constexpr int kOffP = kOffTile + kStages * kTileBytes;
-constexpr int kOffBar = kOffP + 2 * kPBytes;
+constexpr int kOffCs = kOffP + 2 * kPBytes;      // [32] (cos, sin) of the query's rope pairs
+constexpr int kOffBar = kOffCs + 32 * 8;
 enum Bar { kQFull, kQReady, kQEmpty, kKvFull0, kKvEmpty0 = kKvFull0 + kStages,
            kSFull0 = kKvEmpty0 + kStages, kPFull0 = kSFull0 + 2, kPvDone0 = kPFull0 + 2,
            kOFull = kPvDone0 + 2, kOEmpty, kNumBars };
@@ -112,6 +115,15 @@ __device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const
   return p ? p : reinterpret_cast<const __nv_bfloat16*>(a.pool.base);
 }
 
+// Hint: bring a query's 64 KB of rows into L2 ahead of its TMA load (eight 8 KB bulk prefetches).
+__device__ __forceinline__ void prefetch_query_l2(const void* q) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], 8192;" ::"l"(
+                     reinterpret_cast<uint64_t>(q) + (uint64_t)i * 8192)
+                 : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_win_box,
@@ -133,14 +145,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bar[kQEmpty], 2);
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&bar[kKvFull0 + i], 1 + kGroupThreads);  // TMA thread + one gather group
-      tc::mbar_init(&bar[kKvEmpty0 + i], 2);
+      tc::mbar_init(&bar[kKvEmpty0 + i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&bar[kSFull0 + i], 2);
       tc::mbar_init(&bar[kPFull0 + i], 128);
-      tc::mbar_init(&bar[kPvDone0 + i], 2);
+      tc::mbar_init(&bar[kPvDone0 + i], 1);
     }
-    tc::mbar_init(&bar[kOFull], 2);
+    tc::mbar_init(&bar[kOFull], 1);
     tc::mbar_init(&bar[kOEmpty], 128);
     tc::fence_barrier_init();
   }
@@ -166,6 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
         const Row w = locate_row(a, r);
+        if (r + gridDim.x < a.nrows)  // the CTA's next query, loaded by TMA one query later
+          prefetch_query_l2(reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                            (r + gridDim.x) * kHeads * kDim);
         if (qi > 0) ok = tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status);
         if (!ok) break;
         tc::mbar_arrive_expect_tx(&bar[kQFull], kQBytes);
@@ -195,8 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------------------------------ MMA issuers
-    const uint32_t me = warp - 1;  // 0: even partials + O[:,0:256]; 1: odd partials + O[:,256:]
+    // ------------------------------------------------------------------ QK^T issuers
+    const uint32_t me = warp - 1;  // 0: even partials (lanes 0-15); 1: odd partials (lanes 16-31)
     if (lane == 0) {
       uint32_t g0 = 0, qi = 0;
       bool ok = true;
@@ -206,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the query tile has landed; its rope region (the last 128-byte column, K-steps 28..31)
         // is still being rotated, so the first QK^T waits for kQReady only before those steps
         ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
-        for (int j = 0; j <= w.tiles && ok; ++j) {
-          if (j < w.tiles) {  // S(g) = Q K^T over four partial accumulators
+        for (int j = 0; j < w.tiles && ok; ++j) {
+          {  // S(g) = Q K^T over four partial accumulators
             const uint32_t g = g0 + j, b = g % kStages, s = g & 1;
             ok = tc::mbar_wait(&bar[kKvFull0 + b], (g / kStages) & 1, status);
             if (ok && g >= 2) ok = tc::mbar_wait(&bar[kPFull0 + s], ((g - 2) >> 1) & 1, status);
@@ -238,25 +253,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mma_commit(&bar[kSFull0 + s]);
             if (j == w.tiles - 1) tc::mma_commit(&bar[kQEmpty]);
           }
-          if (j >= 1) {  // O += P(g) V(g)
-            const uint32_t g = g0 + j - 1, b = g % kStages, s = g & 1;
-            ok = tc::mbar_wait(&bar[kPFull0 + s], (g >> 1) & 1, status);
-            if (ok && j == 1 && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
-            if (!ok) break;
-            tc::tc_fence_after();
-            const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
-            const uint64_t pd = tc::desc_sw128(tc::smem_u32(smem + kOffP + s * kPBytes), 0, 1024);
-            const uint64_t vd = tc::desc_sw128(v_base + me * 4 * kKRegion, kKRegion, 1024);
-            const uint32_t od = tmem + (me ? (16u << 16) : 0u);
-#pragma unroll
-            for (int kk = 0; kk < kNK / 16; ++kk) {
-              const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
-              tc::mma_bf16_ss(od, pd + kk * 2, vd + kk * 128, kIdescPV, acc);
-            }
-            tc::mma_commit(&bar[kKvEmpty0 + b]);
-            tc::mma_commit(&bar[kPvDone0 + s]);
-            if (j == w.tiles) tc::mma_commit(&bar[kOFull]);
-          }
         }
         g0 += w.tiles;
       }
@@ -264,51 +260,73 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 3) {
     // ------------------------------------------------------------------ query rotation
-    // thread i turns the rope pairs of head rows i and i+32 of the staged query tile (row h's
-    // 16-byte chunk c of a 128-byte region sits at chunk c ^ (h & 7)).
+    // Lane p first writes (cos, sin) of rope pair p at the query's position to a shared table.
+    // Then thread i turns the rope pairs of head rows i and i+32 of the staged query tile (row h's
+    // 16-byte chunk c of a 128-byte region sits at chunk c ^ (h & 7)); when the rope slice starts
+    // on a 16-byte boundary (R a multiple of 8) all of a thread's chunks are loaded before any is
+    // used, so the rotation costs one shared-memory round trip instead of one per chunk.
     const int R = a.rf.R;
     const int p0 = (kDim - R) >> 1;  // first rotated pair among the 256 channel pairs
+    float2* cs_tab = reinterpret_cast<float2*>(smem + kOffCs);
     uint32_t qi = 0;
     bool ok = true;
     for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
       int seq;
       int64_t t;
       a.qr.locate(a.qr.row0 + r, seq, t);
-      float my_c = 1.f, my_s = 0.f;
-      if (lane < R / 2) rope_cos_sin(a.rf, lane, a.pos0 + t, my_c, my_s);
+      if (lane < R / 2) {
+        float c, sn;
+        rope_cos_sin(a.rf, lane, a.pos0 + t, c, sn);
+        cs_tab[lane] = make_float2(c, sn);
+      }
+      __syncwarp();
       ok = __all_sync(~0u, tc::mbar_wait(&bar[kQFull], qi & 1, status));
       if (!ok) break;
-      for (int hh = 0; hh < 2; ++hh) {
-      const int h = hh * 32 + lane;
-      uint8_t* row = smem + kOffQ + h * 128;
-      for (int p = 0; p < R / 2; p += 4) {
-        const int pp = p0 + p;                  // channels 2pp, 2pp+1
-        const int region = pp >> 5;             // 32 pairs per 128-byte region
-        const int chunk = (pp & 31) >> 2;       // 4 pairs per 16-byte chunk
-        uint8_t* cptr = row + region * kQRegion + ((chunk ^ (h & 7)) << 4);
-        if ((pp & 3) == 0 && p + 4 <= R / 2) {
-          uint4 v = *reinterpret_cast<uint4*>(cptr);
-          uint32_t* w4 = reinterpret_cast<uint32_t*>(&v);
+      if ((R & 7) == 0) {
+        constexpr int kMaxChunks = 8;  // R <= 64: at most 8 chunks of 4 pairs
+        const int nch = R >> 3;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float cc = __shfl_sync(~0u, my_c, p + u), ss = __shfl_sync(~0u, my_s, p + u);
-            const float2 x = unpack_bf16(w4[u]);
-            w4[u] = pack_bf16(x.x * cc - x.y * ss, x.x * ss + x.y * cc);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int h = hh * 32 + lane;
+          uint8_t* row = smem + kOffQ + h * 128;
+          uint4 v[kMaxChunks];
+#pragma unroll
+          for (int c = 0; c < kMaxChunks; ++c) {
+            const int pp = p0 + 4 * c;
+            if (c < nch)
+              v[c] = *reinterpret_cast<const uint4*>(row + (pp >> 5) * kQRegion +
+                                                     ((((pp & 31) >> 2) ^ (h & 7)) << 4));
           }
-          *reinterpret_cast<uint4*>(cptr) = v;
-        } else {
-          for (int u = 0; u < 4; ++u) {
-            const int pu = p + u < R / 2 ? p + u : R / 2 - 1;
-            const float cc = __shfl_sync(~0u, my_c, pu), ss = __shfl_sync(~0u, my_s, pu);
-            if (p + u >= R / 2) continue;
-            const int q = p0 + p + u;
-            uint32_t* word = reinterpret_cast<uint32_t*>(
-                row + (q >> 5) * kQRegion + ((((q & 31) >> 2) ^ (h & 7)) << 4) + (q & 3) * 4);
-            const float2 x = unpack_bf16(*word);
-            *word = pack_bf16(x.x * cc - x.y * ss, x.x * ss + x.y * cc);
+#pragma unroll
+          for (int c = 0; c < kMaxChunks; ++c) {
+            if (c >= nch) break;
+            const int pp = p0 + 4 * c;
+            const float4 cs01 = *reinterpret_cast<const float4*>(cs_tab + 4 * c);
+            const float4 cs23 = *reinterpret_cast<const float4*>(cs_tab + 4 * c + 2);
+            const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+            const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+            uint32_t* w4 = reinterpret_cast<uint32_t*>(&v[c]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 x = unpack_bf16(w4[u]);
+              w4[u] = pack_bf16(x.x * cc[u] - x.y * ss[u], x.x * ss[u] + x.y * cc[u]);
+            }
+            *reinterpret_cast<uint4*>(row + (pp >> 5) * kQRegion +
+                                      ((((pp & 31) >> 2) ^ (h & 7)) << 4)) = v[c];
           }
         }
-      }
+      } else {
+        for (int hh = 0; hh < 2; ++hh) {
+          const int h = hh * 32 + lane;
+          uint8_t* row = smem + kOffQ + h * 128;
+          for (int q = p0; q < kDim / 2; ++q) {
+            uint32_t* word = reinterpret_cast<uint32_t*>(
+                row + (q >> 5) * kQRegion + ((((q & 31) >> 2) ^ (h & 7)) << 4) + (q & 3) * 4);
+            const float2 cs = cs_tab[q - p0];
+            const float2 x = unpack_bf16(*word);
+            *word = pack_bf16(x.x * cs.x - x.y * cs.y, x.x * cs.y + x.y * cs.x);
+          }
+        }
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bar[kQReady]);
@@ -390,6 +408,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(&bar[kKvFull0 + b]);
       c = n;
     }
+  } else if (warp == 12) {
+    // ------------------------------------------------------------------ PV issuer
+    // O += P(g) V(g) as soon as the softmax has written P(g), independent of how far the QK^T
+    // issuers have got: O[:, 0:256] accumulates in lanes 0-15 and O[:, 256:512] in lanes 16-31,
+    // and the two halves' MMAs alternate so both lane halves of the tensor core stay busy.
+    if (lane == 0) {
+      uint32_t g0 = 0, qi = 0;
+      bool ok = true;
+      for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
+        const Row w = locate_row(a, r);
+        for (int j = 0; j < w.tiles && ok; ++j) {
+          const uint32_t g = g0 + j, b = g % kStages, s = g & 1;
+          ok = tc::mbar_wait(&bar[kPFull0 + s], (g >> 1) & 1, status);
+          if (ok && j == 0 && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
+          const uint64_t pd = tc::desc_sw128(tc::smem_u32(smem + kOffP + s * kPBytes), 0, 1024);
+          const uint64_t vd0 = tc::desc_sw128(v_base, kKRegion, 1024);
+          const uint64_t vd1 = tc::desc_sw128(v_base + 4 * kKRegion, kKRegion, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kNK / 16; ++kk) {
+            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            tc::mma_bf16_ss(tmem, pd + kk * 2, vd0 + kk * 128, kIdescPV, acc);
+            tc::mma_bf16_ss(tmem + (16u << 16), pd + kk * 2, vd1 + kk * 128, kIdescPV, acc);
+          }
+          tc::mma_commit(&bar[kKvEmpty0 + b]);
+          tc::mma_commit(&bar[kPvDone0 + s]);
+          if (j == w.tiles - 1) tc::mma_commit(&bar[kOFull]);
+        }
+        g0 += w.tiles;
+      }
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax + output
     const int sp = warp & 3;                 // TMEM sub-partition of this warp

@@ -2,9 +2,8 @@
 // paragraph): per query row, the k largest of the (t+1)//m visible scores, ties going to the
 // lower entry index; empty slots (fewer than k visible) hold -1.
 //
-// One block per row; scores become order-preserving uint32 keys, held in registers for rows of up
-// to 32768 entries (block size and keys per thread picked by the longest row) and in shared memory
-// beyond that.
+// One block per row; scores become order-preserving uint32 keys (kept in shared memory for short
+// rows, re-read from L2 by every pass for long ones).
 // The exact k-th largest key T is found by a radix select on digits of 12, 12 and 8 bits. The
 // first digit (sign, exponent and 3 mantissa bits) spreads real score distributions over many
 // bins, so the histogram atomics rarely collide; the keys in the bin that holds T (usually a few
@@ -21,9 +20,11 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxEntries = 49152;   // keys in shared memory: 192 KB
+constexpr int kMaxEntries = 1 << 22;  // longest row (pool entries per sequence) accepted
 constexpr int kBins = 4096;          // 12-bit digits
 constexpr int kCandCap = 2048;       // compacted keys of the threshold bin
+constexpr int kSmemKeyRows = 4096;   // rows up to this length keep their keys in shared memory
+constexpr int kSmemKeyLimit = 49152; // longest row whose keys fit in shared memory (192 KB)
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t u = __float_as_uint(s + 0.0f);  // -0 and +0 compare equal
@@ -97,7 +98,11 @@ __device__ __forceinline__ void find_digit(Shared& sh, int nbins, int rem) {
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __restrict__ scores,
+// kSmemKeys: the row's keys are kept in shared memory (short rows); otherwise every pass
+// re-reads the scores, which the first pass has brought into L2, so that a block needs only
+// ~25 KB of shared memory and several rows run side by side on each SM.
+template <bool kSmemKeys>
+__global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict__ scores,
                                                         int n_stride, QueryRows qr, int m, int k,
                                                         int32_t* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -116,14 +121,17 @@ __global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __rest
     return;
   }
   const float* srow = scores + r * n_stride;
+  auto key_at = [&](int i) -> uint32_t {
+    return kSmemKeys ? keys[i] : order_key(__ldcg(srow + i));
+  };
 
   // ---- digit 1: bits 31..20
   for (int i = tid; i < kBins; i += kThreads) sh.hist[i] = 0;
   if (tid == 0) sh.n_cand = 0;
   __syncthreads();
   for (int i = tid; i < n; i += kThreads) {
-    const uint32_t key = order_key(__ldg(srow + i));
-    keys[i] = key;
+    const uint32_t key = order_key(__ldcg(srow + i));
+    if (kSmemKeys) keys[i] = key;
     atomicAdd(&sh.hist[key >> 20], 1);
   }
   __syncthreads();
@@ -138,7 +146,7 @@ __global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __rest
   if (compact) {
     for (int i0 = warp * 32; i0 < n; i0 += kThreads) {
       const int i = i0 + lane;
-      const uint32_t key = i < n ? keys[i] : 0u;
+      const uint32_t key = i < n ? key_at(i) : 0u;
       const bool hit = i < n && (key >> 20) == d1;
       const uint32_t mask = __ballot_sync(~0u, hit);
       if (mask) {
@@ -149,14 +157,14 @@ __global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __rest
       }
     }
   }
-  const uint32_t* ck = compact ? sh.cand : keys;
   const int nc = compact ? c1 : n;
+  auto cand_at = [&](int i) -> uint32_t { return compact ? sh.cand[i] : key_at(i); };
 
   // ---- digit 2: bits 19..8 among keys with digit 1 == d1
   for (int i = tid; i < kBins; i += kThreads) sh.hist[i] = 0;
   __syncthreads();
   for (int i = tid; i < nc; i += kThreads) {
-    const uint32_t key = ck[i];
+    const uint32_t key = cand_at(i);
     if ((key >> 20) == d1) atomicAdd(&sh.hist[(key >> 8) & 0xFFFu], 1);
   }
   __syncthreads();
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __rest
   for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0;
   __syncthreads();
   for (int i = tid; i < nc; i += kThreads) {
-    const uint32_t key = ck[i];
+    const uint32_t key = cand_at(i);
     if ((key >> 8) == hi24) atomicAdd(&sh.hist[key & 0xFFu], 1);
   }
   __syncthreads();
@@ -184,7 +192,7 @@ __global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __rest
   int gt = 0, eq = 0;
   for (int i0 = s0; i0 < s1; i0 += 32) {
     const int i = i0 + lane;
-    const uint32_t key = i < s1 ? keys[i] : 0u;
+    const uint32_t key = i < s1 ? key_at(i) : 0u;
     gt += __popc(__ballot_sync(~0u, i < s1 && key > T));
     eq += __popc(__ballot_sync(~0u, i < s1 && key == T));
   }
@@ -203,7 +211,7 @@ __global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __rest
   const uint32_t lt = (1u << lane) - 1u;
   for (int i0 = s0; i0 < s1; i0 += 32) {
     const int i = i0 + lane;
-    const uint32_t key = i < s1 ? keys[i] : 0u;
+    const uint32_t key = i < s1 ? key_at(i) : 0u;
     const bool is_gt = i < s1 && key > T;
     const bool is_eq = i < s1 && key == T;
     const uint32_t eq_mask = __ballot_sync(~0u, is_eq);
@@ -215,142 +223,6 @@ __global__ void __launch_bounds__(kThreads) topk_smem_kernel(const float* __rest
   }
 }
 
-// Rows of at most NT * KPT scores: the keys stay in registers. Warp w owns the contiguous segment
-// [w * seg, w * seg + seg) (seg a multiple of 32, the same for every warp) and its lane l holds
-// entries w * seg + 32 j + l, j < KPT: the loads are coalesced and the selection output keeps the
-// in-warp ballot order, exactly as in the shared-memory kernel; the same three digits are used.
-template <int NT, int KPT>
-__global__ void __launch_bounds__(NT, 1) topk_reg_kernel(const float* __restrict__ scores,
-                                                      int n_stride, QueryRows qr, int m, int k,
-                                                      int32_t* __restrict__ out) {
-  constexpr int NW = NT / 32;
-  __shared__ Shared sh;
-  const int64_t r = blockIdx.x;
-  int seq;
-  int64_t t;
-  qr.locate(qr.row0 + r, seq, t);
-  const int n = (int)((t + 1) / m);
-  int32_t* orow = out + r * k;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (n <= k) {
-    for (int i = tid; i < k; i += NT) orow[i] = i < n ? i : -1;
-    return;
-  }
-  const float* srow = scores + r * n_stride;
-  const int seg = ((n + NW * 32 - 1) / (NW * 32)) * 32;
-  const int s0 = warp * seg, s1 = min(n, s0 + seg);
-
-  for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0;
-  if (tid == 0) sh.n_cand = 0;
-  __syncthreads();
-  uint32_t key[KPT];
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    const int i = s0 + 32 * j + lane;
-    key[j] = 0u;
-    if (i < s1) {
-      key[j] = order_key(__ldg(srow + i));
-      atomicAdd(&sh.hist[key[j] >> 20], 1);
-    }
-  }
-  __syncthreads();
-  find_digit<NT>(sh, kBins, k);
-  const uint32_t d1 = (uint32_t)sh.digit;
-  int rem = sh.rem;
-  const int c1 = sh.hist[d1];
-  __syncthreads();
-
-  const bool compact = c1 <= kCandCap;
-  if (compact) {
-#pragma unroll
-    for (int j = 0; j < KPT; ++j) {
-      const int i = s0 + 32 * j + lane;
-      const bool hit = i < s1 && (key[j] >> 20) == d1;
-      const uint32_t mask = __ballot_sync(~0u, hit);
-      if (mask) {
-        int base = 0;
-        if (lane == 0) base = atomicAdd(&sh.n_cand, __popc(mask));
-        base = __shfl_sync(~0u, base, 0);
-        if (hit) sh.cand[base + __popc(mask & ((1u << lane) - 1u))] = key[j];
-      }
-    }
-  }
-  // digit 2 (bits 19..8) among keys with digit 1 == d1
-  for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0;
-  __syncthreads();
-  if (compact) {
-    for (int i = tid; i < c1; i += NT) atomicAdd(&sh.hist[(sh.cand[i] >> 8) & 0xFFFu], 1);
-  } else {
-#pragma unroll
-    for (int j = 0; j < KPT; ++j)
-      if (s0 + 32 * j + lane < s1 && (key[j] >> 20) == d1)
-        atomicAdd(&sh.hist[(key[j] >> 8) & 0xFFFu], 1);
-  }
-  __syncthreads();
-  find_digit<NT>(sh, kBins, rem);
-  const uint32_t d2 = (uint32_t)sh.digit;
-  rem = sh.rem;
-  __syncthreads();
-  // digit 3 (bits 7..0) among keys with bits 31..8 == (d1, d2)
-  const uint32_t hi24 = (d1 << 12) | d2;
-  for (int i = tid; i < 256; i += NT) sh.hist[i] = 0;
-  __syncthreads();
-  if (compact) {
-    for (int i = tid; i < c1; i += NT)
-      if ((sh.cand[i] >> 8) == hi24) atomicAdd(&sh.hist[sh.cand[i] & 0xFFu], 1);
-  } else {
-#pragma unroll
-    for (int j = 0; j < KPT; ++j)
-      if (s0 + 32 * j + lane < s1 && (key[j] >> 8) == hi24)
-        atomicAdd(&sh.hist[key[j] & 0xFFu], 1);
-  }
-  __syncthreads();
-  find_digit<NT>(sh, 256, rem);
-  const uint32_t T = (hi24 << 8) | (uint32_t)sh.digit;
-  const int take_eq = sh.rem;
-
-  int gt = 0, eq = 0;
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    const bool in = s0 + 32 * j + lane < s1;
-    gt += __popc(__ballot_sync(~0u, in && key[j] > T));
-    eq += __popc(__ballot_sync(~0u, in && key[j] == T));
-  }
-  if (lane == 0) {
-    sh.warp_gt[warp] = gt;
-    sh.warp_eq[warp] = eq;
-  }
-  __syncthreads();
-  int eq_before = 0, sel_before = 0;
-  for (int w = 0; w < warp; ++w) {
-    const int e = sh.warp_eq[w];
-    const int take = min(max(take_eq - eq_before, 0), e);
-    sel_before += sh.warp_gt[w] + take;
-    eq_before += e;
-  }
-  const uint32_t lt = (1u << lane) - 1u;
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    const int i = s0 + 32 * j + lane;
-    const bool in = i < s1;
-    const bool is_gt = in && key[j] > T;
-    const bool is_eq = in && key[j] == T;
-    const uint32_t eq_mask = __ballot_sync(~0u, is_eq);
-    const bool sel = is_gt || (is_eq && eq_before + __popc(eq_mask & lt) < take_eq);
-    const uint32_t sel_mask = __ballot_sync(~0u, sel);
-    if (sel) orow[sel_before + __popc(sel_mask & lt)] = i;
-    eq_before += __popc(eq_mask);
-    sel_before += __popc(sel_mask);
-  }
-}
-
-template <int NT, int KPT>
-cudaError_t topk_reg(const float* scores, int n_stride, QueryRows qr, int m, int64_t nrows, int k,
-                     int32_t* out, cudaStream_t st) {
-  topk_reg_kernel<NT, KPT><<<(unsigned)nrows, NT, 0, st>>>(scores, n_stride, qr, m, k, out);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 int topk_max_entries() { return kMaxEntries; }
@@ -359,15 +231,22 @@ cudaError_t launch_topk(const float* scores, int n_stride, QueryRows qr, int m, 
                         int k, int32_t* out, cudaStream_t st) {
   if (nrows == 0) return cudaSuccess;
   if (n_stride > kMaxEntries) return cudaErrorInvalidValue;
-  // rows that fit in registers: block size and keys per thread by the longest row
-  if (n_stride <= 2048) return topk_reg<256, 8>(scores, n_stride, qr, m, nrows, k, out, st);
-  if (n_stride <= 8192) return topk_reg<512, 16>(scores, n_stride, qr, m, nrows, k, out, st);
-  if (n_stride <= 16384) return topk_reg<512, 32>(scores, n_stride, qr, m, nrows, k, out, st);
-  if (n_stride <= 32768) return topk_reg<1024, 32>(scores, n_stride, qr, m, nrows, k, out, st);
-  const size_t smem = sizeof(Shared) + sizeof(uint32_t) * (size_t)(n_stride > 0 ? n_stride : 1);
-  cudaError_t err = ensure_smem_limit((const void*)topk_smem_kernel, (int)smem);
-  if (err != cudaSuccess) return err;
-  topk_smem_kernel<<<(unsigned)nrows, kThreads, smem, st>>>(scores, n_stride, qr, m, k, out);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // keys in shared memory for short rows, and for launches with too few rows to fill the GPU
+  // several times over (there the per-row latency of the L2 re-reads would dominate)
+  const bool smem_keys = n_stride <= kSmemKeyRows || (nrows <= 4 * (int64_t)sms &&
+                                                       n_stride <= kSmemKeyLimit);
+  if (smem_keys) {
+    const size_t smem = sizeof(Shared) + sizeof(uint32_t) * (size_t)(n_stride > 0 ? n_stride : 1);
+    cudaError_t err = ensure_smem_limit((const void*)topk_kernel<true>, (int)smem);
+    if (err != cudaSuccess) return err;
+    topk_kernel<true><<<(unsigned)nrows, kThreads, smem, st>>>(scores, n_stride, qr, m, k, out);
+  } else {
+    topk_kernel<false><<<(unsigned)nrows, kThreads, sizeof(Shared), st>>>(scores, n_stride, qr, m,
+                                                                         k, out);
+  }
   return cudaGetLastError();
 }
 

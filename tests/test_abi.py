@@ -68,7 +68,7 @@ def test_workspace_sizes():
 @pytest.mark.parametrize("bad,code", [
     (dict(D=96), -2), (dict(D=1024), -2), (dict(R=63), -2), (dict(R=66 * 2), -2),
     (dict(dtype="f16"), None), (dict(S=0), -1), (dict(H=0), -1), (dict(sliding_window=0), -1),
-    (dict(idx_dim=48), -2), (dict(topk=0), -1), (dict(m=0), -1), (dict(S=4 * 60000), -2),
+    (dict(idx_dim=48), -2), (dict(topk=0), -1), (dict(m=0), -1), (dict(S=4 * (1 << 22) + 4), -2),
     (dict(softmax_scale=-1.0), -1), (dict(rope_theta=0.0), -1),
 ])
 def test_invalid_params_rejected_on_host(bad, code):
