@@ -115,6 +115,15 @@ class ClockSampler:
                 self.proc.kill()
             self.thread.join(timeout=2)
 
+    def wait_samples(self, n: int, keep_busy, limit_s: float = 5.0):
+        """Keep the GPU busy with keep_busy() (untimed) until n samples have been read, so that
+        a timed region shorter than the sampling period still has samples taken under the same
+        load right before and after it."""
+        t0 = time.time()
+        while self.proc is not None and len(self.lines) < n and time.time() - t0 < limit_s:
+            keep_busy()
+            torch.cuda.synchronize()
+
     def summary(self):
         sm, mx, reasons = [], [], set()
         for line in self.lines:
@@ -132,7 +141,9 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window": "200 ms samples while step replays run back to back, the timed "
+                          "region included"}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -376,7 +387,9 @@ def run_ours(args, wl0):
     graph.replay()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clk:
+        clk.wait_samples(1, graph.replay)
         ms = timed(graph.replay, args.steps, dev)
+        clk.wait_samples(len(clk.lines) + 1, graph.replay)
     ktimes = sac.sac_timing_end()  # per kernel: the last replay, i.e. one step
     ms = max_over_ranks(ms, dev)
     ms_step = ms / args.steps
@@ -499,7 +512,9 @@ def run_decode(args, wl0):
     graph.replay()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clk:
+        clk.wait_samples(1, graph.replay)
         ms = timed_flushed(graph.replay, args.steps, dev)
+        clk.wait_samples(len(clk.lines) + 1, graph.replay)
     ktimes = sac.sac_timing_end()  # per kernel: the last replay, i.e. one step
     ms = max_over_ranks(ms, dev)
     us_step = 1e3 * ms / args.steps

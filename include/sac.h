@@ -177,9 +177,13 @@ SAC_API int csa_forward(const sac_params* p, const void* q, const void* kv, cons
  *   q [nseq,H,D] un-rotated; o [nseq,H,D]; q_idx [nseq,nI,cI], w_idx [nseq,nI] fp32 (CSA);
  *   topk_out [nseq,k] nullable (ascending entries, -1 fill).
  * Workspace: sac_decode_workspace_size() bytes, 16-byte aligned: a 256-byte status word (see
- * sac_device_status) and, for CSA, the scores [nseq, S/m] fp32 and the selection [nseq, k]. ws is
- * required by csa_decode; swa_decode / hca_decode accept NULL (no status word is then kept) or at
- * least 256 bytes. Entries on an unallocated page (block table entry < 0) read as zero keys.
+ * sac_device_status); for CSA the scores [nseq, S/m] fp32 and the selection [nseq, k]; and, for
+ * bf16 layers with 64 heads of 512 when nseq is below the device's SM count, fp32 partial results
+ * that let each sequence's keys be split over several CTAs (nseq * splits * H * (D + 2) floats,
+ * splits = min(8, SMs / nseq)). ws is required by csa_decode; swa_decode / hca_decode accept NULL
+ * (no status word, no split) or any size of at least 256 bytes (the split is used only when the
+ * workspace holds its buffers). Entries on an unallocated page (block table entry < 0) read as
+ * zero keys.
  */
 SAC_API size_t sac_decode_workspace_size(const sac_params* p, int kind, int nseq);
 

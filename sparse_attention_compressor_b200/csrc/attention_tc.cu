@@ -11,8 +11,8 @@
 // groups that take alternate tiles. Tiles never mix window rows and entries.
 //
 // QK^T of a tile is 32 MMAs of K=16. Accumulating them into one TMEM tile would chain each MMA
-// on its predecessor, so they rotate over four partial accumulators and the softmax adds the
-// four partials.
+// on its predecessor, so they rotate over four partial accumulators (one per issuing thread) and
+// the softmax adds the four partials.
 //
 // The query tile arrives un-rotated; one warp turns its rope slice in shared memory before the
 // first QK^T of the row, so no rotated copy of q is written to HBM.
@@ -23,13 +23,13 @@
 // (buffer 0) and 352 (buffer 1). A softmax thread of lane i < 16 and its partner i + 16 own the
 // same head: they add their partials, exchange halves, and each finishes 24 of the 48 keys.
 //
-// Warps: 0 = TMA thread, 1-2 = QK^T issuers (warp 1 also owns TMEM), 3 = query rotation, 4-5 / 6-7
-// = gather groups (even / odd tiles), 8-11 = softmax + output, 12 = PV issuer. Each tcgen05.mma
-// costs its issuing thread a fixed time, so two threads issue QK^T (warp 1 the even partials,
-// warp 2 the odd ones) and a third issues PV the moment P is written, instead of after the next
-// tile's QK^T. An M = 64 MMA occupies one 16-lane half of each TMEM sub-partition, and MMAs into
-// opposite halves run side by side: the two QK^T issuers' partials, and the two halves of O, sit
-// in opposite lane halves. The softmax keeps the running max in log2 units and moves it
+// Warps: 0 = TMA thread, 1-2 = QK^T issuers (warp 1 also owns TMEM), 3 = query rotation, 4-7 =
+// gather (one 128-thread group per tile; idle when every tile arrives by TMA), 8-11 = softmax +
+// output, 12 = PV issuer. Each tcgen05.mma costs its issuing thread a fixed time, so two threads
+// issue QK^T and a third issues PV the moment P is written, instead of after the next tile's
+// QK^T. An M = 64 MMA occupies one 16-lane half of each TMEM sub-partition, and MMAs into
+// opposite halves run side by side: the QK^T partials alternate between the lane halves, and the
+// two halves of O sit in opposite lane halves. The softmax keeps the running max in log2 units and moves it
 // (rescaling O) only when a tile's max exceeds it by more than 8.
 #include <cuda_bf16.h>
 
@@ -51,7 +51,8 @@ constexpr int kKRegion = kNK * 128;              // [48 rows x 128 B]
 constexpr int kQBytes = 8 * kQRegion;            // 64 KB
 constexpr int kTileBytes = 8 * kKRegion;         // 48 KB
 constexpr int kPBytes = kHeads * 128;            // 64 rows x 128 B (48 keys used)
-constexpr int kGroupThreads = 64;                // threads of one gather group
+constexpr int kGatherGroups = 1;                 // producer groups taking tiles in turn
+constexpr int kGroupThreads = 128 / kGatherGroups; // threads of one gather group (warps 4-7)
 constexpr int kThreads = 416;
 
 constexpr int kOffQ = 0;
@@ -68,7 +69,9 @@ constexpr int kSmemBytes = kOffTmemPtr + 16;
 constexpr uint32_t kColS = 256, kSStride = 2 * kNK;  // S buffer s at kColS + s * kSStride
 constexpr uint32_t kIdescQK = tc::idesc_bf16(64, kNK, false, false);
 constexpr uint32_t kIdescPV = tc::idesc_bf16(64, 256, false, true);
-constexpr int kRopeK2 = 14;  // K-step pairs 14,15 (K-steps 28..31) read the last region of Q
+constexpr int kMaxSplits = 8;  // key-tile splits of one row (decode: few rows, many SMs)
+constexpr int kQkIssuers = 2;  // threads issuing QK^T (measured faster than 4 and than 1)
+constexpr int kRopeStep = 28;  // K-steps 28..31 read the last region of Q (the rope slice)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;  // move the running max only when a tile exceeds it by 2^8
 
@@ -76,6 +79,9 @@ struct Row {
   int seq;
   int64_t t, lo;
   int nwin, npool, twin, tiles;
+  int64_t r;   // query row of the work item
+  int sp;      // split of the row's key tiles this item covers
+  int j0, j1;  // tile range [j0, j1) of the item
 };
 
 __device__ __forceinline__ Row locate_row(const AttnArgs& a, int64_t r) {
@@ -90,6 +96,21 @@ __device__ __forceinline__ Row locate_row(const AttnArgs& a, int64_t r) {
   return w;
 }
 
+// Work item it = (row, split): the row's key tiles are divided into a.splits contiguous ranges
+// (a.splits = 1: one item per row, all tiles). Items with an empty range are skipped by every role.
+template <bool kSplit>
+__device__ __forceinline__ Row locate_item(const AttnArgs& a, int64_t it) {
+  const int splits = kSplit ? a.splits : 1;
+  const int64_t r = kSplit ? it / splits : it;
+  const int sp = kSplit ? (int)(it % splits) : 0;
+  Row w = locate_row(a, r);
+  w.r = r;
+  w.sp = sp;
+  w.j0 = kSplit ? (int)((int64_t)w.tiles * sp / splits) : 0;
+  w.j1 = kSplit ? (int)((int64_t)w.tiles * (sp + 1) / splits) : w.tiles;
+  return w;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
   __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -97,6 +118,29 @@ __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
   return __bfloat1622float2(v);
+}
+
+// QK^T K-steps kk = ME (mod NQK) of one tile (fully unrolled, every offset a constant: the issue
+// cost per MMA is what bounds this loop). K-step kk accumulates into partial p = kk & 3 at lanes
+// 16 (p & 1), columns + 48 (p >> 1) of the S buffer at d0. With qready set (a query's first tile)
+// the K-steps of the rope region wait until the query's rope slice has been rotated.
+template <int NQK, int ME>
+__device__ __forceinline__ bool issue_qk(uint32_t d0, uint64_t qd, uint64_t kd, uint64_t* qready,
+                                         uint32_t qparity, int* status) {
+#pragma unroll
+  for (int i = 0; i < kDim / 16 / NQK; ++i) {
+    const int kk = NQK * i + ME;
+    if (kk >= kRopeStep && kk - NQK < kRopeStep && qready != nullptr) {
+      if (!tc::mbar_wait(qready, qparity, status)) return false;
+      tc::tc_fence_after();
+    }
+    const int p = kk & 3;
+    const uint32_t dp = d0 + ((p & 1) ? (16u << 16) : 0u) + ((p & 2) ? (uint32_t)kNK : 0u);
+    const uint32_t qo = ((kk >> 2) * kQRegion + (kk & 3) * 32) >> 4;
+    const uint32_t ko = ((kk >> 2) * kKRegion + (kk & 3) * 32) >> 4;
+    tc::mma_bf16_ss(dp, qd + qo, kd + ko, kIdescQK, kk >= 4 ? 1u : 0u);
+  }
+  return true;
 }
 
 // Global address of key c of tile j (keys past the tile's count reuse a valid row: masked).
@@ -115,15 +159,7 @@ __device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const
   return p ? p : reinterpret_cast<const __nv_bfloat16*>(a.pool.base);
 }
 
-// Hint: bring a query's 64 KB of rows into L2 ahead of its TMA load (eight 8 KB bulk prefetches).
-__device__ __forceinline__ void prefetch_query_l2(const void* q) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], 8192;" ::"l"(
-                     reinterpret_cast<uint64_t>(q) + (uint64_t)i * 8192)
-                 : "memory");
-}
-
+template <bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_win_box,
@@ -139,20 +175,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
+  // window rows of a prefill are consecutive rows of the rotated kv stream, and so are the
+  // entries of an HCA prefill: those tiles load as TMA boxes; the rest are gathered
+  const bool win_contig = a.win.block_table == nullptr;
+  const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
+  const bool any_gather = !win_contig || (a.pool_mode != 0 && !pool_contig);
+  const int64_t n_items = kSplit ? a.nrows * a.splits : a.nrows;
+  // Who issues PV: with gathered tiles the gather latency decides, and a separate thread issues
+  // PV the moment P is ready so that tile buffers free early; with TMA-fed tiles QK^T is the
+  // critical step, and the QK^T threads issue PV right after the next tile's QK^T (measured: 17%
+  // faster at HCA-32k, slower at CSA-8k).
+  const bool pv_by_qk = !any_gather;
+  const uint32_t pv_commits = pv_by_qk ? kQkIssuers : 1;
+
   if (threadIdx.x == 0) {
     tc::mbar_init(&bar[kQFull], 1);
     tc::mbar_init(&bar[kQReady], 32);
-    tc::mbar_init(&bar[kQEmpty], 2);
+    tc::mbar_init(&bar[kQEmpty], kQkIssuers);
     for (int i = 0; i < kStages; ++i) {
-      tc::mbar_init(&bar[kKvFull0 + i], 1 + kGroupThreads);  // TMA thread + one gather group
-      tc::mbar_init(&bar[kKvEmpty0 + i], 1);
+      // TMA thread (+ one gather group when some tiles are gathered)
+      tc::mbar_init(&bar[kKvFull0 + i], any_gather ? 1 + kGroupThreads : 1);
+      tc::mbar_init(&bar[kKvEmpty0 + i], pv_commits);
     }
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bar[kSFull0 + i], 2);
+      tc::mbar_init(&bar[kSFull0 + i], kQkIssuers);
       tc::mbar_init(&bar[kPFull0 + i], 128);
-      tc::mbar_init(&bar[kPvDone0 + i], 1);
+      tc::mbar_init(&bar[kPvDone0 + i], pv_commits);
     }
-    tc::mbar_init(&bar[kOFull], 1);
+    tc::mbar_init(&bar[kOFull], pv_commits);
     tc::mbar_init(&bar[kOEmpty], 128);
     tc::fence_barrier_init();
   }
@@ -166,28 +216,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  // window rows of a prefill are consecutive rows of the rotated kv stream, and so are the
-  // entries of an HCA prefill: those tiles load as TMA boxes; the rest are gathered
-  const bool win_contig = a.win.block_table == nullptr;
-  const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA thread
     if (lane == 0) {
       uint32_t g = 0, qi = 0;
       bool ok = true;
-      for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
-        const Row w = locate_row(a, r);
-        if (r + gridDim.x < a.nrows)  // the CTA's next query, loaded by TMA one query later
-          prefetch_query_l2(reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                            (r + gridDim.x) * kHeads * kDim);
+      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Row w = locate_item<kSplit>(a, it);
+        if (w.j0 == w.j1) continue;
+        const int64_t r = w.r;
         if (qi > 0) ok = tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status);
         if (!ok) break;
         tc::mbar_arrive_expect_tx(&bar[kQFull], kQBytes);
         for (int c = 0; c < 8; ++c)
           tc::tma_load_2d(smem + kOffQ + c * kQRegion, &tm_q, &bar[kQFull], 64 * c,
                           (int32_t)(r * kHeads));
-        for (int j = 0; j < w.tiles && ok; ++j, ++g) {
+        for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
           const uint32_t b = g % kStages;
           if (g >= kStages) ok = tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - kStages) / kStages) & 1,
                                                status);
@@ -206,24 +251,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_arrive(&bar[kKvFull0 + b]);
           }
         }
+        ++qi;
       }
     }
     __syncwarp();
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------------ QK^T issuers
-    const uint32_t me = warp - 1;  // 0: even partials (lanes 0-15); 1: odd partials (lanes 16-31)
+    // issuer me takes the K-steps kk = me (mod 2); K-step kk accumulates into partial p = kk & 3,
+    // which sits in lanes 16 (p & 1), columns + 48 (p >> 1) of the S buffer
+    const uint32_t me = warp - 1;
     if (lane == 0) {
       uint32_t g0 = 0, qi = 0;
       bool ok = true;
       const uint64_t qd = tc::desc_sw128(tc::smem_u32(smem + kOffQ), 0, 1024);
-      for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
-        const Row w = locate_row(a, r);
+      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Row w = locate_item<kSplit>(a, it);
+        if (w.j0 == w.j1) continue;
         // the query tile has landed; its rope region (the last 128-byte column, K-steps 28..31)
         // is still being rotated, so the first QK^T waits for kQReady only before those steps
         ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
-        for (int j = 0; j < w.tiles && ok; ++j) {
-          {  // S(g) = Q K^T over four partial accumulators
-            const uint32_t g = g0 + j, b = g % kStages, s = g & 1;
+        for (int j = w.j0; j < w.j1 + (pv_by_qk ? 1 : 0) && ok; ++j) {
+          if (j < w.j1) {  // S(g) = Q K^T over four partial accumulators
+            const uint32_t g = g0 + (j - w.j0), b = g % kStages, s = g & 1;
             ok = tc::mbar_wait(&bar[kKvFull0 + b], (g / kStages) & 1, status);
             if (ok && g >= 2) ok = tc::mbar_wait(&bar[kPFull0 + s], ((g - 2) >> 1) & 1, status);
             if (!ok) break;
@@ -233,28 +282,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d0 = tmem + kColS + s * kSStride;
             // the descriptor's start-address field counts 16-byte units: advancing along K adds
             // the byte offset >> 4 to the base descriptor
-            // partial p = kk & 3 lives in lanes 16*(p&1), columns + (p>>1)*48; this issuer owns
-            // the partials with (p & 1) == me
-            const uint32_t dme = d0 + (me ? (16u << 16) : 0u);
-#pragma unroll
-            for (int k2 = 0; k2 < kDim / 32; ++k2) {
-              const int kk0 = 2 * k2 + (int)me;  // kk0 & 1 == me
-              if (k2 == kRopeK2 && j == 0) {
-                ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
-                if (!ok) break;
-                tc::tc_fence_after();
-              }
-              const uint32_t qo = ((kk0 >> 2) * kQRegion + (kk0 & 3) * 32) >> 4;
-              const uint32_t ko = ((kk0 >> 2) * kKRegion + (kk0 & 3) * 32) >> 4;
-              tc::mma_bf16_ss(dme + ((kk0 & 2) ? (uint32_t)kNK : 0u), qd + qo, kd + ko, kIdescQK,
-                              kk0 >= 4);
-            }
+            uint64_t* qready = j == w.j0 ? &bar[kQReady] : nullptr;
+            ok = me == 0 ? issue_qk<kQkIssuers, 0>(d0, qd, kd, qready, qi & 1, status)
+                         : issue_qk<kQkIssuers, 1>(d0, qd, kd, qready, qi & 1, status);
             if (!ok) break;
             tc::mma_commit(&bar[kSFull0 + s]);
-            if (j == w.tiles - 1) tc::mma_commit(&bar[kQEmpty]);
+            if (j == w.j1 - 1) tc::mma_commit(&bar[kQEmpty]);
+          }
+          if (pv_by_qk && j > w.j0) {  // O[:, 256 me : 256 me + 256] += P(g) V(g), after QK^T(g+1)
+            const uint32_t g = g0 + (j - 1 - w.j0), b = g % kStages, s = g & 1;
+            ok = tc::mbar_wait(&bar[kPFull0 + s], (g >> 1) & 1, status);
+            if (ok && j - 1 == w.j0 && qi > 0)
+              ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
+            if (!ok) break;
+            tc::tc_fence_after();
+            const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
+            const uint64_t pd = tc::desc_sw128(tc::smem_u32(smem + kOffP + s * kPBytes), 0, 1024);
+            const uint64_t vd = tc::desc_sw128(v_base + me * 4 * kKRegion, kKRegion, 1024);
+            const uint32_t od = tmem + (me ? (16u << 16) : 0u);
+#pragma unroll
+            for (int kk = 0; kk < kNK / 16; ++kk)
+              tc::mma_bf16_ss(od, pd + kk * 2, vd + kk * 128, kIdescPV,
+                              (j - 1 > w.j0 || kk > 0) ? 1u : 0u);
+            tc::mma_commit(&bar[kKvEmpty0 + b]);
+            tc::mma_commit(&bar[kPvDone0 + s]);
+            if (j == w.j1) tc::mma_commit(&bar[kOFull]);
           }
         }
-        g0 += w.tiles;
+        g0 += w.j1 - w.j0;
+        ++qi;
       }
     }
     __syncwarp();
@@ -270,10 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float2* cs_tab = reinterpret_cast<float2*>(smem + kOffCs);
     uint32_t qi = 0;
     bool ok = true;
-    for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
-      int seq;
-      int64_t t;
-      a.qr.locate(a.qr.row0 + r, seq, t);
+    for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const Row w = locate_item<kSplit>(a, it);
+      if (w.j0 == w.j1) continue;
+      const int64_t t = w.t;
       if (lane < R / 2) {
         float c, sn;
         rope_cos_sin(a.rf, lane, a.pos0 + t, c, sn);
@@ -330,18 +386,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bar[kQReady]);
+      ++qi;
     }
   } else if (warp < 8) {
+    if (!any_gather) goto done;  // every tile arrives by TMA
     // ------------------------------------------------------------------ gather groups
-    // group 0 (warps 4-5) fills even tiles, group 1 (warps 6-7) odd tiles. Thread t copies rows
-    // t/8, t/8 + 8, ..., t/8 + 40 of the tile; for each it copies 16-byte slot t%8 of all 8
-    // regions, so a warp instruction reads four whole 128-byte row segments and a thread needs
-    // only six row addresses. Once its copies landed it makes them visible to the tensor core
-    // and arrives on the tile's barrier.
-    const int grp = (warp - 4) >> 1;
-    const int gt = (warp & 1) * 32 + lane;    // 0..63
+    // Warps 4-7 form kGatherGroups groups that take the gathered tiles in turn. Thread t of a
+    // group of G threads copies rows t/8, t/8 + G/8, ... of the tile; for each it copies 16-byte
+    // slot t%8 of all 8 regions, so a warp instruction reads four whole 128-byte row segments and
+    // a thread needs only a few row addresses. Once its copies landed it makes them visible to
+    // the tensor core and arrives on the tile's barrier.
+    constexpr int kWarpsPer = 4 / kGatherGroups;
+    const int grp = (warp - 4) / kWarpsPer;
+    const int gt = ((warp - 4) % kWarpsPer) * 32 + lane;  // thread within the group
     const int row0 = gt >> 3, slot = gt & 7;
-    constexpr int kRowsPer = kNK / 8;         // 6
+    constexpr int kRowStride = kGroupThreads / 8;        // rows a group covers per pass
+    constexpr int kRowsPer = kNK / kRowStride;
     // Walk this group's tiles in order across the CTA's query rows. The source rows of the next
     // tile are resolved while the current tile's copies are in flight, so the selection-index
     // loads do not add to each tile's latency.
@@ -351,34 +411,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       int j;
       uint32_t g;
     };
-    auto valid = [&](const Cursor& c) { return c.r < a.nrows; };
+    auto valid = [&](const Cursor& c) { return c.r < n_items; };  // c.r: the work item
     auto gathered = [&](const Cursor& c) {
       return !(c.j < c.w.twin ? win_contig : pool_contig);
+    };
+    auto first_tile = [&](Cursor& c) {  // c.r: the first non-empty item from c.r on
+      for (; c.r < n_items; c.r += gridDim.x) {
+        c.w = locate_item<kSplit>(a, c.r);
+        if (c.w.j0 < c.w.j1) break;
+      }
+      c.j = c.r < n_items ? c.w.j0 : 0;
     };
     auto advance = [&](Cursor c) {  // next tile of this group after c
       do {
         ++c.g;
-        if (++c.j >= c.w.tiles) {
+        if (++c.j >= c.w.j1) {
           c.r += gridDim.x;
-          c.j = 0;
-          if (c.r >= a.nrows) return c;
-          c.w = locate_row(a, c.r);
+          first_tile(c);
+          if (c.r >= n_items) return c;
         }
-      } while ((int)(c.g & 1) != grp);
+      } while ((int)(c.g % kGatherGroups) != grp);
       return c;
     };
     auto resolve = [&](const Cursor& c, const __nv_bfloat16* (&src)[kRowsPer]) {
 #pragma unroll
-      for (int i = 0; i < kRowsPer; ++i) src[i] = key_ptr(a, c.w, c.r, c.j, row0 + 8 * i);
+      for (int i = 0; i < kRowsPer; ++i) src[i] = key_ptr(a, c.w, c.w.r, c.j, row0 + kRowStride * i);
     };
     Cursor c;
     c.r = blockIdx.x;
-    c.j = 0;
     c.g = 0;
-    if (valid(c)) {
-      c.w = locate_row(a, c.r);
-      if (grp == 1) c = advance(c);
-    }
+    first_tile(c);
+    if (valid(c))
+      for (int i = 0; i < grp; ++i) c = advance(c);
     const __nv_bfloat16* src[kRowsPer];
     if (valid(c) && gathered(c)) resolve(c, src);
     bool ok = true;
@@ -393,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* tile = smem + kOffTile + b * kTileBytes;
 #pragma unroll
         for (int i = 0; i < kRowsPer; ++i) {
-          const int row = row0 + 8 * i;
+          const int row = row0 + kRowStride * i;
           uint8_t* d = tile + row * 128 + ((slot ^ (row & 7)) << 4);
 #pragma unroll
           for (int q = 0; q < 8; ++q) tc::cp_async16(d + q * kKRegion, src[i] + q * 64 + slot * 8);
@@ -413,15 +477,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // O += P(g) V(g) as soon as the softmax has written P(g), independent of how far the QK^T
     // issuers have got: O[:, 0:256] accumulates in lanes 0-15 and O[:, 256:512] in lanes 16-31,
     // and the two halves' MMAs alternate so both lane halves of the tensor core stay busy.
-    if (lane == 0) {
+    if (lane == 0 && !pv_by_qk) {
       uint32_t g0 = 0, qi = 0;
       bool ok = true;
-      for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
-        const Row w = locate_row(a, r);
-        for (int j = 0; j < w.tiles && ok; ++j) {
-          const uint32_t g = g0 + j, b = g % kStages, s = g & 1;
+      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Row w = locate_item<kSplit>(a, it);
+        if (w.j0 == w.j1) continue;
+        for (int j = w.j0; j < w.j1 && ok; ++j) {
+          const uint32_t g = g0 + (j - w.j0), b = g % kStages, s = g & 1;
           ok = tc::mbar_wait(&bar[kPFull0 + s], (g >> 1) & 1, status);
-          if (ok && j == 0 && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
+          if (ok && j == w.j0 && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
           if (!ok) break;
           tc::tc_fence_after();
           const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
@@ -430,15 +495,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t vd1 = tc::desc_sw128(v_base + 4 * kKRegion, kKRegion, 1024);
 #pragma unroll
           for (int kk = 0; kk < kNK / 16; ++kk) {
-            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (j > w.j0 || kk > 0) ? 1u : 0u;
             tc::mma_bf16_ss(tmem, pd + kk * 2, vd0 + kk * 128, kIdescPV, acc);
             tc::mma_bf16_ss(tmem + (16u << 16), pd + kk * 2, vd1 + kk * 128, kIdescPV, acc);
           }
           tc::mma_commit(&bar[kKvEmpty0 + b]);
           tc::mma_commit(&bar[kPvDone0 + s]);
-          if (j == w.tiles - 1) tc::mma_commit(&bar[kOFull]);
+          if (j == w.j1 - 1) tc::mma_commit(&bar[kOFull]);
         }
-        g0 += w.tiles;
+        g0 += w.j1 - w.j0;
+        ++qi;
       }
     }
     __syncwarp();
@@ -452,11 +518,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sink_log2 = __ldg(a.sinks + h) * kLog2e;
     uint32_t g0 = 0, qi = 0;
     bool ok = true;
-    for (int64_t r = blockIdx.x; r < a.nrows && ok; r += gridDim.x, ++qi) {
-      const Row w = locate_row(a, r);
-      float m_run = sink_log2, l_run = 1.f;
-      for (int j = 0; j < w.tiles && ok; ++j) {
-        const uint32_t g = g0 + j, s = g & 1;
+    for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const Row w = locate_item<kSplit>(a, it);
+      if (w.j0 == w.j1) continue;
+      const int64_t r = w.r;
+      // the sink (logit s_h, zero value) is one more term of the normaliser: here, or in the
+      // combine kernel when the row's keys are split
+      float m_run = kSplit ? -INFINITY : sink_log2, l_run = kSplit ? 0.f : 1.f;
+      for (int j = w.j0; j < w.j1 && ok; ++j) {
+        const uint32_t g = g0 + (j - w.j0), s = g & 1;
         ok = __all_sync(~0u, tc::mbar_wait(&bar[kSFull0 + s], (g >> 1) & 1, status));
         if (!ok) break;
         tc::tc_fence_after();
@@ -495,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = move ? mx : m_run;
         const float alpha = exp2f(m_run - m_new);
         // rescale the rows of O this warp owns (rare: only when some row's max moved)
-        if (__any_sync(~0u, move) && j > 0) {
+        if (__any_sync(~0u, move) && j > w.j0) {
           const uint32_t gp = g - 1;
           ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + (gp & 1)], (gp >> 1) & 1, status));
           if (!ok) break;
@@ -538,6 +608,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_arrive(&bar[kPFull0 + s]);
       }
       if (!ok) break;
+      if (kSplit) {
+        // ---- split output: this item's O (relative to its running max), max and normaliser in
+        // fp32 for the combine kernel
+        ok = __all_sync(~0u, tc::mbar_wait(&bar[kOFull], qi & 1, status));
+        if (!ok) break;
+        tc::tc_fence_after();
+        float* po = a.part_o + ((int64_t)it * kHeads + h) * kDim + half * 256;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 256; c0 += 64) {
+          uint32_t v[4][16];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tc::tmem_ld16(t_row + c0 + 16 * q, v[q]);
+          tc::tmem_wait_ld();
+          if (c0 + 64 == 256) {
+            tc::tc_fence_before();
+            tc::mbar_arrive(&bar[kOEmpty]);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              *reinterpret_cast<float4*>(po + c0 + 16 * q + e) =
+                  make_float4(__uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]),
+                              __uint_as_float(v[q][e + 2]), __uint_as_float(v[q][e + 3]));
+        }
+        if (half == 0)
+          *reinterpret_cast<float2*>(a.part_ml + ((int64_t)it * kHeads + h) * 2) =
+              make_float2(m_run, l_run);
+        g0 += w.j1 - w.j0;
+        ++qi;
+        continue;
+      }
       // ---- output: O / l, the rope slice turned by -P_t, bf16 store. Lane p holds the cos/sin
       // of rope pair p; the rotation reads them with warp shuffles.
       const int64_t P = a.pos0 + w.t;
@@ -588,9 +690,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           reinterpret_cast<uint4*>(orow + c)[1] = o1;
         }
       }
-      g0 += w.tiles;
+      g0 += w.j1 - w.j0;
+      ++qi;
     }
   }
+done:
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -599,7 +703,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Combine the splits of each row: O = sum_s 2^(m_s - M) O_s / (2^(sink - M) + sum_s 2^(m_s - M) l_s)
+// with M = max(sink, max_s m_s) over the non-empty splits (all in log2 units), then the rope
+// slice turned by -P_t and the bf16 store. One block per row; thread (h, quarter) owns head h's
+// channels [128 quarter, 128 quarter + 128).
+__global__ void __launch_bounds__(256) attention_combine_kernel(AttnArgs a) {
+  const int64_t r = blockIdx.x;
+  const int h = threadIdx.x >> 2, quarter = threadIdx.x & 3;
+  const Row w = locate_row(a, r);
+  float wgt[kMaxSplits];
+  const float sink = __ldg(a.sinks + h) * kLog2e;
+  float M = sink;
+  for (int sp = 0; sp < a.splits; ++sp) {
+    const bool nonempty = (int64_t)w.tiles * sp / a.splits < (int64_t)w.tiles * (sp + 1) / a.splits;
+    wgt[sp] = nonempty ? a.part_ml[((r * a.splits + sp) * kHeads + h) * 2] : -INFINITY;
+    M = fmaxf(M, wgt[sp]);
+  }
+  float L = exp2f(sink - M);
+  for (int sp = 0; sp < a.splits; ++sp) {
+    const float m = wgt[sp];
+    wgt[sp] = m == -INFINITY ? 0.f : exp2f(m - M);
+    if (wgt[sp] > 0.f) L += wgt[sp] * a.part_ml[((r * a.splits + sp) * kHeads + h) * 2 + 1];
+  }
+  const float inv_l = 1.f / L;
+  const int64_t P = a.pos0 + w.t;
+  const int rope_lo = kDim - a.rf.R;
+  __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (r * kHeads + h) * kDim;
+#pragma unroll 1
+  for (int c = quarter * 128; c < quarter * 128 + 128; c += 8) {
+    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int sp = 0; sp < a.splits; ++sp) {
+      if (wgt[sp] == 0.f) continue;
+      const float* po = a.part_o + ((r * a.splits + sp) * kHeads + h) * kDim + c;
+      const float4 u0 = *reinterpret_cast<const float4*>(po);
+      const float4 u1 = *reinterpret_cast<const float4*>(po + 4);
+      x[0] = fmaf(wgt[sp], u0.x, x[0]); x[1] = fmaf(wgt[sp], u0.y, x[1]);
+      x[2] = fmaf(wgt[sp], u0.z, x[2]); x[3] = fmaf(wgt[sp], u0.w, x[3]);
+      x[4] = fmaf(wgt[sp], u1.x, x[4]); x[5] = fmaf(wgt[sp], u1.y, x[5]);
+      x[6] = fmaf(wgt[sp], u1.z, x[6]); x[7] = fmaf(wgt[sp], u1.w, x[7]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      float x0 = x[e] * inv_l, x1 = x[e + 1] * inv_l;
+      if (c + e >= rope_lo) {
+        float cc, ss;
+        rope_cos_sin(a.rf, (c + e - rope_lo) >> 1, -P, cc, ss);
+        const float y0 = x0 * cc - x1 * ss, y1 = x0 * ss + x1 * cc;
+        x0 = y0;
+        x1 = y1;
+      }
+      x[e] = x0;
+      x[e + 1] = x1;
+    }
+    *reinterpret_cast<uint4*>(orow + c) = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                                     pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+  }
+}
+
 }  // namespace
+
+int attention_tc_max_splits() { return kMaxSplits; }
 
 bool attention_tc_supported(const AttnArgs& a, int dtype) {
   return dtype == 1 && a.H == kHeads && a.D == kDim && a.rf.R <= 64 && a.rf.R % 2 == 0;
@@ -617,13 +780,23 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
   e = make_tmap_bf16_2d(&tpb, has_pool ? a.pool.base : a.win.base,
                         (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
-  e = ensure_smem_limit((const void*)attention_tc_kernel, kSmemBytes);
+  e = ensure_smem_limit(a.splits > 1 ? (const void*)attention_tc_kernel<true>
+                                     : (const void*)attention_tc_kernel<false>, kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = (int)(a.nrows < sms ? a.nrows : sms);
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
+  if (a.splits < 1 || a.splits > kMaxSplits || (a.splits > 1 && (!a.part_o || !a.part_ml)))
+    return cudaErrorInvalidValue;
+  const int64_t items = a.nrows * a.splits;
+  const int grid = (int)(items < sms ? items : sms);
+  if (a.splits > 1)
+    attention_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
+  else
+    attention_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.splits == 1) return e;
+  attention_combine_kernel<<<(unsigned)a.nrows, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -13,7 +13,8 @@
 // counter of its own.
 //
 // One block of 8 warps per sequence: warp 0 writes the new row; on a closing window the warps
-// split the window's rows (all 8 for L >= 64, else warp 0 alone) and merge in shared memory.
+// split the window's rows (all 8 for L >= 64, else warp 0 alone) and merge in shared memory. The
+// pooling reads the new token's row from its input rather than back from the ring.
 #include "pool_window.cuh"
 #include "sac_kernels.h"
 
@@ -54,10 +55,12 @@ __global__ void __launch_bounds__(256) append_kernel(AppendPart a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = (int64_t)__ldg(a.ctx_lens + seq) - 1;
   if (t < 0) return;
+  const T* x_new = reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * C;
   T* ring = a.m > 0 ? reinterpret_cast<T*>(a.ring) + (int64_t)seq * a.L * C : nullptr;
+  const bool closing = a.m > 0 && (t + 1) % a.m == 0;
   if (warp == 0) {
     float v[V];
-    load_lane<T, V>(reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * C, lane, v);
+    load_lane<T, V>(x_new, lane, v);
     if (ring) store_lane<T, V>(ring + (t % a.L) * C, lane, v);
     if (a.kv_pages) {
       T* dst = page_row<T>(a.kv_pages, a.kv_bt, a.kv_max_pages, a.page_size, C, seq, t);
@@ -67,17 +70,20 @@ __global__ void __launch_bounds__(256) append_kernel(AppendPart a) {
       }
     }
   }
-  if (a.m == 0 || (t + 1) % a.m != 0) return;
-  __syncthreads();  // the new ring row is read by every warp below
+  if (!closing) return;
 
+  // The closing window's rows: the new token's row straight from its input, the older ones from
+  // the ring (written by earlier calls), so the pooling needs no barrier after the ring write and
+  // all of its loads start at once.
   const int64_t w = (t + 1) / a.m - 1;
   const int64_t hi = (w + 1) * a.m;
   const int64_t lo = hi - a.L < 0 ? 0 : hi - a.L;
   float u[V], acc[V];
   load_lane<T, V>(reinterpret_cast<const T*>(a.gate), lane, u);
   const int L = a.L;
-  pool_window<T, V, WPE, true>([&](int64_t j) { return ring + (j % L) * C; }, u, a.bias, lo, hi,
-                               L, WPE > 1 || warp == 0, warp, lane, sh, acc);
+  pool_window<T, V, WPE, 4>(
+      [&](int64_t j) { return j == t ? x_new : ring + (j % L) * C; }, u, a.bias, lo, hi, L,
+      WPE > 1 || warp == 0, warp, lane, sh, acc);
   if (warp != 0) return;
   T* dst = page_row<T>(a.pool_pages, a.pool_bt, a.pool_max_pages, a.page_size, C, seq, w);
   if (dst == nullptr) return;

@@ -10,22 +10,20 @@
 
 namespace sac {
 
-// kCoherent: read through L2 (rows written earlier by the same kernel), else the read-only path.
-template <typename T, int V, bool kCoherent = false>
+template <typename T, int V>
 __device__ __forceinline__ void load_lane(const T* row, int lane, float (&v)[V]) {
   const T* p = row + lane * V;
   if constexpr (V * sizeof(T) % 16 == 0) {
 #pragma unroll
     for (int i = 0; i < V * (int)sizeof(T) / 16; ++i) {
-      uint4 u = kCoherent ? __ldcg(reinterpret_cast<const uint4*>(p) + i)
-                          : __ldg(reinterpret_cast<const uint4*>(p) + i);
+      uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + i);
       const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
       for (int k = 0; k < 16 / (int)sizeof(T); ++k) v[i * (16 / sizeof(T)) + k] = to_f<T>(e[k]);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < V; ++i) v[i] = to_f<T>(kCoherent ? __ldcg(p + i) : p[i]);
+    for (int i = 0; i < V; ++i) v[i] = to_f<T>(p[i]);
   }
 }
 
@@ -76,7 +74,7 @@ struct PoolShared {
 // warp % WPE). row(j) gives row j's pointer. On return the group's first warp (sub == 0) holds
 // the normalised pooled row in acc; with WPE > 1 every warp of the block must call (it contains
 // __syncthreads). Rows whose gate logit is -inf get weight 0.
-template <typename T, int V, int WPE, bool kCoherent = false, typename RowFn>
+template <typename T, int V, int WPE, int kBatch = 4, typename RowFn>
 __device__ __forceinline__ void pool_window(RowFn row, const float (&u)[V], const float* bias,
                                             int64_t lo, int64_t hi, int L, bool active, int warp,
                                             int lane, PoolShared<V, WPE>& sh, float (&acc)[V]) {
@@ -87,7 +85,6 @@ __device__ __forceinline__ void pool_window(RowFn row, const float (&u)[V], cons
   if (active) {
     // rows in batches of kBatch: all loads of a batch are issued before any is used, so a
     // window costs ceil(rows / kBatch) memory latencies instead of one per row
-    constexpr int kBatch = 4;
     for (int64_t j0 = lo + sub; j0 < hi; j0 += kBatch * WPE) {
       float xv[kBatch][V];
       float bb[kBatch];
@@ -95,7 +92,7 @@ __device__ __forceinline__ void pool_window(RowFn row, const float (&u)[V], cons
       for (int k = 0; k < kBatch; ++k) {
         const int64_t j = j0 + (int64_t)k * WPE;
         if (j < hi) {
-          load_lane<T, V, kCoherent>(row(j), lane, xv[k]);
+          load_lane<T, V>(row(j), lane, xv[k]);
           bb[k] = __ldg(bias + (j - hi + L));
         }
       }

@@ -183,6 +183,7 @@ sac::AttnArgs attn_common(const sac_params* p, const void* q, void* o, const flo
   a.m = p->m;
   a.k = p->topk;
   a.rf = rope_freqs(p);
+  a.splits = 1;
   return a;
 }
 
@@ -472,13 +473,47 @@ int sac_device_status(const void* ws, int* status, void* stream) {
 // ---------------------------------------------------------------------------------------------
 // decode
 // ---------------------------------------------------------------------------------------------
+// Decode attention on tensor cores splits each sequence's key tiles over several CTAs when there
+// are fewer sequences than SMs; the partial results need nseq * splits * H * (D + 2) floats.
+static int decode_splits(const sac_params* p, int nseq) {
+  if (!use_tc_attention(p)) return 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int sp = sms / nseq;
+  if (sp > sac::attention_tc_max_splits()) sp = sac::attention_tc_max_splits();
+  return sp < 1 ? 1 : sp;
+}
+
+static size_t decode_split_bytes(const sac_params* p, int nseq) {
+  const int sp = decode_splits(p, nseq);
+  if (sp == 1) return 0;
+  return align_up((size_t)nseq * sp * p->H * p->D * 4) + align_up((size_t)nseq * sp * p->H * 2 * 4);
+}
+
+// Point a decode call's attention at its split buffers (after the first `used` bytes of ws) when
+// the workspace holds them; otherwise the attention runs unsplit.
+static void decode_attach_splits(const sac_params* p, int nseq, void* ws, size_t ws_bytes,
+                                 size_t used, sac::AttnArgs& a) {
+  const int sp = decode_splits(p, nseq);
+  const size_t need = decode_split_bytes(p, nseq);
+  if (sp == 1 || ws == nullptr || ws_bytes < used + need) return;
+  char* base = static_cast<char*>(ws) + used;
+  a.splits = sp;
+  a.part_o = reinterpret_cast<float*>(base);
+  a.part_ml = reinterpret_cast<float*>(base + align_up((size_t)nseq * sp * p->H * p->D * 4));
+}
+
 size_t sac_decode_workspace_size(const sac_params* p, int kind, int nseq) {
   if (kind < SAC_KIND_SWA || kind > SAC_KIND_CSA || nseq < 1 ||
       check_params(p, kind, true) != SAC_OK)
     return 0;
-  if (kind != SAC_KIND_CSA) return kStatusBytes;
-  const size_t n = (size_t)(p->S / p->m);
-  return kStatusBytes + align_up((size_t)nseq * n * 4) + align_up((size_t)nseq * p->topk * 4);
+  size_t bytes = kStatusBytes;
+  if (kind == SAC_KIND_CSA) {
+    const size_t n = (size_t)(p->S / p->m);
+    bytes += align_up((size_t)nseq * n * 4) + align_up((size_t)nseq * p->topk * 4);
+  }
+  return bytes + decode_split_bytes(p, nseq);
 }
 
 // Status word of a decode call: the first word of ws when one is given (cleared here), else none
@@ -532,6 +567,7 @@ int swa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.nrows = nseq;
   a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
   a.pool_mode = 0;
+  decode_attach_splits(p, nseq, ws, ws_bytes, kStatusBytes, a);
   cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
@@ -559,6 +595,7 @@ int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
   a.pool_mode = 1;
   a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
+  decode_attach_splits(p, nseq, ws, ws_bytes, kStatusBytes, a);
   cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
@@ -622,6 +659,7 @@ int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
   a.sel = sel;
   a.status = status;
+  decode_attach_splits(p, nseq, ws, ws_bytes, cv.used, a);
   e = run_attention(p, a, 1, 1, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;

@@ -109,6 +109,12 @@ struct AttnArgs {
   int k;
   RopeFreqs rf;
   int* status;           // device status word (tensor-core kernels record wait timeouts)
+  // tensor-core kernel only: each row's key tiles split over `splits` CTAs (1 = no split); with
+  // splits > 1 the partial results go to part_o [nrows*splits, H, D] and part_ml
+  // [nrows*splits, H, 2] (fp32) and a combine kernel writes o
+  int splits;
+  float* part_o;
+  float* part_ml;
 };
 cudaError_t launch_attention_simt(int dtype, const AttnArgs& a, cudaStream_t st);
 
@@ -116,6 +122,7 @@ cudaError_t launch_attention_simt(int dtype, const AttnArgs& a, cudaStream_t st)
 // a.q: [nrows, 64, 512] un-rotated (rotated in the kernel); win/pool bases are [rows, 512]
 // buffers whose row counts (win_rows, pool_rows) bound the TMA coordinates.
 bool attention_tc_supported(const AttnArgs& a, int dtype);
+int attention_tc_max_splits();
 cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t pool_rows,
                                 cudaStream_t st);
 

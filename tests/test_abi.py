@@ -59,10 +59,15 @@ def test_workspace_sizes():
     assert sac.sac_workspace_size(p_csa(m=128, win_len=128), sac.SAC_KIND_HCA) == \
         256 + 8192 * 512 * 2 + 64 * 512 * 2
     assert sac.sac_workspace_size(p_csa(dtype="f32"), sac.SAC_KIND_SWA) == 256 + 8192 * 512 * 4
+    # without a GPU the SM count defaults to 148: 64 sequences -> 2 splits of fp32 partials
+    part = 64 * 2 * 64 * 512 * 4 + 64 * 2 * 64 * 2 * 4
     assert sac.sac_decode_workspace_size(p_csa(S=65536), sac.SAC_KIND_CSA, 64) == \
-        256 + 64 * 16384 * 4 + 64 * 512 * 4
-    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_HCA, 64) == 256
-    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 64) == 256
+        256 + 64 * 16384 * 4 + 64 * 512 * 4 + part
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_HCA, 64) == 256 + part
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 64) == 256 + part
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 200) == 256  # no split
+    p32 = sac.make_params(1, 8192, 8, 128, 32, 1e4, sliding_window=16, dtype="f32")
+    assert sac.sac_decode_workspace_size(p32, sac.SAC_KIND_SWA, 4) == 256  # CUDA-core path
 
 
 @pytest.mark.parametrize("bad,code", [
