@@ -269,9 +269,9 @@ def tensor_kernels(wl) -> set:
 # (workload, kernel); the summary with its command is the named file under profiles/. An entry is
 # removed whenever its kernel changes, and the roofline then reports traffic null.
 NCU_TRAFFIC = {
-    ("csa_8k_bf16", "attention"): (563.197696e6 + 491.843584e6, "attention_tc_csa_8k_bf16.md"),
+    ("csa_8k_bf16", "attention"): (562.846464e6 + 488.891392e6, "attention_tc_csa_8k_bf16.md"),
     ("csa_8k_bf16", "indexer_score"): (136.957696e6 + 25.005312e6, "indexer_tc_csa_8k_bf16.md"),
-    ("csa_8k_bf16", "topk"): (31.865088e6 + 7.68e3, "topk_csa_8k_bf16.md"),
+    ("csa_8k_bf16", "topk"): (31.871744e6 + 3.072e3, "topk_csa_8k_bf16.md"),
 }
 
 
@@ -446,10 +446,10 @@ def decode_bytes(wl, d_csa, d_hca) -> dict:
     out["indexer_score"] = float((nv * wl.cI * esz).sum() + wl.nseq * wl.nI * (wl.cI * esz + 4)
                                  + (nv * 4).sum())
     out["topk"] = float((nv * 4).sum() + wl.nseq * wl.k * 4)
-    att_csa = float(((np.minimum(nv, wl.k) + win) * wl.D * esz).sum() + 2 * qb)
+    out["csa_decode_attention"] = float(((np.minimum(nv, wl.k) + win) * wl.D * esz).sum() + 2 * qb)
     ctx_h = d_hca["ctx_lens"].numpy().astype(np.int64)
-    att_hca = float(((ctx_h // d_hca["m"] + np.minimum(ctx_h, wl.W)) * wl.D * esz).sum() + 2 * qb)
-    out["attention"] = att_csa + att_hca
+    out["hca_decode_attention"] = float(((ctx_h // d_hca["m"] + np.minimum(ctx_h, wl.W))
+                                         * wl.D * esz).sum() + 2 * qb)
     # cache append: the new row read, written rotated to its page and un-rotated to the ring; a
     # closing window (ctx % m == 0) reads its L ring rows and writes one entry
     app = 0.0
@@ -481,6 +481,8 @@ def run_decode(args, wl0):
                          sliding_window=wl.W, dtype=wl.dtype)
     ws = torch.empty(sac.sac_decode_workspace_size(pc, sac.SAC_KIND_CSA, wl.nseq),
                      dtype=torch.uint8, device=dev)
+    ws_h = torch.empty(sac.sac_decode_workspace_size(ph, sac.SAC_KIND_HCA, wl.nseq),
+                       dtype=torch.uint8, device=dev)
     oc = torch.empty_like(gc["q"])
     oh = torch.empty_like(gh["q"])
     ps = wl.page_size
@@ -502,7 +504,7 @@ def run_decode(args, wl0):
                           cmp_gate=gh["cmp_gate"], cmp_bias=gh["cmp_bias"],
                           pool_pages=gh["pool_pages"], pool_block_table=gh["pool_block_table"])
         sac.hca_decode(ph, wl.nseq, gh["q"], gh["kv_pages"], gh["kv_block_table"], gh["ctx_lens"],
-                       ps, gh["pool_pages"], gh["pool_block_table"], gh["sinks"], oh)
+                       ps, gh["pool_pages"], gh["pool_block_table"], gh["sinks"], oh, ws_h)
 
     for _ in range(args.warmup):
         step()
@@ -583,6 +585,76 @@ def run_decode(args, wl0):
         torch.distributed.destroy_process_group()
 
 
+def run_oproj(args, wl0):
+    """The grouped output projection alone: two GEMMs, timed like the prefill path."""
+    import sparse_attention_compressor_b200 as sac
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    wl = rank_workload(wl0, rank)
+    T, G, rk, hid = wl.B * wl.S, wl.o_groups, wl.o_rank, wl.hidden
+    x = W.oproj_inputs(T, wl.H, wl.D, G, rk, hid, wl.seed)
+    g = {k: v.to(dev).contiguous() for k, v in x.items()}
+    p = sac.make_params(1, T, wl.H, wl.D, wl.R, wl.theta)
+    ws = torch.empty(sac.sac_oproj_workspace_size(p, T, G, rk), dtype=torch.uint8, device=dev)
+    out = torch.empty((T, hid), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        sac.o_proj_forward(p, T, G, rk, hid, g["o"], g["w_a"], g["w_b"], out, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sac.sac_timing_begin()
+    graph = capture(step)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        clk.wait_samples(1, graph.replay)
+        ms = timed_flushed(graph.replay, args.steps, dev)
+        clk.wait_samples(len(clk.lines) + 1, graph.replay)
+    ktimes = sac.sac_timing_end()
+    ms = max_over_ranks(ms, dev) / args.steps
+    pin_o = x["o"].pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+    def e2e_step():
+        g["o"].copy_(pin_o, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_graph = capture(e2e_step)
+    e2e_ms = max_over_ranks(timed_flushed(e2e_graph.replay, args.steps, dev), dev) / args.steps
+    peaks = measured_peaks()
+    flops = 2.0 * T * (wl.H * wl.D * rk + G * rk * hid)
+    launches, kms = ktimes.get("o_proj", (1, ms))
+    ach = flops / (kms / max(launches, 1) * 1e-3) / 1e12
+    line = {
+        "metric": "grouped output projection tokens/s", "value": T * world / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic (seeded; see DESIGN.md)",
+        "config": {"workload": wl.name, "tokens": T, "H": wl.H, "head_dim": wl.D,
+                   "o_groups": G, "o_lora_rank": rk, "hidden": hid, "parallelism": f"dp{world}",
+                   "l2": "flushed before every step (252 MiB written, then another 252 MiB read)",
+                   "launch": "one CUDA graph replay per step (two cuBLASLt GEMMs)"},
+        "clocks": clk.summary(),
+        "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": pin_o.numel() * 2, "d2h_bytes_per_step": out.numel() * 2},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"kernel": "o_proj", "bound": "tensor", "achieved": ach,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": peaks["source"]},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def run_reference(args, wl):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -630,6 +702,8 @@ def main(argv=None):
         run_reference(args, wl)
     elif wl.kind == "decode":
         run_decode(args, wl)
+    elif wl.kind == "oproj":
+        run_oproj(args, wl)
     else:
         run_ours(args, wl)
 

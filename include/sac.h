@@ -235,6 +235,26 @@ SAC_API int decode_append(const sac_params* p, int kind, int nseq, const int32_t
                const int32_t* pool_block_table, int pool_max_pages, void* stream);
 
 /*
+ * Grouped low-rank output projection ("Grouped Output Projection" bullet of the architecture
+ * overview; config o_groups, o_lora_rank, hidden_size). The attention output o [T, H, D] of
+ * p->H heads of p->D is cut into `groups` groups of H/groups consecutive heads; group g's
+ * (H/groups)*D features are projected to `rank` features by its own matrix w_a[g] (o_a_proj), the
+ * groups' results are concatenated and projected to `hidden` by w_b (o_b_proj):
+ *   mid[t, g*rank + i] = sum_c o[t, g*(H/groups)*D + c] * w_a[g, i, c]
+ *   out[t, j]          = sum_i mid[t, i] * w_b[j, i]
+ *   o   [T, H*D], w_a [groups, rank, (H/groups)*D], w_b [hidden, groups*rank], out [T, hidden]:
+ *   bf16 (p->dtype must be SAC_BF16), row-major; weights in the nn.Linear [out, in] layout.
+ * The intermediate mid is stored in bf16 (the layer's activation precision); both products
+ * accumulate in fp32. The two GEMMs run on cuBLASLt (a plain dense contraction: the library GEMM).
+ * ws: sac_oproj_workspace_size() bytes (mid plus the GEMM library's scratch), 256-byte aligned.
+ * Returns SAC_ERR_UNSUPPORTED for fp32, groups not dividing H, or rank / hidden not multiples of 8.
+ */
+SAC_API size_t sac_oproj_workspace_size(const sac_params* p, int64_t T, int groups, int rank);
+SAC_API int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank, int hidden,
+               const void* o, const void* w_a, const void* w_b, void* out, void* ws,
+               size_t ws_bytes, void* stream);
+
+/*
  * Device status of the last call that used workspace `ws` (no counterpart on the page: failure
  * reporting). Every prefill call, and every decode call given a workspace, clears the first word
  * of its workspace; a tensor-core

@@ -98,6 +98,9 @@ def _lib():
         lib.orc_csa_index_scores.argtypes = [P, _dp, _dp, _dp, _dp, _dp, _lp, ctypes.c_long, _dp]
         lib.orc_decode.argtypes = [P, ctypes.c_int, _dp, _dp, _ip, ctypes.c_int, _ip, ctypes.c_int,
                                    _dp, _dp, _ip, ctypes.c_int, _dp, _dp, _dp, _dp, _ip, _ip]
+        lib.orc_oproj.restype = None
+        lib.orc_oproj.argtypes = [ctypes.c_int] * 5 + [_dp, _dp, _dp, ctypes.c_int, _lp,
+                                                       ctypes.c_int, _dp, _dp]
         lib.orc_round_bf16.restype = ctypes.c_double
         lib.orc_round_bf16.argtypes = [ctypes.c_double]
         lib.orc_max_threads.restype = ctypes.c_int
@@ -290,3 +293,25 @@ def decode(p: OracleParams, q, kv_pages, kv_block_table, ctx_lens, page_size: in
                       _ptr(pbt, _ip), 0 if pbt is None else pbt.shape[1], _ptr(qI), _ptr(wI),
                       _ptr(_f64(sinks)), _ptr(o), _ptr(tk, _ip), _ptr(tin, _ip))
     return o, tk
+
+
+def o_proj(o, w_a, w_b, groups: int, rows=None, round_mid: bool = False):
+    """Grouped low-rank output projection of the listed token rows (all rows when None).
+    o [T, H, D] or [T, H*D]; w_a [G, rank, (H/G)*D]; w_b [hidden, G*rank]. Returns (mid, out)
+    for those rows, mid [n, G*rank] (rounded to bf16 when round_mid) and out [n, hidden]."""
+    o = _f64(o)
+    T = o.shape[0]
+    o2 = np.ascontiguousarray(o.reshape(T, -1))
+    w_a, w_b = _f64(w_a), _f64(w_b)
+    G, rank, kg = w_a.shape
+    hidden = w_b.shape[0]
+    assert G == groups and w_b.shape[1] == G * rank and o2.shape[1] == G * kg
+    HD = o2.shape[1]
+    # the C routine takes H and D; only H*D and (H/G)*D matter, so pass H = G, D = kg
+    rows = np.arange(T, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    mid = np.zeros((len(rows), G * rank))
+    out = np.zeros((len(rows), hidden))
+    _lib().orc_oproj(G, kg, G, rank, hidden, _ptr(o2), _ptr(w_a), _ptr(w_b), len(rows),
+                     _ptr(rows, _lp), int(round_mid), _ptr(mid), _ptr(out))
+    assert HD == G * kg
+    return mid, out

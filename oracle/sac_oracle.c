@@ -474,3 +474,39 @@ int orc_decode(const orc_params *p, int nseq, const double *q, const double *kv_
   }
   return 0;
 }
+
+/* ---------------------------------------------------------------------------------------------
+ * Grouped low-rank output projection ("Grouped Output Projection" bullet of the architecture
+ * overview; config o_groups, o_lora_rank, hidden_size). For each listed token row t:
+ *   mid[t, g*rank + i] = sum_c o[t, g*Kg + c] * wa[g, i, c]     (Kg = (H/G)*D features per group)
+ *   out[t, j]          = sum_i mid[t, i] * wb[j, i]
+ * o [T, H*D], wa [G, rank, Kg], wb [hidden, G*rank], all row-major fp64; mid [n, G*rank] and
+ * out [n, hidden] for the n listed rows. [reading] mid is an activation stored in the layer's
+ * dtype, so with round_mid it is rounded to bf16 (as orc_round_bf16) before o_b_proj.
+ * ------------------------------------------------------------------------------------------- */
+void orc_oproj(int H, int D, int G, int rank, int hidden, const double *o, const double *wa,
+               const double *wb, int n, const int64_t *rows, int round_mid, double *mid,
+               double *out) {
+  const int Kg = H / G * D;
+  const int M = G * rank;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int r = 0; r < n; ++r) {
+    const double *orow = o + rows[r] * (int64_t)H * D;
+    double *m = mid + (int64_t)r * M;
+    for (int g = 0; g < G; ++g)
+      for (int i = 0; i < rank; ++i) {
+        const double *w = wa + ((int64_t)g * rank + i) * Kg;
+        const double *x = orow + (int64_t)g * Kg;
+        double acc = 0.0;
+        for (int c = 0; c < Kg; ++c) acc += x[c] * w[c];
+        m[g * rank + i] = round_mid ? orc_round_bf16(acc) : acc;
+      }
+    double *y = out + (int64_t)r * hidden;
+    for (int j = 0; j < hidden; ++j) {
+      const double *w = wb + (int64_t)j * M;
+      double acc = 0.0;
+      for (int i = 0; i < M; ++i) acc += m[i] * w[i];
+      y[j] = acc;
+    }
+  }
+}

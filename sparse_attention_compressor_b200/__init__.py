@@ -22,7 +22,7 @@ ABI_SYMBOLS = ("sac_last_error", "sac_version", "sac_workspace_size", "swa_forwa
                "hca_forward", "csa_forward", "sac_decode_workspace_size", "swa_decode",
                "hca_decode", "csa_decode", "sac_timing_begin", "sac_timing_end",
                "sac_static_scratch_bytes", "swa_forward_static", "sac_device_status",
-               "decode_append")
+               "decode_append", "sac_oproj_workspace_size", "o_proj_forward")
 
 
 class SacError(RuntimeError):
@@ -91,6 +91,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                vp, i32p, vp, sz, vp]
     lib.decode_append.argtypes = [P, ci, ci, i32p, vp, vp, vp, fp, vp, fp, vp, i32p, ci, ci, vp,
                                   vp, vp, vp, i32p, ci, vp]
+    lib.sac_oproj_workspace_size.restype = sz
+    lib.sac_oproj_workspace_size.argtypes = [P, ctypes.c_int64, ci, ci]
+    lib.o_proj_forward.restype = ci
+    lib.o_proj_forward.argtypes = [P, ctypes.c_int64, ci, ci, ci, vp, vp, vp, vp, vp, sz, vp]
     lib.sac_device_status.restype = ci
     lib.sac_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
     lib.sac_static_scratch_bytes.restype = sz
@@ -243,3 +247,14 @@ def decode_append(p, kind, nseq, ctx_lens, kv_new, kv_pages, kv_block_table, pag
         _ptr(kv_block_table), kv_block_table.shape[1], page_size, _ptr(cmp_state),
         _ptr(idx_state), _ptr(pool_pages), _ptr(idx_pool_pages), _ptr(pool_block_table), pmax,
         _stream(stream)))
+
+
+def sac_oproj_workspace_size(p: sac_params, T: int, groups: int, rank: int) -> int:
+    return int(load_library().sac_oproj_workspace_size(ctypes.byref(p), T, groups, rank))
+
+
+def o_proj_forward(p, T, groups, rank, hidden, o, w_a, w_b, out, ws, stream=None) -> None:
+    """Grouped low-rank output projection: out = concat_g(o_g w_a[g]^T) w_b^T (see include/sac.h)."""
+    _check("o_proj_forward", load_library().o_proj_forward(
+        ctypes.byref(p), T, groups, rank, hidden, _ptr(o), _ptr(w_a), _ptr(w_b), _ptr(out),
+        _ptr(ws), _nbytes(ws), _stream(stream)))

@@ -160,13 +160,13 @@ sac::RowAddr paged(const void* base, const int32_t* bt, int max_pages, int page_
 // The attention step of a call: the tensor-core kernel for bf16 layers with 64 heads of 512 (it
 // rotates q itself), the CUDA-core kernel otherwise.
 cudaError_t run_attention(const sac_params* p, const sac::AttnArgs& a, int64_t win_rows,
-                          int64_t pool_rows, cudaStream_t st) {
+                          int64_t pool_rows, cudaStream_t st, const char* timer = "attention") {
   if (use_tc_attention(p) && sac::attention_tc_supported(a, p->dtype)) {
-    return sac::timed("attention", st, [&] {
+    return sac::timed(timer, st, [&] {
       return sac::launch_attention_tc(a, win_rows, pool_rows, st);
     });
   }
-  return sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  return sac::timed(timer, st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
 }
 
 sac::AttnArgs attn_common(const sac_params* p, const void* q, void* o, const float* sinks) {
@@ -480,9 +480,12 @@ static int decode_splits(const sac_params* p, int nseq) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Splitting pays only when it multiplies the CTAs several times over: at 2 or 3 splits the
+  // fp32 partials and the combine launch cost more than the shorter key walk saves (64 sequences
+  // on 148 SMs ran 12-25% slower split in two).
   int sp = sms / nseq;
   if (sp > sac::attention_tc_max_splits()) sp = sac::attention_tc_max_splits();
-  return sp < 1 ? 1 : sp;
+  return sp < 4 ? 1 : sp;
 }
 
 static size_t decode_split_bytes(const sac_params* p, int nseq) {
@@ -568,7 +571,7 @@ int swa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
   a.pool_mode = 0;
   decode_attach_splits(p, nseq, ws, ws_bytes, kStatusBytes, a);
-  cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream));
+  cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream), "swa_decode_attention");
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -596,7 +599,7 @@ int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.pool_mode = 1;
   a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
   decode_attach_splits(p, nseq, ws, ws_bytes, kStatusBytes, a);
-  cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream));
+  cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream), "hca_decode_attention");
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -660,7 +663,7 @@ int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
   a.sel = sel;
   a.status = status;
   decode_attach_splits(p, nseq, ws, ws_bytes, cv.used, a);
-  e = run_attention(p, a, 1, 1, st);
+  e = run_attention(p, a, 1, 1, st, "csa_decode_attention");
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -733,6 +736,52 @@ int decode_append(const sac_params* p, int kind, int nseq, const int32_t* ctx_le
       return sac::launch_decode_append(p->dtype, a, true, st);
     });
   if (e != cudaSuccess) return cuda_fail(e, "decode append");
+  return SAC_OK;
+}
+
+size_t sac_oproj_workspace_size(const sac_params* p, int64_t T, int groups, int rank) {
+  if (p == nullptr || T < 0 || groups < 1 || rank < 1) return 0;
+  return align_up((size_t)T * groups * rank * 2) + align_up(sac::oproj_gemm_scratch_bytes());
+}
+
+int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank, int hidden,
+                   const void* o, const void* w_a, const void* w_b, void* out, void* ws,
+                   size_t ws_bytes, void* stream) {
+  REQUIRE(p != nullptr, SAC_ERR_ARG, "params must not be NULL");
+  REQUIRE(p->dtype == SAC_BF16, SAC_ERR_UNSUPPORTED, "the output projection takes bf16");
+  REQUIRE(T >= 0, SAC_ERR_ARG, "T must be >= 0");
+  REQUIRE(p->H >= 1 && p->D >= 8 && p->D % 8 == 0, SAC_ERR_ARG, "bad head shape");
+  REQUIRE(groups >= 1 && p->H % groups == 0, SAC_ERR_UNSUPPORTED,
+          "o_groups (%d) must divide the head count (%d)", groups, p->H);
+  REQUIRE(rank >= 8 && rank % 8 == 0 && hidden >= 8 && hidden % 8 == 0, SAC_ERR_UNSUPPORTED,
+          "o_lora_rank and hidden must be positive multiples of 8");
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(w_a);
+  REQUIRE_PTR(w_b);
+  REQUIRE_PTR(out);
+  const size_t need = sac_oproj_workspace_size(p, T, groups, rank);
+  REQUIRE(ws != nullptr && ws_bytes >= need, SAC_ERR_WORKSPACE,
+          "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255) == 0, SAC_ERR_ARG,
+          "ws must be 256-byte aligned");
+  Carve cv(ws);
+  sac::OProjArgs a;
+  a.T = T;
+  a.H = p->H;
+  a.D = p->D;
+  a.groups = groups;
+  a.rank = rank;
+  a.hidden = hidden;
+  a.o = o;
+  a.w_a = w_a;
+  a.w_b = w_b;
+  a.out = out;
+  a.mid = cv.take((size_t)T * groups * rank * 2);
+  a.scratch_bytes = sac::oproj_gemm_scratch_bytes();
+  a.scratch = cv.take(a.scratch_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = sac::timed("o_proj", st, [&] { return sac::launch_oproj(a, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "output projection");
   return SAC_OK;
 }
 

@@ -51,6 +51,21 @@ struct DecodeAppendArgs {
 cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, bool index_part,
                                  cudaStream_t st);
 
+// ---- grouped output projection (oproj.cu, cuBLASLt GEMMs) ---------------------------------
+struct OProjArgs {
+  int64_t T;             // tokens
+  int H, D, groups, rank, hidden;
+  const void* o;         // [T, H*D] bf16
+  const void* w_a;       // [groups, rank, H/groups*D] bf16 (o_a_proj, nn.Linear layout per group)
+  const void* w_b;       // [hidden, groups*rank] bf16 (o_b_proj)
+  void* mid;             // [T, groups*rank] bf16 intermediate
+  void* out;             // [T, hidden] bf16
+  void* scratch;         // GEMM library workspace
+  size_t scratch_bytes;
+};
+size_t oproj_gemm_scratch_bytes();
+cudaError_t launch_oproj(const OProjArgs& a, cudaStream_t st);
+
 // ---- indexer (indexer.cu) -----------------------------------------------------------------
 struct IndexerArgs {
   const void* q_idx;     // [rows, nI, cI] (flat query rows starting at qr.row0)

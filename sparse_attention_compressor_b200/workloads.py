@@ -25,14 +25,15 @@ _TENSOR_IDS = {"q": 1, "kv": 2, "cmp_gate": 3, "cmp_bias": 4, "q_idx": 5, "w_idx
                "ctx": 12, "pages": 13, "kv_pages": 14, "pool_pages": 15, "idx_pool_pages": 16,
                "hca_kv_pages": 17, "hca_pool_pages": 18, "hca_page_perm": 19, "hca_sinks": 20,
                "kv_new": 21, "k_idx_new": 22, "cmp_state": 23, "idx_state": 24,
-               "hca_cmp_gate": 25, "hca_cmp_bias": 26}
+               "hca_cmp_gate": 25, "hca_cmp_bias": 26, "o_attn": 27, "o_a_proj": 28,
+               "o_b_proj": 29}
 
 ROW_CHUNK = 64  # rows per independently seeded chunk of a per-token tensor
 
 
 @dataclass(frozen=True)
 class Workload:
-    """One synthetic workload. kind: 'csa' | 'hca' | 'swa' prefill, or 'decode'."""
+    """One synthetic workload. kind: 'csa' | 'hca' | 'swa' prefill, 'decode', or 'oproj'."""
     name: str
     kind: str
     dtype: str            # 'f32' or 'bf16'
@@ -55,6 +56,10 @@ class Workload:
     ctx_hi: int = 0
     page_size: int = 64
     hca_m: int = 128
+    # output projection only
+    o_groups: int = 0
+    o_rank: int = 0
+    hidden: int = 0
     seed: int = 1234
 
     @property
@@ -78,6 +83,9 @@ WORKLOADS: Dict[str, Workload] = {
                               cI=128, k=512, spike_frac=0.05, seed=1237),
     "decode_bf16": Workload("decode_bf16", "decode", "bf16", nseq=64, ctx_lo=4096, ctx_hi=65536,
                             page_size=64, m=4, L=8, nI=64, cI=128, k=512, hca_m=128, seed=1238),
+    # Grouped output projection of 8192 tokens: 64 heads of 512 in 8 groups of rank 1024 to 4096.
+    "oproj_8k_bf16": Workload("oproj_8k_bf16", "oproj", "bf16", B=1, S=8192, o_groups=8,
+                              o_rank=1024, hidden=4096, seed=1239),
 }
 
 
@@ -276,3 +284,20 @@ def decode_inputs(wl: Workload, layer: str) -> Dict[str, object]:
         out["w_idx"] = _normal((wl.nseq, wl.nI), 1.0 / math.sqrt(wl.nI), wl.seed, "w_idx",
                                10 ** 6)
     return out
+
+
+# ------------------------------------------------------------------------------------------------
+# Grouped output projection: an attention output o [T, H, D] ~ N(0, 1) and random-init weights
+# (o_a_proj ~ N(0, 1/fan_in) per group, o_b_proj ~ N(0, 1/fan_in)) in the nn.Linear layout.
+# ------------------------------------------------------------------------------------------------
+def oproj_inputs(T: int, H: int, D: int, groups: int, rank: int, hidden: int, seed: int,
+                 dtype=torch.bfloat16) -> Dict[str, torch.Tensor]:
+    kg = H // groups * D
+    o = torch.empty((T, H, D))
+    for c0 in range(0, T, ROW_CHUNK):
+        n = min(ROW_CHUNK, T - c0)
+        o[c0:c0 + n] = _normal((ROW_CHUNK, H, D), 1.0, seed, "o_attn", c0 // ROW_CHUNK)[:n]
+    return {"o": o.to(dtype),
+            "w_a": _normal((groups, rank, kg), 1.0 / math.sqrt(kg), seed, "o_a_proj").to(dtype),
+            "w_b": _normal((hidden, groups * rank), 1.0 / math.sqrt(groups * rank), seed,
+                           "o_b_proj").to(dtype)}

@@ -59,13 +59,18 @@ def test_workspace_sizes():
     assert sac.sac_workspace_size(p_csa(m=128, win_len=128), sac.SAC_KIND_HCA) == \
         256 + 8192 * 512 * 2 + 64 * 512 * 2
     assert sac.sac_workspace_size(p_csa(dtype="f32"), sac.SAC_KIND_SWA) == 256 + 8192 * 512 * 4
-    # without a GPU the SM count defaults to 148: 64 sequences -> 2 splits of fp32 partials
-    part = 64 * 2 * 64 * 512 * 4 + 64 * 2 * 64 * 2 * 4
+    # without a GPU the SM count defaults to 148: 16 sequences -> 8 splits (the cap) of fp32
+    # partials, 37 -> 4; from 38 sequences on (fewer than 4 splits) the attention runs unsplit
+    part = 16 * 8 * 64 * 512 * 4 + 16 * 8 * 64 * 2 * 4
+    assert sac.sac_decode_workspace_size(p_csa(S=65536), sac.SAC_KIND_CSA, 16) == \
+        256 + 16 * 16384 * 4 + 16 * 512 * 4 + part
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_HCA, 16) == 256 + part
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 37) == \
+        256 + 37 * 4 * 64 * 512 * 4 + (37 * 4 * 64 * 2 * 4 + 255) // 256 * 256
     assert sac.sac_decode_workspace_size(p_csa(S=65536), sac.SAC_KIND_CSA, 64) == \
-        256 + 64 * 16384 * 4 + 64 * 512 * 4 + part
-    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_HCA, 64) == 256 + part
-    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 64) == 256 + part
-    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 200) == 256  # no split
+        256 + 64 * 16384 * 4 + 64 * 512 * 4
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 38) == 256
+    assert sac.sac_decode_workspace_size(p_csa(), sac.SAC_KIND_SWA, 200) == 256
     p32 = sac.make_params(1, 8192, 8, 128, 32, 1e4, sliding_window=16, dtype="f32")
     assert sac.sac_decode_workspace_size(p32, sac.SAC_KIND_SWA, 4) == 256  # CUDA-core path
 
@@ -161,3 +166,26 @@ def test_decode_append_validation():
     rc = lib.decode_append(ctypes.byref(p_swa), sac.SAC_KIND_SWA, 2, fake, fake, None, None, None,
                            None, None, fake, fake, 63, 64, None, None, None, None, None, 0, None)
     assert rc == -1 and "block table" in lib.sac_last_error().decode()
+
+
+def test_oproj_validation_and_workspace():
+    lib = sac.load_library()
+    fake = 1 << 20
+    p = sac.make_params(1, 64, 64, 512, 64, 1e4)
+    need = sac.sac_oproj_workspace_size(p, 64, 8, 1024)
+    # bf16 mid [64, 8*1024] plus the GEMM scratch, each 256-byte aligned
+    assert need == 64 * 8 * 1024 * 2 + (32 << 20)
+    assert sac.sac_oproj_workspace_size(p, -1, 8, 1024) == 0
+
+    def call(T=64, groups=8, rank=1024, hidden=4096, ws=fake, ws_bytes=need, params=p):
+        return lib.o_proj_forward(ctypes.byref(params), T, groups, rank, hidden, fake, fake, fake,
+                                  fake, ws, ws_bytes, None)
+
+    assert call(groups=3) == -2
+    assert call(rank=1020) == -2
+    assert call(hidden=4) == -2
+    assert call(ws_bytes=need - 1) == -3
+    assert call(ws=fake + 16) == -1 and "256-byte" in lib.sac_last_error().decode()
+    p32 = sac.make_params(1, 64, 64, 512, 64, 1e4, dtype="f32")
+    assert call(params=p32) == -2
+    assert call(T=0) == 0  # nothing to do: no launch, no device touched

@@ -577,3 +577,62 @@ def test_bf16_pools_round_the_stored_entries():
     _, _, pool_r, kpool_r = oracle.csa_forward(p, *args)
     np.testing.assert_array_equal(pool_r, np.vectorize(oracle.round_bf16)(pool))
     np.testing.assert_array_equal(kpool_r, np.vectorize(oracle.round_bf16)(kpool))
+
+
+# ---- grouped output projection ("Grouped Output Projection" bullet) --------------------------
+def test_oproj_matches_numpy_matmul():
+    rng = np.random.default_rng(3)
+    o = rng.standard_normal((7, 6, 8))
+    wa = rng.standard_normal((3, 5, 16))
+    wb = rng.standard_normal((9, 15))
+    mid, out = oracle.o_proj(o, wa, wb, 3)
+    o2 = o.reshape(7, 48)
+    ref_mid = np.concatenate([o2[:, g * 16:(g + 1) * 16] @ wa[g].T for g in range(3)], axis=1)
+    assert np.allclose(mid, ref_mid, atol=1e-12)
+    assert np.allclose(out, ref_mid @ wb.T, atol=1e-12)
+
+
+def test_oproj_one_hot_selection_is_exact():
+    # o_a_proj rows that pick single features and an o_b_proj permutation give the picked
+    # features back, permuted, exactly
+    rng = np.random.default_rng(4)
+    G, rank, kg = 2, 3, 10
+    o = rng.standard_normal((4, G * kg))
+    wa = np.zeros((G, rank, kg))
+    picks = [[0, 4, 9], [1, 2, 7]]
+    for g in range(G):
+        for i, c in enumerate(picks[g]):
+            wa[g, i, c] = 1.0
+    perm = rng.permutation(G * rank)
+    wb = np.eye(G * rank)[perm]
+    mid, out = oracle.o_proj(o, wa, wb, G)
+    want = np.concatenate([o[:, g * kg + np.array(picks[g])] for g in range(G)], axis=1)
+    assert np.array_equal(mid, want)
+    assert np.array_equal(out, want[:, perm])
+
+
+def test_oproj_groups_are_independent_and_rows_selectable():
+    rng = np.random.default_rng(5)
+    G, rank, kg = 4, 6, 8
+    o = rng.standard_normal((5, G * kg))
+    wa = rng.standard_normal((G, rank, kg))
+    wb = rng.standard_normal((7, G * rank))
+    mid, _ = oracle.o_proj(o, wa, wb, G)
+    o2 = o.copy()
+    o2[:, :kg] += 1.0  # only group 0's features
+    mid2, _ = oracle.o_proj(o2, wa, wb, G)
+    assert not np.allclose(mid2[:, :rank], mid[:, :rank])
+    assert np.array_equal(mid2[:, rank:], mid[:, rank:])
+    mid_r, out_r = oracle.o_proj(o, wa, wb, G, rows=[3, 1])
+    _, out = oracle.o_proj(o, wa, wb, G)
+    assert np.array_equal(out_r, out[[3, 1]])
+
+
+def test_oproj_rounded_intermediate_is_bf16():
+    rng = np.random.default_rng(6)
+    o = rng.standard_normal((3, 16))
+    wa = rng.standard_normal((2, 4, 8))
+    wb = rng.standard_normal((5, 8))
+    mid, _ = oracle.o_proj(o, wa, wb, 2, round_mid=True)
+    as_bf16 = torch.from_numpy(mid).float().to(torch.bfloat16).double().numpy()
+    assert np.array_equal(mid, as_bf16)
