@@ -705,59 +705,78 @@ done:
 
 // Combine the splits of each row: O = sum_s 2^(m_s - M) O_s / (2^(sink - M) + sum_s 2^(m_s - M) l_s)
 // with M = max(sink, max_s m_s) over the non-empty splits (all in log2 units), then the rope
-// slice turned by -P_t and the bf16 store. One block per row; thread (h, quarter) owns head h's
-// channels [128 quarter, 128 quarter + 128).
+// slice turned by -P_t and the bf16 store. Block (row, group of 4 heads); thread (head, chunk)
+// owns 8 consecutive channels, so a warp reads 1 KB of one split's partial O contiguously and
+// every split's loads are issued before the first is used.
+constexpr int kCombineHeads = 4;
 __global__ void __launch_bounds__(256) attention_combine_kernel(AttnArgs a) {
   const int64_t r = blockIdx.x;
-  const int h = threadIdx.x >> 2, quarter = threadIdx.x & 3;
+  const int h = blockIdx.y * kCombineHeads + (threadIdx.x >> 6);
+  const int c = (threadIdx.x & 63) * 8;
   const Row w = locate_row(a, r);
-  float wgt[kMaxSplits];
+  const int splits = a.splits;
+  float wgt[kMaxSplits], lsum[kMaxSplits];
   const float sink = __ldg(a.sinks + h) * kLog2e;
   float M = sink;
-  for (int sp = 0; sp < a.splits; ++sp) {
-    const bool nonempty = (int64_t)w.tiles * sp / a.splits < (int64_t)w.tiles * (sp + 1) / a.splits;
-    wgt[sp] = nonempty ? a.part_ml[((r * a.splits + sp) * kHeads + h) * 2] : -INFINITY;
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplits; ++sp) {
+    wgt[sp] = -INFINITY;
+    lsum[sp] = 0.f;
+    if (sp < splits &&
+        (int64_t)w.tiles * sp / splits < (int64_t)w.tiles * (sp + 1) / splits) {
+      const float2 ml =
+          __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (r * splits + sp) * kHeads + h);
+      wgt[sp] = ml.x;
+      lsum[sp] = ml.y;
+    }
     M = fmaxf(M, wgt[sp]);
   }
   float L = exp2f(sink - M);
-  for (int sp = 0; sp < a.splits; ++sp) {
-    const float m = wgt[sp];
-    wgt[sp] = m == -INFINITY ? 0.f : exp2f(m - M);
-    if (wgt[sp] > 0.f) L += wgt[sp] * a.part_ml[((r * a.splits + sp) * kHeads + h) * 2 + 1];
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplits; ++sp) {
+    wgt[sp] = wgt[sp] == -INFINITY ? 0.f : exp2f(wgt[sp] - M);
+    L += wgt[sp] * lsum[sp];
+  }
+  float4 u[kMaxSplits][2];
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplits; ++sp) {
+    if (wgt[sp] > 0.f) {
+      const float4* po = reinterpret_cast<const float4*>(
+          a.part_o + ((r * splits + sp) * kHeads + h) * kDim + c);
+      u[sp][0] = __ldcs(po);
+      u[sp][1] = __ldcs(po + 1);
+    } else {
+      u[sp][0] = u[sp][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplits; ++sp) {
+    const float g = wgt[sp];
+    x[0] = fmaf(g, u[sp][0].x, x[0]); x[1] = fmaf(g, u[sp][0].y, x[1]);
+    x[2] = fmaf(g, u[sp][0].z, x[2]); x[3] = fmaf(g, u[sp][0].w, x[3]);
+    x[4] = fmaf(g, u[sp][1].x, x[4]); x[5] = fmaf(g, u[sp][1].y, x[5]);
+    x[6] = fmaf(g, u[sp][1].z, x[6]); x[7] = fmaf(g, u[sp][1].w, x[7]);
   }
   const float inv_l = 1.f / L;
   const int64_t P = a.pos0 + w.t;
   const int rope_lo = kDim - a.rf.R;
-  __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (r * kHeads + h) * kDim;
-#pragma unroll 1
-  for (int c = quarter * 128; c < quarter * 128 + 128; c += 8) {
-    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int sp = 0; sp < a.splits; ++sp) {
-      if (wgt[sp] == 0.f) continue;
-      const float* po = a.part_o + ((r * a.splits + sp) * kHeads + h) * kDim + c;
-      const float4 u0 = *reinterpret_cast<const float4*>(po);
-      const float4 u1 = *reinterpret_cast<const float4*>(po + 4);
-      x[0] = fmaf(wgt[sp], u0.x, x[0]); x[1] = fmaf(wgt[sp], u0.y, x[1]);
-      x[2] = fmaf(wgt[sp], u0.z, x[2]); x[3] = fmaf(wgt[sp], u0.w, x[3]);
-      x[4] = fmaf(wgt[sp], u1.x, x[4]); x[5] = fmaf(wgt[sp], u1.y, x[5]);
-      x[6] = fmaf(wgt[sp], u1.z, x[6]); x[7] = fmaf(wgt[sp], u1.w, x[7]);
-    }
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      float x0 = x[e] * inv_l, x1 = x[e + 1] * inv_l;
-      if (c + e >= rope_lo) {
-        float cc, ss;
-        rope_cos_sin(a.rf, (c + e - rope_lo) >> 1, -P, cc, ss);
-        const float y0 = x0 * cc - x1 * ss, y1 = x0 * ss + x1 * cc;
-        x0 = y0;
-        x1 = y1;
-      }
-      x[e] = x0;
-      x[e + 1] = x1;
+  for (int e = 0; e < 8; e += 2) {
+    float x0 = x[e] * inv_l, x1 = x[e + 1] * inv_l;
+    if (c + e >= rope_lo) {
+      float cc, ss;
+      rope_cos_sin(a.rf, (c + e - rope_lo) >> 1, -P, cc, ss);
+      const float y0 = x0 * cc - x1 * ss, y1 = x0 * ss + x1 * cc;
+      x0 = y0;
+      x1 = y1;
     }
-    *reinterpret_cast<uint4*>(orow + c) = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                                                     pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+    x[e] = x0;
+    x[e + 1] = x1;
   }
+  __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (r * kHeads + h) * kDim;
+  *reinterpret_cast<uint4*>(orow + c) = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                                   pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
 }
 
 }  // namespace
@@ -796,7 +815,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
     attention_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.splits == 1) return e;
-  attention_combine_kernel<<<(unsigned)a.nrows, 256, 0, st>>>(a);
+  attention_combine_kernel<<<dim3((unsigned)a.nrows, kHeads / kCombineHeads), 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

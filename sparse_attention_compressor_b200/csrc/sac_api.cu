@@ -481,8 +481,9 @@ static int decode_splits(const sac_params* p, int nseq) {
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // Splitting pays only when it multiplies the CTAs several times over: at 2 or 3 splits the
-  // fp32 partials and the combine launch cost more than the shorter key walk saves (64 sequences
-  // on 148 SMs ran 12-25% slower split in two).
+  // fp32 partials and the combine launch cost about what the shorter key walk saves (64
+  // sequences on 148 SMs: CSA 3% faster, HCA 10% slower split in two; 16 sequences in 8 splits:
+  // 29% and 17% faster).
   int sp = sms / nseq;
   if (sp > sac::attention_tc_max_splits()) sp = sac::attention_tc_max_splits();
   return sp < 4 ? 1 : sp;
