@@ -335,7 +335,7 @@ int hca_forward(const sac_params* p, const void* q, const void* kv, const void* 
   e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
   if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
   e = sac::timed("compress", st, [&] { return sac::launch_compress(p->dtype, kv, cmp_gate, cmp_bias, p->B, p->S, p->D, p->m, p->win_len,
-                           true, rf, p->pos0, pool, st); });
+                           true, rf, p->pos0, pool, status, st); });
   if (e != cudaSuccess) return cuda_fail(e, "compress");
   sac::AttnArgs a = attn_common(p, q, o, sinks);
   a.qr = sac::QueryRows{p->S, nullptr, 0};
@@ -394,10 +394,10 @@ int csa_forward(const sac_params* p, const void* q, const void* kv, const void* 
   e = sac::timed("rotate_kv", st, [&] { return sac::launch_rotate_rows(p->dtype, kv, rows, p->S, p->D, rf, p->pos0, kv_rot, st); });
   if (e != cudaSuccess) return cuda_fail(e, "rotate kv");
   e = sac::timed("compress", st, [&] { return sac::launch_compress(p->dtype, kv, cmp_gate, cmp_bias, p->B, p->S, p->D, p->m, p->win_len,
-                           true, rf, p->pos0, pool, st); });
+                           true, rf, p->pos0, pool, status, st); });
   if (e != cudaSuccess) return cuda_fail(e, "compress");
   e = sac::timed("compress_index", st, [&] { return sac::launch_compress(p->dtype, k_idx, idx_gate, idx_bias, p->B, p->S, p->idx_dim, p->m,
-                           p->win_len, false, rf, p->pos0, ipool, st); });
+                           p->win_len, false, rf, p->pos0, ipool, status, st); });
   if (e != cudaSuccess) return cuda_fail(e, "compress indexer stream");
 
   // indexer + top-k in chunks of query rows of one sequence (bounded scores buffer)

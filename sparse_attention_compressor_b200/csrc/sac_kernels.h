@@ -13,7 +13,7 @@ namespace sac {
 // gate; with rotate != 0 the entry is then rotated at pos0 + w*m. out [B,N,C].
 cudaError_t launch_compress(int dtype, const void* x, const void* gate, const float* bias, int B,
                             int S, int C, int m, int L, bool rotate, const RopeFreqs& rf,
-                            int64_t pos0, void* out, cudaStream_t st);
+                            int64_t pos0, void* out, int* status, cudaStream_t st);
 // out[r] = x[r] with its trailing R channels rotated at pos0 + (r / rows_per_pos) % S.
 // x, out [rows, C] (kv: rows_per_pos = 1; q viewed as [B*S*H, D]: rows_per_pos = H).
 cudaError_t launch_rotate_rows(int dtype, const void* x, int64_t rows, int S, int C,
