@@ -25,6 +25,7 @@ constexpr int kBulkThreads = 32 * (kBulkConsumers + 1);  // + the producer warp
 constexpr int kBulkStages = 3;
 constexpr int kBulkStageBytes = 68 * 1024;            // 16 CSA entries of 1 KB rows + overlap
 constexpr int kBulkPiece = 2048;                       // bytes per bulk copy (multiple of 16)
+constexpr int kBulkMaxRows = kBulkStageBytes / 64;     // rows of a stage at the narrowest row
 
 struct BulkArgs {
   const void* x;
@@ -47,7 +48,6 @@ struct LaneMap {
   static constexpr int NP = V * (int)sizeof(T) / P;
   static constexpr int EPP = P / (int)sizeof(T);  // elements per piece
   static constexpr int NW = (V * (int)sizeof(T) + 3) / 4;
-  static constexpr int kBatch = V * (int)sizeof(T) >= 32 ? 2 : 4;  // window rows per step
   __device__ static int channel(int lane, int i, int k) { return (i * 32 + lane) * EPP + k; }
 };
 
@@ -83,6 +83,32 @@ __device__ __forceinline__ float raw_elem(const uint32_t (&r)[LaneMap<T, V>::NW]
     const uint32_t w = r[k >> 1];
     return __uint_as_float((k & 1) ? (w & 0xFFFF0000u) : (w << 16));
   }
+}
+
+// Elements (2i, 2i+1) of a raw row (V odd: the last pair's second element is 0).
+template <typename T, int V>
+__device__ __forceinline__ float2 raw_pair(const uint32_t (&r)[LaneMap<T, V>::NW], int i) {
+  if constexpr (sizeof(T) == 4 && V == 1) {
+    return make_float2(__uint_as_float(r[0]), 0.f);
+  } else if constexpr (sizeof(T) == 4) {
+    return make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+  } else {
+    const uint32_t w = r[i];
+    return make_float2(__uint_as_float(w << 16),
+                       2 * i + 1 < V ? __uint_as_float(w & 0xFFFF0000u) : 0.f);
+  }
+}
+
+// Named barrier 1 over the consumer warps, AND-reducing a per-thread flag.
+__device__ __forceinline__ bool consumers_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "n"(kBulkConsumers * 32)
+      : "memory");
+  return r != 0;
 }
 
 template <typename T, int V>
@@ -125,6 +151,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) compress_bulk_kernel(BulkArgs
   constexpr int C = 32 * V;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t full[kBulkStages], empty[kBulkStages];
+  __shared__ float g_s[2][kBulkMaxRows];  // gate dots of a chunk's rows, double-buffered
+  __shared__ float bias_s[64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t N = a.S / a.m;
   const int64_t cps = (N + a.E - 1) / a.E;  // chunks per sequence
@@ -182,70 +210,91 @@ __global__ void __launch_bounds__(kBulkThreads, 1) compress_bulk_kernel(BulkArgs
     return;
   }
 
-  // ---- consumers: warp k pools entries w0 + k, w0 + k + 16, ... of each chunk
-  float u[V];
-  load_row_mapped<T, V>(reinterpret_cast<const uint8_t*>(a.gate), lane, u);
+  // ---- consumers, two passes per chunk. Pass 1: the gate dot <x_j, u> of every row of the chunk,
+  // once per row although CSA windows overlap (rows split over the warps, into g_s). Pass 2: warp
+  // k pools entries w0 + k, w0 + k + 16, ... with the softmax of (dot + bias) over its window.
+  float2 u[(V + 1) / 2];
+  {
+    float uf[V];
+    load_row_mapped<T, V>(reinterpret_cast<const uint8_t*>(a.gate), lane, uf);
+#pragma unroll
+    for (int i = 0; i < V / 2; ++i) u[i] = make_float2(uf[2 * i], uf[2 * i + 1]);
+    if constexpr (V % 2) u[V / 2] = make_float2(uf[V - 1], 0.f);
+  }
+  for (int i = threadIdx.x; i < a.L; i += kBulkConsumers * 32) bias_s[i] = a.bias[i];
   int64_t it = 0;
   for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x, ++it) {
     const int s = (int)(it % kBulkStages);
     int b;
     int64_t w0, w1, lo, hi;
     chunk_rows(c, b, w0, w1, lo, hi);
-    if (!__all_sync(~0u, tc::mbar_wait(&full[s], (uint32_t)((it / kBulkStages) & 1), a.status)))
-      return;
+    const bool ok =
+        __all_sync(~0u, tc::mbar_wait(&full[s], (uint32_t)((it / kBulkStages) & 1), a.status));
     const uint8_t* stage = smem + (size_t)s * kBulkStageBytes;
+    float* gs = g_s[it & 1];
+    const int nrows = (int)(hi - lo);
+    if (ok) {
+      for (int r = warp; r < nrows; r += 2 * kBulkConsumers) {
+        const int r2 = r + kBulkConsumers < nrows ? r + kBulkConsumers : r;
+        uint32_t x0[M::NW], x1[M::NW];
+        load_row_raw<T, V>(stage + r * M::kRowBytes, lane, x0);
+        load_row_raw<T, V>(stage + r2 * M::kRowBytes, lane, x1);
+        float2 d0 = make_float2(0.f, 0.f), d1 = d0;
+#pragma unroll
+        for (int i = 0; i < (V + 1) / 2; ++i) {
+          d0 = __ffma2_rn(raw_pair<T, V>(x0, i), u[i], d0);
+          d1 = __ffma2_rn(raw_pair<T, V>(x1, i), u[i], d1);
+        }
+        float g0 = d0.x + d0.y, g1 = d1.x + d1.y;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          g0 += __shfl_xor_sync(~0u, g0, o);
+          g1 += __shfl_xor_sync(~0u, g1, o);
+        }
+        if (lane == 0) {
+          gs[r] = g0;
+          gs[r2] = g1;
+        }
+      }
+    }
+    // every consumer has written its dots (and learns whether all of them got the chunk)
+    if (!consumers_all(ok)) return;
     for (int64_t w = w0 + warp; w < w1; w += kBulkConsumers) {
       const int64_t whi = (w + 1) * a.m;
       const int64_t wlo = whi - a.L < 0 ? 0 : whi - a.L;
-      float acc[V];
+      const int j0 = (int)(wlo - lo), nwin = (int)(whi - wlo), boff = a.L - nwin;
+      // softmax weights of the window's rows, lane t holding rows t and t + 32
+      const float zA = lane < nwin ? gs[j0 + lane] + bias_s[boff + lane] : -INFINITY;
+      const float zB = lane + 32 < nwin ? gs[j0 + lane + 32] + bias_s[boff + lane + 32] : -INFINITY;
+      float mx = fmaxf(zA, zB);
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] = 0.f;
-      float Mx = -INFINITY, Z = 0.f;
-      for (int64_t j0 = wlo; j0 < whi; j0 += M::kBatch) {
-        uint32_t xr[M::kBatch][M::NW];
-        float g[M::kBatch];
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, o));
+      const float pA = zA == -INFINITY ? 0.f : __expf(zA - mx);
+      const float pB = zB == -INFINITY ? 0.f : __expf(zB - mx);
+      float Z = pA + pB;
 #pragma unroll
-        for (int k = 0; k < M::kBatch; ++k) {
-          const int64_t j = j0 + k < whi ? j0 + k : whi - 1;
-          load_row_raw<T, V>(stage + (j - lo) * M::kRowBytes, lane, xr[k]);
-        }
+      for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(~0u, Z, o);
+      float2 acc2[(V + 1) / 2];
 #pragma unroll
-        for (int k = 0; k < M::kBatch; ++k) {
-          float d = 0.f;
+      for (int i = 0; i < (V + 1) / 2; ++i) acc2[i] = make_float2(0.f, 0.f);
+      for (int t = 0; t < nwin; t += 2) {
+        const int t2 = t + 1 < nwin ? t + 1 : t;
+        const float p0 = __shfl_sync(~0u, t < 32 ? pA : pB, t & 31);
+        const float p1 = t + 1 < nwin ? __shfl_sync(~0u, t2 < 32 ? pA : pB, t2 & 31) : 0.f;
+        uint32_t x0[M::NW], x1[M::NW];
+        load_row_raw<T, V>(stage + (j0 + t) * M::kRowBytes, lane, x0);
+        load_row_raw<T, V>(stage + (j0 + t2) * M::kRowBytes, lane, x1);
+        const float2 q0 = make_float2(p0, p0), q1 = make_float2(p1, p1);
 #pragma unroll
-          for (int i = 0; i < V; ++i) d = fmaf(raw_elem<T, V>(xr[k], i), u[i], d);
-          g[k] = d;
-        }
-        // the batch's dot products reduce together (independent shuffle chains)
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-          for (int k = 0; k < M::kBatch; ++k) g[k] += __shfl_xor_sync(~0u, g[k], o);
-        float bm = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < M::kBatch; ++k) {
-          g[k] = j0 + k < whi ? g[k] + __ldg(a.bias + (j0 + k - whi + a.L)) : -INFINITY;
-          bm = fmaxf(bm, g[k]);
-        }
-        if (bm == -INFINITY) continue;
-        if (bm > Mx) {
-          const float sc = __expf(Mx - bm);  // 0 when Mx = -inf
-          Z *= sc;
-#pragma unroll
-          for (int i = 0; i < V; ++i) acc[i] *= sc;
-          Mx = bm;
-        }
-#pragma unroll
-        for (int k = 0; k < M::kBatch; ++k) {
-          const float p = g[k] == -INFINITY ? 0.f : __expf(g[k] - Mx);
-          Z += p;
-#pragma unroll
-          for (int i = 0; i < V; ++i) acc[i] = fmaf(p, raw_elem<T, V>(xr[k], i), acc[i]);
+        for (int i = 0; i < (V + 1) / 2; ++i) {
+          acc2[i] = __ffma2_rn(raw_pair<T, V>(x0, i), q0, acc2[i]);
+          acc2[i] = __ffma2_rn(raw_pair<T, V>(x1, i), q1, acc2[i]);
         }
       }
       const float inv = 1.f / Z;
+      float acc[V];
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] *= inv;
+      for (int i = 0; i < V; ++i) acc[i] = ((i & 1) ? acc2[i / 2].y : acc2[i / 2].x) * inv;
       if (a.rotate) {
         const int R = a.rf.R;
         const int64_t pos = a.pos0 + w * a.m;
