@@ -178,9 +178,9 @@ SAC_API int csa_forward(const sac_params* p, const void* q, const void* kv, cons
  *   topk_out [nseq,k] nullable (ascending entries, -1 fill).
  * Workspace: sac_decode_workspace_size() bytes, 16-byte aligned: a 256-byte status word (see
  * sac_device_status); for CSA the scores [nseq, S/m] fp32 and the selection [nseq, k]; and, for
- * bf16 layers with 64 heads of 512 when nseq is below the device's SM count, fp32 partial results
- * that let each sequence's keys be split over several CTAs (nseq * splits * H * (D + 2) floats,
- * splits = min(8, SMs / nseq)). ws is required by csa_decode; swa_decode / hca_decode accept NULL
+ * bf16 layers with 64 heads of 512 when nseq is at most a quarter of the device's SM count, fp32
+ * partial results that let each sequence's keys be split over several CTAs
+ * (nseq * splits * H * (D + 2) floats, splits = min(8, SMs / nseq), used only when >= 4). ws is required by csa_decode; swa_decode / hca_decode accept NULL
  * (no status word, no split) or any size of at least 256 bytes (the split is used only when the
  * workspace holds its buffers). Entries on an unallocated page (block table entry < 0) read as
  * zero keys.
@@ -233,6 +233,60 @@ SAC_API int decode_append(const sac_params* p, int kind, int nseq, const int32_t
                void* kv_pages, const int32_t* kv_block_table, int kv_max_pages, int page_size,
                void* cmp_state, void* idx_state, void* pool_pages, void* idx_pool_pages,
                const int32_t* pool_block_table, int pool_max_pages, void* stream);
+
+/*
+ * Chunked prefill over the paged caches: n query tokens per sequence, the LAST n tokens of each
+ * context (t = ctx - n .. ctx - 1, positions pos0 + t), all of which are already in the caches
+ * (prefill_chunk_append below). Each query row sees exactly what a decode step at ctx = t + 1
+ * would see: the window rows t - W + 1 .. t and the entries closed by then, (t + 1) // m of them
+ * (CSA: the indexer's top-k of those). Later tokens of the chunk already in the caches are masked
+ * by position, so the chunk attends to the cached prefix plus itself, causally.
+ * Arguments as in *_decode, with n rows per sequence: q, o [nseq, n, H, D]; q_idx [nseq, n, nI,
+ * cI]; w_idx [nseq, n, nI]; topk_out [nseq, n, k]; every ctx must satisfy n <= ctx <= p->S
+ * (rows of a sequence with ctx < n have t < 0 and see no key).
+ * Workspace: sac_chunk_workspace_size() bytes (the decode layout for nseq * n query rows; the
+ * CSA scores hold at most 1 GiB of rows at once, the indexer and top-k then run in row blocks).
+ * Decode is the case n = 1.
+ */
+SAC_API size_t sac_chunk_workspace_size(const sac_params* p, int kind, int nseq, int n);
+
+SAC_API int swa_prefill_chunk(const sac_params* p, int nseq, int n, const void* q,
+               const void* kv_pages, const int32_t* kv_block_table, int kv_max_pages,
+               const int32_t* ctx_lens, int page_size, const float* sinks, void* o, void* ws,
+               size_t ws_bytes, void* stream);
+
+SAC_API int hca_prefill_chunk(const sac_params* p, int nseq, int n, const void* q,
+               const void* kv_pages, const int32_t* kv_block_table, int kv_max_pages,
+               const int32_t* ctx_lens, int page_size, const void* pool_pages,
+               const int32_t* pool_block_table, int pool_max_pages, const float* sinks, void* o,
+               void* ws, size_t ws_bytes, void* stream);
+
+SAC_API int csa_prefill_chunk(const sac_params* p, int nseq, int n, const void* q,
+               const void* kv_pages, const int32_t* kv_block_table, int kv_max_pages,
+               const int32_t* ctx_lens, int page_size, const void* pool_pages,
+               const void* idx_pool_pages, const int32_t* pool_block_table, int pool_max_pages,
+               const void* q_idx, const float* w_idx, const float* sinks, void* o,
+               int32_t* topk_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Cache append of a prefill chunk: decode_append for n tokens per sequence at once. ctx_lens
+ * already counts the chunk, whose tokens are t = ctx - n .. ctx - 1; kv_new [nseq, n, D] and
+ * (CSA) k_idx_new [nseq, n, cI] are their un-rotated rows; every other argument as in
+ * decode_append. Each entry w that closes inside the chunk ((w+1)m - 1 >= ctx - n) is pooled
+ * exactly as the prefill compressor pools it, its rows taken from kv_new where they belong to the
+ * chunk and from the ring (which holds the win_len rows before the chunk) otherwise; then every
+ * chunk row is written rotated to the window pages and the ring keeps the sequence's last
+ * win_len rows. Appending a stream chunk by chunk (any sizes, decode steps mixed
+ * in) leaves the same caches as appending it token by token. Sequences with ctx < n are left
+ * untouched. No workspace.
+ */
+SAC_API int prefill_chunk_append(const sac_params* p, int kind, int nseq, int n,
+               const int32_t* ctx_lens, const void* kv_new, const void* k_idx_new,
+               const void* cmp_gate, const float* cmp_bias, const void* idx_gate,
+               const float* idx_bias, void* kv_pages, const int32_t* kv_block_table,
+               int kv_max_pages, int page_size, void* cmp_state, void* idx_state,
+               void* pool_pages, void* idx_pool_pages, const int32_t* pool_block_table,
+               int pool_max_pages, void* stream);
 
 /*
  * Grouped low-rank output projection ("Grouped Output Projection" bullet of the architecture

@@ -22,7 +22,9 @@ ABI_SYMBOLS = ("sac_last_error", "sac_version", "sac_workspace_size", "swa_forwa
                "hca_forward", "csa_forward", "sac_decode_workspace_size", "swa_decode",
                "hca_decode", "csa_decode", "sac_timing_begin", "sac_timing_end",
                "sac_static_scratch_bytes", "swa_forward_static", "sac_device_status",
-               "decode_append", "sac_oproj_workspace_size", "o_proj_forward")
+               "decode_append", "sac_oproj_workspace_size", "o_proj_forward",
+               "sac_chunk_workspace_size", "swa_prefill_chunk", "hca_prefill_chunk",
+               "csa_prefill_chunk", "prefill_chunk_append")
 
 
 class SacError(RuntimeError):
@@ -91,6 +93,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                vp, i32p, vp, sz, vp]
     lib.decode_append.argtypes = [P, ci, ci, i32p, vp, vp, vp, fp, vp, fp, vp, i32p, ci, ci, vp,
                                   vp, vp, vp, i32p, ci, vp]
+    lib.sac_chunk_workspace_size.restype = sz
+    lib.sac_chunk_workspace_size.argtypes = [P, ci, ci, ci]
+    for name, decode_name in (("swa_prefill_chunk", "swa_decode"),
+                              ("hca_prefill_chunk", "hca_decode"),
+                              ("csa_prefill_chunk", "csa_decode")):
+        fn = getattr(lib, name)  # the decode signature with n after nseq
+        dec = getattr(lib, decode_name).argtypes
+        fn.argtypes = dec[:2] + [ci] + dec[2:]
+    lib.prefill_chunk_append.argtypes = lib.decode_append.argtypes[:3] + [ci] + \
+        lib.decode_append.argtypes[3:]
     lib.sac_oproj_workspace_size.restype = sz
     lib.sac_oproj_workspace_size.argtypes = [P, ctypes.c_int64, ci, ci]
     lib.o_proj_forward.restype = ci
@@ -230,6 +242,54 @@ def csa_decode(p, nseq, q, kv_pages, kv_block_table, ctx_lens, page_size, pool_p
         kv_block_table.shape[1], _ptr(ctx_lens), page_size, _ptr(pool_pages),
         _ptr(idx_pool_pages), _ptr(pool_block_table), pool_block_table.shape[1], _ptr(q_idx),
         _ptr(w_idx), _ptr(sinks), _ptr(o), _ptr(topk_out), _ptr(ws), _nbytes(ws),
+        _stream(stream)))
+
+
+def sac_chunk_workspace_size(p: sac_params, kind: int, nseq: int, n: int) -> int:
+    return int(load_library().sac_chunk_workspace_size(ctypes.byref(p), kind, nseq, n))
+
+
+def swa_prefill_chunk(p, nseq, n, q, kv_pages, kv_block_table, ctx_lens, page_size, sinks, o,
+                      ws=None, stream=None) -> None:
+    """Attention of each sequence's last n tokens over the paged caches (see include/sac.h)."""
+    _check("swa_prefill_chunk", load_library().swa_prefill_chunk(
+        ctypes.byref(p), nseq, n, _ptr(q), _ptr(kv_pages), _ptr(kv_block_table),
+        kv_block_table.shape[1], _ptr(ctx_lens), page_size, _ptr(sinks), _ptr(o), _ptr(ws),
+        _nbytes(ws), _stream(stream)))
+
+
+def hca_prefill_chunk(p, nseq, n, q, kv_pages, kv_block_table, ctx_lens, page_size, pool_pages,
+                      pool_block_table, sinks, o, ws=None, stream=None) -> None:
+    _check("hca_prefill_chunk", load_library().hca_prefill_chunk(
+        ctypes.byref(p), nseq, n, _ptr(q), _ptr(kv_pages), _ptr(kv_block_table),
+        kv_block_table.shape[1], _ptr(ctx_lens), page_size, _ptr(pool_pages),
+        _ptr(pool_block_table), pool_block_table.shape[1], _ptr(sinks), _ptr(o), _ptr(ws),
+        _nbytes(ws), _stream(stream)))
+
+
+def csa_prefill_chunk(p, nseq, n, q, kv_pages, kv_block_table, ctx_lens, page_size, pool_pages,
+                      idx_pool_pages, pool_block_table, q_idx, w_idx, sinks, o, topk_out, ws,
+                      stream=None) -> None:
+    _check("csa_prefill_chunk", load_library().csa_prefill_chunk(
+        ctypes.byref(p), nseq, n, _ptr(q), _ptr(kv_pages), _ptr(kv_block_table),
+        kv_block_table.shape[1], _ptr(ctx_lens), page_size, _ptr(pool_pages),
+        _ptr(idx_pool_pages), _ptr(pool_block_table), pool_block_table.shape[1], _ptr(q_idx),
+        _ptr(w_idx), _ptr(sinks), _ptr(o), _ptr(topk_out), _ptr(ws), _nbytes(ws),
+        _stream(stream)))
+
+
+def prefill_chunk_append(p, kind, nseq, n, ctx_lens, kv_new, kv_pages, kv_block_table,
+                         page_size, cmp_state=None, cmp_gate=None, cmp_bias=None,
+                         pool_pages=None, pool_block_table=None, k_idx_new=None, idx_state=None,
+                         idx_gate=None, idx_bias=None, idx_pool_pages=None, stream=None) -> None:
+    """Append each sequence's last n tokens (kv_new [nseq, n, D]) to the caches: decode_append
+    for a whole chunk."""
+    pmax = pool_block_table.shape[1] if pool_block_table is not None else 0
+    _check("prefill_chunk_append", load_library().prefill_chunk_append(
+        ctypes.byref(p), kind, nseq, n, _ptr(ctx_lens), _ptr(kv_new), _ptr(k_idx_new),
+        _ptr(cmp_gate), _ptr(cmp_bias), _ptr(idx_gate), _ptr(idx_bias), _ptr(kv_pages),
+        _ptr(kv_block_table), kv_block_table.shape[1], page_size, _ptr(cmp_state),
+        _ptr(idx_state), _ptr(pool_pages), _ptr(idx_pool_pages), _ptr(pool_block_table), pmax,
         _stream(stream)))
 
 

@@ -91,6 +91,91 @@ __global__ void __launch_bounds__(256) append_kernel(AppendPart a) {
   store_lane<T, V>(dst, lane, acc);
 }
 
+// ---- prefill chunk: n tokens per sequence, t0 = ctx - n.
+// Entries w in [t0 / m, ctx / m) close inside the chunk (their last row (w+1)m - 1 >= t0). Their
+// rows j >= t0 come from the chunk's input, rows j < t0 from the ring, which still holds the L rows
+// before the chunk (j > t0 - L for every such window), so all entries pool in parallel; the ring
+// and page writes of the chunk's rows follow in a second launch.
+template <typename T, int V, int WPE>
+__global__ void __launch_bounds__(256) chunk_pool_kernel(AppendPart a, int n) {
+  constexpr int C = 32 * V;
+  constexpr int EPB = 8 / WPE;  // entries per block
+  __shared__ PoolShared<V, WPE> sh;
+  const int seq = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ctx = __ldg(a.ctx_lens + seq), t0 = ctx - n;
+  if (t0 < 0) return;  // fewer tokens than the chunk: left untouched
+  const int64_t w = t0 / a.m + (int64_t)blockIdx.x * EPB + warp / WPE;
+  const bool active = w < ctx / a.m;
+  if (!__syncthreads_or(active)) return;
+  const T* x_new = reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * n * C;
+  const T* ring = reinterpret_cast<const T*>(a.ring) + (int64_t)seq * a.L * C;
+  const int64_t hi = (w + 1) * a.m;
+  const int64_t lo = hi - a.L < 0 ? 0 : hi - a.L;
+  float u[V], acc[V];
+  load_lane<T, V>(reinterpret_cast<const T*>(a.gate), lane, u);
+  const int L = a.L;
+  pool_window<T, V, WPE, 4>(
+      [&](int64_t j) { return j >= t0 ? x_new + (j - t0) * C : ring + (j % L) * C; }, u, a.bias,
+      lo, hi, L, active, warp, lane, sh, acc);
+  if (!active || warp % WPE != 0) return;
+  T* dst = page_row<T>(a.pool_pages, a.pool_bt, a.pool_max_pages, a.page_size, C, seq, w);
+  if (dst == nullptr) return;
+  if (a.rotate) rotate_lane<V>(acc, lane, C, a.rf, a.pos0 + w * a.m);
+  store_lane<T, V>(dst, lane, acc);
+}
+
+// Warp per chunk token: the rotated row into the window pages, the un-rotated row into the ring
+// when it is among the sequence's last L rows.
+template <typename T, int V>
+__global__ void __launch_bounds__(256) chunk_rows_kernel(AppendPart a, int n) {
+  constexpr int C = 32 * V;
+  const int seq = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int64_t i = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int64_t ctx = __ldg(a.ctx_lens + seq), t0 = ctx - n;
+  if (t0 < 0 || i >= n) return;
+  const int64_t t = t0 + i;
+  float v[V];
+  load_lane<T, V>(reinterpret_cast<const T*>(a.x_new) + ((int64_t)seq * n + i) * C, lane, v);
+  if (a.m > 0 && t >= ctx - a.L)
+    store_lane<T, V>(reinterpret_cast<T*>(a.ring) + ((int64_t)seq * a.L + t % a.L) * C, lane, v);
+  if (a.kv_pages) {
+    T* dst = page_row<T>(a.kv_pages, a.kv_bt, a.kv_max_pages, a.page_size, C, seq, t);
+    if (dst) {
+      rotate_lane<V>(v, lane, C, a.rf, a.pos0 + t);
+      store_lane<T, V>(dst, lane, v);
+    }
+  }
+}
+
+template <typename T, int V>
+cudaError_t chunk_t(const AppendPart& a, int nseq, int n, cudaStream_t st) {
+  if (a.m > 0) {
+    const int64_t entries = (int64_t)n / a.m + 1;  // closing entries per sequence, at most
+    if (a.L >= 64)
+      chunk_pool_kernel<T, V, 8><<<dim3((unsigned)entries, nseq), 256, 0, st>>>(a, n);
+    else
+      chunk_pool_kernel<T, V, 1><<<dim3((unsigned)((entries + 7) / 8), nseq), 256, 0, st>>>(a, n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  chunk_rows_kernel<T, V><<<dim3((unsigned)((n + 7) / 8), nseq), 256, 0, st>>>(a, n);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t chunk_dispatch(const AppendPart& a, int C, int nseq, int n, cudaStream_t st) {
+  switch (C) {
+    case 32: return chunk_t<T, 1>(a, nseq, n, st);
+    case 64: return chunk_t<T, 2>(a, nseq, n, st);
+    case 128: return chunk_t<T, 4>(a, nseq, n, st);
+    case 256: return chunk_t<T, 8>(a, nseq, n, st);
+    case 512: return chunk_t<T, 16>(a, nseq, n, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <typename T, int V>
 cudaError_t append_t(const AppendPart& a, int nseq, cudaStream_t st) {
   if (a.m > 0 && a.L >= 64)
@@ -114,9 +199,7 @@ cudaError_t append_dispatch(const AppendPart& a, int C, int nseq, cudaStream_t s
 
 }  // namespace
 
-cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, bool index_part,
-                                 cudaStream_t st) {
-  if (a.nseq == 0) return cudaSuccess;
+static AppendPart make_part(const DecodeAppendArgs& a, bool index_part) {
   AppendPart p{};
   p.ctx_lens = a.ctx_lens;
   p.m = a.m;
@@ -136,18 +219,34 @@ cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, bool inde
     p.kv_max_pages = a.kv_max_pages;
     p.pool_pages = a.pool_pages;
     p.rotate = 1;
-    return dtype == 0 ? append_dispatch<float>(p, a.D, a.nseq, st)
-                      : append_dispatch<__nv_bfloat16>(p, a.D, a.nseq, st);
+  } else {
+    // the indexer part: its own ring, gate and pool, no window cache, no rotation
+    p.x_new = a.k_idx_new;
+    p.ring = a.idx_state;
+    p.gate = a.idx_gate;
+    p.bias = a.idx_bias;
+    p.pool_pages = a.idx_pool_pages;
+    p.rotate = 0;
   }
-  // the indexer part: its own ring, gate and pool, no window cache, no rotation
-  p.x_new = a.k_idx_new;
-  p.ring = a.idx_state;
-  p.gate = a.idx_gate;
-  p.bias = a.idx_bias;
-  p.pool_pages = a.idx_pool_pages;
-  p.rotate = 0;
-  return dtype == 0 ? append_dispatch<float>(p, a.cI, a.nseq, st)
-                    : append_dispatch<__nv_bfloat16>(p, a.cI, a.nseq, st);
+  return p;
+}
+
+cudaError_t launch_chunk_append(int dtype, const DecodeAppendArgs& a, int n, bool index_part,
+                                cudaStream_t st) {
+  if (a.nseq == 0 || n == 0) return cudaSuccess;
+  const AppendPart p = make_part(a, index_part);
+  const int C = index_part ? a.cI : a.D;
+  return dtype == 0 ? chunk_dispatch<float>(p, C, a.nseq, n, st)
+                    : chunk_dispatch<__nv_bfloat16>(p, C, a.nseq, n, st);
+}
+
+cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, bool index_part,
+                                 cudaStream_t st) {
+  if (a.nseq == 0) return cudaSuccess;
+  const AppendPart p = make_part(a, index_part);
+  const int C = index_part ? a.cI : a.D;
+  return dtype == 0 ? append_dispatch<float>(p, C, a.nseq, st)
+                    : append_dispatch<__nv_bfloat16>(p, C, a.nseq, st);
 }
 
 }  // namespace sac

@@ -1,7 +1,8 @@
-// Tensor-core (tcgen05) Lightning Indexer score of a decode step ("Hybrid attention", CSA bullet,
-// eq. 13-17; "Cache layers": paged indexer pool): for each sequence's single new query at
-// t = ctx - 1, I[w] = sum_h w_idx[h] * max(0, <q_idx[h], KI_w>) over the visible entries
-// w < ctx // m, bf16 layers with 64 indexer heads of dim 128.
+// Tensor-core (tcgen05) Lightning Indexer score over a paged indexer pool ("Hybrid attention",
+// CSA bullet, eq. 13-17; "Cache layers": paged indexer pool): for each query row at position t
+// (a decode step's new token t = ctx - 1, or one of a prefill chunk's last positions),
+// I[w] = sum_h w_idx[h] * max(0, <q_idx[h], KI_w>) over the visible entries w < (t + 1) // m,
+// bf16 layers with 64 indexer heads of dim 128.
 //
 // The step reads every visible indexer-pool entry once (256 bytes each) and does 64 x 128 MACs per
 // entry, so it is bound by HBM. One MMA per 128 entries puts all 64 head dot products of each
@@ -11,8 +12,8 @@
 //
 // Pool pages may have any size, so entries are gathered with 16-byte cp.async copies: sixteen
 // threads per 256-byte entry row (one fully used 512-byte span per warp instruction), three
-// 32 KB stages in flight per CTA and two CTAs per SM. Each CTA takes one (sequence, 1024-entry
-// chunk) pair; chunks past a sequence's visible entries exit at once.
+// 32 KB stages in flight per CTA and two CTAs per SM. Each CTA takes one (query row, 1024-entry
+// chunk) pair; chunks past the row's visible entries exit at once.
 //
 // Warps: 0..3 gather (q_idx once, then entry blocks), 4..7 drain, 8 issues the MMAs and owns TMEM.
 #include <cuda_bf16.h>
@@ -63,8 +64,12 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c, int region_bytes) {
 
 __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerArgs a, int* status) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int seq = blockIdx.y;
-  const int64_t t = (int64_t)__ldg(a.qr.ctx_lens + seq) - 1;
+  // row = blockIdx.y of this launch (q_idx, w_idx and scores start at the launch's first row);
+  // its sequence selects the block-table row
+  const int row = blockIdx.y;
+  int seq;
+  int64_t t;
+  a.qr.locate(a.qr.row0 + row, seq, t);
   const int64_t nvis = (t + 1) / a.m;
   const int64_t e_begin = (int64_t)blockIdx.x * kChunkBlocks * kBE;
   if (t < 0 || e_begin >= nvis) return;
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
   // head weights: plain loads before the start barrier (the drain reads them from shared memory)
   if (threadIdx.x >= 128 && threadIdx.x < 128 + kNI)
     reinterpret_cast<float*>(smem + kOffW)[threadIdx.x - 128] =
-        __ldg(a.w_idx + (int64_t)seq * kNI + (threadIdx.x - 128));
+        __ldg(a.w_idx + (int64_t)row * kNI + (threadIdx.x - 128));
 
   // Gather thread g copies 16-byte chunk (g & 15) of rows (g >> 4) + 8j; its rows share r & 7, so
   // the swizzle term is fixed per thread. Lane l of gather warp w resolves the address of row
@@ -130,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
 
   if (warp < 4) {
     // q_idx [64 heads x 128] of this sequence, then the first blocks, before the start barrier
-    const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q_idx) + (int64_t)seq * kNI * kCI;
+    const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q_idx) + (int64_t)row * kNI * kCI;
 #pragma unroll
     for (int j = 0; j < kNI / 8; ++j) {
       const int r = gr + 8 * j;
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
       tc::tc_fence_before();
       tc::mbar_arrive(&bar[kAccEmpty0 + acc]);
       const int64_t e = e_begin + (int64_t)kb * kBE + sp * 32 + lane;
-      if (e < e_end) a.scores[(int64_t)seq * a.n_stride + e] = (s0.x + s0.y) + (s1.x + s1.y);
+      if (e < e_end) a.scores[(int64_t)row * a.n_stride + e] = (s0.x + s0.y) + (s1.x + s1.y);
     }
   }
   tc::tc_fence_before();
@@ -245,9 +250,21 @@ cudaError_t launch_indexer_decode_tc(const IndexerArgs& a, int max_visible, int*
   cudaError_t e = ensure_smem_limit((const void*)indexer_decode_tc_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int chunk = kChunkBlocks * kBE;
-  dim3 grid((unsigned)((max_visible + chunk - 1) / chunk), (unsigned)a.nrows);
-  indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, status);
-  return cudaGetLastError();
+  // one launch per 65535 query rows (the grid's y limit), each with its rows' pointers
+  constexpr int64_t kMaxRowsPerLaunch = 65535;
+  for (int64_t r0 = 0; r0 < a.nrows; r0 += kMaxRowsPerLaunch) {
+    IndexerArgs b = a;
+    b.nrows = a.nrows - r0 < kMaxRowsPerLaunch ? a.nrows - r0 : kMaxRowsPerLaunch;
+    b.qr.row0 = a.qr.row0 + r0;
+    b.q_idx = reinterpret_cast<const __nv_bfloat16*>(a.q_idx) + r0 * kNI * kCI;
+    b.w_idx = a.w_idx + r0 * kNI;
+    b.scores = a.scores + r0 * a.n_stride;
+    dim3 grid((unsigned)((max_visible + chunk - 1) / chunk), (unsigned)b.nrows);
+    indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(b, status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace sac

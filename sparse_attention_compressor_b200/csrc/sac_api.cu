@@ -475,7 +475,7 @@ int sac_device_status(const void* ws, int* status, void* stream) {
 // ---------------------------------------------------------------------------------------------
 // Decode attention on tensor cores splits each sequence's key tiles over several CTAs when there
 // are fewer sequences than SMs; the partial results need nseq * splits * H * (D + 2) floats.
-static int decode_splits(const sac_params* p, int nseq) {
+static int decode_splits(const sac_params* p, int64_t rows) {
   if (!use_tc_attention(p)) return 1;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -484,40 +484,60 @@ static int decode_splits(const sac_params* p, int nseq) {
   // fp32 partials and the combine launch cost about what the shorter key walk saves (64
   // sequences on 148 SMs: CSA 3% faster, HCA 10% slower split in two; 16 sequences in 8 splits:
   // 29% and 17% faster).
-  int sp = sms / nseq;
+  int64_t sp = sms / rows;
   if (sp > sac::attention_tc_max_splits()) sp = sac::attention_tc_max_splits();
-  return sp < 4 ? 1 : sp;
+  return sp < 4 ? 1 : (int)sp;
 }
 
-static size_t decode_split_bytes(const sac_params* p, int nseq) {
-  const int sp = decode_splits(p, nseq);
+static size_t decode_split_bytes(const sac_params* p, int64_t rows) {
+  const int sp = decode_splits(p, rows);
   if (sp == 1) return 0;
-  return align_up((size_t)nseq * sp * p->H * p->D * 4) + align_up((size_t)nseq * sp * p->H * 2 * 4);
+  return align_up((size_t)rows * sp * p->H * p->D * 4) + align_up((size_t)rows * sp * p->H * 2 * 4);
 }
 
-// Point a decode call's attention at its split buffers (after the first `used` bytes of ws) when
+// Point a paged call's attention at its split buffers (after the first `used` bytes of ws) when
 // the workspace holds them; otherwise the attention runs unsplit.
-static void decode_attach_splits(const sac_params* p, int nseq, void* ws, size_t ws_bytes,
+static void decode_attach_splits(const sac_params* p, int64_t rows, void* ws, size_t ws_bytes,
                                  size_t used, sac::AttnArgs& a) {
-  const int sp = decode_splits(p, nseq);
-  const size_t need = decode_split_bytes(p, nseq);
+  const int sp = decode_splits(p, rows);
+  const size_t need = decode_split_bytes(p, rows);
   if (sp == 1 || ws == nullptr || ws_bytes < used + need) return;
   char* base = static_cast<char*>(ws) + used;
   a.splits = sp;
   a.part_o = reinterpret_cast<float*>(base);
-  a.part_ml = reinterpret_cast<float*>(base + align_up((size_t)nseq * sp * p->H * p->D * 4));
+  a.part_ml = reinterpret_cast<float*>(base + align_up((size_t)rows * sp * p->H * p->D * 4));
+}
+
+// CSA query rows whose indexer scores share the workspace at once (the rest run in blocks).
+static int64_t paged_score_rows(const sac_params* p, int64_t rows) {
+  const int64_t n = p->S / p->m;
+  int64_t per = n > 0 ? (int64_t)(kScoresBudget / ((size_t)n * 4)) : rows;
+  if (per < 1) per = 1;
+  return rows < per ? rows : per;
+}
+
+static size_t paged_workspace_size(const sac_params* p, int kind, int64_t rows) {
+  size_t bytes = kStatusBytes;
+  if (kind == SAC_KIND_CSA) {
+    const size_t n = (size_t)(p->S / p->m);
+    bytes += align_up((size_t)paged_score_rows(p, rows) * n * 4) +
+             align_up((size_t)rows * p->topk * 4);
+  }
+  return bytes + decode_split_bytes(p, rows);
 }
 
 size_t sac_decode_workspace_size(const sac_params* p, int kind, int nseq) {
   if (kind < SAC_KIND_SWA || kind > SAC_KIND_CSA || nseq < 1 ||
       check_params(p, kind, true) != SAC_OK)
     return 0;
-  size_t bytes = kStatusBytes;
-  if (kind == SAC_KIND_CSA) {
-    const size_t n = (size_t)(p->S / p->m);
-    bytes += align_up((size_t)nseq * n * 4) + align_up((size_t)nseq * p->topk * 4);
-  }
-  return bytes + decode_split_bytes(p, nseq);
+  return paged_workspace_size(p, kind, nseq);
+}
+
+size_t sac_chunk_workspace_size(const sac_params* p, int kind, int nseq, int n) {
+  if (kind < SAC_KIND_SWA || kind > SAC_KIND_CSA || nseq < 1 || n < 1 ||
+      check_params(p, kind, true) != SAC_OK)
+    return 0;
+  return paged_workspace_size(p, kind, (int64_t)nseq * n);
 }
 
 // Status word of a decode call: the first word of ws when one is given (cleared here), else none
@@ -555,26 +575,144 @@ static int check_decode_common(const sac_params* p, int kind, int nseq, const vo
   return SAC_OK;
 }
 
+// Attention of nq query rows per sequence (the last nq positions of each context; nq = 1 for a
+// decode step) over the paged caches: window keys from the kv pages, HCA pool entries or the CSA
+// indexer's top-k of the pool pages.
+struct PagedCall {
+  int kind, nseq, nq;
+  const void *q, *kv_pages;
+  const int32_t *kv_block_table, *ctx_lens;
+  int kv_max_pages, page_size;
+  const void *pool_pages, *idx_pool_pages;
+  const int32_t* pool_block_table;
+  int pool_max_pages;
+  const void* q_idx;
+  const float *w_idx, *sinks;
+  void* o;
+  int32_t* topk_out;
+  void* ws;
+  size_t ws_bytes;
+  void* stream;
+  const char* timer;  // attention timer name
+};
+
+static int paged_attention(const sac_params* p, const PagedCall& c) {
+  int rc = check_decode_common(p, c.kind, c.nseq, c.q, c.kv_pages, c.kv_block_table,
+                               c.kv_max_pages, c.ctx_lens, c.page_size, c.sinks, c.o);
+  if (rc) return rc;
+  REQUIRE(c.nq >= 1, SAC_ERR_ARG, "query rows per sequence must be >= 1 (got %d)", c.nq);
+  const int64_t rows = (int64_t)c.nseq * c.nq;
+  if (c.kind != SAC_KIND_SWA) {
+    REQUIRE(c.pool_pages != nullptr, SAC_ERR_ARG, "pool_pages must not be NULL");
+    REQUIRE(aligned16(c.pool_pages), SAC_ERR_ARG, "pool_pages must be 16-byte aligned");
+    REQUIRE(c.pool_block_table != nullptr, SAC_ERR_ARG, "pool_block_table must not be NULL");
+    REQUIRE((int64_t)c.pool_max_pages * c.page_size >= p->S / p->m, SAC_ERR_ARG,
+            "pool block table too short for S/m entries");
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(c.stream);
+  sac::QueryRows qr{0, c.ctx_lens, 0, c.nq};
+  sac::AttnArgs a = attn_common(p, c.q, c.o, c.sinks);
+  a.qr = qr;
+  a.nrows = rows;
+  a.win = paged(c.kv_pages, c.kv_block_table, c.kv_max_pages, c.page_size, p->D);
+  a.pool_mode = c.kind == SAC_KIND_SWA ? 0 : c.kind == SAC_KIND_HCA ? 1 : 2;
+  if (c.kind != SAC_KIND_SWA)
+    a.pool = paged(c.pool_pages, c.pool_block_table, c.pool_max_pages, c.page_size, p->D);
+  size_t used = kStatusBytes;
+  int* status = nullptr;
+  if (c.kind == SAC_KIND_CSA) {
+    REQUIRE(c.idx_pool_pages != nullptr, SAC_ERR_ARG, "idx_pool_pages must not be NULL");
+    REQUIRE(aligned16(c.idx_pool_pages), SAC_ERR_ARG, "idx_pool_pages must be 16-byte aligned");
+    REQUIRE(c.q_idx != nullptr, SAC_ERR_ARG, "q_idx must not be NULL");
+    REQUIRE(aligned16(c.q_idx), SAC_ERR_ARG, "q_idx must be 16-byte aligned");
+    REQUIRE(c.w_idx != nullptr, SAC_ERR_ARG, "w_idx must not be NULL");
+    REQUIRE(aligned16(c.w_idx), SAC_ERR_ARG, "w_idx must be 16-byte aligned");
+    REQUIRE(c.topk_out == nullptr || aligned16(c.topk_out), SAC_ERR_ARG,
+            "topk_out must be 16-byte aligned");
+    const int N = p->S / p->m;
+    const int64_t score_rows = paged_score_rows(p, rows);
+    const size_t need = kStatusBytes + align_up((size_t)score_rows * N * 4) +
+                        (c.topk_out ? 0 : align_up((size_t)rows * p->topk * 4));
+    REQUIRE(c.ws != nullptr && c.ws_bytes >= need, SAC_ERR_WORKSPACE,
+            "workspace of %zu bytes needed (got %zu)", need, c.ws_bytes);
+    rc = decode_status(c.ws, c.ws_bytes, st, &status);
+    if (rc) return rc;
+    Carve cv(c.ws);
+    cv.take(kStatusBytes);
+    float* scores = static_cast<float*>(cv.take((size_t)score_rows * N * 4));
+    int32_t* sel =
+        c.topk_out ? c.topk_out : static_cast<int32_t*>(cv.take((size_t)rows * p->topk * 4));
+    used = cv.used;
+    const size_t qi_row = (size_t)p->n_idx_heads * p->idx_dim * esize(p->dtype);
+    for (int64_t r0 = 0; r0 < rows; r0 += score_rows) {
+      const int64_t nr = rows - r0 < score_rows ? rows - r0 : score_rows;
+      sac::QueryRows bq{0, c.ctx_lens, r0, c.nq};
+      sac::IndexerArgs ia;
+      ia.q_idx = static_cast<const char*>(c.q_idx) + (size_t)r0 * qi_row;
+      ia.w_idx = c.w_idx + (size_t)r0 * p->n_idx_heads;
+      ia.kpool = paged(c.idx_pool_pages, c.pool_block_table, c.pool_max_pages, c.page_size,
+                       p->idx_dim);
+      ia.qr = bq;
+      ia.nI = p->n_idx_heads;
+      ia.cI = p->idx_dim;
+      ia.m = p->m;
+      ia.nrows = nr;
+      ia.n_stride = N;
+      ia.scores = scores;
+      cudaError_t e = sac::timed("indexer_score", st, [&] {
+        if (sac::indexer_decode_tc_supported(p->dtype, p->n_idx_heads, p->idx_dim))
+          return sac::launch_indexer_decode_tc(ia, N, status, st);
+        return sac::launch_indexer(p->dtype, ia, N, st);
+      });
+      if (e != cudaSuccess) return cuda_fail(e, "indexer");
+      e = sac::timed("topk", st, [&] {
+        return sac::launch_topk(scores, N, bq, p->m, nr, p->topk, sel + r0 * p->topk, st);
+      });
+      if (e != cudaSuccess) return cuda_fail(e, "top-k");
+    }
+    a.sel = sel;
+  } else {
+    rc = decode_status(c.ws, c.ws_bytes, st, &status);
+    if (rc) return rc;
+  }
+  a.status = status;
+  decode_attach_splits(p, rows, c.ws, c.ws_bytes, used, a);
+  cudaError_t e = run_attention(p, a, 1, 1, st, c.timer);
+  if (e != cudaSuccess) return cuda_fail(e, "attention");
+  return SAC_OK;
+}
+
+static PagedCall paged_call(int kind, int nseq, int nq, const void* q, const void* kv_pages,
+                            const int32_t* kv_block_table, int kv_max_pages,
+                            const int32_t* ctx_lens, int page_size, const float* sinks, void* o,
+                            void* ws, size_t ws_bytes, void* stream, const char* timer) {
+  PagedCall c;
+  std::memset(&c, 0, sizeof(c));
+  c.kind = kind;
+  c.nseq = nseq;
+  c.nq = nq;
+  c.q = q;
+  c.kv_pages = kv_pages;
+  c.kv_block_table = kv_block_table;
+  c.kv_max_pages = kv_max_pages;
+  c.ctx_lens = ctx_lens;
+  c.page_size = page_size;
+  c.sinks = sinks;
+  c.o = o;
+  c.ws = ws;
+  c.ws_bytes = ws_bytes;
+  c.stream = stream;
+  c.timer = timer;
+  return c;
+}
+
 int swa_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
                const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
                int page_size, const float* sinks, void* o, void* ws, size_t ws_bytes,
                void* stream) {
-  int rc = check_decode_common(p, SAC_KIND_SWA, nseq, q, kv_pages, kv_block_table, kv_max_pages,
-                               ctx_lens, page_size, sinks, o);
-  if (rc) return rc;
-  int* status = nullptr;
-  rc = decode_status(ws, ws_bytes, static_cast<cudaStream_t>(stream), &status);
-  if (rc) return rc;
-  sac::AttnArgs a = attn_common(p, q, o, sinks);
-  a.status = status;
-  a.qr = sac::QueryRows{0, ctx_lens, 0};
-  a.nrows = nseq;
-  a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
-  a.pool_mode = 0;
-  decode_attach_splits(p, nseq, ws, ws_bytes, kStatusBytes, a);
-  cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream), "swa_decode_attention");
-  if (e != cudaSuccess) return cuda_fail(e, "attention");
-  return SAC_OK;
+  return paged_attention(p, paged_call(SAC_KIND_SWA, nseq, 1, q, kv_pages, kv_block_table,
+                                       kv_max_pages, ctx_lens, page_size, sinks, o, ws, ws_bytes,
+                                       stream, "swa_decode_attention"));
 }
 
 int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
@@ -582,27 +720,13 @@ int hca_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
                int page_size, const void* pool_pages, const int32_t* pool_block_table,
                int pool_max_pages, const float* sinks, void* o, void* ws, size_t ws_bytes,
                void* stream) {
-  int rc = check_decode_common(p, SAC_KIND_HCA, nseq, q, kv_pages, kv_block_table, kv_max_pages,
-                               ctx_lens, page_size, sinks, o);
-  if (rc) return rc;
-  REQUIRE_PTR(pool_pages);
-  REQUIRE(pool_block_table != nullptr, SAC_ERR_ARG, "pool_block_table must not be NULL");
-  REQUIRE((int64_t)pool_max_pages * page_size >= p->S / p->m, SAC_ERR_ARG,
-          "pool block table too short for S/m entries");
-  int* status = nullptr;
-  rc = decode_status(ws, ws_bytes, static_cast<cudaStream_t>(stream), &status);
-  if (rc) return rc;
-  sac::AttnArgs a = attn_common(p, q, o, sinks);
-  a.status = status;
-  a.qr = sac::QueryRows{0, ctx_lens, 0};
-  a.nrows = nseq;
-  a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
-  a.pool_mode = 1;
-  a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
-  decode_attach_splits(p, nseq, ws, ws_bytes, kStatusBytes, a);
-  cudaError_t e = run_attention(p, a, 1, 1, static_cast<cudaStream_t>(stream), "hca_decode_attention");
-  if (e != cudaSuccess) return cuda_fail(e, "attention");
-  return SAC_OK;
+  PagedCall c = paged_call(SAC_KIND_HCA, nseq, 1, q, kv_pages, kv_block_table, kv_max_pages,
+                           ctx_lens, page_size, sinks, o, ws, ws_bytes, stream,
+                           "hca_decode_attention");
+  c.pool_pages = pool_pages;
+  c.pool_block_table = pool_block_table;
+  c.pool_max_pages = pool_max_pages;
+  return paged_attention(p, c);
 }
 
 int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_pages,
@@ -611,74 +735,75 @@ int csa_decode(const sac_params* p, int nseq, const void* q, const void* kv_page
                const int32_t* pool_block_table, int pool_max_pages, const void* q_idx,
                const float* w_idx, const float* sinks, void* o, int32_t* topk_out, void* ws,
                size_t ws_bytes, void* stream) {
-  int rc = check_decode_common(p, SAC_KIND_CSA, nseq, q, kv_pages, kv_block_table, kv_max_pages,
-                               ctx_lens, page_size, sinks, o);
-  if (rc) return rc;
-  REQUIRE_PTR(pool_pages);
-  REQUIRE_PTR(idx_pool_pages);
-  REQUIRE(pool_block_table != nullptr, SAC_ERR_ARG, "pool_block_table must not be NULL");
-  REQUIRE((int64_t)pool_max_pages * page_size >= p->S / p->m, SAC_ERR_ARG,
-          "pool block table too short for S/m entries");
-  REQUIRE_PTR(q_idx);
-  REQUIRE_PTR(w_idx);
-  OPTIONAL_PTR(topk_out);
-  const int N = p->S / p->m;
-  size_t need = kStatusBytes + align_up((size_t)nseq * N * 4) +
-                (topk_out ? 0 : align_up((size_t)nseq * p->topk * 4));
-  REQUIRE(ws != nullptr && ws_bytes >= need, SAC_ERR_WORKSPACE,
-          "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int* status = nullptr;
-  rc = decode_status(ws, ws_bytes, st, &status);
-  if (rc) return rc;
-  Carve cv(ws);
-  cv.take(kStatusBytes);
-  float* scores = static_cast<float*>(cv.take((size_t)nseq * N * 4));
-  int32_t* sel = topk_out ? topk_out : static_cast<int32_t*>(cv.take((size_t)nseq * p->topk * 4));
-  sac::QueryRows qr{0, ctx_lens, 0};
-  sac::IndexerArgs ia;
-  ia.q_idx = q_idx;
-  ia.w_idx = w_idx;
-  ia.kpool = paged(idx_pool_pages, pool_block_table, pool_max_pages, page_size, p->idx_dim);
-  ia.qr = qr;
-  ia.nI = p->n_idx_heads;
-  ia.cI = p->idx_dim;
-  ia.m = p->m;
-  ia.nrows = nseq;
-  ia.n_stride = N;
-  ia.scores = scores;
-  cudaError_t e = sac::timed("indexer_score", st, [&] {
-    if (sac::indexer_decode_tc_supported(p->dtype, p->n_idx_heads, p->idx_dim))
-      return sac::launch_indexer_decode_tc(ia, N, status, st);
-    return sac::launch_indexer(p->dtype, ia, N, st);
-  });
-  if (e != cudaSuccess) return cuda_fail(e, "indexer");
-  e = sac::timed("topk", st, [&] { return sac::launch_topk(scores, N, qr, p->m, nseq, p->topk, sel, st); });
-  if (e != cudaSuccess) return cuda_fail(e, "top-k");
-  sac::AttnArgs a = attn_common(p, q, o, sinks);
-  a.qr = qr;
-  a.nrows = nseq;
-  a.win = paged(kv_pages, kv_block_table, kv_max_pages, page_size, p->D);
-  a.pool_mode = 2;
-  a.pool = paged(pool_pages, pool_block_table, pool_max_pages, page_size, p->D);
-  a.sel = sel;
-  a.status = status;
-  decode_attach_splits(p, nseq, ws, ws_bytes, cv.used, a);
-  e = run_attention(p, a, 1, 1, st, "csa_decode_attention");
-  if (e != cudaSuccess) return cuda_fail(e, "attention");
-  return SAC_OK;
+  PagedCall c = paged_call(SAC_KIND_CSA, nseq, 1, q, kv_pages, kv_block_table, kv_max_pages,
+                           ctx_lens, page_size, sinks, o, ws, ws_bytes, stream,
+                           "csa_decode_attention");
+  c.pool_pages = pool_pages;
+  c.idx_pool_pages = idx_pool_pages;
+  c.pool_block_table = pool_block_table;
+  c.pool_max_pages = pool_max_pages;
+  c.q_idx = q_idx;
+  c.w_idx = w_idx;
+  c.topk_out = topk_out;
+  return paged_attention(p, c);
 }
 
-int decode_append(const sac_params* p, int kind, int nseq, const int32_t* ctx_lens,
-                  const void* kv_new, const void* k_idx_new, const void* cmp_gate,
-                  const float* cmp_bias, const void* idx_gate, const float* idx_bias,
-                  void* kv_pages, const int32_t* kv_block_table, int kv_max_pages, int page_size,
-                  void* cmp_state, void* idx_state, void* pool_pages, void* idx_pool_pages,
-                  const int32_t* pool_block_table, int pool_max_pages, void* stream) {
+int swa_prefill_chunk(const sac_params* p, int nseq, int n, const void* q, const void* kv_pages,
+                      const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+                      int page_size, const float* sinks, void* o, void* ws, size_t ws_bytes,
+                      void* stream) {
+  return paged_attention(p, paged_call(SAC_KIND_SWA, nseq, n, q, kv_pages, kv_block_table,
+                                       kv_max_pages, ctx_lens, page_size, sinks, o, ws, ws_bytes,
+                                       stream, "swa_chunk_attention"));
+}
+
+int hca_prefill_chunk(const sac_params* p, int nseq, int n, const void* q, const void* kv_pages,
+                      const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+                      int page_size, const void* pool_pages, const int32_t* pool_block_table,
+                      int pool_max_pages, const float* sinks, void* o, void* ws, size_t ws_bytes,
+                      void* stream) {
+  PagedCall c = paged_call(SAC_KIND_HCA, nseq, n, q, kv_pages, kv_block_table, kv_max_pages,
+                           ctx_lens, page_size, sinks, o, ws, ws_bytes, stream,
+                           "hca_chunk_attention");
+  c.pool_pages = pool_pages;
+  c.pool_block_table = pool_block_table;
+  c.pool_max_pages = pool_max_pages;
+  return paged_attention(p, c);
+}
+
+int csa_prefill_chunk(const sac_params* p, int nseq, int n, const void* q, const void* kv_pages,
+                      const int32_t* kv_block_table, int kv_max_pages, const int32_t* ctx_lens,
+                      int page_size, const void* pool_pages, const void* idx_pool_pages,
+                      const int32_t* pool_block_table, int pool_max_pages, const void* q_idx,
+                      const float* w_idx, const float* sinks, void* o, int32_t* topk_out,
+                      void* ws, size_t ws_bytes, void* stream) {
+  PagedCall c = paged_call(SAC_KIND_CSA, nseq, n, q, kv_pages, kv_block_table, kv_max_pages,
+                           ctx_lens, page_size, sinks, o, ws, ws_bytes, stream,
+                           "csa_chunk_attention");
+  c.pool_pages = pool_pages;
+  c.idx_pool_pages = idx_pool_pages;
+  c.pool_block_table = pool_block_table;
+  c.pool_max_pages = pool_max_pages;
+  c.q_idx = q_idx;
+  c.w_idx = w_idx;
+  c.topk_out = topk_out;
+  return paged_attention(p, c);
+}
+
+// Cache append of n tokens per sequence (the last n of each context); n = 0 is a decode step
+// (one token, the decode kernel), n >= 1 a prefill chunk (the chunk kernels).
+static int append_paged(const sac_params* p, int kind, int nseq, int n, const int32_t* ctx_lens,
+                        const void* kv_new, const void* k_idx_new, const void* cmp_gate,
+                        const float* cmp_bias, const void* idx_gate, const float* idx_bias,
+                        void* kv_pages, const int32_t* kv_block_table, int kv_max_pages,
+                        int page_size, void* cmp_state, void* idx_state, void* pool_pages,
+                        void* idx_pool_pages, const int32_t* pool_block_table, int pool_max_pages,
+                        void* stream) {
   REQUIRE(kind >= SAC_KIND_SWA && kind <= SAC_KIND_CSA, SAC_ERR_ARG, "unknown layer kind %d", kind);
   int rc = check_params(p, kind, true);
   if (rc) return rc;
   REQUIRE(nseq >= 1, SAC_ERR_ARG, "nseq must be >= 1 (got %d)", nseq);
+  REQUIRE(n >= 0, SAC_ERR_ARG, "chunk tokens must be >= 1 (got %d)", n);
   REQUIRE(page_size >= 1, SAC_ERR_ARG, "page_size must be >= 1 (got %d)", page_size);
   REQUIRE(ctx_lens != nullptr, SAC_ERR_ARG, "ctx_lens must not be NULL");
   REQUIRE_PTR(kv_new);
@@ -729,15 +854,52 @@ int decode_append(const sac_params* p, int kind, int nseq, const int32_t* ctx_le
     a.idx_pool_pages = idx_pool_pages;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = sac::timed("decode_append", st, [&] {
-    return sac::launch_decode_append(p->dtype, a, false, st);
-  });
-  if (e == cudaSuccess && kind == SAC_KIND_CSA)
-    e = sac::timed("decode_append_index", st, [&] {
-      return sac::launch_decode_append(p->dtype, a, true, st);
+  cudaError_t e;
+  if (n == 0) {
+    e = sac::timed("decode_append", st, [&] {
+      return sac::launch_decode_append(p->dtype, a, false, st);
     });
-  if (e != cudaSuccess) return cuda_fail(e, "decode append");
+    if (e == cudaSuccess && kind == SAC_KIND_CSA)
+      e = sac::timed("decode_append_index", st, [&] {
+        return sac::launch_decode_append(p->dtype, a, true, st);
+      });
+  } else {
+    e = sac::timed("chunk_append", st, [&] {
+      return sac::launch_chunk_append(p->dtype, a, n, false, st);
+    });
+    if (e == cudaSuccess && kind == SAC_KIND_CSA)
+      e = sac::timed("chunk_append_index", st, [&] {
+        return sac::launch_chunk_append(p->dtype, a, n, true, st);
+      });
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "cache append");
   return SAC_OK;
+}
+
+int decode_append(const sac_params* p, int kind, int nseq, const int32_t* ctx_lens,
+                  const void* kv_new, const void* k_idx_new, const void* cmp_gate,
+                  const float* cmp_bias, const void* idx_gate, const float* idx_bias,
+                  void* kv_pages, const int32_t* kv_block_table, int kv_max_pages, int page_size,
+                  void* cmp_state, void* idx_state, void* pool_pages, void* idx_pool_pages,
+                  const int32_t* pool_block_table, int pool_max_pages, void* stream) {
+  return append_paged(p, kind, nseq, 0, ctx_lens, kv_new, k_idx_new, cmp_gate, cmp_bias,
+                      idx_gate, idx_bias, kv_pages, kv_block_table, kv_max_pages, page_size,
+                      cmp_state, idx_state, pool_pages, idx_pool_pages, pool_block_table,
+                      pool_max_pages, stream);
+}
+
+int prefill_chunk_append(const sac_params* p, int kind, int nseq, int n, const int32_t* ctx_lens,
+                         const void* kv_new, const void* k_idx_new, const void* cmp_gate,
+                         const float* cmp_bias, const void* idx_gate, const float* idx_bias,
+                         void* kv_pages, const int32_t* kv_block_table, int kv_max_pages,
+                         int page_size, void* cmp_state, void* idx_state, void* pool_pages,
+                         void* idx_pool_pages, const int32_t* pool_block_table,
+                         int pool_max_pages, void* stream) {
+  REQUIRE(n >= 1, SAC_ERR_ARG, "chunk tokens must be >= 1 (got %d)", n);
+  return append_paged(p, kind, nseq, n, ctx_lens, kv_new, k_idx_new, cmp_gate, cmp_bias,
+                      idx_gate, idx_bias, kv_pages, kv_block_table, kv_max_pages, page_size,
+                      cmp_state, idx_state, pool_pages, idx_pool_pages, pool_block_table,
+                      pool_max_pages, stream);
 }
 
 size_t sac_oproj_workspace_size(const sac_params* p, int64_t T, int groups, int rank) {

@@ -72,13 +72,16 @@ struct RowAddr {
 // Query rows: prefill row r = seq*S + t; decode row r = seq with t = ctx_lens[seq] - 1.
 struct QueryRows {
   int S;                     // prefill tokens per sequence (0 for decode)
-  const int32_t* ctx_lens;   // decode only
+  const int32_t* ctx_lens;   // decode / chunked prefill only
   int64_t row0;              // first flat row of this launch (prefill chunking)
+  int nq;                    // with ctx_lens: query rows per sequence, the last nq positions
+                             // (0 or 1: one query per sequence, decode)
 
   __device__ __forceinline__ void locate(int64_t r, int& seq, int64_t& t) const {
     if (ctx_lens != nullptr) {
-      seq = (int)r;
-      t = (int64_t)__ldg(ctx_lens + r) - 1;
+      const int q = nq > 1 ? nq : 1;
+      seq = (int)(r / q);
+      t = (int64_t)__ldg(ctx_lens + seq) - q + r % q;
     } else {
       seq = (int)(r / S);
       t = r % S;

@@ -31,8 +31,8 @@ struct DecodeAppendArgs {
   int D, cI, m, L;
   int64_t pos0;
   RopeFreqs rf;
-  const void* kv_new;         // [nseq, D] un-rotated
-  const void* k_idx_new;      // [nseq, cI] (CSA)
+  const void* kv_new;         // [nseq, n, D] un-rotated (n = 1 for a decode step)
+  const void* k_idx_new;      // [nseq, n, cI] (CSA)
   const void* cmp_gate;       // [D]
   const float* cmp_bias;      // [L]
   const void* idx_gate;       // [cI] (CSA)
@@ -50,6 +50,10 @@ struct DecodeAppendArgs {
 // index_part = false: the kv row and the main pool; true: the indexer ring and pool (CSA).
 cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, bool index_part,
                                  cudaStream_t st);
+// The same for a prefill chunk of n tokens per sequence at t = ctx - n .. ctx - 1 (two launches:
+// the entries that close inside the chunk, then the rows' page and ring writes).
+cudaError_t launch_chunk_append(int dtype, const DecodeAppendArgs& a, int n, bool index_part,
+                                cudaStream_t st);
 
 // ---- grouped output projection (oproj.cu, cuBLASLt GEMMs) ---------------------------------
 struct OProjArgs {

@@ -189,3 +189,30 @@ def test_oproj_validation_and_workspace():
     p32 = sac.make_params(1, 64, 64, 512, 64, 1e4, dtype="f32")
     assert call(params=p32) == -2
     assert call(T=0) == 0  # nothing to do: no launch, no device touched
+
+
+def test_chunk_validation_and_workspace():
+    lib = sac.load_library()
+    fake = 1 << 20
+    p = p_csa(S=65536)
+    # the decode layout for nseq * n rows: 4 * 16 = 64 rows -> no split; the CSA scores of all
+    # 64 rows fit the 1 GiB budget
+    assert sac.sac_chunk_workspace_size(p, sac.SAC_KIND_CSA, 4, 16) == \
+        sac.sac_decode_workspace_size(p, sac.SAC_KIND_CSA, 64)
+    assert sac.sac_chunk_workspace_size(p, sac.SAC_KIND_CSA, 4, 0) == 0
+    # 16 Ki rows of 16 Ki entries: scores capped at 1 GiB (16 Ki rows x 64 KiB = 1 GiB exactly)
+    big = sac.sac_chunk_workspace_size(p, sac.SAC_KIND_CSA, 8, 4096)
+    assert big == 256 + (1 << 30) + 8 * 4096 * 512 * 4
+    big2 = sac.sac_chunk_workspace_size(p, sac.SAC_KIND_CSA, 16, 4096)
+    assert big2 == 256 + (1 << 30) + 16 * 4096 * 512 * 4
+    # n < 1 is rejected before any device work
+    rc = lib.swa_prefill_chunk(ctypes.byref(p), 2, 0, fake, fake, fake, 64, fake, 1024, fake,
+                               fake, None, 0, None)
+    assert rc == -1 and "query rows" in lib.sac_last_error().decode()
+    rc = lib.prefill_chunk_append(ctypes.byref(p), sac.SAC_KIND_SWA, 2, 0, fake, fake, None, None,
+                                  None, None, None, fake, fake, 64, 1024, None, None, None, None,
+                                  None, 0, None)
+    assert rc == -1 and "chunk tokens" in lib.sac_last_error().decode()
+    rc = lib.hca_prefill_chunk(ctypes.byref(p), 2, 8, fake, fake, fake, 64, fake, 1024, None,
+                               fake, 16, fake, fake, None, 0, None)
+    assert rc == -1 and "pool_pages" in lib.sac_last_error().decode()
