@@ -462,6 +462,37 @@ def decode_bytes(wl, d_csa, d_hca) -> dict:
     return out
 
 
+def chunk_work(wl, d_csa, d_hca) -> dict:
+    """Algorithmic work per chunked-prefill step: FLOPs of the contractions (indexer scores and
+    attention, tensor-bound: every chunk row re-uses the same cached rows), bytes of the rest."""
+    esz, n = 2, wl.chunk
+    out = {}
+    ctx = d_csa["ctx_lens"].numpy().astype(np.int64)
+    t = (ctx[:, None] - n + np.arange(n)[None, :])  # [nseq, n] positions of the chunk rows
+    nv = (t + 1) // wl.m
+    win = np.minimum(t + 1, wl.W)
+    out["indexer_score"] = ("flops", float((nv * 2 * wl.nI * wl.cI).sum()))
+    out["topk"] = ("bytes", float((nv * 4).sum() + t.size * wl.k * 4))
+    out["csa_chunk_attention"] = ("flops", float(((np.minimum(nv, wl.k) + win)
+                                                  * 4 * wl.H * wl.D).sum()))
+    ctx_h = d_hca["ctx_lens"].numpy().astype(np.int64)
+    th = (ctx_h[:, None] - n + np.arange(n)[None, :])
+    out["hca_chunk_attention"] = ("flops", float(((th + 1) // d_hca["m"] + np.minimum(th + 1, wl.W))
+                                                 .sum() * 4 * wl.H * wl.D))
+    # append: every chunk row read once and written rotated (plus the ring's last L rows); each
+    # closing entry reads its L rows and writes one
+    app = 0.0
+    for d, m, L in ((d_csa, wl.m, wl.L), (d_hca, d_hca["m"], d_hca["m"])):
+        c = d["ctx_lens"].numpy().astype(np.int64)
+        closing = (c // m - (c - n) // m).sum()
+        app += (2 * t.size + wl.nseq * min(L, n)) * wl.D * esz + closing * (L + 1) * wl.D * esz
+    out["chunk_append"] = ("bytes", float(app))
+    closing = (ctx // wl.m - (ctx - n) // wl.m).sum()
+    out["chunk_append_index"] = ("bytes", float((t.size + wl.nseq * min(wl.L, n)) * wl.cI * esz
+                                                + closing * (wl.L + 1) * wl.cI * esz))
+    return out
+
+
 def run_decode(args, wl0):
     import sparse_attention_compressor_b200 as sac
     world, rank, local = dist_env()
@@ -479,15 +510,45 @@ def run_decode(args, wl0):
                          dtype=wl.dtype)
     ph = sac.make_params(1, max_ctx, wl.H, wl.D, wl.R, wl.theta, m=dh["m"], win_len=dh["m"],
                          sliding_window=wl.W, dtype=wl.dtype)
-    ws = torch.empty(sac.sac_decode_workspace_size(pc, sac.SAC_KIND_CSA, wl.nseq),
-                     dtype=torch.uint8, device=dev)
-    ws_h = torch.empty(sac.sac_decode_workspace_size(ph, sac.SAC_KIND_HCA, wl.nseq),
-                       dtype=torch.uint8, device=dev)
+    n = wl.chunk
+    if n > 1:
+        ws = torch.empty(sac.sac_chunk_workspace_size(pc, sac.SAC_KIND_CSA, wl.nseq, n),
+                         dtype=torch.uint8, device=dev)
+        ws_h = torch.empty(sac.sac_chunk_workspace_size(ph, sac.SAC_KIND_HCA, wl.nseq, n),
+                           dtype=torch.uint8, device=dev)
+    else:
+        ws = torch.empty(sac.sac_decode_workspace_size(pc, sac.SAC_KIND_CSA, wl.nseq),
+                         dtype=torch.uint8, device=dev)
+        ws_h = torch.empty(sac.sac_decode_workspace_size(ph, sac.SAC_KIND_HCA, wl.nseq),
+                           dtype=torch.uint8, device=dev)
     oc = torch.empty_like(gc["q"])
     oh = torch.empty_like(gh["q"])
     ps = wl.page_size
 
-    def step():
+    def chunk_step():
+        # each layer: append the chunk's tokens to its caches, then attend
+        sac.prefill_chunk_append(pc, sac.SAC_KIND_CSA, wl.nseq, n, gc["ctx_lens"], gc["kv_new"],
+                                 gc["kv_pages"], gc["kv_block_table"], ps,
+                                 cmp_state=gc["cmp_state"], cmp_gate=gc["cmp_gate"],
+                                 cmp_bias=gc["cmp_bias"], pool_pages=gc["pool_pages"],
+                                 pool_block_table=gc["pool_block_table"],
+                                 k_idx_new=gc["k_idx_new"], idx_state=gc["idx_state"],
+                                 idx_gate=gc["idx_gate"], idx_bias=gc["idx_bias"],
+                                 idx_pool_pages=gc["idx_pool_pages"])
+        sac.csa_prefill_chunk(pc, wl.nseq, n, gc["q"], gc["kv_pages"], gc["kv_block_table"],
+                              gc["ctx_lens"], ps, gc["pool_pages"], gc["idx_pool_pages"],
+                              gc["pool_block_table"], gc["q_idx"], gc["w_idx"], gc["sinks"], oc,
+                              None, ws)
+        sac.prefill_chunk_append(ph, sac.SAC_KIND_HCA, wl.nseq, n, gh["ctx_lens"], gh["kv_new"],
+                                 gh["kv_pages"], gh["kv_block_table"], ps,
+                                 cmp_state=gh["cmp_state"], cmp_gate=gh["cmp_gate"],
+                                 cmp_bias=gh["cmp_bias"], pool_pages=gh["pool_pages"],
+                                 pool_block_table=gh["pool_block_table"])
+        sac.hca_prefill_chunk(ph, wl.nseq, n, gh["q"], gh["kv_pages"], gh["kv_block_table"],
+                              gh["ctx_lens"], ps, gh["pool_pages"], gh["pool_block_table"],
+                              gh["sinks"], oh, ws_h)
+
+    def decode_step():
         # each layer: append the new token to its caches, then attend
         sac.decode_append(pc, sac.SAC_KIND_CSA, wl.nseq, gc["ctx_lens"], gc["kv_new"],
                           gc["kv_pages"], gc["kv_block_table"], ps, cmp_state=gc["cmp_state"],
@@ -506,6 +567,7 @@ def run_decode(args, wl0):
         sac.hca_decode(ph, wl.nseq, gh["q"], gh["kv_pages"], gh["kv_block_table"], gh["ctx_lens"],
                        ps, gh["pool_pages"], gh["pool_block_table"], gh["sinks"], oh, ws_h)
 
+    step = chunk_step if n > 1 else decode_step
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -546,33 +608,56 @@ def run_decode(args, wl0):
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
     d2h = (oc.numel() + oh.numel()) * oc.element_size()
     peaks = measured_peaks()
-    wb = decode_bytes(wl, dc, dh)
+    if n > 1:
+        wb = chunk_work(wl, dc, dh)
+    else:
+        wb = {k: ("bytes", v) for k, v in decode_bytes(wl, dc, dh).items()}
     krows = {}
     total = sum(v[1] for v in ktimes.values()) or 1.0
     for name, (launches, kms) in ktimes.items():
         per = kms / max(launches, 1)
         row = {"launches": launches, "ms_per_launch": per, "share": kms / total}
         if name in wb:
-            per_launch_bytes = wb[name] / launches
-            ach = per_launch_bytes / (per * 1e-3) / 1e9
-            row.update(bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
-                       frac=ach / peaks["hbm_gbs"])
+            kind, amount = wb[name]
+            if kind == "bytes":
+                ach = amount / launches / (per * 1e-3) / 1e9
+                row.update(bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
+                           frac=ach / peaks["hbm_gbs"])
+            else:
+                ach = amount / launches / (per * 1e-3) / 1e12
+                row.update(bound="tensor", achieved=ach, peak=peaks["bf16_tflops"],
+                           unit="TFLOP/s", frac=ach / peaks["bf16_tflops"])
         krows[name] = row
     dom = max(ktimes, key=lambda k: ktimes[k][1])
     d = krows[dom]
+    cfg = {"workload": wl.name, "nseq": wl.nseq, "ctx": f"U[{wl.ctx_lo},{wl.ctx_hi}]",
+           "page_size": wl.page_size, "H": wl.H, "head_dim": wl.D, "csa_m": wl.m,
+           "hca_m": dh["m"], "index_topk": wl.k, "sliding_window": wl.W,
+           "parallelism": f"dp{world}",
+           "l2": "flushed before every step (252 MiB written, then another 252 MiB read)",
+           "launch": "one CUDA graph replay per step (cache append + both layers)"}
+    if n > 1:
+        cfg["chunk"] = n
+        tok_s = wl.nseq * n * world / (us_step * 1e-6)
+        head = {"metric": f"chunked prefill tokens/s (CSA + HCA layer, {wl.nseq} sequences x {n}"
+                          " tokens against a cached prefix)",
+                "value": tok_s, "unit": "tokens/s", "higher_is_better": True}
+        e2e = {"value": wl.nseq * n * world / (e2e_us * 1e-6), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    else:
+        head = {"metric": "decode us/step (CSA + HCA layer, 64 sequences)", "value": us_step,
+                "unit": "us/step", "higher_is_better": False}
+        e2e = {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
     line = {
-        "metric": "decode us/step (CSA + HCA layer, 64 sequences)", "value": us_step,
-        "unit": "us/step", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": us_step / 1e3, "higher_is_better": False, "scaling": "weak",
+        "metric": head["metric"], "value": head["value"],
+        "unit": head["unit"], "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us_step / 1e3, "higher_is_better": head["higher_is_better"],
+        "scaling": "weak",
         "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded; see DESIGN.md)",
-        "config": {"workload": wl.name, "nseq": wl.nseq, "ctx": f"U[{wl.ctx_lo},{wl.ctx_hi}]",
-                   "page_size": wl.page_size, "H": wl.H, "head_dim": wl.D, "csa_m": wl.m,
-                   "hca_m": dh["m"], "index_topk": wl.k, "sliding_window": wl.W,
-                   "parallelism": f"dp{world}", "l2": "flushed before every step (252 MiB written, then another 252 MiB read)",
-                   "launch": "one CUDA graph replay per step (cache append + both layers)"},
+        "config": cfg,
         "clocks": clk.summary(),
-        "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "e2e": e2e,
         "gpu_launches": sum(v[0] for v in ktimes.values()) * args.steps,
         "roofline": {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
                      "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),

@@ -56,6 +56,7 @@ class Workload:
     ctx_hi: int = 0
     page_size: int = 64
     hca_m: int = 128
+    chunk: int = 1            # query tokens per sequence and step (> 1: chunked prefill)
     # output projection only
     o_groups: int = 0
     o_rank: int = 0
@@ -83,6 +84,10 @@ WORKLOADS: Dict[str, Workload] = {
                               cI=128, k=512, spike_frac=0.05, seed=1237),
     "decode_bf16": Workload("decode_bf16", "decode", "bf16", nseq=64, ctx_lo=4096, ctx_hi=65536,
                             page_size=64, m=4, L=8, nI=64, cI=128, k=512, hca_m=128, seed=1238),
+    # Chunked prefill: 8 sequences each take their next 1024 tokens against a cached prefix.
+    "chunk_bf16": Workload("chunk_bf16", "decode", "bf16", nseq=8, ctx_lo=16384, ctx_hi=65536,
+                           page_size=64, m=4, L=8, nI=64, cI=128, k=512, hca_m=128, chunk=1024,
+                           seed=1240),
     # Grouped output projection of 8192 tokens: 64 heads of 512 in 8 groups of rank 1024 to 4096.
     "oproj_8k_bf16": Workload("oproj_8k_bf16", "oproj", "bf16", B=1, S=8192, o_groups=8,
                               o_rank=1024, hidden=4096, seed=1239),
@@ -245,14 +250,18 @@ def _paged(wl: Workload, tensor: str, perm_tensor: str, lens: np.ndarray, width:
 
 
 def decode_inputs(wl: Workload, layer: str) -> Dict[str, object]:
-    """Inputs of one decode step of the CSA layer ('csa') or the HCA layer ('hca')."""
+    """Inputs of one decode step of the CSA layer ('csa') or the HCA layer ('hca'); with
+    wl.chunk = n > 1, of one prefill chunk: the per-token tensors gain an n axis after the
+    sequence axis and ctx counts the chunk."""
     dt = wl.torch_dtype
     g = _gen(wl.seed, "ctx", 0)
     ctx = torch.randint(wl.ctx_lo, wl.ctx_hi + 1, (wl.nseq,), generator=g).to(torch.int32)
     lens = ctx.numpy()
     pfx = "" if layer == "csa" else "hca_"
     m = wl.m if layer == "csa" else wl.hca_m
-    win_start = np.maximum(lens - wl.W, 0)
+    n = wl.chunk
+    tok = (wl.nseq,) if n == 1 else (wl.nseq, n)  # leading shape of the per-token tensors
+    win_start = np.maximum(lens - wl.W - (n - 1), 0)
     kv = _paged(wl, pfx + "kv_pages", "pages" if layer == "csa" else "hca_page_perm", lens,
                 wl.D, win_start, dt)
     npool = lens // m
@@ -260,12 +269,12 @@ def decode_inputs(wl: Workload, layer: str) -> Dict[str, object]:
                   np.maximum(npool, 1), wl.D, None, dt)
     out = {"ctx_lens": ctx, "kv_pages": kv.pages, "kv_block_table": kv.block_table,
            "pool_pages": pool.pages, "pool_block_table": pool.block_table, "m": m,
-           "q": _normal((wl.nseq, wl.H, wl.D), 1.0, wl.seed, "q", 10 ** 6 + (layer == "hca"))
+           "q": _normal(tok + (wl.H, wl.D), 1.0, wl.seed, "q", 10 ** 6 + (layer == "hca"))
            .to(dt),
            "sinks": _normal((wl.H,), 1.0, wl.seed, "sinks" if layer == "csa" else "hca_sinks")}
     # the step's cache append: the new token's un-rotated kv row, the compressor gate and ring
     L = wl.L if layer == "csa" else m
-    out["kv_new"] = _normal((wl.nseq, wl.D), 1.0, wl.seed, "kv_new", layer == "hca").to(dt)
+    out["kv_new"] = _normal(tok + (wl.D,), 1.0, wl.seed, "kv_new", layer == "hca").to(dt)
     out["cmp_gate"] = _normal((wl.D,), 1.0 / math.sqrt(wl.D), wl.seed,
                               "cmp_gate" if layer == "csa" else "hca_cmp_gate").to(dt)
     out["cmp_bias"] = _normal((L,), 1.0 / math.sqrt(L), wl.seed,
@@ -273,15 +282,15 @@ def decode_inputs(wl: Workload, layer: str) -> Dict[str, object]:
     out["cmp_state"] = _normal((wl.nseq, L, wl.D), 1.0, wl.seed, "cmp_state",
                                layer == "hca").to(dt)
     if layer == "csa":
-        out["k_idx_new"] = _normal((wl.nseq, wl.cI), 1.0, wl.seed, "k_idx_new").to(dt)
+        out["k_idx_new"] = _normal(tok + (wl.cI,), 1.0, wl.seed, "k_idx_new").to(dt)
         out["idx_gate"] = _normal((wl.cI,), 1.0 / math.sqrt(wl.cI), wl.seed, "idx_gate").to(dt)
         out["idx_bias"] = _normal((L,), 1.0 / math.sqrt(L), wl.seed, "idx_bias")
         out["idx_state"] = _normal((wl.nseq, L, wl.cI), 1.0, wl.seed, "idx_state").to(dt)
         ipool = _paged(wl, "idx_pool_pages", "pages", np.maximum(npool, 1), wl.cI, None, dt)
         assert torch.equal(ipool.block_table, pool.block_table)
         out["idx_pool_pages"] = ipool.pages
-        out["q_idx"] = _normal((wl.nseq, wl.nI, wl.cI), 1.0, wl.seed, "q_idx", 10 ** 6).to(dt)
-        out["w_idx"] = _normal((wl.nseq, wl.nI), 1.0 / math.sqrt(wl.nI), wl.seed, "w_idx",
+        out["q_idx"] = _normal(tok + (wl.nI, wl.cI), 1.0, wl.seed, "q_idx", 10 ** 6).to(dt)
+        out["w_idx"] = _normal(tok + (wl.nI,), 1.0 / math.sqrt(wl.nI), wl.seed, "w_idx",
                                10 ** 6)
     return out
 
