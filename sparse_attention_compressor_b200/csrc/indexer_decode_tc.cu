@@ -34,18 +34,25 @@ constexpr int kGatherThreads = 128;
 constexpr int kThreads = 288;
 constexpr int kRegion = kBE * 128;        // one 64-dim half of a block: [128 rows x 128 B]
 constexpr int kBlockBytes = 2 * kRegion;  // 32 KB
-constexpr int kQRegion = kNI * 128;       // [64 rows x 128 B]
-constexpr int kQBytes = 2 * kQRegion;     // 16 KB
-
-constexpr int kOffKv = 0;
-constexpr int kOffQ = kOffKv + kStages * kBlockBytes;
-constexpr int kOffW = kOffQ + kQBytes;
-constexpr int kOffBar = kOffW + kNI * 4;
 enum Bar { kFull0, kEmpty0 = kFull0 + kStages, kAccFull0 = kEmpty0 + kStages, kAccEmpty0 = kAccFull0 + 2,
            kNumBars = kAccEmpty0 + 2 };
-constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffTmemPtr + 16;  // two CTAs per SM fit in 228 KB
-constexpr uint32_t kIdesc = tc::idesc_bf16(kBE, kNI, false, false);
+
+// Layout for Q query rows per CTA (Q = 1: a decode step; Q = 4: four consecutive rows of one
+// sequence in a prefill chunk, which then share every gathered entry block). MMA N = 64 Q.
+template <int Q>
+struct Cfg {
+  static constexpr int kN = kNI * Q;
+  static constexpr int kQRegion = kN * 128;  // [N rows x 128 B]
+  static constexpr int kQBytes = 2 * kQRegion;
+  static constexpr int kOffKv = 0;
+  static constexpr int kOffQ = kOffKv + kStages * kBlockBytes;
+  static constexpr int kOffW = kOffQ + kQBytes;
+  static constexpr int kOffBar = kOffW + kN * 4;
+  static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffTmemPtr + 16;  // Q = 1: two CTAs per SM fit
+  static constexpr uint32_t kTmemCols = 2 * kN < 32 ? 32 : 2 * kN;  // two accumulators
+  static constexpr uint32_t kIdesc = tc::idesc_bf16(kBE, kN, false, false);
+};
 
 // cp.async.wait_group with the stage depth as its immediate.
 __device__ __forceinline__ void cp_async_commit() {
@@ -62,15 +69,20 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c, int region_bytes) {
   return (uint32_t)((c >> 3) * region_bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+template <int Q>
 __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerArgs a, int* status) {
+  using K = Cfg<Q>;
+  constexpr int kOffQ = K::kOffQ, kOffW = K::kOffW, kOffBar = K::kOffBar;
+  constexpr int kOffKv = K::kOffKv, kOffTmemPtr = K::kOffTmemPtr, kQRegion = K::kQRegion;
   extern __shared__ __align__(1024) uint8_t smem[];
-  // row = blockIdx.y of this launch (q_idx, w_idx and scores start at the launch's first row);
-  // its sequence selects the block-table row
-  const int row = blockIdx.y;
+  // rows row .. row + Q - 1 of this launch (q_idx, w_idx and scores start at the launch's first
+  // row), all of one sequence, whose block-table row the gathers use
+  const int row = blockIdx.y * Q;
   int seq;
-  int64_t t;
-  a.qr.locate(a.qr.row0 + row, seq, t);
-  const int64_t nvis = (t + 1) / a.m;
+  int64_t t_first, t;
+  a.qr.locate(a.qr.row0 + row, seq, t_first);
+  a.qr.locate(a.qr.row0 + row + Q - 1, seq, t);  // the last row sees the most entries
+  const int64_t nvis = t < 0 ? 0 : (t + 1) / a.m;
   const int64_t e_begin = (int64_t)blockIdx.x * kChunkBlocks * kBE;
   if (t < 0 || e_begin >= nvis) return;
   const int64_t e_end = nvis < e_begin + kChunkBlocks * kBE ? nvis : e_begin + kChunkBlocks * kBE;
@@ -97,11 +109,10 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
     }
     tc::fence_barrier_init();
   }
-  if (warp == 8) tc::tmem_alloc(tmem_ptr, 128);
+  if (warp == 8) tc::tmem_alloc(tmem_ptr, K::kTmemCols);
   // head weights: plain loads before the start barrier (the drain reads them from shared memory)
-  if (threadIdx.x >= 128 && threadIdx.x < 128 + kNI)
-    reinterpret_cast<float*>(smem + kOffW)[threadIdx.x - 128] =
-        __ldg(a.w_idx + (int64_t)row * kNI + (threadIdx.x - 128));
+  for (int i = threadIdx.x - 128; i >= 0 && i < K::kN && threadIdx.x < 256; i += 128)
+    reinterpret_cast<float*>(smem + kOffW)[i] = __ldg(a.w_idx + (int64_t)row * kNI + i);
 
   // Gather thread g copies 16-byte chunk (g & 15) of rows (g >> 4) + 8j; its rows share r & 7, so
   // the swizzle term is fixed per thread. Lane l of gather warp w resolves the address of row
@@ -134,10 +145,11 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
   };
 
   if (warp < 4) {
-    // q_idx [64 heads x 128] of this sequence, then the first blocks, before the start barrier
+    // q_idx [Q rows x 64 heads x 128] (consecutive in memory), then the first blocks, before the
+    // start barrier
     const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q_idx) + (int64_t)row * kNI * kCI;
 #pragma unroll
-    for (int j = 0; j < kNI / 8; ++j) {
+    for (int j = 0; j < K::kN / 8; ++j) {
       const int r = gr + 8 * j;
       tc::cp_async16(smem + kOffQ + sw_off(r, gc, kQRegion), q + r * kCI + gc * 8);
     }
@@ -187,10 +199,10 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
         const uint32_t kv_base = tc::smem_u32(smem + kOffKv + s * kBlockBytes);
 #pragma unroll
         for (int kk = 0; kk < kCI / 16; ++kk)
-          tc::mma_bf16_ss(tmem + acc * kNI,
+          tc::mma_bf16_ss(tmem + acc * K::kN,
                           tc::desc_sw128(kv_base + (kk >> 2) * kRegion + (kk & 3) * 32, 0, 1024),
                           tc::desc_sw128(q_base + (kk >> 2) * kQRegion + (kk & 3) * 32, 0, 1024),
-                          kIdesc, kk > 0);
+                          K::kIdesc, kk > 0);
         tc::mma_commit(&bar[kEmpty0 + s]);
         tc::mma_commit(&bar[kAccFull0 + acc]);
       }
@@ -207,35 +219,67 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
       ok = __all_sync(~0u, tc::mbar_wait(&bar[kAccFull0 + acc], (kb >> 1) & 1, status));
       if (!ok) break;
       tc::tc_fence_after();
-      float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+      const int64_t e = e_begin + (int64_t)kb * kBE + sp * 32 + lane;
+      float score[Q];
 #pragma unroll
-      for (int c = 0; c < kNI; c += 16) {
-        uint32_t v[16];
-        tc::tmem_ld16(t_lane + acc * kNI + c, v);
-        tc::tmem_wait_ld();
+      for (int qi = 0; qi < Q; ++qi) {
+        float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int u = 0; u < 16; u += 4) {
-          const float4 wv = w4[(c + u) / 4];
-          const float2 x0 = make_float2(fmaxf(__uint_as_float(v[u]), 0.f),
-                                        fmaxf(__uint_as_float(v[u + 1]), 0.f));
-          const float2 x1 = make_float2(fmaxf(__uint_as_float(v[u + 2]), 0.f),
-                                        fmaxf(__uint_as_float(v[u + 3]), 0.f));
-          s0 = __ffma2_rn(x0, make_float2(wv.x, wv.y), s0);
-          s1 = __ffma2_rn(x1, make_float2(wv.z, wv.w), s1);
+        for (int c = 0; c < kNI; c += 16) {
+          uint32_t v[16];
+          tc::tmem_ld16(t_lane + acc * K::kN + qi * kNI + c, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 16; u += 4) {
+            const float4 wv = w4[(qi * kNI + c + u) / 4];
+            const float2 x0 = make_float2(fmaxf(__uint_as_float(v[u]), 0.f),
+                                          fmaxf(__uint_as_float(v[u + 1]), 0.f));
+            const float2 x1 = make_float2(fmaxf(__uint_as_float(v[u + 2]), 0.f),
+                                          fmaxf(__uint_as_float(v[u + 3]), 0.f));
+            s0 = __ffma2_rn(x0, make_float2(wv.x, wv.y), s0);
+            s1 = __ffma2_rn(x1, make_float2(wv.z, wv.w), s1);
+          }
         }
+        score[qi] = (s0.x + s0.y) + (s1.x + s1.y);
       }
       tc::tc_fence_before();
       tc::mbar_arrive(&bar[kAccEmpty0 + acc]);
-      const int64_t e = e_begin + (int64_t)kb * kBE + sp * 32 + lane;
-      if (e < e_end) a.scores[(int64_t)row * a.n_stride + e] = (s0.x + s0.y) + (s1.x + s1.y);
+      // row qi sees the entries w < (t_first + qi + 1) // m (consecutive positions)
+#pragma unroll
+      for (int qi = 0; qi < Q; ++qi)
+        if (e < e_end && e < (t_first + qi + 1) / a.m)
+          a.scores[(int64_t)(row + qi) * a.n_stride + e] = score[qi];
     }
   }
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 8) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, 128);
+    tc::tmem_dealloc(tmem, K::kTmemCols);
   }
+}
+
+template <int Q>
+cudaError_t launch_q(const IndexerArgs& a, int max_visible, int* status, cudaStream_t st) {
+  using K = Cfg<Q>;
+  cudaError_t e = ensure_smem_limit((const void*)indexer_decode_tc_kernel<Q>, K::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int chunk = kChunkBlocks * kBE;
+  // one launch per 65535 CTA rows (the grid's y limit), each with its rows' pointers
+  constexpr int64_t kMaxRowsPerLaunch = 65535 * (int64_t)Q;
+  for (int64_t r0 = 0; r0 < a.nrows; r0 += kMaxRowsPerLaunch) {
+    IndexerArgs b = a;
+    b.nrows = a.nrows - r0 < kMaxRowsPerLaunch ? a.nrows - r0 : kMaxRowsPerLaunch;
+    b.qr.row0 = a.qr.row0 + r0;
+    b.q_idx = reinterpret_cast<const __nv_bfloat16*>(a.q_idx) + r0 * kNI * kCI;
+    b.w_idx = a.w_idx + r0 * kNI;
+    b.scores = a.scores + r0 * a.n_stride;
+    dim3 grid((unsigned)((max_visible + chunk - 1) / chunk), (unsigned)(b.nrows / Q));
+    indexer_decode_tc_kernel<Q><<<grid, kThreads, K::kSmemBytes, st>>>(b, status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -247,24 +291,12 @@ bool indexer_decode_tc_supported(int dtype, int nI, int cI) {
 cudaError_t launch_indexer_decode_tc(const IndexerArgs& a, int max_visible, int* status,
                                      cudaStream_t st) {
   if (a.nrows == 0 || max_visible == 0) return cudaSuccess;
-  cudaError_t e = ensure_smem_limit((const void*)indexer_decode_tc_kernel, kSmemBytes);
-  if (e != cudaSuccess) return e;
-  const int chunk = kChunkBlocks * kBE;
-  // one launch per 65535 query rows (the grid's y limit), each with its rows' pointers
-  constexpr int64_t kMaxRowsPerLaunch = 65535;
-  for (int64_t r0 = 0; r0 < a.nrows; r0 += kMaxRowsPerLaunch) {
-    IndexerArgs b = a;
-    b.nrows = a.nrows - r0 < kMaxRowsPerLaunch ? a.nrows - r0 : kMaxRowsPerLaunch;
-    b.qr.row0 = a.qr.row0 + r0;
-    b.q_idx = reinterpret_cast<const __nv_bfloat16*>(a.q_idx) + r0 * kNI * kCI;
-    b.w_idx = a.w_idx + r0 * kNI;
-    b.scores = a.scores + r0 * a.n_stride;
-    dim3 grid((unsigned)((max_visible + chunk - 1) / chunk), (unsigned)b.nrows);
-    indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(b, status);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  // groups of four rows when every group lies in one sequence (rows per sequence a multiple of 4,
+  // launches starting on a sequence boundary)
+  const int nq = a.qr.nq > 1 ? a.qr.nq : 1;
+  if (a.qr.ctx_lens != nullptr && nq % 4 == 0 && a.qr.row0 % nq == 0 && a.nrows % 4 == 0)
+    return launch_q<4>(a, max_visible, status, st);
+  return launch_q<1>(a, max_visible, status, st);
 }
 
 }  // namespace sac
