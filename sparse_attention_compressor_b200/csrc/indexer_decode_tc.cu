@@ -28,7 +28,8 @@ namespace {
 constexpr int kNI = 64;                   // indexer heads (MMA N)
 constexpr int kCI = 128;                  // indexer head dim (MMA K)
 constexpr int kBE = 128;                  // entries per block (MMA M)
-constexpr int kChunkBlocks = 8;           // blocks per CTA
+constexpr int kChunkBlocks = 8;           // blocks per CTA (one query row)
+constexpr int kChunkBlocksQ4 = 32;        // blocks per CTA (four rows: fewer, longer CTAs)
 constexpr int kStages = 3;
 constexpr int kGatherThreads = 128;
 constexpr int kThreads = 288;
@@ -52,6 +53,7 @@ struct Cfg {
   static constexpr int kSmemBytes = kOffTmemPtr + 16;  // Q = 1: two CTAs per SM fit
   static constexpr uint32_t kTmemCols = 2 * kN < 32 ? 32 : 2 * kN;  // two accumulators
   static constexpr uint32_t kIdesc = tc::idesc_bf16(kBE, kN, false, false);
+  static constexpr int kChunk = (Q == 1 ? kChunkBlocks : kChunkBlocksQ4) * kBE;  // entries per CTA
 };
 
 // cp.async.wait_group with the stage depth as its immediate.
@@ -83,9 +85,9 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
   a.qr.locate(a.qr.row0 + row, seq, t_first);
   a.qr.locate(a.qr.row0 + row + Q - 1, seq, t);  // the last row sees the most entries
   const int64_t nvis = t < 0 ? 0 : (t + 1) / a.m;
-  const int64_t e_begin = (int64_t)blockIdx.x * kChunkBlocks * kBE;
+  const int64_t e_begin = (int64_t)blockIdx.x * K::kChunk;
   if (t < 0 || e_begin >= nvis) return;
-  const int64_t e_end = nvis < e_begin + kChunkBlocks * kBE ? nvis : e_begin + kChunkBlocks * kBE;
+  const int64_t e_end = nvis < e_begin + K::kChunk ? nvis : e_begin + K::kChunk;
   const int nkb = (int)((e_end - e_begin + kBE - 1) / kBE);
 
   // The 128-byte swizzle needs 1024-byte aligned tiles; the dynamic window starts aligned.
@@ -264,7 +266,7 @@ cudaError_t launch_q(const IndexerArgs& a, int max_visible, int* status, cudaStr
   using K = Cfg<Q>;
   cudaError_t e = ensure_smem_limit((const void*)indexer_decode_tc_kernel<Q>, K::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int chunk = kChunkBlocks * kBE;
+  const int chunk = K::kChunk;
   // one launch per 65535 CTA rows (the grid's y limit), each with its rows' pointers
   constexpr int64_t kMaxRowsPerLaunch = 65535 * (int64_t)Q;
   for (int64_t r0 = 0; r0 < a.nrows; r0 += kMaxRowsPerLaunch) {
