@@ -23,9 +23,9 @@
 // (buffer 0) and 352 (buffer 1). A softmax thread of lane i < 16 and its partner i + 16 own the
 // same head: they add their partials, exchange halves, and each finishes 24 of the 48 keys.
 //
-// Warps: 0 = TMA thread, 1-2 = QK^T issuers (warp 1 also owns TMEM), 3 = query rotation, 4-7 =
-// gather (one 128-thread group per tile; idle when every tile arrives by TMA), 8-11 = softmax +
-// output, 12 = PV issuer. Each tcgen05.mma costs its issuing thread a fixed time, so two threads
+// Warps: 0 = TMA thread, 1-2 = QK^T issuers (warp 1 also owns TMEM), 3 = query rotation, 4-7 and
+// 13-16 = two gather groups of 128 threads taking the gathered tiles in turn (idle when every
+// tile arrives by TMA), 8-11 = softmax + output, 12 = PV issuer. Each tcgen05.mma costs its issuing thread a fixed time, so two threads
 // issue QK^T and a third issues PV the moment P is written, instead of after the next tile's
 // QK^T. An M = 64 MMA occupies one 16-lane half of each TMEM sub-partition, and MMAs into
 // opposite halves run side by side: the QK^T partials alternate between the lane halves, and the
@@ -51,9 +51,9 @@ constexpr int kKRegion = kNK * 128;              // [48 rows x 128 B]
 constexpr int kQBytes = 8 * kQRegion;            // 64 KB
 constexpr int kTileBytes = 8 * kKRegion;         // 48 KB
 constexpr int kPBytes = kHeads * 128;            // 64 rows x 128 B (48 keys used)
-constexpr int kGatherGroups = 1;                 // producer groups taking tiles in turn
-constexpr int kGroupThreads = 128 / kGatherGroups; // threads of one gather group (warps 4-7)
-constexpr int kThreads = 416;
+constexpr int kGatherGroups = 2;                 // producer groups taking tiles in turn
+constexpr int kGroupThreads = 128;               // threads of one gather group (warps 4-7, 13-16)
+constexpr int kThreads = 544;
 
 constexpr int kOffQ = 0;
 constexpr int kOffTile = kOffQ + kQBytes;
@@ -388,17 +388,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(&bar[kQReady]);
       ++qi;
     }
-  } else if (warp < 8) {
+  } else if (warp < 8 || warp >= 13) {
     if (!any_gather) goto done;  // every tile arrives by TMA
     // ------------------------------------------------------------------ gather groups
-    // Warps 4-7 form kGatherGroups groups that take the gathered tiles in turn. Thread t of a
+    // Warps 4-7 and 13-16 form two groups that take the gathered tiles in turn. Thread t of a
     // group of G threads copies rows t/8, t/8 + G/8, ... of the tile; for each it copies 16-byte
     // slot t%8 of all 8 regions, so a warp instruction reads four whole 128-byte row segments and
     // a thread needs only a few row addresses. Once its copies landed it makes them visible to
     // the tensor core and arrives on the tile's barrier.
-    constexpr int kWarpsPer = 4 / kGatherGroups;
-    const int grp = (warp - 4) / kWarpsPer;
-    const int gt = ((warp - 4) % kWarpsPer) * 32 + lane;  // thread within the group
+    const int grp = warp < 8 ? 0 : 1;
+    const int gt = (warp < 8 ? warp - 4 : warp - 13) * 32 + lane;  // thread within the group
     const int row0 = gt >> 3, slot = gt & 7;
     constexpr int kRowStride = kGroupThreads / 8;        // rows a group covers per pass
     constexpr int kRowsPer = kNK / kRowStride;
