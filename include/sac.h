@@ -311,10 +311,11 @@ SAC_API int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank,
 /*
  * Device status of the last call that used workspace `ws` (no counterpart on the page: failure
  * reporting). Every prefill call, and every decode call given a workspace, clears the first word
- * of its workspace; a tensor-core
- * kernel that gives up a bounded wait (2 s) writes a nonzero code there and returns instead of
- * hanging. This call waits for `stream`, copies the word to *status (0 = ok, 1 = a wait timed
- * out, 2 = misaligned shared memory) and returns SAC_OK, or SAC_ERR_LAUNCH if the copy fails.
+ * of its workspace; a tensor-core kernel that gives up a bounded wait (2 s) writes a nonzero code
+ * there and returns instead of hanging. This call waits for `stream`, copies the word to *status
+ * (0 = ok, 1 = a wait timed out, 2 = misaligned shared memory, 3 = a kernel launched with a block
+ * size its arguments do not allow: an internal error) and returns SAC_OK, or SAC_ERR_LAUNCH if
+ * the copy fails.
  */
 SAC_API int sac_device_status(const void* ws, int* status, void* stream);
 

@@ -53,7 +53,8 @@ constexpr int kTileBytes = 8 * kKRegion;         // 48 KB
 constexpr int kPBytes = kHeads * 128;            // 64 rows x 128 B (48 keys used)
 constexpr int kGatherGroups = 2;                 // producer groups taking tiles in turn
 constexpr int kGroupThreads = 128;               // threads of one gather group (warps 4-7, 13-16)
-constexpr int kThreads = 544;
+constexpr int kThreads = 544;                    // with the gather groups
+constexpr int kThreadsTma = 416;                 // every tile by TMA: warps 13-16 not launched
 
 constexpr int kOffQ = 0;
 constexpr int kOffTile = kOffQ + kQBytes;
@@ -159,8 +160,10 @@ __device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const
   return p ? p : reinterpret_cast<const __nv_bfloat16*>(a.pool.base);
 }
 
-template <bool kSplit>
-__global__ void __launch_bounds__(kThreads, 1)
+// kNThreads: kThreads when some tile is gathered, else kThreadsTma (the smaller block keeps the
+// register budget of the TMA-only layers at 152 per thread instead of 120).
+template <bool kSplit, int kNThreads>
+__global__ void __launch_bounds__(kNThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_win_box,
                         const __grid_constant__ CUtensorMap tm_pool_box, AttnArgs a) {
@@ -180,6 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool win_contig = a.win.block_table == nullptr;
   const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
   const bool any_gather = !win_contig || (a.pool_mode != 0 && !pool_contig);
+  if (any_gather && kNThreads < kThreads) {  // the launcher sizes the block from the same rule
+    if (threadIdx.x == 0 && status) atomicExch(status, tc::kStatusConfig);
+    return;
+  }
   const int64_t n_items = kSplit ? a.nrows * a.splits : a.nrows;
   // Who issues PV: with gathered tiles the gather latency decides, and a separate thread issues
   // PV the moment P is ready so that tile buffers free early; with TMA-fed tiles QK^T is the
@@ -798,8 +805,15 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
   e = make_tmap_bf16_2d(&tpb, has_pool ? a.pool.base : a.win.base,
                         (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
-  e = ensure_smem_limit(a.splits > 1 ? (const void*)attention_tc_kernel<true>
-                                     : (const void*)attention_tc_kernel<false>, kSmemBytes);
+  // the same rule as the kernel's any_gather: paged rows or CSA selections are gathered
+  const bool win_contig = a.win.block_table == nullptr;
+  const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
+  const bool any_gather = !win_contig || (a.pool_mode != 0 && !pool_contig);
+  const void* kern = a.splits > 1 ? (any_gather ? (const void*)attention_tc_kernel<true, kThreads>
+                                                : (const void*)attention_tc_kernel<true, kThreadsTma>)
+                                  : (any_gather ? (const void*)attention_tc_kernel<false, kThreads>
+                                                : (const void*)attention_tc_kernel<false, kThreadsTma>);
+  e = ensure_smem_limit(kern, kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -808,10 +822,18 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
     return cudaErrorInvalidValue;
   const int64_t items = a.nrows * a.splits;
   const int grid = (int)(items < sms ? items : sms);
-  if (a.splits > 1)
-    attention_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
-  else
-    attention_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
+  if (a.splits > 1) {
+    if (any_gather)
+      attention_tc_kernel<true, kThreads><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
+    else
+      attention_tc_kernel<true, kThreadsTma><<<grid, kThreadsTma, kSmemBytes, st>>>(tq, twb, tpb, a);
+  } else {
+    if (any_gather)
+      attention_tc_kernel<false, kThreads><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
+    else
+      attention_tc_kernel<false, kThreadsTma><<<grid, kThreadsTma, kSmemBytes, st>>>(tq, twb, tpb,
+                                                                                    a);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess || a.splits == 1) return e;
   attention_combine_kernel<<<dim3((unsigned)a.nrows, kHeads / kCombineHeads), 256, 0, st>>>(a);

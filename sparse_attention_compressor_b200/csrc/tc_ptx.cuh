@@ -13,7 +13,7 @@ namespace tc {
 // ---------------------------------------------------------------------------------------------
 // status word: kernels that give up a wait record the reason here and return
 // ---------------------------------------------------------------------------------------------
-enum : int { kStatusOk = 0, kStatusWaitTimeout = 1, kStatusMisaligned = 2 };
+enum : int { kStatusOk = 0, kStatusWaitTimeout = 1, kStatusMisaligned = 2, kStatusConfig = 3 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
