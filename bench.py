@@ -36,6 +36,9 @@ N_SM = 148
 # ------------------------------------------------------------------------------------------------
 # algorithmic work (only the causal, visible work)
 # ------------------------------------------------------------------------------------------------
+DATA = "synthetic (seeded generators; the shapes and distributions of the workload)"
+
+
 def visible(wl, S=None):
     S = wl.S if S is None else S
     t = np.arange(S, dtype=np.int64)
@@ -418,7 +421,7 @@ def run_ours(args, wl0):
         "metric": f"{wl.kind.upper()} attention fwd tokens/s (prefill)", "value": value,
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded; see DESIGN.md)",
+        "vs_baseline": None, "dtype": wl.dtype, "data": DATA,
         "config": config_of(wl, world), "clocks": clk.summary(),
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -654,7 +657,7 @@ def run_decode(args, wl0):
         "unit": head["unit"], "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": us_step / 1e3, "higher_is_better": head["higher_is_better"],
         "scaling": "weak",
-        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded; see DESIGN.md)",
+        "vs_baseline": None, "dtype": wl.dtype, "data": DATA,
         "config": cfg,
         "clocks": clk.summary(),
         "e2e": e2e,
@@ -720,7 +723,7 @@ def run_oproj(args, wl0):
         "metric": "grouped output projection tokens/s", "value": T * world / (ms * 1e-3),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": wl.dtype, "data": "synthetic (seeded; see DESIGN.md)",
+        "dtype": wl.dtype, "data": DATA,
         "config": {"workload": wl.name, "tokens": T, "H": wl.H, "head_dim": wl.D,
                    "o_groups": G, "o_lora_rank": rk, "hidden": hid, "parallelism": f"dp{world}",
                    "l2": "flushed before every step (252 MiB written, then another 252 MiB read)",
