@@ -18,8 +18,10 @@
 namespace sac {
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
+constexpr int kThreads = 512;       // rows re-read from L2, and long rows with keys in smem
+// rows of at most kSmemKeyRows scores: more rows side by side per SM (measured at CSA-8k: 112 us
+// with 512 threads, 87 us with 256, 108 us with 128)
+constexpr int kShortThreads = 256;
 constexpr int kMaxEntries = 1 << 22;  // longest row (pool entries per sequence) accepted
 constexpr int kBins = 4096;          // 12-bit digits
 constexpr int kCandCap = 2048;       // compacted keys of the threshold bin
@@ -101,8 +103,8 @@ __device__ __forceinline__ void find_digit(Shared& sh, int nbins, int rem) {
 // kSmemKeys: the row's keys are kept in shared memory (short rows); otherwise every pass
 // re-reads the scores, which the first pass has brought into L2, so that a block needs only
 // ~25 KB of shared memory and several rows run side by side on each SM.
-template <bool kSmemKeys>
-__global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict__ scores,
+template <bool kSmemKeys, int NT>
+__global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scores,
                                                         int n_stride, QueryRows qr, int m, int k,
                                                         int32_t* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
   int32_t* orow = out + r * k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (n <= k) {
-    for (int i = tid; i < k; i += kThreads) orow[i] = i < n ? i : -1;
+    for (int i = tid; i < k; i += NT) orow[i] = i < n ? i : -1;
     return;
   }
   const float* srow = scores + r * n_stride;
@@ -126,16 +128,16 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
   };
 
   // ---- digit 1: bits 31..20
-  for (int i = tid; i < kBins; i += kThreads) sh.hist[i] = 0;
+  for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0;
   if (tid == 0) sh.n_cand = 0;
   __syncthreads();
-  for (int i = tid; i < n; i += kThreads) {
+  for (int i = tid; i < n; i += NT) {
     const uint32_t key = order_key(__ldcg(srow + i));
     if (kSmemKeys) keys[i] = key;
     atomicAdd(&sh.hist[key >> 20], 1);
   }
   __syncthreads();
-  find_digit<kThreads>(sh, kBins, k);
+  find_digit<NT>(sh, kBins, k);
   const uint32_t d1 = (uint32_t)sh.digit;
   int rem = sh.rem;
   const int c1 = sh.hist[d1];
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
   // ---- compact the keys of digit d1 when they fit; otherwise scan the whole row with a mask
   const bool compact = c1 <= kCandCap;
   if (compact) {
-    for (int i0 = warp * 32; i0 < n; i0 += kThreads) {
+    for (int i0 = warp * 32; i0 < n; i0 += NT) {
       const int i = i0 + lane;
       const uint32_t key = i < n ? key_at(i) : 0u;
       const bool hit = i < n && (key >> 20) == d1;
@@ -161,33 +163,33 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
   auto cand_at = [&](int i) -> uint32_t { return compact ? sh.cand[i] : key_at(i); };
 
   // ---- digit 2: bits 19..8 among keys with digit 1 == d1
-  for (int i = tid; i < kBins; i += kThreads) sh.hist[i] = 0;
+  for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0;
   __syncthreads();
-  for (int i = tid; i < nc; i += kThreads) {
+  for (int i = tid; i < nc; i += NT) {
     const uint32_t key = cand_at(i);
     if ((key >> 20) == d1) atomicAdd(&sh.hist[(key >> 8) & 0xFFFu], 1);
   }
   __syncthreads();
-  find_digit<kThreads>(sh, kBins, rem);
+  find_digit<NT>(sh, kBins, rem);
   const uint32_t d2 = (uint32_t)sh.digit;
   rem = sh.rem;
   __syncthreads();
 
   // ---- digit 3: bits 7..0 among keys with bits 31..8 == (d1, d2)
   const uint32_t hi24 = (d1 << 12) | d2;
-  for (int i = tid; i < 256; i += kThreads) sh.hist[i] = 0;
+  for (int i = tid; i < 256; i += NT) sh.hist[i] = 0;
   __syncthreads();
-  for (int i = tid; i < nc; i += kThreads) {
+  for (int i = tid; i < nc; i += NT) {
     const uint32_t key = cand_at(i);
     if ((key >> 8) == hi24) atomicAdd(&sh.hist[key & 0xFFu], 1);
   }
   __syncthreads();
-  find_digit<kThreads>(sh, 256, rem);
+  find_digit<NT>(sh, 256, rem);
   const uint32_t T = (hi24 << 8) | (uint32_t)sh.digit;
   const int take_eq = sh.rem;  // keys equal to T to keep, lowest indices first
 
   // ---- selection: warp w owns the contiguous segment [w*seg, (w+1)*seg)
-  const int seg = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int seg = ((n + (NT / 32) * 32 - 1) / ((NT / 32) * 32)) * 32;
   const int s0 = warp * seg, s1 = min(n, s0 + seg);
   int gt = 0, eq = 0;
   for (int i0 = s0; i0 < s1; i0 += 32) {
@@ -240,12 +242,20 @@ cudaError_t launch_topk(const float* scores, int n_stride, QueryRows qr, int m, 
                                                        n_stride <= kSmemKeyLimit);
   if (smem_keys) {
     const size_t smem = sizeof(Shared) + sizeof(uint32_t) * (size_t)(n_stride > 0 ? n_stride : 1);
-    cudaError_t err = ensure_smem_limit((const void*)topk_kernel<true>, (int)smem);
+    if (n_stride <= kSmemKeyRows) {
+      cudaError_t err = ensure_smem_limit((const void*)topk_kernel<true, kShortThreads>, (int)smem);
+      if (err != cudaSuccess) return err;
+      topk_kernel<true, kShortThreads><<<(unsigned)nrows, kShortThreads, smem, st>>>(
+          scores, n_stride, qr, m, k, out);
+      return cudaGetLastError();
+    }
+    cudaError_t err = ensure_smem_limit((const void*)topk_kernel<true, kThreads>, (int)smem);
     if (err != cudaSuccess) return err;
-    topk_kernel<true><<<(unsigned)nrows, kThreads, smem, st>>>(scores, n_stride, qr, m, k, out);
-  } else {
-    topk_kernel<false><<<(unsigned)nrows, kThreads, sizeof(Shared), st>>>(scores, n_stride, qr, m,
+    topk_kernel<true, kThreads><<<(unsigned)nrows, kThreads, smem, st>>>(scores, n_stride, qr, m,
                                                                          k, out);
+  } else {
+    topk_kernel<false, kThreads><<<(unsigned)nrows, kThreads, sizeof(Shared), st>>>(
+        scores, n_stride, qr, m, k, out);
   }
   return cudaGetLastError();
 }
