@@ -222,6 +222,23 @@ def capture(fn):
     return g
 
 
+def kernel_times(fn, dev, flush: bool = False) -> dict:
+    """Per-kernel device times of one step: fn captured into a second graph with the library's
+    timing events around every launch and replayed once (the timed graph carries no events);
+    with flush, L2 is flushed before that replay as timed_flushed() does before every step."""
+    import sparse_attention_compressor_b200 as sac
+    sac.sac_timing_begin()
+    g = capture(fn)
+    if flush:
+        torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev).fill_(0)
+        torch.zeros(2 * L2_BYTES // 4, dtype=torch.int32, device=dev).sum()
+    g.replay()
+    torch.cuda.synchronize(dev)
+    out = sac.sac_timing_end()
+    del g
+    return out
+
+
 def timed(step, steps, dev):
     barrier(dev)
     torch.cuda.synchronize(dev)
@@ -384,8 +401,7 @@ def run_ours(args, wl0):
         step()
     torch.cuda.synchronize(dev)
 
-    # one step captured as a CUDA graph (with the per-kernel timing events inside it)
-    sac.sac_timing_begin()
+    # one step captured as a CUDA graph
     graph = capture(step)
     graph.replay()
     torch.cuda.synchronize(dev)
@@ -393,7 +409,7 @@ def run_ours(args, wl0):
         clk.wait_samples(1, graph.replay)
         ms = timed(graph.replay, args.steps, dev)
         clk.wait_samples(len(clk.lines) + 1, graph.replay)
-    ktimes = sac.sac_timing_end()  # per kernel: the last replay, i.e. one step
+    ktimes = kernel_times(step, dev)
     ms = max_over_ranks(ms, dev)
     ms_step = ms / args.steps
     tokens = wl.B * wl.S * world
@@ -574,7 +590,6 @@ def run_decode(args, wl0):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    sac.sac_timing_begin()
     graph = capture(step)
     graph.replay()
     torch.cuda.synchronize(dev)
@@ -582,7 +597,7 @@ def run_decode(args, wl0):
         clk.wait_samples(1, graph.replay)
         ms = timed_flushed(graph.replay, args.steps, dev)
         clk.wait_samples(len(clk.lines) + 1, graph.replay)
-    ktimes = sac.sac_timing_end()  # per kernel: the last replay, i.e. one step
+    ktimes = kernel_times(step, dev, flush=True)
     ms = max_over_ranks(ms, dev)
     us_step = 1e3 * ms / args.steps
     # end to end: the step's new-token inputs from pinned host memory, outputs back
@@ -694,7 +709,6 @@ def run_oproj(args, wl0):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    sac.sac_timing_begin()
     graph = capture(step)
     graph.replay()
     torch.cuda.synchronize(dev)
@@ -702,7 +716,7 @@ def run_oproj(args, wl0):
         clk.wait_samples(1, graph.replay)
         ms = timed_flushed(graph.replay, args.steps, dev)
         clk.wait_samples(len(clk.lines) + 1, graph.replay)
-    ktimes = sac.sac_timing_end()
+    ktimes = kernel_times(step, dev, flush=True)
     ms = max_over_ranks(ms, dev) / args.steps
     pin_o = x["o"].pin_memory()
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
