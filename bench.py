@@ -629,7 +629,10 @@ def run_decode(args, wl0):
     if n > 1:
         wb = chunk_work(wl, dc, dh)
     else:
-        wb = {k: ("bytes", v) for k, v in decode_bytes(wl, dc, dh).items()}
+        db = decode_bytes(wl, dc, dh)
+        if "decode_append_index" not in ktimes:  # both CSA parts ran as one launch
+            db["decode_append"] += db.pop("decode_append_index")
+        wb = {k: ("bytes", v) for k, v in db.items()}
     krows = {}
     total = sum(v[1] for v in ktimes.values()) or 1.0
     for name, (launches, kms) in ktimes.items():

@@ -47,6 +47,55 @@ __device__ __forceinline__ T* page_row(void* base, const int32_t* bt, int max_pa
   return reinterpret_cast<T*>(base) + ((int64_t)page * page_size + j % page_size) * C;
 }
 
+// One warp's append of sequence seq when a single warp pools a window (L < 64): the new row to
+// the ring and the window pages, and on a closing window the pooled entry.
+template <typename T, int V>
+__device__ __forceinline__ void append_warp(const AppendPart& a, int seq, int lane,
+                                            PoolShared<V, 1>& sh) {
+  constexpr int C = 32 * V;
+  const int64_t t = (int64_t)__ldg(a.ctx_lens + seq) - 1;
+  if (t < 0) return;
+  const T* x_new = reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * C;
+  T* ring = a.m > 0 ? reinterpret_cast<T*>(a.ring) + (int64_t)seq * a.L * C : nullptr;
+  float v[V];
+  load_lane<T, V>(x_new, lane, v);
+  if (ring) store_lane<T, V>(ring + (t % a.L) * C, lane, v);
+  if (a.kv_pages) {
+    T* dst = page_row<T>(a.kv_pages, a.kv_bt, a.kv_max_pages, a.page_size, C, seq, t);
+    if (dst) {
+      rotate_lane<V>(v, lane, C, a.rf, a.pos0 + t);
+      store_lane<T, V>(dst, lane, v);
+    }
+  }
+  if (a.m == 0 || (t + 1) % a.m != 0) return;
+  const int64_t w = (t + 1) / a.m - 1;
+  const int64_t hi = (w + 1) * a.m;
+  const int64_t lo = hi - a.L < 0 ? 0 : hi - a.L;
+  float u[V], acc[V];
+  load_lane<T, V>(reinterpret_cast<const T*>(a.gate), lane, u);
+  const int L = a.L;
+  pool_window<T, V, 1, 4>([&](int64_t j) { return j == t ? x_new : ring + (j % L) * C; }, u,
+                          a.bias, lo, hi, L, true, 0, lane, sh, acc);
+  T* dst = page_row<T>(a.pool_pages, a.pool_bt, a.pool_max_pages, a.page_size, C, seq, w);
+  if (dst == nullptr) return;
+  if (a.rotate) rotate_lane<V>(acc, lane, C, a.rf, a.pos0 + w * a.m);
+  store_lane<T, V>(dst, lane, acc);
+}
+
+// Both parts of a CSA layer's append in one launch: warp 0 the kv row and the main pool, warp 1
+// the indexer row and its pool (one launch fewer per decode step).
+template <typename T, int V0, int V1>
+__global__ void __launch_bounds__(64) append_pair_kernel(AppendPart main_part,
+                                                         AppendPart index_part) {
+  __shared__ PoolShared<V0, 1> sh0;
+  __shared__ PoolShared<V1, 1> sh1;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32)
+    append_warp<T, V0>(main_part, blockIdx.x, lane, sh0);
+  else
+    append_warp<T, V1>(index_part, blockIdx.x, lane, sh1);
+}
+
 template <typename T, int V, int WPE>
 __global__ void __launch_bounds__(256) append_kernel(AppendPart a) {
   constexpr int C = 32 * V;
@@ -238,6 +287,21 @@ cudaError_t launch_chunk_append(int dtype, const DecodeAppendArgs& a, int n, boo
   const int C = index_part ? a.cI : a.D;
   return dtype == 0 ? chunk_dispatch<float>(p, C, a.nseq, n, st)
                     : chunk_dispatch<__nv_bfloat16>(p, C, a.nseq, n, st);
+}
+
+bool decode_append_pair_supported(const DecodeAppendArgs& a) {
+  return a.D == 512 && a.cI == 128 && a.m > 0 && a.L < 64;
+}
+
+cudaError_t launch_decode_append_pair(int dtype, const DecodeAppendArgs& a, cudaStream_t st) {
+  if (a.nseq == 0) return cudaSuccess;
+  if (!decode_append_pair_supported(a)) return cudaErrorInvalidValue;
+  const AppendPart p0 = make_part(a, false), p1 = make_part(a, true);
+  if (dtype == 0)
+    append_pair_kernel<float, 16, 4><<<a.nseq, 64, 0, st>>>(p0, p1);
+  else
+    append_pair_kernel<__nv_bfloat16, 16, 4><<<a.nseq, 64, 0, st>>>(p0, p1);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, bool index_part,

@@ -856,13 +856,20 @@ static int append_paged(const sac_params* p, int kind, int nseq, int n, const in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (n == 0) {
-    e = sac::timed("decode_append", st, [&] {
-      return sac::launch_decode_append(p->dtype, a, false, st);
-    });
-    if (e == cudaSuccess && kind == SAC_KIND_CSA)
-      e = sac::timed("decode_append_index", st, [&] {
-        return sac::launch_decode_append(p->dtype, a, true, st);
+    if (kind == SAC_KIND_CSA && sac::decode_append_pair_supported(a)) {
+      // both parts in one launch
+      e = sac::timed("decode_append", st, [&] {
+        return sac::launch_decode_append_pair(p->dtype, a, st);
       });
+    } else {
+      e = sac::timed("decode_append", st, [&] {
+        return sac::launch_decode_append(p->dtype, a, false, st);
+      });
+      if (e == cudaSuccess && kind == SAC_KIND_CSA)
+        e = sac::timed("decode_append_index", st, [&] {
+          return sac::launch_decode_append(p->dtype, a, true, st);
+        });
+    }
   } else {
     e = sac::timed("chunk_append", st, [&] {
       return sac::launch_chunk_append(p->dtype, a, n, false, st);

@@ -50,6 +50,10 @@ struct DecodeAppendArgs {
 // index_part = false: the kv row and the main pool; true: the indexer ring and pool (CSA).
 cudaError_t launch_decode_append(int dtype, const DecodeAppendArgs& a, bool index_part,
                                  cudaStream_t st);
+// Both parts of a CSA layer in one launch, for the shapes decode_append_pair_supported() accepts
+// (D = 512, cI = 128, L < 64); other shapes launch the parts one by one.
+bool decode_append_pair_supported(const DecodeAppendArgs& a);
+cudaError_t launch_decode_append_pair(int dtype, const DecodeAppendArgs& a, cudaStream_t st);
 // The same for a prefill chunk of n tokens per sequence at t = ctx - n .. ctx - 1 (two launches:
 // the entries that close inside the chunk, then the rows' page and ring writes).
 cudaError_t launch_chunk_append(int dtype, const DecodeAppendArgs& a, int n, bool index_part,
