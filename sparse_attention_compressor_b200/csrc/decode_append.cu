@@ -8,13 +8,16 @@
 // the overlap carried from the previous window. When t + 1 is a multiple of m, entry
 // w = (t+1)/m - 1 closes: it pools the ring rows of its window [(w+1)m - L, (w+1)m) (clipped at
 // 0) with the prefill compressor's pooling (pool_window.cuh) and is written, rotated at
-// pos0 + w*m, to the pool pages. CSA runs the same kernel a second time for the indexer key row
-// (its own ring and gate, no rotation). The token count is ctx itself, so the state needs no
-// counter of its own.
+// pos0 + w*m, to the pool pages. CSA does the same for the indexer key row (its own ring and
+// gate, no rotation). The token count is ctx itself, so the state needs no counter of its own.
 //
-// One block of 8 warps per sequence: warp 0 writes the new row; on a closing window the warps
-// split the window's rows (all 8 for L >= 64, else warp 0 alone) and merge in shared memory. The
-// pooling reads the new token's row from its input rather than back from the ring.
+// Windows of L >= 64 rows (HCA): one block of 8 warps per sequence; warp 0 writes the new row and
+// on a closing window the 8 warps split the window's rows and merge in shared memory. Shorter
+// windows take one warp per part: a CSA layer with D = 512 and cI = 128 runs both parts in one
+// 64-thread block per sequence (warp 0 the kv row and main pool, warp 1 the indexer's), other
+// shapes one launch per part. The pooling reads the new token's row from its input rather than
+// back from the ring. Prefill chunks (several tokens per sequence) have their own two kernels
+// below.
 #include "pool_window.cuh"
 #include "sac_kernels.h"
 
