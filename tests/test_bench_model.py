@@ -1,0 +1,60 @@
+"""Host logic of bench.py: the algorithmic work each roofline divides by, against direct
+per-query loops on small workloads (no GPU)."""
+from dataclasses import replace
+
+import numpy as np
+import torch
+
+import bench
+from sparse_attention_compressor_b200 import workloads as W
+
+
+def test_prefill_work_matches_per_query_counts():
+    wl = W.Workload("t", "csa", "bf16", B=2, S=37, H=4, D=64, m=4, L=8, W=8, nI=3, cI=32, k=5)
+    w = bench.work(wl)
+    keys = sum(min(t + 1, wl.W) + min((t + 1) // wl.m, wl.k) for t in range(wl.S)) * wl.B
+    assert w["attention"] == ("flops", keys * 4 * wl.H * wl.D)
+    pairs = sum((t + 1) // wl.m for t in range(wl.S)) * wl.B
+    assert w["indexer_score"] == ("flops", pairs * 2 * wl.nI * wl.cI)
+    assert w["topk"] == ("bytes", float((pairs // wl.B * 4 + wl.S * wl.k * 4) * wl.B))
+    # compressor: every token row read once, every entry written once (bf16)
+    assert w["compress"] == ("bytes", float((wl.S + wl.S // wl.m) * wl.D * 2 * wl.B))
+    hca = replace(wl, kind="hca", m=16, L=16)
+    keys = sum(min(t + 1, wl.W) + (t + 1) // 16 for t in range(wl.S)) * wl.B
+    assert bench.work(hca)["attention"] == ("flops", keys * 4 * wl.H * wl.D)
+
+
+def _paged_ctx(ctx, m):
+    return {"ctx_lens": torch.tensor(ctx, dtype=torch.int32), "m": m}
+
+
+def test_chunk_work_matches_per_row_counts():
+    wl = W.Workload("c", "decode", "bf16", nseq=2, H=4, D=64, m=4, L=8, W=8, nI=3, cI=32, k=5,
+                    hca_m=16, chunk=6)
+    dc, dh = _paged_ctx([20, 9], 4), _paged_ctx([33, 6], 16)
+    w = bench.chunk_work(wl, dc, dh)
+    rows = [(c, t) for c in (20, 9) for t in range(c - 6, c)]
+    assert w["indexer_score"] == ("flops", float(sum((t + 1) // 4 for _, t in rows) * 2 * 3 * 32))
+    csa_keys = sum(min((t + 1) // 4, wl.k) + min(t + 1, wl.W) for _, t in rows)
+    assert w["csa_chunk_attention"] == ("flops", float(csa_keys * 4 * wl.H * wl.D))
+    hrows = [t for c in (33, 6) for t in range(c - 6, c)]
+    hca_keys = sum((t + 1) // 16 + min(t + 1, wl.W) for t in hrows)
+    assert w["hca_chunk_attention"] == ("flops", float(hca_keys * 4 * wl.H * wl.D))
+    # entries closing inside the chunks: CSA 20 -> 5 - 3 = 2, 9 -> 2 - 0 = 2; HCA 33 -> 2 - 1 = 1
+    closing_csa = (20 // 4 - 14 // 4) + (9 // 4 - 3 // 4)
+    assert w["chunk_append_index"][1] == float((12 + 2 * min(wl.L, 6)) * wl.cI * 2
+                                               + closing_csa * (wl.L + 1) * wl.cI * 2)
+
+
+def test_decode_bytes_fold_the_index_part_when_fused():
+    wl = W.Workload("d", "decode", "bf16", nseq=3, H=4, D=64, m=4, L=8, W=8, nI=3, cI=32, k=5,
+                    hca_m=16)
+    dc, dh = _paged_ctx([8, 9, 40], 4), _paged_ctx([16, 17, 5], 16)
+    db = bench.decode_bytes(wl, dc, dh)
+    assert set(db) >= {"decode_append", "decode_append_index", "indexer_score", "topk",
+                       "csa_decode_attention", "hca_decode_attention"}
+    # closing windows: CSA ctx 8 and 40 (multiples of 4), HCA ctx 16
+    app = 3 * 3 * wl.D * 2 + 2 * (wl.L + 1) * wl.D * 2 + 3 * 3 * wl.D * 2 + 1 * 17 * wl.D * 2
+    assert db["decode_append"] == float(app)
+    nv = np.array([8, 9, 40]) // 4
+    assert db["topk"] == float((nv * 4).sum() + 3 * wl.k * 4)
