@@ -8,12 +8,19 @@
  * partial RoPE and the -i output rotation, eq. 26; per-head sink, eq. 27; sliding-window branch),
  * "Attention mask layout" (sliding mask, CSA slots with the -1 sentinel, HCA visibility
  * w < (t+1)//m), "Cache layers" (compressor / indexer buffer, pool, count, overlap) and
- * "DeepseekV4Config" (head_dim, sliding_window, compress_rates, index_* fields, rope bases).
+ * "DeepseekV4Config" (head_dim, sliding_window, compress_rates, index_* fields, rope bases,
+ * o_groups, o_lora_rank), and the "Grouped Output Projection" bullet of the architecture overview.
+ *
+ * Entry points: prefill (swa/hca/csa_forward, swa_forward_static), decode over paged caches
+ * (swa/hca/csa_decode, decode_append), chunked prefill over the same caches
+ * (swa/hca/csa_prefill_chunk, prefill_chunk_append), the grouped output projection
+ * (o_proj_forward), workspace sizes, the device status word and per-kernel timing.
  *
  * Conventions shared by every entry point
  *  - Tensors are caller-owned DEVICE pointers, dense row-major, 16-byte aligned. The library
  *    never allocates device memory; scratch space is a caller-provided workspace of at least
- *    sac_workspace_size() / sac_decode_workspace_size() bytes (256-byte aligned).
+ *    sac_workspace_size() / sac_decode_workspace_size() / sac_chunk_workspace_size() /
+ *    sac_oproj_workspace_size() bytes (256-byte aligned).
  *  - Element type of q, kv, k_idx, q_idx, gates, pools and o is params.dtype (SAC_F32 or
  *    SAC_BF16). Biases, sinks and indexer head weights are always fp32; indices are int32.
  *  - Every call enqueues kernels on `stream` (a cudaStream_t passed as void*; NULL = legacy
