@@ -760,9 +760,138 @@ def run_oproj(args, wl0):
         torch.distributed.destroy_process_group()
 
 
+def _logical_rows(pages, bt, s, lo, hi):
+    """Rows lo..hi-1 of sequence s of a paged cache (CPU tensors) as float64 numpy."""
+    ps = pages.shape[1]
+    idx = np.arange(lo, hi)
+    pg = bt[s, idx // ps].numpy()
+    return pages[torch.from_numpy(pg).long(), torch.from_numpy(idx % ps)].double().numpy()
+
+
+def _oracle_paged_step(wl, d, layer, rows):
+    """The oracle's attention of the listed (sequence, position) rows of one layer over the rows of
+    the paged caches they read (copied once per sequence to a page-size-1 layout); seconds."""
+    import oracle
+    m = d["m"]
+    seqs = sorted({s for s, _ in rows})
+    slot = {s: i for i, s in enumerate(seqs)}
+    ctx = d["ctx_lens"].numpy()
+    kv_rows, pool_rows, ipool_rows = [], [], []
+    maxc = int(max(ctx[s] for s in seqs))
+    kbt = np.full((len(seqs), maxc), -1, dtype=np.int32)
+    pbt = np.full((len(seqs), max(1, maxc // m)), -1, dtype=np.int32)
+    nk = npl = 0
+    for s in seqs:
+        c, i = int(ctx[s]), slot[s]
+        lo = max(0, min(t for ss, t in rows if ss == s) - wl.W + 1)
+        kv_rows.append(_logical_rows(d["kv_pages"], d["kv_block_table"], s, lo, c))
+        kbt[i, lo:c] = np.arange(nk, nk + c - lo)
+        nk += c - lo
+        nv = c // m
+        if nv:
+            pool_rows.append(_logical_rows(d["pool_pages"], d["pool_block_table"], s, 0, nv))
+            if layer == "csa":
+                ipool_rows.append(_logical_rows(d["idx_pool_pages"], d["pool_block_table"], s, 0,
+                                                nv))
+            pbt[i, :nv] = np.arange(npl, npl + nv)
+            npl += nv
+    p = oracle.OracleParams(1, maxc, wl.H, wl.D, wl.R, wl.theta, wl.W, m=m,
+                            L=wl.L if layer == "csa" else m, nI=wl.nI if layer == "csa" else 0,
+                            cI=wl.cI if layer == "csa" else 0, k=wl.k if layer == "csa" else 0)
+    n = wl.chunk
+    def tok(name, s, t):  # the per-token tensor row of (s, t)
+        x = d[name]
+        return x[s] if n == 1 else x[s, t - (int(ctx[s]) - n)]
+    q = np.stack([tok("q", s, t).double().numpy() for s, t in rows])
+    kw = {}
+    if layer == "csa":
+        kw = dict(q_idx=np.stack([tok("q_idx", s, t).double().numpy() for s, t in rows]),
+                  w_idx=np.stack([tok("w_idx", s, t).double().numpy() for s, t in rows]),
+                  idx_pool_pages=np.concatenate(ipool_rows)[:, None, :])
+    sl = [slot[s] for s, _ in rows]
+    t0 = time.perf_counter()
+    oracle.decode(p, q, np.concatenate(kv_rows)[:, None, :], kbt[sl],
+                  np.array([t + 1 for _, t in rows], dtype=np.int32), 1,
+                  pool_pages=np.concatenate(pool_rows)[:, None, :], pool_block_table=pbt[sl],
+                  sinks=d["sinks"].double().numpy(), **kw)
+    return time.perf_counter() - t0
+
+
+def run_reference_paged(args, wl):
+    """The oracle on a bounded sample of a decode (or chunked-prefill) step: the attention of a
+    few query rows of each layer, scaled to the step's rows by count."""
+    import oracle
+    oracle.build()
+    world, _, _ = dist_env()
+    dc, dh = W.decode_inputs(wl, "csa"), W.decode_inputs(wl, "hca")
+    n = wl.chunk
+    rng = np.random.default_rng(2)
+    ctx_c, ctx_h = dc["ctx_lens"].numpy(), dh["ctx_lens"].numpy()
+    per = 4  # sampled rows per layer and step
+    def sample(ctx):
+        ss = rng.choice(wl.nseq, size=per)
+        return [(int(s), int(ctx[s]) - 1 - int(rng.integers(0, n))) for s in ss]
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = _oracle_paged_step(wl, dc, "csa", sample(ctx_c)) + \
+            _oracle_paged_step(wl, dh, "hca", sample(ctx_h))
+        if i >= args.warmup:
+            times.append(t)
+    rows_step = wl.nseq * n
+    s_per_step = sum(times) / len(times) * rows_step / per
+    threads = oracle.max_threads()
+    sample_txt = (f"each step: {per} random query rows of each layer (CSA with its indexer and "
+                  f"top-k, HCA) through the oracle's paged attention, scaled by count to the "
+                  f"{rows_step} rows of a step")
+    if n > 1:
+        value, unit, hib = rows_step / s_per_step, "tokens/s", True
+        metric = (f"chunked prefill tokens/s (CSA + HCA layer, {wl.nseq} sequences x {n} tokens "
+                  "against a cached prefix)")
+    else:
+        value, unit, hib = s_per_step * 1e6, "us/step", False
+        metric = "decode us/step (CSA + HCA layer, 64 sequences)"
+    return metric, value, unit, hib, s_per_step * 1e3, threads, sample_txt
+
+
+def run_reference_oproj(args, wl):
+    """The oracle's grouped output projection of a bounded sample of token rows."""
+    import oracle
+    oracle.build()
+    T = wl.B * wl.S
+    x = W.oproj_inputs(T, wl.H, wl.D, wl.o_groups, wl.o_rank, wl.hidden, wl.seed)
+    o, wa, wb = (x[k].double().numpy() for k in ("o", "w_a", "w_b"))
+    rng = np.random.default_rng(3)
+    per = 64
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(T, size=per, replace=False))
+        t0 = time.perf_counter()
+        oracle.o_proj(o, wa, wb, wl.o_groups, rows=rows, round_mid=True)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    s = sum(times) / len(times)
+    return ("grouped output projection tokens/s", per / s, "tokens/s", True, s * 1e3,
+            oracle.max_threads(), f"each step: {per} random token rows of {T}")
+
+
 def run_reference(args, wl):
     world, rank, _ = dist_env()
     if rank != 0:
+        return
+    if wl.kind in ("decode", "oproj"):
+        fn = run_reference_paged if wl.kind == "decode" else run_reference_oproj
+        metric, value, unit, hib, ms_step, threads, sample = fn(args, wl)
+        line = {
+            "impl": "reference", "metric": metric, "value": value, "unit": unit,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": hib, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "parallelism": f"dp{world}"},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
         return
     import oracle
     oracle.build()
