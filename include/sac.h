@@ -250,7 +250,8 @@ SAC_API int decode_append(const sac_params* p, int kind, int nseq, const int32_t
  * by position, so the chunk attends to the cached prefix plus itself, causally.
  * Arguments as in *_decode, with n rows per sequence: q, o [nseq, n, H, D]; q_idx [nseq, n, nI,
  * cI]; w_idx [nseq, n, nI]; topk_out [nseq, n, k]; every ctx must satisfy n <= ctx <= p->S
- * (rows of a sequence with ctx < n have t < 0 and see no key).
+ * (the device cannot check it: rows of a sequence with ctx < n have t < 0, see no key, and their
+ * output rows are left undefined).
  * Workspace: sac_chunk_workspace_size() bytes (the decode layout for nseq * n query rows; the
  * CSA scores hold at most 1 GiB of rows at once, the indexer and top-k then run in row blocks).
  * Decode is the case n = 1.
