@@ -164,12 +164,15 @@ def oracle_caches(wl, x, lens, dtype):
     return out
 
 
-@pytest.mark.parametrize("kind,dtype", [("csa", "bf16"), ("hca", "bf16"), ("swa", "bf16"),
-                                        ("csa", "f32"), ("hca", "f32"), ("swa", "f32")])
-def test_chunk_attention_matches_oracle(kind, dtype):
+@pytest.mark.parametrize("kind,dtype,n", [("csa", "bf16", 64), ("hca", "bf16", 64),
+                                          ("swa", "bf16", 64), ("csa", "f32", 64),
+                                          ("hca", "f32", 64), ("swa", "f32", 64),
+                                          # 3 x 8 rows: each row's keys split over several CTAs
+                                          ("csa", "bf16", 8), ("hca", "bf16", 8)])
+def test_chunk_attention_matches_oracle(kind, dtype, n):
+    """The last n tokens of each sequence (all in the caches) attended as one chunk."""
     wl, x, g, p, ps, c, extra, lens = build_caches(kind, dtype)
     dev = torch.device("cuda", 0)
-    n = CHUNKS[-1]
     ctx = torch.tensor(lens, dtype=torch.int32, device=dev)
     rows = [(s, t) for s in range(wl.B) for t in range(lens[s] - n, lens[s])]
     q = torch.stack([g["q"][s, t] for s, t in rows]).reshape(wl.B, n, wl.H, wl.D).contiguous()
