@@ -58,3 +58,24 @@ def test_decode_bytes_fold_the_index_part_when_fused():
     assert db["decode_append"] == float(app)
     nv = np.array([8, 9, 40]) // 4
     assert db["topk"] == float((nv * 4).sum() + 3 * wl.k * 4)
+
+
+def test_chunk_inputs_shapes_and_reproducibility():
+    """A chunk workload's per-token tensors gain the chunk axis, the contexts hold the chunk, and
+    the window pages cover the rows every chunk row can see; a decode workload keeps its shapes."""
+    wl = W.Workload("c", "decode", "bf16", nseq=2, H=4, D=64, R=16, m=4, L=8, W=8, nI=3, cI=32,
+                    k=5, hca_m=16, ctx_lo=40, ctx_hi=90, page_size=16, chunk=6, seed=5)
+    d = W.decode_inputs(wl, "csa")
+    assert d["q"].shape == (2, 6, 4, 64) and d["kv_new"].shape == (2, 6, 64)
+    assert d["q_idx"].shape == (2, 6, 3, 32) and d["w_idx"].shape == (2, 6, 3)
+    ctx = d["ctx_lens"].numpy()
+    assert (ctx >= wl.chunk).all()
+    for s in range(2):  # rows ctx - chunk - W + 1 .. ctx - 1 sit on filled pages
+        lo = ctx[s] - wl.chunk - wl.W + 1
+        for j in range(max(lo, 0), ctx[s]):
+            page = int(d["kv_block_table"][s, j // wl.page_size])
+            assert d["kv_pages"][page, j % wl.page_size].abs().sum() > 0, (s, j)
+    d2 = W.decode_inputs(wl, "csa")
+    assert torch.equal(d["q"], d2["q"]) and torch.equal(d["kv_pages"], d2["kv_pages"])
+    dec = W.decode_inputs(replace(wl, chunk=1), "csa")
+    assert dec["q"].shape == (2, 4, 64) and dec["q_idx"].shape == (2, 3, 32)
