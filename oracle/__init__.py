@@ -257,7 +257,10 @@ def csa_forward(p: OracleParams, q, kv, cmp_gate, cmp_bias, q_idx, w_idx, k_idx,
 
 
 def csa_index_scores(p: OracleParams, q_idx, w_idx, k_idx, idx_gate, idx_bias, rows):
-    """Indexer scores [len(rows), N] of the listed rows (q_idx/w_idx given for those rows)."""
+    """Indexer scores [len(rows), N] of the listed rows (q_idx/w_idx given for those rows), over
+    the oracle's own indexer pool (rounded to bf16 with p.bf16_pools), -inf past (t+1)//m.
+    Pinned by tests/test_oracle_index_pins.py: its top-k equals csa_forward's selection, and its
+    scores equal index_scores over the pool csa_forward returns."""
     r, n = _rows(p, rows)
     qI = _f64(q_idx).reshape(n, p.nI, p.cI)
     wI = _f64(w_idx).reshape(n, p.nI)
