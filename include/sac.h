@@ -118,20 +118,24 @@ SAC_API int swa_forward(const sac_params* p, const void* q, const void* kv, cons
                 void* ws, size_t ws_bytes, void* stream);
 
 /*
- * swa_forward without any device allocation by the caller: the same computation and kernels as
- * swa_forward, with the scratch that swa_forward takes from `ws` (the rotated kv stream,
- * B*S*D elements of dtype) held instead in a fixed 16 MiB array inside this library (a static
- * __device__ array present on every GPU that loads the library, until the process exits).
- * The page has no counterpart of this entry point; it exists for callers that cannot call
- * cudaMalloc: code that runs inside a host framework whose caching allocator owns all device
- * memory and does not lend it to plug-ins, and serving loops that forbid any allocation after
- * start-up so that memory use stays fixed.
+ * swa_forward without any device allocation by the caller: the same computation and the same
+ * kernels as swa_forward (the tensor-core attention for bf16 layers of 64 heads of 512, the
+ * CUDA-core one otherwise), with the one piece of scratch swa_forward takes from `ws` -- the
+ * rotated kv stream, B*S*D elements of dtype -- held instead in a fixed 16 MiB array inside this
+ * library (a static __device__ array present on every GPU that loads the library, until the
+ * process exits). The page has no counterpart of this entry point. It exists for callers that
+ * cannot call cudaMalloc: code that runs inside a host framework whose caching allocator owns
+ * all device memory and does not lend it to plug-ins, and serving loops that forbid any
+ * allocation after start-up so that memory use stays fixed.
  *   - Returns SAC_ERR_UNSUPPORTED when B*S*D*sizeof(dtype) exceeds sac_static_scratch_bytes().
  *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current); make that first call before any stream capture.
+ *     with that device current); make that first call before any stream capture. Later calls
+ *     look the address up again whenever their stream is not capturing, so that a context torn
+ *     down and created again (cudaDeviceReset) never leaves a stale address behind.
  *   - All calls share the one array and it keeps the last call's contents; every byte a call
  *     reads is first written by the same call. Calls that overlap on the GPU (concurrent streams
- *     or devices sharing nothing but this array per device) race on it: serialise them.
+ *     sharing a device) race on it: serialise them.
+ *   - There is no status word: a tensor-core kernel that gives up a bounded wait returns silently.
  *   - Allocates nothing: no cudaMalloc / cudaFree and no allocating library routine.
  */
 SAC_API size_t sac_static_scratch_bytes(void);
@@ -180,7 +184,9 @@ SAC_API int csa_forward(const sac_params* p, const void* q, const void* kv, cons
  *     pool_block_table [nseq, pool_max_pages] with entry w at page w/page_size, row w%page_size.
  *   - ctx_lens [nseq] int32 (device) counts the new token: the query is token t = ctx-1 at
  *     position pos0 + t, it sees the last min(ctx, W) tokens and floor(ctx/m) entries.
- *     Every ctx must satisfy 1 <= ctx <= p->S.
+ *     Every ctx must satisfy 1 <= ctx <= p->S. The kernels check the upper bound (the block
+ *     tables cover p->S rows): a sequence with ctx > p->S reads no cache row, its output row is
+ *     left undefined and status 4 is recorded in the workspace's status word (sac_device_status).
  *   q [nseq,H,D] un-rotated; o [nseq,H,D]; q_idx [nseq,nI,cI], w_idx [nseq,nI] fp32 (CSA);
  *   topk_out [nseq,k] nullable (ascending entries, -1 fill).
  * Workspace: sac_decode_workspace_size() bytes, 16-byte aligned: a 256-byte status word (see
@@ -232,7 +238,9 @@ SAC_API int csa_decode(const sac_params* p, int nseq, const void* q, const void*
  * CSA also takes k_idx_new [nseq, cI], idx_state [nseq, win_len, cI], idx_gate [cI], idx_bias
  * [win_len] fp32 and idx_pool_pages, and closes the indexer entry the same way without rotation.
  * SWA uses only kv_new and the kv pages (the other pointers may be NULL). Rows on unallocated
- * pages (block table entry < 0) are skipped. No workspace; returns before the kernel runs.
+ * pages (block table entry < 0) are skipped, and so are sequences whose ctx lies outside
+ * [1, p->S] (the block tables cover p->S rows): nothing of theirs is read or written. No
+ * workspace; returns before the kernel runs.
  */
 SAC_API int decode_append(const sac_params* p, int kind, int nseq, const int32_t* ctx_lens,
                const void* kv_new, const void* k_idx_new, const void* cmp_gate,
@@ -250,8 +258,8 @@ SAC_API int decode_append(const sac_params* p, int kind, int nseq, const int32_t
  * by position, so the chunk attends to the cached prefix plus itself, causally.
  * Arguments as in *_decode, with n rows per sequence: q, o [nseq, n, H, D]; q_idx [nseq, n, nI,
  * cI]; w_idx [nseq, n, nI]; topk_out [nseq, n, k]; every ctx must satisfy n <= ctx <= p->S
- * (the device cannot check it: rows of a sequence with ctx < n have t < 0, see no key, and their
- * output rows are left undefined).
+ * (rows of a sequence with ctx < n have t < 0, see no key, and their output rows are left
+ * undefined; a sequence with ctx > p->S is handled as in decode, with status 4).
  * Workspace: sac_chunk_workspace_size() bytes (the decode layout for nseq * n query rows; the
  * CSA scores hold at most 1 GiB of rows at once, the indexer and top-k then run in row blocks).
  * Decode is the case n = 1.
@@ -286,7 +294,7 @@ SAC_API int csa_prefill_chunk(const sac_params* p, int nseq, int n, const void* 
  * chunk row is written rotated to the window pages and the ring keeps the sequence's last
  * win_len rows. Appending a stream chunk by chunk (any sizes, decode steps mixed
  * in) leaves the same caches as appending it token by token. Sequences with ctx < n are left
- * untouched. No workspace.
+ * untouched, and so are sequences with ctx > p->S (as in decode_append). No workspace.
  */
 SAC_API int prefill_chunk_append(const sac_params* p, int kind, int nseq, int n,
                const int32_t* ctx_lens, const void* kv_new, const void* k_idx_new,
@@ -322,8 +330,8 @@ SAC_API int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank,
  * of its workspace; a tensor-core kernel that gives up a bounded wait (2 s) writes a nonzero code
  * there and returns instead of hanging. This call waits for `stream`, copies the word to *status
  * (0 = ok, 1 = a wait timed out, 2 = misaligned shared memory, 3 = a kernel launched with a block
- * size its arguments do not allow: an internal error) and returns SAC_OK, or SAC_ERR_LAUNCH if
- * the copy fails.
+ * size its arguments do not allow: an internal error, 4 = a decode / chunk context length above
+ * p->S, whose rows were skipped) and returns SAC_OK, or SAC_ERR_LAUNCH if the copy fails.
  */
 SAC_API int sac_device_status(const void* ws, int* status, void* stream);
 
@@ -337,8 +345,8 @@ SAC_API int sac_device_status(const void* ws, int* status, void* stream);
  * records then hold the times of the graph's most recent replay.
  *
  * CUDA graphs: after one eager call with the same shapes (which performs the one-time per-device
- * setup), every entry point except sac_device_status and swa_forward_static's first call may be
- * captured into a CUDA graph; nothing they enqueue synchronises or allocates.
+ * setup), the prefill, decode, chunk, append and projection entry points that take a workspace
+ * may be captured into a CUDA graph; nothing they enqueue synchronises or allocates.
  */
 typedef struct {
   char name[32];

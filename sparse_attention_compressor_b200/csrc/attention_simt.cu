@@ -49,7 +49,8 @@ __global__ void attention_simt_kernel(AttnArgs a, int HG) {
   const int nh = min(HG, a.H - h0);
   int seq;
   int64_t t;
-  a.qr.locate(a.qr.row0 + row, seq, t);
+  if (!a.qr.locate(a.qr.row0 + row, seq, t) && threadIdx.x == 0 && blockIdx.y == 0 && a.status)
+    atomicExch(a.status, 4);  // a context beyond the block tables: the row sees no key
   const int64_t P = a.pos0 + t;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int R = a.rf.R;

@@ -83,11 +83,17 @@ struct Row {
   int64_t r;   // query row of the work item
   int sp;      // split of the row's key tiles this item covers
   int j0, j1;  // tile range [j0, j1) of the item
+  bool bad;    // the row's context lies beyond the block tables (no key is read)
 };
 
 __device__ __forceinline__ Row locate_row(const AttnArgs& a, int64_t r) {
   Row w;
-  a.qr.locate(a.qr.row0 + r, w.seq, w.t);
+  w.bad = !a.qr.locate(a.qr.row0 + r, w.seq, w.t);
+  if (w.t < 0) {  // no key: a bad context, or a chunk row before its sequence's start
+    w.lo = 0;
+    w.nwin = w.npool = w.twin = w.tiles = 0;
+    return w;
+  }
   w.lo = w.t - a.W + 1 < 0 ? 0 : w.t - a.W + 1;
   w.nwin = (int)(w.t - w.lo + 1);
   const int nvis = a.pool_mode ? (int)((w.t + 1) / a.m) : 0;
@@ -231,6 +237,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
       bool ok = true;
       for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const Row w = locate_item<kSplit>(a, it);
+        if (w.bad && status) atomicExch(status, tc::kStatusBadInput);
         if (w.j0 == w.j1) continue;
         const int64_t r = w.r;
         if (qi > 0) ok = tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status);

@@ -26,6 +26,7 @@ namespace {
 
 struct AppendPart {
   const int32_t* ctx_lens;
+  int64_t max_ctx;               // contexts above this (beyond the block tables) are skipped
   int m, L, page_size;
   int64_t pos0;
   RopeFreqs rf;
@@ -42,6 +43,13 @@ struct AppendPart {
   int rotate;
 };
 
+// Context length of sequence seq; 0 (the sequence is skipped) when it exceeds max_ctx, a bad
+// input the block tables do not cover.
+__device__ __forceinline__ int64_t checked_ctx(const AppendPart& a, int seq) {
+  const int64_t c = __ldg(a.ctx_lens + seq);
+  return c > a.max_ctx ? 0 : c;
+}
+
 template <typename T>
 __device__ __forceinline__ T* page_row(void* base, const int32_t* bt, int max_pages, int page_size,
                                        int C, int seq, int64_t j) {
@@ -56,7 +64,7 @@ template <typename T, int V>
 __device__ __forceinline__ void append_warp(const AppendPart& a, int seq, int lane,
                                             PoolShared<V, 1>& sh) {
   constexpr int C = 32 * V;
-  const int64_t t = (int64_t)__ldg(a.ctx_lens + seq) - 1;
+  const int64_t t = checked_ctx(a, seq) - 1;
   if (t < 0) return;
   const T* x_new = reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * C;
   T* ring = a.m > 0 ? reinterpret_cast<T*>(a.ring) + (int64_t)seq * a.L * C : nullptr;
@@ -105,7 +113,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendPart a) {
   __shared__ PoolShared<V, WPE> sh;
   const int seq = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)__ldg(a.ctx_lens + seq) - 1;
+  const int64_t t = checked_ctx(a, seq) - 1;
   if (t < 0) return;
   const T* x_new = reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * C;
   T* ring = a.m > 0 ? reinterpret_cast<T*>(a.ring) + (int64_t)seq * a.L * C : nullptr;
@@ -155,7 +163,7 @@ __global__ void __launch_bounds__(256) chunk_pool_kernel(AppendPart a, int n) {
   __shared__ PoolShared<V, WPE> sh;
   const int seq = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t ctx = __ldg(a.ctx_lens + seq), t0 = ctx - n;
+  const int64_t ctx = checked_ctx(a, seq), t0 = ctx - n;
   if (t0 < 0) return;  // fewer tokens than the chunk: left untouched
   const int64_t w = t0 / a.m + (int64_t)blockIdx.x * EPB + warp / WPE;
   const bool active = w < ctx / a.m;
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(256) chunk_rows_kernel(AppendPart a, int n) {
   const int seq = blockIdx.y;
   const int lane = threadIdx.x & 31;
   const int64_t i = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int64_t ctx = __ldg(a.ctx_lens + seq), t0 = ctx - n;
+  const int64_t ctx = checked_ctx(a, seq), t0 = ctx - n;
   if (t0 < 0 || i >= n) return;
   const int64_t t = t0 + i;
   float v[V];
@@ -254,6 +262,7 @@ cudaError_t append_dispatch(const AppendPart& a, int C, int nseq, cudaStream_t s
 static AppendPart make_part(const DecodeAppendArgs& a, bool index_part) {
   AppendPart p{};
   p.ctx_lens = a.ctx_lens;
+  p.max_ctx = a.max_ctx;
   p.m = a.m;
   p.L = a.L;
   p.page_size = a.page_size;

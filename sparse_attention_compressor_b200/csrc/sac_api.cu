@@ -251,20 +251,28 @@ namespace {
 std::mutex g_static_scratch_mu;
 void* g_static_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device, looked up once per device (the host
-// symbol is only a stand-in: kernels must be given this address).
-int static_scratch_address(void** out) {
+// Device address of g_static_scratch on the current device (the host symbol is only a stand-in:
+// kernels must be given this address). The first call on a device looks it up with that device
+// current; later calls look it up again whenever their stream is not capturing, so a context torn
+// down and created again (cudaDeviceReset) gets the address of its own copy. A capturing stream
+// takes the address found by the device's last look-up (none yet: an error).
+int static_scratch_address(cudaStream_t st, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   REQUIRE(dev >= 0 && dev < kMaxDevices, SAC_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cap);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
   std::lock_guard<std::mutex> lk(g_static_scratch_mu);
-  if (g_static_scratch_addr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
     g_static_scratch_addr[dev] = ptr;
   }
+  REQUIRE(g_static_scratch_addr[dev] != nullptr, SAC_ERR_ARG,
+          "swa_forward_static: the first call on a device must come before any stream capture");
   *out = g_static_scratch_addr[dev];
   return SAC_OK;
 }
@@ -282,14 +290,15 @@ int swa_forward_static(const sac_params* p, const void* q, const void* kv, const
   REQUIRE_PTR(kv);
   REQUIRE_PTR(sinks);
   REQUIRE_PTR(o);
+  // the scratch swa_forward takes from its workspace for the rotated kv stream
   const size_t need = (size_t)p->B * p->S * p->D * esize(p->dtype);
   REQUIRE(need <= kStaticScratchBytes, SAC_ERR_UNSUPPORTED,
           "B*S*head_dim needs %zu bytes of scratch; the static scratch holds %zu", need,
           kStaticScratchBytes);
-  void* kv_rot = nullptr;
-  rc = static_scratch_address(&kv_rot);
-  if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* kv_rot = nullptr;
+  rc = static_scratch_address(st, &kv_rot);
+  if (rc) return rc;
   sac::RopeFreqs rf = rope_freqs(p);
   const int64_t rows = (int64_t)p->B * p->S;
   cudaError_t e = sac::timed("rotate_kv", st, [&] {
@@ -301,7 +310,8 @@ int swa_forward_static(const sac_params* p, const void* q, const void* kv, const
   a.nrows = rows;
   a.win = contiguous(kv_rot, p->S, p->D);
   a.pool_mode = 0;
-  e = sac::timed("attention", st, [&] { return sac::launch_attention_simt(p->dtype, a, st); });
+  // no status word: a kernel giving up a bounded wait returns silently
+  e = run_attention(p, a, rows, 0, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }
@@ -610,7 +620,7 @@ static int paged_attention(const sac_params* p, const PagedCall& c) {
             "pool block table too short for S/m entries");
   }
   cudaStream_t st = static_cast<cudaStream_t>(c.stream);
-  sac::QueryRows qr{0, c.ctx_lens, 0, c.nq};
+  sac::QueryRows qr{0, c.ctx_lens, 0, c.nq, (int64_t)p->S};
   sac::AttnArgs a = attn_common(p, c.q, c.o, c.sinks);
   a.qr = qr;
   a.nrows = rows;
@@ -646,7 +656,7 @@ static int paged_attention(const sac_params* p, const PagedCall& c) {
     const size_t qi_row = (size_t)p->n_idx_heads * p->idx_dim * esize(p->dtype);
     for (int64_t r0 = 0; r0 < rows; r0 += score_rows) {
       const int64_t nr = rows - r0 < score_rows ? rows - r0 : score_rows;
-      sac::QueryRows bq{0, c.ctx_lens, r0, c.nq};
+      sac::QueryRows bq{0, c.ctx_lens, r0, c.nq, (int64_t)p->S};
       sac::IndexerArgs ia;
       ia.q_idx = static_cast<const char*>(c.q_idx) + (size_t)r0 * qi_row;
       ia.w_idx = c.w_idx + (size_t)r0 * p->n_idx_heads;
@@ -815,6 +825,7 @@ static int append_paged(const sac_params* p, int kind, int nseq, int n, const in
   std::memset(&a, 0, sizeof(a));
   a.nseq = nseq;
   a.ctx_lens = ctx_lens;
+  a.max_ctx = p->S;
   a.D = p->D;
   a.pos0 = p->pos0;
   a.rf = rope_freqs(p);

@@ -76,16 +76,27 @@ struct QueryRows {
   int64_t row0;              // first flat row of this launch (prefill chunking)
   int nq;                    // with ctx_lens: query rows per sequence, the last nq positions
                              // (0 or 1: one query per sequence, decode)
+  int64_t max_ctx;           // with ctx_lens: the longest context the block tables cover
+                             // (0: not checked)
 
-  __device__ __forceinline__ void locate(int64_t r, int& seq, int64_t& t) const {
+  // Sequence and position of row r. A context above max_ctx is a bad input: the row then gets
+  // t = -1, so it sees no key and addresses no cache row, and locate returns false. Rows with
+  // t < 0 (also those of a context shorter than nq) see no key; their output rows are undefined.
+  __device__ __forceinline__ bool locate(int64_t r, int& seq, int64_t& t) const {
     if (ctx_lens != nullptr) {
       const int q = nq > 1 ? nq : 1;
       seq = (int)(r / q);
-      t = (int64_t)__ldg(ctx_lens + seq) - q + r % q;
+      const int64_t ctx = __ldg(ctx_lens + seq);
+      if (max_ctx > 0 && ctx > max_ctx) {
+        t = -1;
+        return false;
+      }
+      t = ctx - q + r % q;
     } else {
       seq = (int)(r / S);
       t = r % S;
     }
+    return true;
   }
 };
 

@@ -28,6 +28,7 @@ cudaError_t launch_rotate_rows(int dtype, const void* x, int64_t rows, int S, in
 struct DecodeAppendArgs {
   int nseq;
   const int32_t* ctx_lens;
+  int64_t max_ctx;            // the longest context the block tables cover; longer: skipped
   int D, cI, m, L;
   int64_t pos0;
   RopeFreqs rf;

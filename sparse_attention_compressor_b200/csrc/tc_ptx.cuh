@@ -13,7 +13,13 @@ namespace tc {
 // ---------------------------------------------------------------------------------------------
 // status word: kernels that give up a wait record the reason here and return
 // ---------------------------------------------------------------------------------------------
-enum : int { kStatusOk = 0, kStatusWaitTimeout = 1, kStatusMisaligned = 2, kStatusConfig = 3 };
+enum : int {
+  kStatusOk = 0,
+  kStatusWaitTimeout = 1,
+  kStatusMisaligned = 2,
+  kStatusConfig = 3,
+  kStatusBadInput = 4,  // a context length beyond the range the call's block tables cover
+};
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
