@@ -1,7 +1,7 @@
 """Benchmark of the hybrid-attention forward on B200 (one process per GPU).
 
 `python bench.py --gpus N --steps K --warmup W` times K steps of one workload (default: the CSA
-prefill at 8k tokens, bf16) and rank 0 prints one JSON line. A step is one csa_forward call: the
+prefill at 128k tokens, bf16) and rank 0 prints one JSON line. A step is one csa_forward call: the
 compressor over kv and over the indexer key stream, the indexer score, top-k, and the sparse +
 sliding attention with the sink and both RoPE rotations. With N > 1 (torchrun, NCCL) every rank
 runs its own sequence (data parallel, no collective on the data path; weak scaling) and the time
@@ -285,14 +285,47 @@ def tensor_kernels(wl) -> set:
     return out
 
 
-# DRAM bytes (read + write) per launch from one ncu capture of the kernel as it stands, keyed by
-# (workload, kernel); the summary with its command is the named file under profiles/. An entry is
-# removed whenever its kernel changes, and the roofline then reports traffic null.
-NCU_TRAFFIC = {
-    ("csa_8k_bf16", "attention"): (563.554048e6 + 490.33856e6, "attention_tc_csa_8k_bf16.md"),
-    ("csa_8k_bf16", "indexer_score"): (136.957696e6 + 25.005312e6, "indexer_tc_csa_8k_bf16.md"),
-    ("csa_8k_bf16", "topk"): (31.872256e6 + 12.288e3, "topk_csa_8k_bf16.md"),
+# DRAM bytes (read + write) per launch of a kernel come from one ncu capture, recorded in
+# profiles/ncu_traffic.json with the SHA-256 of the kernel's sources at capture time. A record
+# whose sources have changed since is stale and the roofline reports traffic null.
+CSRC = os.path.join(ROOT, "sparse_attention_compressor_b200", "csrc")
+KERNEL_SOURCES = {
+    "attention": ["attention_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
+    "csa_decode_attention": ["attention_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
+    "hca_decode_attention": ["attention_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
+    "indexer_score": ["indexer_tc.cu", "indexer_decode_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
+    "topk": ["topk.cu", "sac_common.cuh"],
+    "compress": ["compress.cu", "pool_window.cuh", "tc_ptx.cuh", "sac_common.cuh"],
+    "compress_index": ["compress.cu", "pool_window.cuh", "tc_ptx.cuh", "sac_common.cuh"],
+    "decode_append": ["decode_append.cu", "pool_window.cuh", "sac_common.cuh"],
+    "o_proj": ["oproj.cu", "tc_ptx.cuh"],
 }
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+
+
+def source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        path = os.path.join(CSRC, f)
+        if os.path.exists(path):
+            with open(path, "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(workload: str, kernel: str):
+    """(bytes per launch, record) of a current ncu record of the kernel on this workload, or
+    (None, None) when there is none or its sources changed since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, None
+    with open(TRAFFIC_FILE) as f:
+        recs = json.load(f)
+    for r in recs:
+        if r["workload"] == workload and r["kernel"] == kernel and \
+                r["source_sha256"] == source_hash(kernel):
+            return float(r["dram_bytes_per_launch"]), r
+    return None, None
 
 
 def roofline(wl, ktimes: dict, peaks: dict, steps: int, tensor_kernels: set) -> tuple:
@@ -321,36 +354,69 @@ def roofline(wl, ktimes: dict, peaks: dict, steps: int, tensor_kernels: set) -> 
                              frac=achieved / peaks["hbm_gbs"])
         rows[name] = entry
     dom = max(ktimes, key=lambda k: ktimes[k][1])
-    d = rows[dom]
-    tr = NCU_TRAFFIC.get((wl.name, dom))
-    roof = {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
+    return roof_of(wl.name, dom, rows[dom], peaks), rows
+
+
+def roof_of(workload: str, kernel: str, d: dict, peaks: dict) -> dict:
+    traffic, rec = ncu_traffic(workload, kernel)
+    roof = {"kernel": kernel, "bound": d.get("bound"), "achieved": d.get("achieved"),
             "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),
-            "traffic": tr[0] if tr else None, "peak_source": peaks["source"]}
-    if tr:
-        roof["traffic_source"] = "profiles/" + tr[1]
-    return roof, rows
+            "traffic": traffic, "peak_source": peaks["source"]}
+    if rec is not None:
+        roof["traffic_source"] = rec["summary"]
+        if rec.get("scaled_from"):
+            roof["traffic_note"] = rec["scaled_from"]
+    return roof
 
 
-def cpu_baseline(wl, budget_s: float = 12.0) -> dict:
-    """The fp64 oracle on a bounded sample of query rows of the same workload (rank 0, N=1)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(wl, budget_s: float = 12.0, single_budget_s: float = 4.0) -> dict:
+    """The fp64 oracle on a bounded sample of query rows of the same workload (rank 0, N=1):
+    first on all host threads, then single-threaded. Rows are drawn uniformly, so rows / time
+    estimates the tokens/s of the whole sequence (each row's work, indexer scores over its visible
+    entries included, is independent given the pools); the estimate is marked extrapolated when
+    the sample is smaller than the workload."""
     import oracle
     t0 = time.perf_counter()
     threads = oracle.max_threads()
     n = max(1, threads)
-    value, sample = None, None
     x = W.prefill_inputs(wl, with_queries=False)
     rng = np.random.default_rng(0)
+    total = wl.B * wl.S
     while True:
-        rows = np.sort(rng.choice(wl.B * wl.S, size=min(n, wl.B * wl.S), replace=False))
+        rows = np.sort(rng.choice(total, size=min(n, total), replace=False))
         dt = oracle_rows(wl, x, rows)
-        if dt > budget_s / 3 or n >= wl.B * wl.S or time.perf_counter() - t0 > budget_s:
-            value = len(rows) / dt
-            sample = (f"{len(rows)} random query rows of {wl.name} (full path incl. compressor "
-                      f"over all {wl.S} tokens), {dt:.2f} s")
+        if dt > budget_s / 3 or n >= total or time.perf_counter() - t0 > budget_s:
             break
         n = int(n * min(8.0, max(2.0, (budget_s / 3) / max(dt, 1e-3))))
-    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": sample}
+    out = {"value": len(rows) / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "cpu_model": cpu_model(),
+           "sample": f"{len(rows)} random query rows of {wl.name} (full path incl. compressor "
+                     f"over all {wl.S} tokens), {dt:.2f} s on {threads} threads",
+           "extrapolated": len(rows) < total}
+    # single-threaded point on a smaller sample of the same rows
+    oracle.set_threads(1)
+    try:
+        n1 = max(1, min(len(rows), int(len(rows) * single_budget_s / max(dt * threads, 1e-3))))
+        rows1 = rows[:n1]
+        dt1 = oracle_rows(wl, x, rows1)
+        out["single_thread"] = {"value": len(rows1) / dt1, "unit": "tokens/s", "cores": 1,
+                                "sample": f"{len(rows1)} of the same rows, {dt1:.2f} s",
+                                "extrapolated": len(rows1) < total}
+    finally:
+        oracle.set_threads(threads)
+    return out
 
 
 def oracle_rows(wl, x, rows) -> float:
@@ -680,9 +746,7 @@ def run_decode(args, wl0):
         "clocks": clk.summary(),
         "e2e": e2e,
         "gpu_launches": sum(v[0] for v in ktimes.values()) * args.steps,
-        "roofline": {"kernel": dom, "bound": d.get("bound"), "achieved": d.get("achieved"),
-                     "peak": d.get("peak"), "unit": d.get("unit"), "frac": d.get("frac"),
-                     "traffic": None, "peak_source": peaks["source"]},
+        "roofline": roof_of(wl.name, dom, d, peaks),
         "kernels": krows,
     }
     if rank == 0:
@@ -749,10 +813,9 @@ def run_oproj(args, wl0):
         "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": pin_o.numel() * 2, "d2h_bytes_per_step": out.numel() * 2},
         "gpu_launches": 2 * args.steps,
-        "roofline": {"kernel": "o_proj", "bound": "tensor", "achieved": ach,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": ach / peaks["bf16_tflops"], "traffic": None,
-                     "peak_source": peaks["source"]},
+        "roofline": roof_of(wl.name, "o_proj", {"bound": "tensor", "achieved": ach,
+                                                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                                 "frac": ach / peaks["bf16_tflops"]}, peaks),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -897,7 +960,8 @@ def run_reference(args, wl):
     oracle.build()
     x = W.prefill_inputs(wl, with_queries=False)
     threads = oracle.max_threads()
-    n = max(32, 32 * threads)
+    # rows per step: long sequences cost more per row (the indexer scores every visible entry)
+    n = max(16, int(32 * threads * min(1.0, 32768 / wl.S)))
     rng = np.random.default_rng(1)
     samples = [np.sort(rng.choice(wl.B * wl.S, size=n, replace=False))
                for _ in range(args.warmup + args.steps)]
@@ -922,16 +986,32 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def launch_ranks(n: int, argv: list) -> int:
+    """Run this script on n local ranks (torch.distributed.run, rendezvous on 127.0.0.1) and return
+    the launcher's exit status; rank 0 prints the JSON line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + argv
+    return subprocess.call(cmd)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="csa_8k_bf16", choices=list(W.WORKLOADS))
+    ap.add_argument("--workload", default="csa_128k_bf16", choices=list(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     wl = W.WORKLOADS[args.workload]
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: relaunch this command under torch.distributed.run
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv)))
     if args.impl == "reference":
         run_reference(args, wl)
     elif wl.kind == "decode":

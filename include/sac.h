@@ -80,6 +80,15 @@ extern "C" {
  *   softmax_scale   logit scale (e.g. 1/sqrt(D)).
  *   pos0            absolute position of token 0 (prefill); added to every decode position.
  *   dtype           SAC_F32 or SAC_BF16.
+ *   rope_factor, rope_orig_max_pos, yarn_beta_fast, yarn_beta_slow
+ *                   YaRN frequency scaling of every rotation of the layer [the rope scaling the
+ *                   config pairs with compress_rope_theta; the page gives no values]. With
+ *                   rope_factor s > 1, pair i (base frequency f_i) completes
+ *                   r_i = rope_orig_max_pos * f_i / (2 pi) turns over the original context and
+ *                   turns at (1 - g) f_i / s + g f_i, g = clamp((r_i - yarn_beta_slow) /
+ *                   (yarn_beta_fast - yarn_beta_slow), 0, 1) (YaRN, Peng et al. 2023; usual values
+ *                   32 and 1). YaRN's attention temperature scales the logits only: fold it into
+ *                   softmax_scale. rope_factor <= 1: plain RoPE, the other three are ignored.
  */
 typedef struct {
   int B, S, H, D, R;
@@ -90,12 +99,15 @@ typedef struct {
   float softmax_scale;
   int64_t pos0;
   int dtype;
+  double rope_factor;
+  int rope_orig_max_pos;
+  double yarn_beta_fast, yarn_beta_slow;
 } sac_params;
 
 /* Message of the calling thread's last failed call ("" if none). Static storage. */
 SAC_API const char* sac_last_error(void);
 
-/* ABI version (major*100 + minor). */
+/* ABI version (major*100 + minor): 200 (sac_params carries the YaRN fields). */
 SAC_API int sac_version(void);
 
 /*

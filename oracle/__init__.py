@@ -34,7 +34,9 @@ class _Params(ctypes.Structure):
         ("R", ctypes.c_int), ("theta", ctypes.c_double), ("m", ctypes.c_int),
         ("L", ctypes.c_int), ("W", ctypes.c_int), ("nI", ctypes.c_int), ("cI", ctypes.c_int),
         ("k", ctypes.c_int), ("scale", ctypes.c_double), ("pos0", ctypes.c_int64),
-        ("bf16_pools", ctypes.c_int),
+        ("bf16_pools", ctypes.c_int), ("yarn_factor", ctypes.c_double),
+        ("yarn_orig", ctypes.c_int), ("yarn_beta_fast", ctypes.c_double),
+        ("yarn_beta_slow", ctypes.c_double),
     ]
 
 
@@ -56,12 +58,17 @@ class OracleParams:
     scale: float = 0.0
     pos0: int = 0
     bf16_pools: bool = False  # pools cached in bf16 (the layer's working dtype)
+    yarn_factor: float = 1.0  # YaRN context scale s (<= 1: plain RoPE)
+    yarn_orig: int = 0        # YaRN original context length
+    yarn_beta_fast: float = 32.0
+    yarn_beta_slow: float = 1.0
 
     def c(self) -> _Params:
         scale = self.scale if self.scale > 0 else 1.0 / np.sqrt(self.D)
         return _Params(self.B, self.S, self.H, self.D, self.R, float(self.theta), self.m,
                        self.L, self.W, self.nI, self.cI, self.k, float(scale), int(self.pos0),
-                       int(self.bf16_pools))
+                       int(self.bf16_pools), float(self.yarn_factor), int(self.yarn_orig),
+                       float(self.yarn_beta_fast), float(self.yarn_beta_slow))
 
 
 def build(force: bool = False) -> str:
@@ -82,6 +89,13 @@ def _lib():
     if _lib_handle is None:
         lib = ctypes.CDLL(build())
         lib.orc_rope.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double]
+        lib.orc_rope_yarn.argtypes = [_dp, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                      ctypes.c_double, ctypes.c_int, ctypes.c_double,
+                                      ctypes.c_double, ctypes.c_double]
+        lib.orc_rope_freq.restype = ctypes.c_double
+        lib.orc_rope_freq.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                      ctypes.c_double, ctypes.c_int, ctypes.c_double,
+                                      ctypes.c_double]
         lib.orc_compress.restype = ctypes.c_long
         lib.orc_compress.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, _dp, _dp, _dp, _dp]
@@ -153,6 +167,24 @@ def rope(x, R: int, theta: float, pos: float) -> np.ndarray:
     for r in rows:
         _lib().orc_rope(_ptr(r), a.shape[-1], R, float(theta), float(pos))
     return rows.reshape(a.shape)
+
+
+def rope_yarn(x, R: int, theta: float, pos: float, factor: float, orig: int,
+              beta_fast: float = 32.0, beta_slow: float = 1.0) -> np.ndarray:
+    """rope() with YaRN frequencies (context scale `factor` over an original length `orig`)."""
+    a = _f64(x).copy()
+    rows = a.reshape(-1, a.shape[-1])
+    for r in rows:
+        _lib().orc_rope_yarn(_ptr(r), a.shape[-1], R, float(theta), float(factor), int(orig),
+                             float(beta_fast), float(beta_slow), float(pos))
+    return rows.reshape(a.shape)
+
+
+def rope_freq(i: int, R: int, theta: float, factor: float = 1.0, orig: int = 1,
+              beta_fast: float = 32.0, beta_slow: float = 1.0) -> float:
+    """Frequency of rope pair i (YaRN-scaled when factor > 1)."""
+    return float(_lib().orc_rope_freq(i, R, float(theta), float(factor), int(orig),
+                                      float(beta_fast), float(beta_slow)))
 
 
 def compress(x, u, bias, m: int, L: int) -> np.ndarray:

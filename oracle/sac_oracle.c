@@ -37,6 +37,9 @@ typedef struct {
   double scale;        /* softmax scale tau                                                   */
   int64_t pos0;        /* absolute position of token 0                                        */
   int bf16_pools;      /* 1: pools are cached in bf16 (see orc_round_bf16)                     */
+  double yarn_factor;  /* YaRN context scale s (<= 1: plain RoPE)                             */
+  int yarn_orig;       /* YaRN original context length L                                      */
+  double yarn_beta_fast, yarn_beta_slow;  /* YaRN ramp bounds beta (fast) and alpha (slow)    */
 } orc_params;
 
 int orc_max_threads(void) {
@@ -77,19 +80,52 @@ static void round_pool(const orc_params *p, double *x, size_t n) {
 /* ---------------------------------------------------------------------------------------------
  * Partial interleaved-pair RoPE ("Hybrid attention", shared skeleton, partial RoPE bullet):
  * only the trailing R channels of a head rotate; channel pairs are (D-R+2i, D-R+2i+1);
- * pair i turns by angle pos * theta^(-2i/R). A negative pos gives the inverse rotation
- * (the "-i" rotation the page applies to the rope slice of the attention output, eq. 26).
+ * pair i turns by angle pos * f_i. A negative pos gives the inverse rotation (the "-i" rotation
+ * the page applies to the rope slice of the attention output, eq. 26).
+ *
+ * Frequencies. Plain RoPE: f_i = theta^(-2i/R). The config pairs compress_rope_theta with a YaRN
+ * rope scaling ("DeepseekV4Config") but gives none of its parameters, so they are arguments here
+ * ([reading]: factor <= 1 means no scaling). YaRN (Peng et al. 2023, "YaRN:
+ * Efficient Context Window Extension of Large Language Models", the "NTK-by-parts"
+ * interpolation): with context scale s and original context length L, pair i completes
+ * r_i = L / (2 pi / f_i) turns over L tokens; the ramp gamma_i = 0 for r_i < alpha, 1 for
+ * r_i > beta and (r_i - alpha) / (beta - alpha) between; the scaled frequency is
+ * (1 - gamma_i) * f_i / s + gamma_i * f_i (slow pairs interpolated, fast pairs kept). YaRN's
+ * attention temperature multiplies the logits only, so it lives in the softmax scale (an input).
  * ------------------------------------------------------------------------------------------- */
-void orc_rope(double *x, int D, int R, double theta, double pos) {
+double orc_rope_freq(int i, int R, double theta, double s, int L, double beta_fast,
+                     double beta_slow) {
+  double f = pow(theta, -2.0 * (double)i / (double)R);
+  if (!(s > 1.0)) return f;
+  const double pi = 3.14159265358979323846;
+  double r = (double)L / (2.0 * pi / f);
+  double gamma;
+  if (r < beta_slow) gamma = 0.0;
+  else if (r > beta_fast) gamma = 1.0;
+  else gamma = (r - beta_slow) / (beta_fast - beta_slow);
+  return (1.0 - gamma) * f / s + gamma * f;
+}
+
+void orc_rope_yarn(double *x, int D, int R, double theta, double s, int L, double beta_fast,
+                   double beta_slow, double pos) {
   for (int i = 0; i < R / 2; ++i) {
-    double freq = pow(theta, -2.0 * (double)i / (double)R);
-    double phi = pos * freq;
-    double c = cos(phi), s = sin(phi);
+    double phi = pos * orc_rope_freq(i, R, theta, s, L, beta_fast, beta_slow);
+    double c = cos(phi), sn = sin(phi);
     double *p = x + (D - R) + 2 * i;
     double a = p[0], b = p[1];
-    p[0] = a * c - b * s;
-    p[1] = a * s + b * c;
+    p[0] = a * c - b * sn;
+    p[1] = a * sn + b * c;
   }
+}
+
+void orc_rope(double *x, int D, int R, double theta, double pos) {
+  orc_rope_yarn(x, D, R, theta, 1.0, 1, 0.0, 0.0, pos);
+}
+
+/* The rotation of a layer: its base and, when yarn_factor > 1, its YaRN frequencies. */
+static void layer_rope(const orc_params *p, double *x, double pos) {
+  orc_rope_yarn(x, p->D, p->R, p->theta, p->yarn_factor, p->yarn_orig, p->yarn_beta_fast,
+                p->yarn_beta_slow, pos);
 }
 
 /* ---------------------------------------------------------------------------------------------
@@ -221,9 +257,9 @@ static void attend_row(const orc_params *p, const double *q_t, double pos_t, lon
   size_t hd = (size_t)p->H * p->D;
   double *qr = (double *)malloc(sizeof(double) * hd);
   memcpy(qr, q_t, sizeof(double) * hd);
-  for (int h = 0; h < p->H; ++h) orc_rope(qr + (size_t)h * p->D, p->D, p->R, p->theta, pos_t);
+  for (int h = 0; h < p->H; ++h) layer_rope(p, qr + (size_t)h * p->D, pos_t);
   orc_attend(p->H, p->D, p->scale, qr, nk, keys, sinks, o_t);
-  for (int h = 0; h < p->H; ++h) orc_rope(o_t + (size_t)h * p->D, p->D, p->R, p->theta, -pos_t);
+  for (int h = 0; h < p->H; ++h) layer_rope(p, o_t + (size_t)h * p->D, -pos_t);
   free(qr);
 }
 
@@ -238,7 +274,7 @@ static long window_lo(long t, int W) {
 /* Copy kv row j of batch b, rotated at its absolute position. */
 static void rotated_kv_row(const orc_params *p, const double *kv, int b, long j, double *dst) {
   memcpy(dst, kv + ((size_t)b * p->S + j) * p->D, sizeof(double) * p->D);
-  orc_rope(dst, p->D, p->R, p->theta, (double)(p->pos0 + j));
+  layer_rope(p, dst, (double)(p->pos0 + j));
 }
 
 /* [reading] pool entry w is rotated at the first position of the block it stands for,
@@ -284,7 +320,7 @@ static long rotated_pool(const orc_params *p, const double *kv, const double *u,
   long N = orc_compress(p->B, p->S, p->D, p->m, p->L, kv, u, bias, pool);
   for (int b = 0; b < p->B; ++b)
     for (long w = 0; w < N; ++w)
-      orc_rope(pool + ((size_t)b * N + w) * p->D, p->D, p->R, p->theta, entry_pos(p, w));
+      layer_rope(p, pool + ((size_t)b * N + w) * p->D, entry_pos(p, w));
   round_pool(p, pool, (size_t)p->B * N * p->D);
   return N;
 }

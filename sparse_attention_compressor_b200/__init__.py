@@ -42,17 +42,22 @@ class sac_params(ctypes.Structure):
                 ("m", ctypes.c_int), ("win_len", ctypes.c_int), ("sliding_window", ctypes.c_int),
                 ("n_idx_heads", ctypes.c_int), ("idx_dim", ctypes.c_int), ("topk", ctypes.c_int),
                 ("softmax_scale", ctypes.c_float), ("pos0", ctypes.c_int64),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("rope_factor", ctypes.c_double),
+                ("rope_orig_max_pos", ctypes.c_int), ("yarn_beta_fast", ctypes.c_double),
+                ("yarn_beta_slow", ctypes.c_double)]
 
 
 def make_params(B: int, S: int, H: int, D: int, R: int, rope_theta: float, *, m: int = 0,
                 win_len: int = 0, sliding_window: int = 128, n_idx_heads: int = 0,
                 idx_dim: int = 0, topk: int = 0, softmax_scale: Optional[float] = None,
-                pos0: int = 0, dtype: str = "bf16") -> sac_params:
+                pos0: int = 0, dtype: str = "bf16", rope_factor: float = 1.0,
+                rope_orig_max_pos: int = 0, yarn_beta_fast: float = 32.0,
+                yarn_beta_slow: float = 1.0) -> sac_params:
     scale = softmax_scale if softmax_scale is not None else D ** -0.5
     return sac_params(B, S, H, D, R, float(rope_theta), m, win_len, sliding_window, n_idx_heads,
                       idx_dim, topk, float(scale), int(pos0),
-                      SAC_F32 if dtype in ("f32", "float32") else SAC_BF16)
+                      SAC_F32 if dtype in ("f32", "float32") else SAC_BF16, float(rope_factor),
+                      int(rope_orig_max_pos), float(yarn_beta_fast), float(yarn_beta_slow))
 
 
 class sac_kernel_time(ctypes.Structure):

@@ -67,6 +67,13 @@ int check_params(const sac_params* p, int kind, bool decode) {
   REQUIRE(p->R >= 0 && p->R <= p->D && p->R % 2 == 0 && p->R / 2 <= sac::kMaxRopePairs,
           SAC_ERR_UNSUPPORTED, "rope dim must be even, <= head_dim and <= 128 (got %d)", p->R);
   REQUIRE(p->rope_theta > 0 && std::isfinite(p->rope_theta), SAC_ERR_ARG, "rope_theta must be > 0");
+  if (p->rope_factor > 1.0) {
+    REQUIRE(std::isfinite(p->rope_factor) && p->rope_orig_max_pos >= 1, SAC_ERR_ARG,
+            "YaRN needs a finite rope_factor and rope_orig_max_pos >= 1");
+    REQUIRE(std::isfinite(p->yarn_beta_fast) && p->yarn_beta_slow > 0 &&
+                p->yarn_beta_fast > p->yarn_beta_slow,
+            SAC_ERR_ARG, "YaRN needs yarn_beta_fast > yarn_beta_slow > 0");
+  }
   REQUIRE(p->sliding_window >= 1, SAC_ERR_ARG, "sliding_window must be >= 1");
   REQUIRE(p->softmax_scale > 0 && std::isfinite(p->softmax_scale), SAC_ERR_ARG,
           "softmax_scale must be > 0");
@@ -91,11 +98,27 @@ int check_params(const sac_params* p, int kind, bool decode) {
   return SAC_OK;
 }
 
+// Frequencies of the layer's rope pairs, in double precision. With rope_factor s > 1 they follow
+// YaRN's "NTK-by-parts" interpolation (Peng et al. 2023): a pair that turns fewer than
+// yarn_beta_slow times over the original context is slowed by s (position interpolation), one
+// that turns more than yarn_beta_fast times is kept, and the pairs between blend the two linearly
+// in their turn count.
 sac::RopeFreqs rope_freqs(const sac_params* p) {
   sac::RopeFreqs rf;
   std::memset(&rf, 0, sizeof(rf));
   rf.R = p->R;
-  for (int i = 0; i < p->R / 2; ++i) rf.inv_freq[i] = std::pow(p->rope_theta, -2.0 * i / p->R);
+  constexpr double kTwoPi = 6.283185307179586476925;
+  for (int i = 0; i < p->R / 2; ++i) {
+    const double f = std::pow(p->rope_theta, -2.0 * i / p->R);
+    if (!(p->rope_factor > 1.0)) {
+      rf.inv_freq[i] = f;
+      continue;
+    }
+    const double turns = (double)p->rope_orig_max_pos * f / kTwoPi;
+    double keep = (turns - p->yarn_beta_slow) / (p->yarn_beta_fast - p->yarn_beta_slow);
+    keep = keep < 0.0 ? 0.0 : keep > 1.0 ? 1.0 : keep;
+    rf.inv_freq[i] = keep * f + (1.0 - keep) * (f / p->rope_factor);
+  }
   return rf;
 }
 
@@ -193,7 +216,7 @@ extern "C" {
 
 const char* sac_last_error(void) { return g_err; }
 
-int sac_version(void) { return 100; }
+int sac_version(void) { return 200; }
 
 size_t sac_workspace_size(const sac_params* p, int kind) {
   if (kind < SAC_KIND_SWA || kind > SAC_KIND_CSA || check_params(p, kind, false) != SAC_OK)

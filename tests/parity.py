@@ -16,25 +16,33 @@ TOL = {"bf16": (2e-2, 2e-3), "f32": (1e-4, 1e-5)}
 TIE_REL = 1e-3
 
 
-def oracle_params(wl: W.Workload, pos0: int = 0) -> oracle.OracleParams:
-    return oracle.OracleParams(wl.B, wl.S, wl.H, wl.D, wl.R, wl.theta, wl.W, m=wl.m, L=wl.L,
-                               nI=wl.nI, cI=wl.cI, k=wl.k, pos0=pos0,
-                               bf16_pools=wl.dtype == "bf16")
+def oracle_params(wl: W.Workload, pos0: int = 0, yarn=None) -> oracle.OracleParams:
+    """yarn: None, or (factor, original context, beta_fast, beta_slow) of a YaRN-scaled RoPE."""
+    p = oracle.OracleParams(wl.B, wl.S, wl.H, wl.D, wl.R, wl.theta, wl.W, m=wl.m, L=wl.L,
+                            nI=wl.nI, cI=wl.cI, k=wl.k, pos0=pos0, bf16_pools=wl.dtype == "bf16")
+    if yarn is not None:
+        p.yarn_factor, p.yarn_orig, p.yarn_beta_fast, p.yarn_beta_slow = yarn
+    return p
 
 
-def sac_params(wl: W.Workload, pos0: int = 0):
+def sac_params(wl: W.Workload, pos0: int = 0, yarn=None):
+    kw = {}
+    if yarn is not None:
+        kw = dict(rope_factor=yarn[0], rope_orig_max_pos=yarn[1], yarn_beta_fast=yarn[2],
+                  yarn_beta_slow=yarn[3])
     return sac.make_params(wl.B, wl.S, wl.H, wl.D, wl.R, wl.theta, m=wl.m, win_len=wl.L,
                            sliding_window=wl.W, n_idx_heads=wl.nI, idx_dim=wl.cI, topk=wl.k,
-                           pos0=pos0, dtype=wl.dtype)
+                           pos0=pos0, dtype=wl.dtype, **kw)
 
 
 KIND = {"swa": sac.SAC_KIND_SWA, "hca": sac.SAC_KIND_HCA, "csa": sac.SAC_KIND_CSA}
 
 
-def gpu_prefill(wl: W.Workload, x: dict, pos0: int = 0, with_aux: bool = True) -> dict:
+def gpu_prefill(wl: W.Workload, x: dict, pos0: int = 0, with_aux: bool = True,
+                yarn=None) -> dict:
     """Run the layer's forward on cuda:0; returns CPU tensors o (and topk / pools)."""
     dev = torch.device("cuda", 0)
-    p = sac_params(wl, pos0)
+    p = sac_params(wl, pos0, yarn)
     g = {k: v.to(dev).contiguous() for k, v in x.items()}
     o = torch.empty_like(g["q"])
     ws = torch.empty(sac.sac_workspace_size(p, KIND[wl.kind]), dtype=torch.uint8, device=dev)

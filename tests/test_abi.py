@@ -30,15 +30,17 @@ def test_header_declares_the_abi():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert sac.sac_version() == 100
+    assert sac.sac_version() == 200
 
 
 def test_params_struct_layout_matches_header():
     # B,S,H,D,R ints (20) + pad (4) + double (8) + 6 ints (24) + float (4) + pad (4) + int64 (8)
-    # + int (4) + pad (4)
-    assert ctypes.sizeof(sac.sac_params) == 80
+    # + int (4) + pad (4) + double (8) + int (4) + pad (4) + 2 doubles (16)
+    assert ctypes.sizeof(sac.sac_params) == 112
     assert sac.sac_params.rope_theta.offset == 24
     assert sac.sac_params.pos0.offset == 64
+    assert sac.sac_params.rope_factor.offset == 80
+    assert sac.sac_params.yarn_beta_slow.offset == 104
 
 
 def p_csa(**kw):
@@ -80,6 +82,8 @@ def test_workspace_sizes():
     (dict(dtype="f16"), None), (dict(S=0), -1), (dict(H=0), -1), (dict(sliding_window=0), -1),
     (dict(idx_dim=48), -2), (dict(topk=0), -1), (dict(m=0), -1), (dict(S=4 * (1 << 22) + 4), -2),
     (dict(softmax_scale=-1.0), -1), (dict(rope_theta=0.0), -1),
+    (dict(rope_factor=4.0, rope_orig_max_pos=0), -1),
+    (dict(rope_factor=4.0, rope_orig_max_pos=4096, yarn_beta_fast=1.0, yarn_beta_slow=32.0), -1),
 ])
 def test_invalid_params_rejected_on_host(bad, code):
     kw = dict(bad)

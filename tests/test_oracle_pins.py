@@ -636,3 +636,81 @@ def test_oproj_rounded_intermediate_is_bf16():
     mid, _ = oracle.o_proj(o, wa, wb, 2, round_mid=True)
     as_bf16 = torch.from_numpy(mid).float().to(torch.bfloat16).double().numpy()
     assert np.array_equal(mid, as_bf16)
+
+
+# ---- YaRN-scaled RoPE (the config pairs compress_rope_theta with a YaRN rope scaling) ---------
+# Pair i of R rope channels turns r_i = L f_i / (2 pi) times over the original context L. YaRN
+# keeps the pairs with r_i above beta_fast, interpolates those below beta_slow like position
+# interpolation (position / s), and ramps between.
+YARN = dict(theta=160000.0, R=64, factor=4.0, orig=4096, beta_fast=32.0, beta_slow=1.0)
+
+
+def _turns(i, R, theta, orig):
+    return orig * theta ** (-2.0 * i / R) / (2 * math.pi)
+
+
+def _yarn(x, pos, **over):
+    c = dict(YARN, **over)
+    return oracle.rope_yarn(x, c["R"], c["theta"], pos, c["factor"], c["orig"], c["beta_fast"],
+                            c["beta_slow"])
+
+
+def test_yarn_with_factor_one_is_plain_rope():
+    x = rng(80).standard_normal((5, 96))
+    for pos in (0.0, 7.0, 123456.0, -99.0):
+        np.testing.assert_array_equal(_yarn(x, pos, factor=1.0),
+                                      oracle.rope(x, YARN["R"], YARN["theta"], pos))
+
+
+def test_yarn_keeps_fast_pairs_and_interpolates_slow_pairs():
+    R, D = YARN["R"], 96
+    turns = [_turns(i, R, YARN["theta"], YARN["orig"]) for i in range(R // 2)]
+    fast = [i for i, r in enumerate(turns) if r > YARN["beta_fast"]]
+    slow = [i for i, r in enumerate(turns) if r < YARN["beta_slow"]]
+    assert fast and slow  # the configuration exercises both ends of the ramp
+    for i in fast + slow:
+        x = np.zeros(D)
+        x[D - R + 2 * i] = 1.0  # one-hot on pair i: the result is (cos phi, sin phi)
+        for pos in (3.0, 1000.0, 77777.0):
+            got = _yarn(x, pos)
+            # fast pairs rotate like plain RoPE at pos; slow pairs like plain RoPE at pos / s
+            ref_pos = pos if i in fast else pos / YARN["factor"]
+            ref = oracle.rope(x, R, YARN["theta"], ref_pos)
+            np.testing.assert_allclose(got, ref, atol=1e-9, err_msg=f"pair {i} pos {pos}")
+
+
+def test_yarn_ramp_midpoint_is_the_mean_of_both_frequencies():
+    # choose the original length so that pair 5 completes exactly (alpha + beta) / 2 turns:
+    # its frequency is then halfway between f (kept) and f / s (interpolated)
+    R, theta, i = 64, 10000.0, 5
+    f = theta ** (-2.0 * i / R)
+    mid = (YARN["beta_fast"] + YARN["beta_slow"]) / 2
+    L_real = mid * 2 * math.pi / f
+    L = int(round(L_real))
+    r = L * f / (2 * math.pi)
+    gamma = (r - YARN["beta_slow"]) / (YARN["beta_fast"] - YARN["beta_slow"])
+    assert abs(gamma - 0.5) < 0.01
+    got = oracle.rope_freq(i, R, theta, 4.0, L, YARN["beta_fast"], YARN["beta_slow"])
+    np.testing.assert_allclose(got, (1 - gamma) * f / 4.0 + gamma * f, rtol=1e-14)
+    assert f / 4.0 < got < f
+
+
+def test_yarn_rotation_preserves_norm_and_inverts():
+    x = rng(81).standard_normal((4, 96))
+    y = _yarn(x, 4321.0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(_yarn(y, -4321.0), x, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["hca", "csa"])
+def test_yarn_layers_stay_shift_invariant(kind):
+    base = _tiny(kind, pos0=0)
+    d = _inputs(base, 82)
+    outs = []
+    for pos0 in (0, 50000):
+        p = _tiny(kind, pos0=pos0)
+        p.yarn_factor, p.yarn_orig = 4.0, 64
+        outs.append(_run(kind, p, d))
+    np.testing.assert_allclose(outs[1], outs[0], atol=1e-11)
+    plain = _run(kind, base, d)
+    assert np.abs(outs[0] - plain).max() > 1e-6  # the scaling does change the output
