@@ -518,6 +518,55 @@ def run_ours(args, wl0):
 
 
 # ------------------------------------------------------------------------------------------------
+# query-sharded prefill: one sequence over N ranks (halo send / recv, pool all-gather)
+# ------------------------------------------------------------------------------------------------
+def run_sharded(args, wl):
+    """One step = sharded_forward on every rank: the halo exchange, the local cache append, the
+    NCCL all-gather of the pools and the rank's chunk of queries. Strong scaling: the sequence is
+    fixed, each rank takes S/N of its queries."""
+    import sparse_attention_compressor_b200 as sac
+    from sparse_attention_compressor_b200 import sharded
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    kind = sac.SAC_KIND_CSA if wl.kind == "csa" else sac.SAC_KIND_HCA
+    sp = sharded.plan(wl.S, world, rank, wl.m, wl.L, wl.W, page_size=64)
+    x = {k: v.to(dev) for k, v in W.prefill_slice_inputs(wl, sp.s0, sp.s1).items()}
+    p = sac.make_params(1, wl.S, wl.H, wl.D, wl.R, wl.theta, m=wl.m, win_len=wl.L,
+                        sliding_window=wl.W, n_idx_heads=wl.nI, idx_dim=wl.cI, topk=wl.k,
+                        dtype=wl.dtype)
+    o = torch.empty_like(x["q"])
+    ws = torch.empty(sac.sac_chunk_workspace_size(p, kind, 1, sp.n), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        sharded.sharded_forward(sp, kind, p, x, o, ws=ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        clk.wait_samples(1, step)
+        ms = timed(step, args.steps, dev)
+        clk.wait_samples(len(clk.lines) + 1, step)
+    ms = max_over_ranks(ms, dev) / args.steps
+    line = {
+        "metric": f"{wl.kind.upper()} attention fwd tokens/s (prefill)",
+        "value": wl.S / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": wl.dtype, "data": DATA,
+        "config": dict(config_of(wl, world), parallelism=f"seq{world}",
+                       launch="eager launches per step (halo send / recv and pool all-gather on "
+                              "NCCL, then the chunk kernels)"),
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------------------------
 # decode: one step = the CSA layer and the HCA layer, each over its paged cache
 # ------------------------------------------------------------------------------------------------
 def decode_bytes(wl, d_csa, d_hca) -> dict:
@@ -1007,6 +1056,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="csa_128k_bf16", choices=list(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", choices=["dp", "seq"], default="dp",
+                    help="dp: every rank its own sequence (weak scaling); seq: one sequence "
+                         "split by queries over the ranks (CSA / HCA prefill, strong scaling)")
     args = ap.parse_args(argv)
     wl = W.WORKLOADS[args.workload]
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
@@ -1018,6 +1070,8 @@ def main(argv=None):
         run_decode(args, wl)
     elif wl.kind == "oproj":
         run_oproj(args, wl)
+    elif args.shard == "seq" and wl.kind in ("csa", "hca"):
+        run_sharded(args, wl)
     else:
         run_ours(args, wl)
 

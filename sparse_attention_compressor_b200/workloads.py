@@ -216,6 +216,19 @@ def prefill_inputs(wl: Workload, with_queries: bool = True) -> Dict[str, torch.T
     return out
 
 
+def prefill_slice_inputs(wl: Workload, s0: int, s1: int) -> Dict[str, torch.Tensor]:
+    """The inputs of tokens [s0, s1) of sequence 0 (the same bytes prefill_inputs draws for those
+    rows), plus the weights: q [n,H,D], kv [n,D]; CSA: k_idx [n,cI], q_idx [n,nI,cI], w_idx
+    [n,nI]. One rank's share of a query-sharded prefill."""
+    rows = np.arange(s0, s1, dtype=np.int64)
+    out = dict(prefill_weights(wl))
+    out["kv"] = _rows_tensor(wl, "kv", (wl.D,), 1.0, rows).to(wl.torch_dtype)
+    out.update(prefill_row_inputs(wl, rows))
+    if wl.kind == "csa":
+        out["k_idx"] = _rows_tensor(wl, "k_idx", (wl.cI,), 1.0, rows).to(wl.torch_dtype)
+    return out
+
+
 # ------------------------------------------------------------------------------------------------
 # Decode: nseq sequences, one new token each, paged caches of page_size rows with physical pages
 # shuffled through a pool. kv pages hold rotated kv, pool pages rotated entries, indexer pool pages
