@@ -857,7 +857,7 @@ def run_oproj(args, wl0):
         "config": {"workload": wl.name, "tokens": T, "H": wl.H, "head_dim": wl.D,
                    "o_groups": G, "o_lora_rank": rk, "hidden": hid, "parallelism": f"dp{world}",
                    "l2": "flushed before every step (252 MiB written, then another 252 MiB read)",
-                   "launch": "one CUDA graph replay per step (two cuBLASLt GEMMs)"},
+                   "launch": "one CUDA graph replay per step (two tcgen05 GEMM launches)"},
         "clocks": clk.summary(),
         "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": pin_o.numel() * 2, "d2h_bytes_per_step": out.numel() * 2},

@@ -327,9 +327,12 @@ SAC_API int prefill_chunk_append(const sac_params* p, int kind, int nseq, int n,
  *   o   [T, H*D], w_a [groups, rank, (H/groups)*D], w_b [hidden, groups*rank], out [T, hidden]:
  *   bf16 (p->dtype must be SAC_BF16), row-major; weights in the nn.Linear [out, in] layout.
  * The intermediate mid is stored in bf16 (the layer's activation precision); both products
- * accumulate in fp32. The two GEMMs run on cuBLASLt (a plain dense contraction: the library GEMM).
- * ws: sac_oproj_workspace_size() bytes (mid plus the GEMM library's scratch), 256-byte aligned.
- * Returns SAC_ERR_UNSUPPORTED for fp32, groups not dividing H, or rank / hidden not multiples of 8.
+ * accumulate in fp32. Both products run on the library's tcgen05 GEMM kernel (256 x 256 output
+ * tiles, operands streamed by TMA, fp32 accumulators in tensor memory).
+ * ws: sac_oproj_workspace_size() bytes (the 256-byte status word of sac_device_status, then mid),
+ * 256-byte aligned.
+ * Returns SAC_ERR_UNSUPPORTED for fp32, groups not dividing H, rank / hidden not multiples of 8, or
+ * a group width (H/groups)*D that is not a multiple of 64.
  */
 SAC_API size_t sac_oproj_workspace_size(const sac_params* p, int64_t T, int groups, int rank);
 SAC_API int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank, int hidden,

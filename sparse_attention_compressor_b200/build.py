@@ -2,7 +2,7 @@
 
 Each ``csrc/*.cu`` compiles with nvcc (``-gencode arch=compute_100a,code=sm_100a``) to an object in
 ``_build/``; the objects link into ``sparse_attention_compressor_b200/libsac.so`` with a static
-CUDA runtime and the toolkit's cuBLASLt (the output projection's plain GEMMs). Rebuilds only what changed (sources or any header under csrc/ and include/).
+CUDA runtime. Rebuilds only what changed (sources or any header under csrc/ and include/).
 """
 from __future__ import annotations
 
@@ -70,7 +70,7 @@ def build(verbose: bool = False, extra_flags=()) -> str:
                 raise RuntimeError(f"nvcc failed on {cmd[-3]}")
     if _stale(LIB, objs):
         tmp = LIB + f".tmp{os.getpid()}"
-        cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static", "-lcublasLt"]
+        cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n" + r.stdout + r.stderr)

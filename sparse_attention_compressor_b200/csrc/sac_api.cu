@@ -945,7 +945,7 @@ int prefill_chunk_append(const sac_params* p, int kind, int nseq, int n, const i
 
 size_t sac_oproj_workspace_size(const sac_params* p, int64_t T, int groups, int rank) {
   if (p == nullptr || T < 0 || groups < 1 || rank < 1) return 0;
-  return align_up((size_t)T * groups * rank * 2) + align_up(sac::oproj_gemm_scratch_bytes());
+  return kStatusBytes + align_up((size_t)T * groups * rank * 2);
 }
 
 int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank, int hidden,
@@ -959,6 +959,8 @@ int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank, int hid
           "o_groups (%d) must divide the head count (%d)", groups, p->H);
   REQUIRE(rank >= 8 && rank % 8 == 0 && hidden >= 8 && hidden % 8 == 0, SAC_ERR_UNSUPPORTED,
           "o_lora_rank and hidden must be positive multiples of 8");
+  REQUIRE((p->H / groups) * p->D % 64 == 0, SAC_ERR_UNSUPPORTED,
+          "a group's features ((H/o_groups)*head_dim) must be a multiple of 64");
   REQUIRE_PTR(o);
   REQUIRE_PTR(w_a);
   REQUIRE_PTR(w_b);
@@ -968,7 +970,12 @@ int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank, int hid
           "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
   REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255) == 0, SAC_ERR_ARG,
           "ws must be 256-byte aligned");
+  if (T == 0) return SAC_OK;  // nothing to do: no device work
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carve cv(ws);
+  int* status = static_cast<int*>(cv.take(kStatusBytes));
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
   sac::OProjArgs a;
   a.T = T;
   a.H = p->H;
@@ -981,10 +988,8 @@ int o_proj_forward(const sac_params* p, int64_t T, int groups, int rank, int hid
   a.w_b = w_b;
   a.out = out;
   a.mid = cv.take((size_t)T * groups * rank * 2);
-  a.scratch_bytes = sac::oproj_gemm_scratch_bytes();
-  a.scratch = cv.take(a.scratch_bytes);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = sac::timed("o_proj", st, [&] { return sac::launch_oproj(a, st); });
+  a.status = status;
+  e = sac::timed("o_proj", st, [&] { return sac::launch_oproj(a, st); });
   if (e != cudaSuccess) return cuda_fail(e, "output projection");
   return SAC_OK;
 }

@@ -60,7 +60,7 @@ cudaError_t launch_decode_append_pair(int dtype, const DecodeAppendArgs& a, cuda
 cudaError_t launch_chunk_append(int dtype, const DecodeAppendArgs& a, int n, bool index_part,
                                 cudaStream_t st);
 
-// ---- grouped output projection (oproj.cu, cuBLASLt GEMMs) ---------------------------------
+// ---- grouped output projection (oproj.cu, tcgen05 GEMM) ----------------------------------
 struct OProjArgs {
   int64_t T;             // tokens
   int H, D, groups, rank, hidden;
@@ -69,10 +69,8 @@ struct OProjArgs {
   const void* w_b;       // [hidden, groups*rank] bf16 (o_b_proj)
   void* mid;             // [T, groups*rank] bf16 intermediate
   void* out;             // [T, hidden] bf16
-  void* scratch;         // GEMM library workspace
-  size_t scratch_bytes;
+  int* status;           // device status word
 };
-size_t oproj_gemm_scratch_bytes();
 cudaError_t launch_oproj(const OProjArgs& a, cudaStream_t st);
 
 // ---- indexer (indexer.cu) -----------------------------------------------------------------

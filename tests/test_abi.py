@@ -177,8 +177,8 @@ def test_oproj_validation_and_workspace():
     fake = 1 << 20
     p = sac.make_params(1, 64, 64, 512, 64, 1e4)
     need = sac.sac_oproj_workspace_size(p, 64, 8, 1024)
-    # bf16 mid [64, 8*1024] plus the GEMM scratch, each 256-byte aligned
-    assert need == 64 * 8 * 1024 * 2 + (32 << 20)
+    # the status word, then the bf16 mid [64, 8*1024], each 256-byte aligned
+    assert need == 256 + 64 * 8 * 1024 * 2
     assert sac.sac_oproj_workspace_size(p, -1, 8, 1024) == 0
 
     def call(T=64, groups=8, rank=1024, hidden=4096, ws=fake, ws_bytes=need, params=p):
@@ -192,6 +192,8 @@ def test_oproj_validation_and_workspace():
     assert call(ws=fake + 16) == -1 and "256-byte" in lib.sac_last_error().decode()
     p32 = sac.make_params(1, 64, 64, 512, 64, 1e4, dtype="f32")
     assert call(params=p32) == -2
+    p_odd = sac.make_params(1, 64, 6, 40, 0, 1e4)  # groups of 3 heads x 40 = 120 features
+    assert call(params=p_odd, groups=2, rank=64, hidden=64) == -2
     assert call(T=0) == 0  # nothing to do: no launch, no device touched
 
 

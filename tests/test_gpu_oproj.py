@@ -1,6 +1,8 @@
-"""GPU parity of the grouped low-rank output projection (o_proj_forward) against the fp64
-oracle, whose intermediate is rounded to bf16 as the kernel stores it: a small case with several
-groups and a ragged row count, and the page's configuration (64 heads of 512, 8 groups of rank
+"""GPU parity of the grouped low-rank output projection (o_proj_forward, the tcgen05 GEMM) against
+the fp64 oracle, whose intermediate is rounded to bf16 as the kernel stores it: small cases with
+several groups, row counts that are not a multiple of the 256-row tile, output widths that are not
+a multiple of the 256-column tile and an o_b_proj contraction (G*rank = 120) that is not a
+multiple of the 64-wide K step; and the page's configuration (64 heads of 512, 8 groups of rank
 1024, hidden 4096) checked on all rows of a short run and on sampled rows of a long one."""
 import numpy as np
 import pytest
@@ -31,7 +33,9 @@ def f64(t):
 
 
 @pytest.mark.parametrize("T,H,D,G,rank,hidden", [(77, 8, 64, 4, 32, 96), (5, 4, 64, 1, 64, 64),
-                                                 (200, 16, 128, 2, 256, 512)])
+                                                 (200, 16, 128, 2, 256, 512),
+                                                 (300, 6, 64, 3, 40, 72),
+                                                 (513, 8, 128, 4, 264, 520)])
 def test_oproj_small(T, H, D, G, rank, hidden):
     x, out = run(T, H, D, G, rank, hidden, 41)
     _, want = oracle.o_proj(f64(x["o"]), f64(x["w_a"]), f64(x["w_b"]), G, round_mid=True)
