@@ -2,35 +2,37 @@
 // 64 query heads and head_dim 512 ("Hybrid attention": shared K=V MQA; per-head sink, eq. 27;
 // partial RoPE with the -i output rotation, eq. 26; sliding-window branch + compressor entries).
 //
-// One query row at a time per CTA (persistent over rows). Its 64 heads are the M = 64 rows of
-// both contractions:  S = Q K^T  (M=64, N=48 keys, K=512)  and  O += P V  (M=64, N=256 x 2, K=48).
-// Because K = V, one shared-memory key tile serves as the K-major B operand of QK^T and as the
-// MN-major B operand of PV. Tiles of 48 keys keep three tile buffers resident next to the 64 KB
-// query tile. Window rows and HCA entries are consecutive rows and load as 8 TMA boxes per tile;
-// CSA selections (and paged rows) are gathered with 16-byte cp.async copies by two producer
-// groups that take alternate tiles. Tiles never mix window rows and entries.
+// One query row at a time per CTA (persistent over rows). Both contractions put the 128 keys of a
+// tile, or the 128 channels of a dimension block, on the MMA's M = 128 side and the 64 heads on
+// N = 64, so every MMA runs at the full tcgen05 rate (an M = 64 MMA of the heads would run at
+// half of it):
+//   S^T[key, head]  = K[128 keys x 512] . Q^T                  (M = 128, N = 64, K = 512)
+//   O^T[dim, head] += V^T[128 dims x 128 keys] . P^T[keys, heads]  per block of 128 dims
+//                                                              (M = 128, N = 64, K = 128)
+// Because K = V, one key tile in shared memory is the K-major A operand of the first product and
+// the MN-major A operand of the second. It is held as four 32 KB dimension blocks ("pairs": two
+// 128-byte swizzle columns of 64 channels); the next tile refills a pair as soon as the PV MMAs of
+// its block have completed, so the loads of tile g+1 overlap the end of tile g.
 //
-// QK^T of a tile is 32 MMAs of K=16. Accumulating them into one TMEM tile would chain each MMA
-// on its predecessor, so they rotate over four partial accumulators (one per issuing thread) and
-// the softmax adds the four partials.
+// MMA issue: one thread issuing a chain of MMAs into the same accumulator keeps them pipelined,
+// while switching accumulators between consecutive MMAs of one thread drains the pipe (measured:
+// ~55 vs ~220 cycles per M = 128, N = 64 MMA). So four issuer threads each own one chain: issuer
+// i computes S^T over dimension block i (8 K-steps, partial accumulator S_i) and then O^T block i
+// (8 K-steps of 16 keys); the softmax adds the four partials of S^T.
 //
-// The query tile arrives un-rotated; one warp turns its rope slice in shared memory before the
-// first QK^T of the row, so no rotated copy of q is written to HBM.
+// Tensor memory (512 columns, fp32): O^T block i at columns 64i (128 lanes = 128 channels), S_i at
+// 256 + 64i.
 //
-// Tensor memory (512 columns, fp32): O[:, 0:256] in lanes 0-15 of each sub-partition and
-// O[:, 256:512] in lanes 16-31 (the M = 64 layout leaves half the lanes free); for each of the two
-// S buffers, partials 0/2 in lanes 0-15 and partials 1/3 in lanes 16-31 of 96 columns at 256
-// (buffer 0) and 352 (buffer 1). A softmax thread of lane i < 16 and its partner i + 16 own the
-// same head: they add their partials, exchange halves, and each finishes 24 of the 48 keys.
+// Softmax: thread = key (TMEM lane); per-head running max in shared memory, moved only when a
+// tile's logit exceeds it by more than 2^8 (log2 units), which a block-wide vote detects; then the
+// exact per-head tile max is taken with warp shuffles and O^T is rescaled in TMEM. The
+// normaliser's per-head sums over keys are reduce-scattered across each warp with shuffles (a lane
+// keeps two heads) and summed over the four warps at the end of the row.
 //
-// Warps: 0 = TMA thread, 1-2 = QK^T issuers (warp 1 also owns TMEM), 3 = query rotation, 4-7 and
-// 13-16 = two gather groups of 128 threads taking the gathered tiles in turn (idle when every
-// tile arrives by TMA), 8-11 = softmax + output, 12 = PV issuer. Each tcgen05.mma costs its issuing thread a fixed time, so two threads
-// issue QK^T and a third issues PV the moment P is written, instead of after the next tile's
-// QK^T. An M = 64 MMA occupies one 16-lane half of each TMEM sub-partition, and MMAs into
-// opposite halves run side by side: the QK^T partials alternate between the lane halves, and the
-// two halves of O sit in opposite lane halves. The softmax keeps the running max in log2 units and moves it
-// (rescaling O) only when a tile's max exceeds it by more than 8.
+// Warps: 0 = TMA producer (query, contiguous key tiles), 1-4 = MMA issuers (warp 1 owns TMEM),
+// 5 = query rotation, 8-11 = softmax and output, 12-15 = gather group for tiles whose rows are
+// not consecutive (CSA selections, paged caches). Layers whose every tile arrives by TMA launch
+// without the gather warps.
 #include <cuda_bf16.h>
 
 #include "launch_util.h"
@@ -43,38 +45,42 @@ namespace {
 
 constexpr int kHeads = 64;
 constexpr int kDim = 512;
-constexpr int kNK = 48;                          // keys per tile
-constexpr int kHalfNK = kNK / 2;
-constexpr int kStages = 3;                       // key tiles in flight
-constexpr int kQRegion = 64 * 128;               // [64 rows x 128 B]: one swizzle column of Q
-constexpr int kKRegion = kNK * 128;              // [48 rows x 128 B]
+constexpr int kNK = 128;                         // keys per tile (MMA M of S^T)
+constexpr int kPairs = kDim / 128;               // dimension blocks of a key tile
+constexpr int kRegion = kNK * 128;               // 16 KB: 128 keys x 64 channels, 128-B rows
+constexpr int kPairBytes = 2 * kRegion;          // 32 KB: one dimension block
+constexpr int kQRegion = kHeads * 128;           // 8 KB: 64 heads x 64 channels
 constexpr int kQBytes = 8 * kQRegion;            // 64 KB
-constexpr int kTileBytes = 8 * kKRegion;         // 48 KB
-constexpr int kPBytes = kHeads * 128;            // 64 rows x 128 B (48 keys used)
-constexpr int kGatherGroups = 2;                 // producer groups taking tiles in turn
-constexpr int kGroupThreads = 128;               // threads of one gather group (warps 4-7, 13-16)
-constexpr int kThreads = 544;                    // with the gather groups
-constexpr int kThreadsTma = 416;                 // every tile by TMA: warps 13-16 not launched
+constexpr int kPBytes = kNK * 128;               // 16 KB: P^T, 128 keys x 64 heads
+constexpr int kGroupThreads = 128;               // the gather group
+constexpr int kThreads = 512;                    // with the gather group
+constexpr int kThreadsTma = 384;                 // every tile by TMA: warps 12-15 not launched
+constexpr int kIssuers = kPairs;                 // MMA issuer threads, one per dimension block
+constexpr int kSoftmaxWarp0 = 8;                 // warps 8-11: softmax and output
 
 constexpr int kOffQ = 0;
-constexpr int kOffTile = kOffQ + kQBytes;
-constexpr int kOffP = kOffTile + kStages * kTileBytes;
-constexpr int kOffCs = kOffP + 2 * kPBytes;      // [32] (cos, sin) of the query's rope pairs
+constexpr int kOffPair = kOffQ + kQBytes;
+constexpr int kOffP = kOffPair + kPairs * kPairBytes;
+constexpr int kOffM = kOffP + kPBytes;           // [64] running max per head (log2 units)
+constexpr int kOffAlpha = kOffM + 256;           // [64] rescale factors of a moved max
+constexpr int kOffL = kOffAlpha + 256;           // [64] normaliser of the output
+constexpr int kOffWmax = kOffL + 256;            // [4][64] per-warp tile maxima / normalisers
+constexpr int kOffCs = kOffWmax + 1024;          // [32] (cos, sin) of the query's rope pairs
 constexpr int kOffBar = kOffCs + 32 * 8;
-enum Bar { kQFull, kQReady, kQEmpty, kKvFull0, kKvEmpty0 = kKvFull0 + kStages,
-           kSFull0 = kKvEmpty0 + kStages, kPFull0 = kSFull0 + 2, kPvDone0 = kPFull0 + 2,
-           kOFull = kPvDone0 + 2, kOEmpty, kNumBars };
+enum Bar { kQFull, kQReady, kQEmpty, kPairFull0, kPairEmpty0 = kPairFull0 + kPairs,
+           kSFull = kPairEmpty0 + kPairs, kSEmpty, kPFull, kPEmpty, kOFull, kOEmpty, kNumBars };
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemPtr + 16;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-constexpr uint32_t kColS = 256, kSStride = 2 * kNK;  // S buffer s at kColS + s * kSStride
-constexpr uint32_t kIdescQK = tc::idesc_bf16(64, kNK, false, false);
-constexpr uint32_t kIdescPV = tc::idesc_bf16(64, 256, false, true);
+constexpr uint32_t kColO = 0, kColS = 256;       // O^T block i at 64 i, S_i at 256 + 64 i
+constexpr uint32_t kIdescQK = tc::idesc_bf16(128, kHeads, false, false);
+constexpr uint32_t kIdescPV = tc::idesc_bf16(128, kHeads, true, true);
 constexpr int kMaxSplits = 8;  // key-tile splits of one row (decode: few rows, many SMs)
-constexpr int kQkIssuers = 2;  // threads issuing QK^T (measured faster than 4 and than 1)
 constexpr int kRopeStep = 28;  // K-steps 28..31 read the last region of Q (the rope slice)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;  // move the running max only when a tile exceeds it by 2^8
+constexpr int kSoftmaxBar = 1; // named barrier of the 128 softmax threads
 
 struct Row {
   int seq;
@@ -118,6 +124,11 @@ __device__ __forceinline__ Row locate_item(const AttnArgs& a, int64_t it) {
   return w;
 }
 
+// keys of tile j of a row
+__device__ __forceinline__ int tile_keys(const Row& w, int j) {
+  return j < w.twin ? min(kNK, w.nwin - j * kNK) : min(kNK, w.npool - (j - w.twin) * kNK);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
   __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -127,32 +138,32 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return __bfloat1622float2(v);
 }
 
-// QK^T K-steps kk = ME (mod NQK) of one tile (fully unrolled, every offset a constant: the issue
-// cost per MMA is what bounds this loop). K-step kk accumulates into partial p = kk & 3 at lanes
-// 16 (p & 1), columns + 48 (p >> 1) of the S buffer at d0. With qready set (a query's first tile)
-// the K-steps of the rope region wait until the query's rope slice has been rotated.
-template <int NQK, int ME>
-__device__ __forceinline__ bool issue_qk(uint32_t d0, uint64_t qd, uint64_t kd, uint64_t* qready,
-                                         uint32_t qparity, int* status) {
-#pragma unroll
-  for (int i = 0; i < kDim / 16 / NQK; ++i) {
-    const int kk = NQK * i + ME;
-    if (kk >= kRopeStep && kk - NQK < kRopeStep && qready != nullptr) {
-      if (!tc::mbar_wait(qready, qparity, status)) return false;
-      tc::tc_fence_after();
-    }
-    const int p = kk & 3;
-    const uint32_t dp = d0 + ((p & 1) ? (16u << 16) : 0u) + ((p & 2) ? (uint32_t)kNK : 0u);
-    const uint32_t qo = ((kk >> 2) * kQRegion + (kk & 3) * 32) >> 4;
-    const uint32_t ko = ((kk >> 2) * kKRegion + (kk & 3) * 32) >> 4;
-    tc::mma_bf16_ss(dp, qd + qo, kd + ko, kIdescQK, kk >= 4 ? 1u : 0u);
-  }
-  return true;
+__device__ __forceinline__ void bar_sync_softmax() {
+  asm volatile("barrier.sync %0, %1;" ::"r"(kSoftmaxBar), "r"(128) : "memory");
+}
+// true on every softmax thread when v is true on any of them
+__device__ __forceinline__ bool bar_any_softmax(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(kSoftmaxBar), "r"(128)
+      : "memory");
+  return r != 0;
+}
+
+// Wait on an mbarrier phase from the 128 softmax threads. The group meets at named barriers, so
+// whether the wait timed out is decided for the whole group: if any thread gave up, all do.
+__device__ __forceinline__ bool softmax_wait(uint64_t* bar, uint32_t parity, int* status) {
+  return !bar_any_softmax(!tc::mbar_wait(bar, parity, status));
 }
 
 // Global address of key c of tile j (keys past the tile's count reuse a valid row: masked).
-__device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const Row& w,
-                                                        int64_t r, int j, int c) {
+__device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const Row& w, int j,
+                                                        int c) {
   if (j < w.twin) {
     int x = j * kNK + c;
     if (x >= w.nwin) x = 0;
@@ -161,13 +172,11 @@ __device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const
   }
   int i = (j - w.twin) * kNK + c;
   if (i >= w.npool) i = 0;
-  int64_t e = a.pool_mode == 2 ? (int64_t)__ldg(a.sel + r * a.k + i) : i;
+  int64_t e = a.pool_mode == 2 ? (int64_t)__ldg(a.sel + w.r * a.k + i) : i;
   const __nv_bfloat16* p = a.pool.row<__nv_bfloat16>(w.seq, e < 0 ? 0 : e);
   return p ? p : reinterpret_cast<const __nv_bfloat16*>(a.pool.base);
 }
 
-// kNThreads: kThreads when some tile is gathered, else kThreadsTma (the smaller block keeps the
-// register budget of the TMA-only layers at 152 per thread instead of 120).
 template <bool kSplit, int kNThreads>
 __global__ void __launch_bounds__(kNThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -183,7 +192,6 @@ __global__ void __launch_bounds__(kNThreads, 1)
     if (threadIdx.x == 0 && status) atomicExch(status, tc::kStatusMisaligned);
     return;
   }
-
   // window rows of a prefill are consecutive rows of the rotated kv stream, and so are the
   // entries of an HCA prefill: those tiles load as TMA boxes; the rest are gathered
   const bool win_contig = a.win.block_table == nullptr;
@@ -194,28 +202,21 @@ __global__ void __launch_bounds__(kNThreads, 1)
     return;
   }
   const int64_t n_items = kSplit ? a.nrows * a.splits : a.nrows;
-  // Who issues PV: with gathered tiles the gather latency decides, and a separate thread issues
-  // PV the moment P is ready so that tile buffers free early; with TMA-fed tiles QK^T is the
-  // critical step, and the QK^T threads issue PV right after the next tile's QK^T (measured: 17%
-  // faster at HCA-32k, slower at CSA-8k).
-  const bool pv_by_qk = !any_gather;
-  const uint32_t pv_commits = pv_by_qk ? kQkIssuers : 1;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bar[kQFull], 1);
     tc::mbar_init(&bar[kQReady], 32);
-    tc::mbar_init(&bar[kQEmpty], kQkIssuers);
-    for (int i = 0; i < kStages; ++i) {
-      // TMA thread (+ one gather group when some tiles are gathered)
-      tc::mbar_init(&bar[kKvFull0 + i], any_gather ? 1 + kGroupThreads : 1);
-      tc::mbar_init(&bar[kKvEmpty0 + i], pv_commits);
+    tc::mbar_init(&bar[kQEmpty], kIssuers);
+    for (int b = 0; b < kPairs; ++b) {
+      // TMA thread (+ the gather group when some tiles are gathered)
+      tc::mbar_init(&bar[kPairFull0 + b], any_gather ? 1 + kGroupThreads : 1);
+      tc::mbar_init(&bar[kPairEmpty0 + b], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bar[kSFull0 + i], kQkIssuers);
-      tc::mbar_init(&bar[kPFull0 + i], 128);
-      tc::mbar_init(&bar[kPvDone0 + i], pv_commits);
-    }
-    tc::mbar_init(&bar[kOFull], pv_commits);
+    tc::mbar_init(&bar[kSFull], kIssuers);
+    tc::mbar_init(&bar[kSEmpty], 128);
+    tc::mbar_init(&bar[kPFull], 128);
+    tc::mbar_init(&bar[kPEmpty], kIssuers);
+    tc::mbar_init(&bar[kOFull], kIssuers);
     tc::mbar_init(&bar[kOEmpty], 128);
     tc::fence_barrier_init();
   }
@@ -231,7 +232,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
   const uint32_t tmem = *tmem_ptr;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA thread
+    // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t g = 0, qi = 0;
       bool ok = true;
@@ -239,102 +240,97 @@ __global__ void __launch_bounds__(kNThreads, 1)
         const Row w = locate_item<kSplit>(a, it);
         if (w.bad && status) atomicExch(status, tc::kStatusBadInput);
         if (w.j0 == w.j1) continue;
-        const int64_t r = w.r;
         if (qi > 0) ok = tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status);
         if (!ok) break;
         tc::mbar_arrive_expect_tx(&bar[kQFull], kQBytes);
         for (int c = 0; c < 8; ++c)
           tc::tma_load_2d(smem + kOffQ + c * kQRegion, &tm_q, &bar[kQFull], 64 * c,
-                          (int32_t)(r * kHeads));
+                          (int32_t)(w.r * kHeads));
         for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
-          const uint32_t b = g % kStages;
-          if (g >= kStages) ok = tc::mbar_wait(&bar[kKvEmpty0 + b], ((g - kStages) / kStages) & 1,
-                                               status);
-          if (!ok) break;
           const bool is_win = j < w.twin;
-          if (is_win ? win_contig : pool_contig) {
-            tc::mbar_arrive_expect_tx(&bar[kKvFull0 + b], kTileBytes);
-            const int64_t y0 = is_win ? a.win.row_index(w.seq, w.lo + (int64_t)j * kNK)
-                                      : a.pool.row_index(w.seq, (int64_t)(j - w.twin) * kNK);
-            const CUtensorMap* map = is_win ? &tm_win_box : &tm_pool_box;
-            uint8_t* tile = smem + kOffTile + b * kTileBytes;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              tc::tma_load_2d(tile + c * kKRegion, map, &bar[kKvFull0 + b], 64 * c, (int32_t)y0);
-          } else {
-            tc::mbar_arrive(&bar[kKvFull0 + b]);
+          const bool contig = is_win ? win_contig : pool_contig;
+          const int64_t y0 = contig ? (is_win ? a.win.row_index(w.seq, w.lo + (int64_t)j * kNK)
+                                              : a.pool.row_index(w.seq, (int64_t)(j - w.twin) * kNK))
+                                    : 0;
+          const CUtensorMap* map = is_win ? &tm_win_box : &tm_pool_box;
+          for (int b = 0; b < kPairs && ok; ++b) {
+            if (g > 0) ok = tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status);
+            if (!ok) break;
+            if (contig) {
+              uint8_t* dst = smem + kOffPair + b * kPairBytes;
+              tc::mbar_arrive_expect_tx(&bar[kPairFull0 + b], kPairBytes);
+              tc::tma_load_2d(dst, map, &bar[kPairFull0 + b], 128 * b, (int32_t)y0);
+              tc::tma_load_2d(dst + kRegion, map, &bar[kPairFull0 + b], 128 * b + 64, (int32_t)y0);
+            } else {
+              tc::mbar_arrive(&bar[kPairFull0 + b]);
+            }
           }
         }
         ++qi;
       }
     }
     __syncwarp();
-  } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------------------------------ QK^T issuers
-    // issuer me takes the K-steps kk = me (mod 2); K-step kk accumulates into partial p = kk & 3,
-    // which sits in lanes 16 (p & 1), columns + 48 (p >> 1) of the S buffer
-    const uint32_t me = warp - 1;
+  } else if (warp >= 1 && warp <= kIssuers) {
+    // ------------------------------------------------------------------ MMA issuers
+    // Issuer i: S_i = K[:, block i] Q[:, block i]^T (8 K-steps), then O^T block i += V^T P^T
+    // (8 steps of 16 keys); each chain stays on one accumulator.
+    const int bi = warp - 1;
     if (lane == 0) {
-      uint32_t g0 = 0, qi = 0;
+      uint32_t g = 0, qi = 0;
       bool ok = true;
-      const uint64_t qd = tc::desc_sw128(tc::smem_u32(smem + kOffQ), 0, 1024);
+      const uint32_t q_base = tc::smem_u32(smem + kOffQ) + bi * 2 * kQRegion;
+      const uint32_t pair = tc::smem_u32(smem + kOffPair) + bi * kPairBytes;
+      const uint64_t p_desc = tc::desc_sw128(tc::smem_u32(smem + kOffP), 0, 1024);
+      const uint32_t s_acc = tmem + kColS + 64 * bi, o_acc = tmem + kColO + 64 * bi;
       for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const Row w = locate_item<kSplit>(a, it);
         if (w.j0 == w.j1) continue;
-        // the query tile has landed; its rope region (the last 128-byte column, K-steps 28..31)
-        // is still being rotated, so the first QK^T waits for kQReady only before those steps
         ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
-        for (int j = w.j0; j < w.j1 + (pv_by_qk ? 1 : 0) && ok; ++j) {
-          if (j < w.j1) {  // S(g) = Q K^T over four partial accumulators
-            const uint32_t g = g0 + (j - w.j0), b = g % kStages, s = g & 1;
-            ok = tc::mbar_wait(&bar[kKvFull0 + b], (g / kStages) & 1, status);
-            if (ok && g >= 2) ok = tc::mbar_wait(&bar[kPFull0 + s], ((g - 2) >> 1) & 1, status);
-            if (!ok) break;
-            tc::tc_fence_after();
-            const uint64_t kd =
-                tc::desc_sw128(tc::smem_u32(smem + kOffTile + b * kTileBytes), 0, 1024);
-            const uint32_t d0 = tmem + kColS + s * kSStride;
-            // the descriptor's start-address field counts 16-byte units: advancing along K adds
-            // the byte offset >> 4 to the base descriptor
-            uint64_t* qready = j == w.j0 ? &bar[kQReady] : nullptr;
-            ok = me == 0 ? issue_qk<kQkIssuers, 0>(d0, qd, kd, qready, qi & 1, status)
-                         : issue_qk<kQkIssuers, 1>(d0, qd, kd, qready, qi & 1, status);
-            if (!ok) break;
-            tc::mma_commit(&bar[kSFull0 + s]);
-            if (j == w.j1 - 1) tc::mma_commit(&bar[kQEmpty]);
-          }
-          if (pv_by_qk && j > w.j0) {  // O[:, 256 me : 256 me + 256] += P(g) V(g), after QK^T(g+1)
-            const uint32_t g = g0 + (j - 1 - w.j0), b = g % kStages, s = g & 1;
-            ok = tc::mbar_wait(&bar[kPFull0 + s], (g >> 1) & 1, status);
-            if (ok && j - 1 == w.j0 && qi > 0)
-              ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
-            if (!ok) break;
-            tc::tc_fence_after();
-            const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
-            const uint64_t pd = tc::desc_sw128(tc::smem_u32(smem + kOffP + s * kPBytes), 0, 1024);
-            const uint64_t vd = tc::desc_sw128(v_base + me * 4 * kKRegion, kKRegion, 1024);
-            const uint32_t od = tmem + (me ? (16u << 16) : 0u);
+        for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
+          const bool first = j == w.j0, last = j == w.j1 - 1;
+          if (g > 0) ok = tc::mbar_wait(&bar[kSEmpty], (g - 1) & 1, status);
+          if (ok) ok = tc::mbar_wait(&bar[kPairFull0 + bi], g & 1, status);
+          if (!ok) break;
+          tc::tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kNK / 16; ++kk)
-              tc::mma_bf16_ss(od, pd + kk * 2, vd + kk * 128, kIdescPV,
-                              (j - 1 > w.j0 || kk > 0) ? 1u : 0u);
-            tc::mma_commit(&bar[kKvEmpty0 + b]);
-            tc::mma_commit(&bar[kPvDone0 + s]);
-            if (j == w.j1) tc::mma_commit(&bar[kOFull]);
+          for (int kk = 0; kk < 8; ++kk) {
+            // K-steps 8 bi + kk; the last block holds the rope slice of Q (K-steps 28..31),
+            // rotated in place before the row's first tile reads it
+            if (bi == kPairs - 1 && first && kk == kRopeStep - 8 * (kPairs - 1)) {
+              ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
+              if (!ok) break;
+              tc::tc_fence_after();
+            }
+            const uint32_t off = (uint32_t)((kk >> 2) * kRegion + (kk & 3) * 32);
+            const uint32_t qoff = (uint32_t)((kk >> 2) * kQRegion + (kk & 3) * 32);
+            tc::mma_bf16_ss(s_acc, tc::desc_sw128(pair + off, 0, 1024),
+                            tc::desc_sw128(q_base + qoff, 0, 1024), kIdescQK, kk > 0 ? 1u : 0u);
           }
+          if (!ok) break;
+          tc::mma_commit(&bar[kSFull]);
+          if (last) tc::mma_commit(&bar[kQEmpty]);
+          ok = tc::mbar_wait(&bar[kPFull], g & 1, status);
+          if (ok && first && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
+          if (!ok) break;
+          tc::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kNK / 16; ++kk)
+            tc::mma_bf16_ss(o_acc, tc::desc_sw128(pair + kk * 2048, kRegion, 1024),
+                            p_desc + (uint64_t)(kk * 2048 >> 4), kIdescPV,
+                            (first && kk == 0) ? 0u : 1u);
+          tc::mma_commit(&bar[kPairEmpty0 + bi]);
+          tc::mma_commit(&bar[kPEmpty]);
+          if (last) tc::mma_commit(&bar[kOFull]);
         }
-        g0 += w.j1 - w.j0;
         ++qi;
       }
     }
     __syncwarp();
-  } else if (warp == 3) {
+  } else if (warp == kIssuers + 1) {
     // ------------------------------------------------------------------ query rotation
     // Lane p first writes (cos, sin) of rope pair p at the query's position to a shared table.
     // Then thread i turns the rope pairs of head rows i and i+32 of the staged query tile (row h's
-    // 16-byte chunk c of a 128-byte region sits at chunk c ^ (h & 7)); when the rope slice starts
-    // on a 16-byte boundary (R a multiple of 8) all of a thread's chunks are loaded before any is
-    // used, so the rotation costs one shared-memory round trip instead of one per chunk.
+    // 16-byte chunk c of a 128-byte region sits at chunk c ^ (h & 7)).
     const int R = a.rf.R;
     const int p0 = (kDim - R) >> 1;  // first rotated pair among the 256 channel pairs
     float2* cs_tab = reinterpret_cast<float2*>(smem + kOffCs);
@@ -343,10 +339,9 @@ __global__ void __launch_bounds__(kNThreads, 1)
     for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const Row w = locate_item<kSplit>(a, it);
       if (w.j0 == w.j1) continue;
-      const int64_t t = w.t;
       if (lane < R / 2) {
         float c, sn;
-        rope_cos_sin(a.rf, lane, a.pos0 + t, c, sn);
+        rope_cos_sin(a.rf, lane, a.pos0 + w.t, c, sn);
         cs_tab[lane] = make_float2(c, sn);
       }
       __syncwarp();
@@ -402,308 +397,304 @@ __global__ void __launch_bounds__(kNThreads, 1)
       tc::mbar_arrive(&bar[kQReady]);
       ++qi;
     }
-  } else if (warp < 8 || warp >= 13) {
+  } else if (warp >= kSoftmaxWarp0 + 4) {
     if (!any_gather) goto done;  // every tile arrives by TMA
-    // ------------------------------------------------------------------ gather groups
-    // Warps 4-7 and 13-16 form two groups that take the gathered tiles in turn. Thread t of a
-    // group of G threads copies rows t/8, t/8 + G/8, ... of the tile; for each it copies 16-byte
-    // slot t%8 of all 8 regions, so a warp instruction reads four whole 128-byte row segments and
-    // a thread needs only a few row addresses. Once its copies landed it makes them visible to
-    // the tensor core and arrives on the tile's barrier.
-    const int grp = warp < 8 ? 0 : 1;
-    const int gt = (warp < 8 ? warp - 4 : warp - 13) * 32 + lane;  // thread within the group
+    // ------------------------------------------------------------------ gather group
+    // Thread t copies 16-byte slot t % 8 of key rows t / 8 + 16 i of both 64-channel regions of a
+    // dimension block, so a warp instruction reads four whole 128-byte row segments. Blocks are
+    // issued in order as soon as each is free; a block is handed over (wait_group) once the next
+    // block's copies are in flight. The pair barriers count this group's threads for every tile,
+    // so it also arrives for tiles that TMA fills (after the same wait for the block to be free,
+    // which keeps the barrier phases in tile order).
+    const int gt = (warp - kSoftmaxWarp0 - 4) * 32 + lane;
     const int row0 = gt >> 3, slot = gt & 7;
-    constexpr int kRowStride = kGroupThreads / 8;        // rows a group covers per pass
-    constexpr int kRowsPer = kNK / kRowStride;
-    // Walk this group's tiles in order across the CTA's query rows. The source rows of the next
-    // tile are resolved while the current tile's copies are in flight, so the selection-index
-    // loads do not add to each tile's latency.
-    struct Cursor {
-      int64_t r;
-      Row w;
-      int j;
-      uint32_t g;
-    };
-    auto valid = [&](const Cursor& c) { return c.r < n_items; };  // c.r: the work item
-    auto gathered = [&](const Cursor& c) {
-      return !(c.j < c.w.twin ? win_contig : pool_contig);
-    };
-    auto first_tile = [&](Cursor& c) {  // c.r: the first non-empty item from c.r on
-      for (; c.r < n_items; c.r += gridDim.x) {
-        c.w = locate_item<kSplit>(a, c.r);
-        if (c.w.j0 < c.w.j1) break;
-      }
-      c.j = c.r < n_items ? c.w.j0 : 0;
-    };
-    auto advance = [&](Cursor c) {  // next tile of this group after c
-      do {
-        ++c.g;
-        if (++c.j >= c.w.j1) {
-          c.r += gridDim.x;
-          first_tile(c);
-          if (c.r >= n_items) return c;
-        }
-      } while ((int)(c.g % kGatherGroups) != grp);
-      return c;
-    };
-    auto resolve = [&](const Cursor& c, const __nv_bfloat16* (&src)[kRowsPer]) {
-#pragma unroll
-      for (int i = 0; i < kRowsPer; ++i) src[i] = key_ptr(a, c.w, c.w.r, c.j, row0 + kRowStride * i);
-    };
-    Cursor c;
-    c.r = blockIdx.x;
-    c.g = 0;
-    first_tile(c);
-    if (valid(c))
-      for (int i = 0; i < grp; ++i) c = advance(c);
-    const __nv_bfloat16* src[kRowsPer];
-    if (valid(c) && gathered(c)) resolve(c, src);
-    bool ok = true;
-    while (valid(c) && ok) {
-      const uint32_t b = c.g % kStages;
-      if (c.g >= kStages)
-        ok = __all_sync(~0u, tc::mbar_wait(&bar[kKvEmpty0 + b], ((c.g - kStages) / kStages) & 1,
-                                           status));
-      if (!ok) break;
-      const bool gath = gathered(c);
-      if (gath) {
-        uint8_t* tile = smem + kOffTile + b * kTileBytes;
-#pragma unroll
-        for (int i = 0; i < kRowsPer; ++i) {
-          const int row = row0 + kRowStride * i;
-          uint8_t* d = tile + row * 128 + ((slot ^ (row & 7)) << 4);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) tc::cp_async16(d + q * kKRegion, src[i] + q * 64 + slot * 8);
-        }
-      }
-      const Cursor n = advance(c);
-      if (valid(n) && gathered(n)) resolve(n, src);  // overlaps the copies in flight
-      if (gath) {
-        tc::cp_async_wait_all();
-        tc::fence_proxy_async_smem();
-      }
-      tc::mbar_arrive(&bar[kKvFull0 + b]);
-      c = n;
-    }
-  } else if (warp == 12) {
-    // ------------------------------------------------------------------ PV issuer
-    // O += P(g) V(g) as soon as the softmax has written P(g), independent of how far the QK^T
-    // issuers have got: O[:, 0:256] accumulates in lanes 0-15 and O[:, 256:512] in lanes 16-31,
-    // and the two halves' MMAs alternate so both lane halves of the tensor core stay busy.
-    if (lane == 0 && !pv_by_qk) {
-      uint32_t g0 = 0, qi = 0;
-      bool ok = true;
-      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const Row w = locate_item<kSplit>(a, it);
-        if (w.j0 == w.j1) continue;
-        for (int j = w.j0; j < w.j1 && ok; ++j) {
-          const uint32_t g = g0 + (j - w.j0), b = g % kStages, s = g & 1;
-          ok = tc::mbar_wait(&bar[kPFull0 + s], (g >> 1) & 1, status);
-          if (ok && j == w.j0 && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
-          if (!ok) break;
-          tc::tc_fence_after();
-          const uint32_t v_base = tc::smem_u32(smem + kOffTile + b * kTileBytes);
-          const uint64_t pd = tc::desc_sw128(tc::smem_u32(smem + kOffP + s * kPBytes), 0, 1024);
-          const uint64_t vd0 = tc::desc_sw128(v_base, kKRegion, 1024);
-          const uint64_t vd1 = tc::desc_sw128(v_base + 4 * kKRegion, kKRegion, 1024);
-#pragma unroll
-          for (int kk = 0; kk < kNK / 16; ++kk) {
-            const uint32_t acc = (j > w.j0 || kk > 0) ? 1u : 0u;
-            tc::mma_bf16_ss(tmem, pd + kk * 2, vd0 + kk * 128, kIdescPV, acc);
-            tc::mma_bf16_ss(tmem + (16u << 16), pd + kk * 2, vd1 + kk * 128, kIdescPV, acc);
-          }
-          tc::mma_commit(&bar[kKvEmpty0 + b]);
-          tc::mma_commit(&bar[kPvDone0 + s]);
-          if (j == w.j1 - 1) tc::mma_commit(&bar[kOFull]);
-        }
-        g0 += w.j1 - w.j0;
-        ++qi;
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------------ softmax + output
-    const int sp = warp & 3;                 // TMEM sub-partition of this warp
-    const int half = lane >> 4;              // 0: keys 0..23, O[:,0:256]; 1: keys 24..47, O[:,256:]
-    const int h = 16 * sp + (lane & 15);     // head of this thread's row
-    const uint32_t t_row = tmem + ((uint32_t)(32 * sp) << 16);
-    const float scale_log2 = a.scale * kLog2e;
-    const float sink_log2 = __ldg(a.sinks + h) * kLog2e;
-    uint32_t g0 = 0, qi = 0;
+    constexpr int kRowsPer = kNK / 16;
+    uint32_t g = 0;
     bool ok = true;
     for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const Row w = locate_item<kSplit>(a, it);
       if (w.j0 == w.j1) continue;
-      const int64_t r = w.r;
-      // the sink (logit s_h, zero value) is one more term of the normaliser: here, or in the
-      // combine kernel when the row's keys are split
-      float m_run = kSplit ? -INFINITY : sink_log2, l_run = kSplit ? 0.f : 1.f;
-      for (int j = w.j0; j < w.j1 && ok; ++j) {
-        const uint32_t g = g0 + (j - w.j0), s = g & 1;
-        ok = __all_sync(~0u, tc::mbar_wait(&bar[kSFull0 + s], (g >> 1) & 1, status));
+      for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
+        const bool gath = !(j < w.twin ? win_contig : pool_contig);
+        const __nv_bfloat16* src[kRowsPer];
+        if (gath) {
+#pragma unroll
+          for (int i = 0; i < kRowsPer; ++i) src[i] = key_ptr(a, w, j, row0 + 16 * i);
+        }
+#pragma unroll
+        for (int b = 0; b < kPairs; ++b) {
+          if (g > 0) ok = __all_sync(~0u, tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status));
+          if (!ok) break;
+          if (!gath) {
+            tc::mbar_arrive(&bar[kPairFull0 + b]);
+            continue;
+          }
+          uint8_t* pr = smem + kOffPair + b * kPairBytes;
+#pragma unroll
+          for (int i = 0; i < kRowsPer; ++i) {
+            const int row = row0 + 16 * i;
+            uint8_t* d = pr + row * 128 + ((slot ^ (row & 7)) << 4);
+            tc::cp_async16(d, src[i] + 128 * b + slot * 8);
+            tc::cp_async16(d + kRegion, src[i] + 128 * b + 64 + slot * 8);
+          }
+          asm volatile("cp.async.commit_group;" ::: "memory");
+          if (b > 0) {  // the previous block's copies have landed: hand it over
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&bar[kPairFull0 + b - 1]);
+          }
+        }
+        if (!ok || !gath) continue;
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&bar[kPairFull0 + kPairs - 1]);
+      }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------------ softmax + output
+    const int sp = warp & 3;                  // TMEM sub-partition of this warp
+    const int tid = threadIdx.x - 32 * kSoftmaxWarp0;  // 0..127
+    const int key = 32 * sp + lane;           // key of the tile (TMEM lane) / channel in a block
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * sp) << 16);
+    float* m_sm = reinterpret_cast<float*>(smem + kOffM);
+    float* alpha_sm = reinterpret_cast<float*>(smem + kOffAlpha);
+    float* l_sm = reinterpret_cast<float*>(smem + kOffL);
+    float* wred_sm = reinterpret_cast<float*>(smem + kOffWmax);
+    uint8_t* prow = smem + kOffP + key * 128;
+    const float scale_log2 = a.scale * kLog2e;
+    // the two heads whose normaliser this lane keeps after the warp's reduce-scatter: bit 4 of
+    // the lane picks the half of the 64 heads, bit 3 the quarter, ... bit 0 the pair
+    const int h_mine = ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
+                       ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+    uint32_t g = 0, qi = 0;
+    bool ok = true;
+    for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const Row w = locate_item<kSplit>(a, it);
+      if (w.j0 == w.j1) continue;
+      // running max per head: starts at the sink logit (unsplit rows) or -inf (splits, whose
+      // combine adds the sink); O^T starts fresh with the item's first PV
+      if (tid < kHeads) m_sm[tid] = kSplit ? -INFINITY : __ldg(a.sinks + tid) * kLog2e;
+      float l0 = 0.f, l1 = 0.f;  // this warp's sums of p for heads h_mine, h_mine + 1
+      bar_sync_softmax();
+      for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
+        const bool first = j == w.j0;
+        ok = softmax_wait(&bar[kSFull], g & 1, status);
         if (!ok) break;
         tc::tc_fence_after();
-        // own partials: columns [0,48) and [48,96) of this S buffer in this thread's lane
-        float own[kNK];
-        {
-          uint32_t v[16];
+        const bool valid = key < tile_keys(w, j);
+        float x[kHeads];
 #pragma unroll
-          for (int c = 0; c < kNK; c += 16) {
-            uint32_t u[16];
-            tc::tmem_ld16(t_row + kColS + s * kSStride + c, v);
-            tc::tmem_ld16(t_row + kColS + s * kSStride + kNK + c, u);
-            tc::tmem_wait_ld();
+        for (int c = 0; c < kHeads; c += 16) {
+          uint32_t v0[16], v1[16], v2[16], v3[16];
+          tc::tmem_ld16(t_lane + kColS + c, v0);
+          tc::tmem_ld16(t_lane + kColS + 64 + c, v1);
+          tc::tmem_ld16(t_lane + kColS + 128 + c, v2);
+          tc::tmem_ld16(t_lane + kColS + 192 + c, v3);
+          tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) own[c + e] = __uint_as_float(v[e]) + __uint_as_float(u[e]);
+          for (int e = 0; e < 16; ++e)
+            x[c + e] = valid ? ((__uint_as_float(v0[e]) + __uint_as_float(v1[e])) +
+                                (__uint_as_float(v2[e]) + __uint_as_float(v3[e]))) * scale_log2
+                             : -INFINITY;
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(&bar[kSEmpty]);
+        // does any logit exceed its head's running max by more than the lazy margin?
+        bool exceed = false;
+#pragma unroll
+        for (int c = 0; c < kHeads; c += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(m_sm + c);
+          exceed |= (x[c] > m4.x + kLazy) | (x[c + 1] > m4.y + kLazy) |
+                    (x[c + 2] > m4.z + kLazy) | (x[c + 3] > m4.w + kLazy);
+        }
+        if (bar_any_softmax(exceed)) {
+          // exact per-head maximum of this tile, then move the heads that exceed by the margin
+#pragma unroll
+          for (int h = 0; h < kHeads; ++h) {
+            const float v = warp_max(x[h]);
+            if (lane == 0) wred_sm[sp * kHeads + h] = v;
           }
-        }
-        // exchange: this thread finishes keys [half*24, half*24+24) of the row
-        float sv[kHalfNK];
-#pragma unroll
-        for (int k = 0; k < kHalfNK; ++k) {
-          const float send = half ? own[k] : own[kHalfNK + k];
-          const float recv = __shfl_xor_sync(~0u, send, 16);
-          sv[k] = (half ? own[kHalfNK + k] : own[k]) + recv;
-        }
-        const int nk = j < w.twin ? min(kNK, w.nwin - j * kNK)
-                                  : min(kNK, w.npool - (j - w.twin) * kNK);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < kHalfNK; ++k) {
-          sv[k] = half * kHalfNK + k < nk ? sv[k] * scale_log2 : -INFINITY;
-          mx = fmaxf(mx, sv[k]);
-        }
-        mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, 16));
-        const bool move = mx > m_run + kLazy;
-        const float m_new = move ? mx : m_run;
-        const float alpha = exp2f(m_run - m_new);
-        // rescale the rows of O this warp owns (rare: only when some row's max moved)
-        if (__any_sync(~0u, move) && j > w.j0) {
-          const uint32_t gp = g - 1;
-          ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + (gp & 1)], (gp >> 1) & 1, status));
-          if (!ok) break;
-          tc::tc_fence_after();
+          bar_sync_softmax();
+          if (tid < kHeads) {
+            const float tm = fmaxf(fmaxf(wred_sm[tid], wred_sm[kHeads + tid]),
+                                   fmaxf(wred_sm[2 * kHeads + tid], wred_sm[3 * kHeads + tid]));
+            const float old = m_sm[tid];
+            const float nm = tm > old + kLazy ? tm : old;
+            alpha_sm[tid] = exp2f(old - nm);
+            m_sm[tid] = nm;
+          }
+          bar_sync_softmax();
+          l0 *= alpha_sm[h_mine];
+          l1 *= alpha_sm[h_mine + 1];
+          if (!first) {
+            // rescale this thread's channel row of every O^T block by alpha per head; PV of the
+            // previous tile has completed: its commit preceded this tile's S commits
 #pragma unroll 1
-          for (int c = 0; c < 256; c += 16) {
-            uint32_t v[16];
-            tc::tmem_ld16(t_row + c, v);
-            tc::tmem_wait_ld();
+            for (int blk = 0; blk < kPairs; ++blk) {
+#pragma unroll 1
+              for (int c = 0; c < kHeads; c += 16) {
+                uint32_t v[16];
+                tc::tmem_ld16(t_lane + kColO + 64 * blk + c, v);
+                tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            tc::tmem_st16(t_row + c, v);
+                for (int e = 0; e < 16; ++e)
+                  v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha_sm[c + e]);
+                tc::tmem_st16(t_lane + kColO + 64 * blk + c, v);
+              }
+            }
+            tc::tmem_wait_st();
           }
-          tc::tmem_wait_st();
         }
-        float sum = 0.f;
-        uint32_t pk[kHalfNK / 2];
-#pragma unroll
-        for (int k = 0; k < kHalfNK; k += 2) {
-          const float e0 = exp2f(sv[k] - m_new), e1 = exp2f(sv[k + 1] - m_new);
-          sum += e0 + e1;
-          pk[k / 2] = pack_bf16(e0, e1);
-        }
-        sum += __shfl_xor_sync(~0u, sum, 16);
-        l_run = l_run * alpha + sum;
-        m_run = m_new;
-        // P buffer s is free once PV(g-2) completed
-        if (g >= 2)
-          ok = __all_sync(~0u, tc::mbar_wait(&bar[kPvDone0 + s], ((g - 2) >> 1) & 1, status));
+        // P^T row of this key: 64 heads of bf16 in one 128-byte swizzled row
+        if (g > 0) ok = softmax_wait(&bar[kPEmpty], (g - 1) & 1, status);
         if (!ok) break;
-        uint8_t* prow = smem + kOffP + s * kPBytes + h * 128;
 #pragma unroll
-        for (int ch = 0; ch < kHalfNK / 8; ++ch) {
-          const int cg = half * (kHalfNK / 8) + ch;  // 16-byte chunk of keys 8cg..8cg+7
-          *reinterpret_cast<uint4*>(prow + ((cg ^ (h & 7)) << 4)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        for (int ch = 0; ch < 8; ++ch) {
+          const float4 ma = *reinterpret_cast<const float4*>(m_sm + 8 * ch);
+          const float4 mb = *reinterpret_cast<const float4*>(m_sm + 8 * ch + 4);
+          float* xs = x + 8 * ch;
+          xs[0] = exp2f(xs[0] - ma.x); xs[1] = exp2f(xs[1] - ma.y);
+          xs[2] = exp2f(xs[2] - ma.z); xs[3] = exp2f(xs[3] - ma.w);
+          xs[4] = exp2f(xs[4] - mb.x); xs[5] = exp2f(xs[5] - mb.y);
+          xs[6] = exp2f(xs[6] - mb.z); xs[7] = exp2f(xs[7] - mb.w);
+          const uint4 pk = make_uint4(pack_bf16(xs[0], xs[1]), pack_bf16(xs[2], xs[3]),
+                                      pack_bf16(xs[4], xs[5]), pack_bf16(xs[6], xs[7]));
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (key & 7)) << 4)) = pk;
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
-        tc::mbar_arrive(&bar[kPFull0 + s]);
+        tc::mbar_arrive(&bar[kPFull]);
+        // reduce-scatter the 64 per-head probabilities over the warp's 32 keys: each step keeps
+        // half of the heads (chosen by one lane bit) and adds the partner's copy of that half
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool up = lane & 16;
+          const float send = up ? x[e] : x[e + 32];
+          const float keep = up ? x[e + 32] : x[e];
+          x[e] = keep + __shfl_xor_sync(~0u, send, 16);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const bool up = lane & 8;
+          const float send = up ? x[e] : x[e + 16];
+          const float keep = up ? x[e + 16] : x[e];
+          x[e] = keep + __shfl_xor_sync(~0u, send, 8);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const bool up = lane & 4;
+          const float send = up ? x[e] : x[e + 8];
+          const float keep = up ? x[e + 8] : x[e];
+          x[e] = keep + __shfl_xor_sync(~0u, send, 4);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool up = lane & 2;
+          const float send = up ? x[e] : x[e + 4];
+          const float keep = up ? x[e + 4] : x[e];
+          x[e] = keep + __shfl_xor_sync(~0u, send, 2);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool up = lane & 1;
+          const float send = up ? x[e] : x[e + 2];
+          const float keep = up ? x[e + 2] : x[e];
+          x[e] = keep + __shfl_xor_sync(~0u, send, 1);
+        }
+        l0 += x[0];
+        l1 += x[1];
       }
       if (!ok) break;
+      // ---- output of the item: the normaliser per head from the four warps' sums
+      wred_sm[sp * kHeads + h_mine] = l0;
+      wred_sm[sp * kHeads + h_mine + 1] = l1;
+      bar_sync_softmax();
+      if (tid < kHeads)
+        l_sm[tid] = (wred_sm[tid] + wred_sm[kHeads + tid]) +
+                    (wred_sm[2 * kHeads + tid] + wred_sm[3 * kHeads + tid]);
+      ok = softmax_wait(&bar[kOFull], qi & 1, status);
+      if (!ok) break;
+      tc::tc_fence_after();
       if (kSplit) {
-        // ---- split output: this item's O (relative to its running max), max and normaliser in
-        // fp32 for the combine kernel
-        ok = __all_sync(~0u, tc::mbar_wait(&bar[kOFull], qi & 1, status));
-        if (!ok) break;
-        tc::tc_fence_after();
-        float* po = a.part_o + ((int64_t)it * kHeads + h) * kDim + half * 256;
+        // this item's O (relative to its running max), max and normaliser in fp32 for the
+        // combine kernel: thread = channel of each block, 64 heads
+        float* po = a.part_o + (int64_t)it * kHeads * kDim;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 64) {
-          uint32_t v[4][16];
+        for (int blk = 0; blk < kPairs; ++blk) {
+          const int d = 128 * blk + key;
+#pragma unroll 1
+          for (int c = 0; c < kHeads; c += 16) {
+            uint32_t v[16];
+            tc::tmem_ld16(t_lane + kColO + 64 * blk + c, v);
+            tc::tmem_wait_ld();
+            if (blk == kPairs - 1 && c + 16 == kHeads) {
+              tc::tc_fence_before();
+              tc::mbar_arrive(&bar[kOEmpty]);
+            }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) tc::tmem_ld16(t_row + c0 + 16 * q, v[q]);
-          tc::tmem_wait_ld();
-          if (c0 + 64 == 256) {
-            tc::tc_fence_before();
-            tc::mbar_arrive(&bar[kOEmpty]);
+            for (int e = 0; e < 16; ++e) __stcg(po + (int64_t)(c + e) * kDim + d, __uint_as_float(v[e]));
           }
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              *reinterpret_cast<float4*>(po + c0 + 16 * q + e) =
-                  make_float4(__uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]),
-                              __uint_as_float(v[q][e + 2]), __uint_as_float(v[q][e + 3]));
         }
-        if (half == 0)
-          *reinterpret_cast<float2*>(a.part_ml + ((int64_t)it * kHeads + h) * 2) =
-              make_float2(m_run, l_run);
-        g0 += w.j1 - w.j0;
+        if (tid < kHeads)
+          *reinterpret_cast<float2*>(a.part_ml + ((int64_t)it * kHeads + tid) * 2) =
+              make_float2(m_sm[tid], l_sm[tid]);
+        bar_sync_softmax();  // m_sm, l_sm and the warp sums are rewritten by the next item
         ++qi;
         continue;
       }
-      // ---- output: O / l, the rope slice turned by -P_t, bf16 store. Lane p holds the cos/sin
-      // of rope pair p; the rotation reads them with warp shuffles.
+      // O / (l + sink term), the rope slice turned by -P_t, bf16. A lane pair (2i, 2i+1) holds
+      // channels d, d+1: after exchanging halves the even lane stores heads c..c+7 and the odd
+      // lane heads c+8..c+15 of each group of 16, as bf16 pairs (64 contiguous bytes per warp and
+      // head).
+      if (tid < kHeads) l_sm[tid] = 1.f / (l_sm[tid] + exp2f(__ldg(a.sinks + tid) * kLog2e - m_sm[tid]));
+      bar_sync_softmax();
       const int64_t P = a.pos0 + w.t;
-      float my_c = 1.f, my_s = 0.f;
-      if (lane < a.rf.R / 2) rope_cos_sin(a.rf, lane, -P, my_c, my_s);
-      ok = __all_sync(~0u, tc::mbar_wait(&bar[kOFull], qi & 1, status));
-      if (!ok) break;
-      tc::tc_fence_after();
-      const float inv_l = 1.f / l_run;
-      __nv_bfloat16* orow =
-          reinterpret_cast<__nv_bfloat16*>(a.o) + ((int64_t)r * kHeads + h) * kDim + half * 256;
-      const int rope_lo = kDim - a.rf.R;  // first rotated channel (always in the upper half)
+      const int rope_lo = kDim - a.rf.R;  // first rotated channel
+      __nv_bfloat16* obase = reinterpret_cast<__nv_bfloat16*>(a.o) + w.r * kHeads * kDim;
+      const int odd = lane & 1;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 64) {
-        uint32_t v[4][16];
+      for (int blk = 0; blk < kPairs; ++blk) {
+        const int d = 128 * blk + key;   // this thread's channel
+        const int d0 = d - odd;          // even channel of the lane pair
+        float cc = 1.f, ss = 0.f;
+        const bool rot = d0 >= rope_lo;  // the same for both lanes of a pair
+        if (rot) rope_cos_sin(a.rf, (d0 - rope_lo) >> 1, -P, cc, ss);
+#pragma unroll 1
+        for (int c = 0; c < kHeads; c += 16) {
+          uint32_t v[16];
+          tc::tmem_ld16(t_lane + kColO + 64 * blk + c, v);
+          tc::tmem_wait_ld();
+          if (blk == kPairs - 1 && c + 16 == kHeads) {
+            tc::tc_fence_before();
+            tc::mbar_arrive(&bar[kOEmpty]);
+          }
+          float y[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tc::tmem_ld16(t_row + c0 + 16 * q, v[q]);
-        tc::tmem_wait_ld();
-        if (c0 + 64 == 256) {  // last chunk: every upper-half lane holds rope channels here
-          tc::tc_fence_before();
-          tc::mbar_arrive(&bar[kOEmpty]);
-        }
+          for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(v[e]) * l_sm[c + e];
+          // partner's channel values for the same heads; on rope channels (the same decision for
+          // both lanes of a pair) each lane turns its own coordinate of (x0, x1) = (even, odd)
+          float z[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = c0 + 16 * q;
-          float x[16];
+          for (int e = 0; e < 16; ++e) z[e] = __shfl_xor_sync(~0u, y[e], 1);
+          if (rot) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[q][e]) * inv_l;
-          if (256 + c + 16 > rope_lo) {  // warp-uniform: some upper-half lane rotates here
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const int ch = half * 256 + c + e;
-              const int p = ch >= rope_lo ? (ch - rope_lo) >> 1 : 0;
-              const float cc = __shfl_sync(~0u, my_c, p);
-              const float ss = __shfl_sync(~0u, my_s, p);
-              if (ch >= rope_lo) {
-                const float x0 = x[e], x1 = x[e + 1];
-                x[e] = x0 * cc - x1 * ss;
-                x[e + 1] = x0 * ss + x1 * cc;
-              }
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = odd ? z[e] : y[e], x1 = odd ? y[e] : z[e];
+              y[e] = odd ? x0 * ss + x1 * cc : x0 * cc - x1 * ss;
             }
           }
-          uint4 o0 = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                                pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-          uint4 o1 = make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]),
-                                pack_bf16(x[12], x[13]), pack_bf16(x[14], x[15]));
-          reinterpret_cast<uint4*>(orow + c)[0] = o0;
-          reinterpret_cast<uint4*>(orow + c)[1] = o1;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) z[e] = __shfl_xor_sync(~0u, y[e], 1);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float lo = odd ? z[e + 8] : y[e], hi = odd ? y[e + 8] : z[e];
+            *reinterpret_cast<uint32_t*>(obase + (int64_t)(c + e + 8 * odd) * kDim + d0) =
+                pack_bf16(lo, hi);
+          }
         }
       }
-      g0 += w.j1 - w.j0;
+      bar_sync_softmax();  // m_sm, l_sm and the warp sums are rewritten by the next item
       ++qi;
     }
   }

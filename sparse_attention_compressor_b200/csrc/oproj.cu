@@ -14,8 +14,10 @@
 // 8.4 MFLOP (32 B per cycle per SM at the bf16 rate) instead of the 48 KB per 4.2 MFLOP of a single
 // 128 x 256 tile. The two accumulators take all 512 TMEM columns, so the epilogue of a tile drains
 // them before the next tile's first MMA; the TMA producer runs ahead meanwhile (3 stages of 64 KB).
-// Warps: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2-5 = epilogue (one TMEM lane
-// quarter each: thread = tile row, 256 fp32 columns per accumulator -> bf16 -> global).
+// Warps: 0 = TMA producer, 1 and 6 = MMA issuers (warp 1 owns TMEM), 2-5 = epilogue (one TMEM
+// lane quarter each: thread = tile row, 256 fp32 columns per accumulator -> bf16 -> global). Each
+// issuer feeds one accumulator, so consecutive MMAs of a thread chain on the same accumulator
+// (switching accumulators between consecutive MMAs of one thread drains the MMA pipe).
 // No cluster multicast: every CTA loads its own tiles.
 #include <cuda_bf16.h>
 
@@ -37,7 +39,7 @@ enum Bar { kFull0, kEmpty0 = kFull0 + kStages, kAccFull = kEmpty0 + kStages, kAc
            kNumBars };
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemPtr + 16;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr uint32_t kIdesc = tc::idesc_bf16(128, kBN, false, false);
 
 struct GemmArgs {
@@ -88,9 +90,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&bar[kFull0 + i], 1);
-      tc::mbar_init(&bar[kEmpty0 + i], 1);
+      tc::mbar_init(&bar[kEmpty0 + i], 2);  // both issuers
     }
-    tc::mbar_init(&bar[kAccFull], 1);
+    tc::mbar_init(&bar[kAccFull], 2);
     tc::mbar_init(&bar[kAccEmpty], 128);
     tc::fence_barrier_init();
   }
@@ -125,8 +127,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 6) {
+    // ------------------------------------------------------------------ MMA issuers
+    // warp 1: rows 0-127 of the tile (accumulator at column 0); warp 6: rows 128-255 (column 256)
+    const uint32_t half = warp == 6 ? 1u : 0u;
     if (lane == 0) {
       uint32_t g = 0, tc_count = 0;
       bool ok = true;
@@ -142,20 +146,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_base = tc::smem_u32(smem + s * kStageBytes);
           const uint32_t w_base = a_base + kABytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t wd = tc::desc_sw128(w_base + kk * 32, 0, 1024);
-            const uint32_t acc = (k > 0 || kk > 0) ? 1u : 0u;
-            tc::mma_bf16_ss(tmem, tc::desc_sw128(a_base + kk * 32, 0, 1024), wd, kIdesc, acc);
-            tc::mma_bf16_ss(tmem + kBN, tc::desc_sw128(a_base + kABytes / 2 + kk * 32, 0, 1024),
-                            wd, kIdesc, acc);
-          }
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            tc::mma_bf16_ss(tmem + half * kBN,
+                            tc::desc_sw128(a_base + half * (kABytes / 2) + kk * 32, 0, 1024),
+                            tc::desc_sw128(w_base + kk * 32, 0, 1024), kIdesc,
+                            (k > 0 || kk > 0) ? 1u : 0u);
           tc::mma_commit(&bar[kEmpty0 + s]);
         }
         tc::mma_commit(&bar[kAccFull]);
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;                   // TMEM lane quarter this warp may read
     const int r = q * 32 + lane;              // row within each accumulator
