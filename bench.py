@@ -328,6 +328,53 @@ def ncu_traffic(workload: str, kernel: str):
     return None, None
 
 
+def record_traffic(raw_csv: str, workload: str, kernel: str, name_regex: str, summary: str,
+                   scale: float = 1.0, scaled_from: str = "") -> dict:
+    """Add (or replace) the ncu traffic record of one kernel on one workload.
+
+    raw_csv is `ncu -i <report> --page raw --csv` of a capture of that kernel; the record keeps
+    the mean dram__bytes_read.sum + dram__bytes_write.sum over the captured launches whose name
+    matches name_regex, times `scale` when the capture ran a smaller case than the workload (the
+    ratio of units processed, stated in scaled_from), with the SHA-256 of the kernel's sources."""
+    import csv
+    import re
+    to_bytes = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}
+    with open(raw_csv) as f:
+        rows = [r for r in csv.reader(f)]
+    # ncu prints its own log lines before the table: the header row names the kernel column
+    start = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    head, units, data = rows[start], rows[start + 1], rows[start + 2:]
+    ik = head.index("Kernel Name")
+    per = []
+    for r in data:
+        if len(r) != len(head) or not re.search(name_regex, r[ik]):
+            continue
+        tot = 0.0
+        for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            i = head.index(m)
+            tot += float(r[i].replace(",", "")) * to_bytes[units[i]]
+        per.append(tot)
+    if not per:
+        raise SystemExit(f"no launch of {name_regex!r} in {raw_csv}")
+    rec = {"workload": workload, "kernel": kernel,
+           "dram_bytes_per_launch": sum(per) / len(per) * scale,
+           "launches_captured": len(per), "source_sha256": source_hash(kernel),
+           "summary": summary}
+    if scaled_from:
+        rec["scaled_from"] = scaled_from
+    recs = []
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            recs = [r for r in json.load(f)
+                    if not (r["workload"] == workload and r["kernel"] == kernel)]
+    recs.append(rec)
+    recs.sort(key=lambda r: (r["workload"], r["kernel"]))
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(recs, f, indent=1)
+        f.write("\n")
+    return rec
+
+
 def roofline(wl, ktimes: dict, peaks: dict, steps: int, tensor_kernels: set) -> tuple:
     wk = work(wl)
     total = sum(v[1] for v in ktimes.values()) or 1.0
@@ -1059,8 +1106,18 @@ def main(argv=None):
     ap.add_argument("--shard", choices=["dp", "seq"], default="dp",
                     help="dp: every rank its own sequence (weak scaling); seq: one sequence "
                          "split by queries over the ranks (CSA / HCA prefill, strong scaling)")
+    ap.add_argument("--record-traffic", nargs=4, metavar=("RAW_CSV", "KERNEL", "REGEX", "SUMMARY"),
+                    help="write the ncu traffic record of KERNEL on --workload from a raw-page "
+                         "CSV of its capture (no GPU work)")
+    ap.add_argument("--traffic-scale", type=float, default=1.0)
+    ap.add_argument("--traffic-scaled-from", default="")
     args = ap.parse_args(argv)
     wl = W.WORKLOADS[args.workload]
+    if args.record_traffic:
+        raw, kern, rx, summ = args.record_traffic
+        print(json.dumps(record_traffic(raw, args.workload, kern, rx, summ, args.traffic_scale,
+                                        args.traffic_scaled_from)))
+        return
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         # one process per GPU: relaunch this command under torch.distributed.run
         sys.exit(launch_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv)))

@@ -16,23 +16,24 @@
 //
 // MMA issue: one thread issuing a chain of MMAs into the same accumulator keeps them pipelined,
 // while switching accumulators between consecutive MMAs of one thread drains the pipe (measured:
-// ~55 vs ~220 cycles per M = 128, N = 64 MMA). So four issuer threads each own one chain: issuer
-// i computes S^T over dimension block i (8 K-steps, partial accumulator S_i) and then O^T block i
-// (8 K-steps of 16 keys); the softmax adds the four partials of S^T.
+// ~55 vs ~220 cycles per M = 128, N = 64 MMA), and two chains already reach the shared-memory
+// operand rate (~48 cycles per MMA). So issuers 0 and 1 each compute one partial of S^T over two
+// dimension blocks (16 K-steps, accumulator S_c), the softmax adds the two, and issuer i adds
+// V^T P^T of dimension block i into O^T block i (8 K-steps of 16 keys).
 //
-// Tensor memory (512 columns, fp32): O^T block i at columns 64i (128 lanes = 128 channels), S_i at
-// 256 + 64i.
+// Tensor memory (512 columns, fp32): O^T block i at columns 64i (128 lanes = 128 channels), S_c at
+// 256 + 64c.
 //
-// Softmax: thread = key (TMEM lane); per-head running max in shared memory, moved only when a
-// tile's logit exceeds it by more than 2^8 (log2 units), which a block-wide vote detects; then the
-// exact per-head tile max is taken with warp shuffles and O^T is rescaled in TMEM. The
-// normaliser's per-head sums over keys are reduce-scattered across each warp with shuffles (a lane
-// keeps two heads) and summed over the four warps at the end of the row.
+// Softmax: thread = key (TMEM lane) for 32 of the heads, two warps per TMEM sub-partition; per-head
+// running max in shared memory, moved only when a tile's logit exceeds it by more than 2^8 (log2
+// units), which a vote of the softmax threads detects; then the exact per-head tile max is taken
+// with warp shuffles and O^T is rescaled in TMEM. The normaliser's per-head sums over keys are
+// reduce-scattered across each warp with shuffles (lane i keeps one head) and summed over the
+// four sub-partitions at the end of the row.
 //
 // Warps: 0 = TMA producer (query, contiguous key tiles), 1-4 = MMA issuers (warp 1 owns TMEM),
-// 5 = query rotation, 8-11 = softmax and output, 12-15 = gather group for tiles whose rows are
-// not consecutive (CSA selections, paged caches). Layers whose every tile arrives by TMA launch
-// without the gather warps.
+// 5 = query rotation, 6-7 = gather group for tiles whose rows are not consecutive (CSA
+// selections, paged caches; idle when every tile arrives by TMA), 8-15 = softmax and output.
 #include <cuda_bf16.h>
 
 #include "launch_util.h"
@@ -52,11 +53,13 @@ constexpr int kPairBytes = 2 * kRegion;          // 32 KB: one dimension block
 constexpr int kQRegion = kHeads * 128;           // 8 KB: 64 heads x 64 channels
 constexpr int kQBytes = 8 * kQRegion;            // 64 KB
 constexpr int kPBytes = kNK * 128;               // 16 KB: P^T, 128 keys x 64 heads
-constexpr int kGroupThreads = 128;               // the gather group
-constexpr int kThreads = 512;                    // with the gather group
-constexpr int kThreadsTma = 384;                 // every tile by TMA: warps 12-15 not launched
+constexpr int kGatherWarp0 = 6;                  // warps 6-7: the gather group
+constexpr int kGroupThreads = 64;
+constexpr int kThreads = 512;                    // 16 warps: 128 registers a thread
 constexpr int kIssuers = kPairs;                 // MMA issuer threads, one per dimension block
-constexpr int kSoftmaxWarp0 = 8;                 // warps 8-11: softmax and output
+constexpr int kSoftmaxWarp0 = 8;                 // warps 8-15: softmax and output
+constexpr int kSoftmaxThreads = 256;
+constexpr int kQkChains = 2;                     // S^T partial accumulators
 
 constexpr int kOffQ = 0;
 constexpr int kOffPair = kOffQ + kQBytes;
@@ -64,16 +67,16 @@ constexpr int kOffP = kOffPair + kPairs * kPairBytes;
 constexpr int kOffM = kOffP + kPBytes;           // [64] running max per head (log2 units)
 constexpr int kOffAlpha = kOffM + 256;           // [64] rescale factors of a moved max
 constexpr int kOffL = kOffAlpha + 256;           // [64] normaliser of the output
-constexpr int kOffWmax = kOffL + 256;            // [4][64] per-warp tile maxima / normalisers
+constexpr int kOffWmax = kOffL + 256;            // [4][64] per-sub-partition maxima / normalisers
 constexpr int kOffCs = kOffWmax + 1024;          // [32] (cos, sin) of the query's rope pairs
 constexpr int kOffBar = kOffCs + 32 * 8;
 enum Bar { kQFull, kQReady, kQEmpty, kPairFull0, kPairEmpty0 = kPairFull0 + kPairs,
-           kSFull = kPairEmpty0 + kPairs, kSEmpty, kPFull, kPEmpty, kOFull, kOEmpty, kNumBars };
+           kSFull = kPairEmpty0 + kPairs, kSEmpty, kPFull, kOFull, kOEmpty, kNumBars };
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemPtr + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-constexpr uint32_t kColO = 0, kColS = 256;       // O^T block i at 64 i, S_i at 256 + 64 i
+constexpr uint32_t kColO = 0, kColS = 256;       // O^T block i at 64 i, S^T partial c at 256 + 64 c
 constexpr uint32_t kIdescQK = tc::idesc_bf16(128, kHeads, false, false);
 constexpr uint32_t kIdescPV = tc::idesc_bf16(128, kHeads, true, true);
 constexpr int kMaxSplits = 8;  // key-tile splits of one row (decode: few rows, many SMs)
@@ -81,6 +84,7 @@ constexpr int kRopeStep = 28;  // K-steps 28..31 read the last region of Q (the 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;  // move the running max only when a tile exceeds it by 2^8
 constexpr int kSoftmaxBar = 1; // named barrier of the 128 softmax threads
+constexpr int kGatherBar = 2;  // named barrier of the gather group
 
 struct Row {
   int seq;
@@ -139,7 +143,7 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
 }
 
 __device__ __forceinline__ void bar_sync_softmax() {
-  asm volatile("barrier.sync %0, %1;" ::"r"(kSoftmaxBar), "r"(128) : "memory");
+  asm volatile("barrier.sync %0, %1;" ::"r"(kSoftmaxBar), "r"(kSoftmaxThreads) : "memory");
 }
 // true on every softmax thread when v is true on any of them
 __device__ __forceinline__ bool bar_any_softmax(bool v) {
@@ -150,38 +154,88 @@ __device__ __forceinline__ bool bar_any_softmax(bool v) {
       "barrier.red.or.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v), "r"(kSoftmaxBar), "r"(128)
+      : "r"((uint32_t)v), "r"(kSoftmaxBar), "r"(kSoftmaxThreads)
       : "memory");
   return r != 0;
 }
 
-// Wait on an mbarrier phase from the 128 softmax threads. The group meets at named barriers, so
+// Reduce-scatter of 32 per-head values over the 32 lanes of a warp (sum, or max with kMax):
+// each step keeps the half of the heads that one lane bit selects and combines it with the
+// partner lane's copy, so after five steps lane l holds head l. v is left unchanged.
+template <bool kMax>
+__device__ __forceinline__ float reduce_scatter32(const float (&v)[32], int lane) {
+  float t[16];
+  const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4, u2 = lane & 2, u1 = lane & 1;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float keep = u16 ? v[e + 16] : v[e];
+    const float recv = __shfl_xor_sync(~0u, u16 ? v[e] : v[e + 16], 16);
+    t[e] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float keep = u8 ? t[e + 8] : t[e];
+    const float recv = __shfl_xor_sync(~0u, u8 ? t[e] : t[e + 8], 8);
+    t[e] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float keep = u4 ? t[e + 4] : t[e];
+    const float recv = __shfl_xor_sync(~0u, u4 ? t[e] : t[e + 4], 4);
+    t[e] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const float keep = u2 ? t[e + 2] : t[e];
+    const float recv = __shfl_xor_sync(~0u, u2 ? t[e] : t[e + 2], 2);
+    t[e] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+  const float keep = u1 ? t[1] : t[0];
+  const float recv = __shfl_xor_sync(~0u, u1 ? t[0] : t[1], 1);
+  return kMax ? fmaxf(keep, recv) : keep + recv;
+}
+
+// true on every gather thread when v is true on any of them
+__device__ __forceinline__ bool bar_any_gather(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(kGatherBar), "r"(kGroupThreads)
+      : "memory");
+  return r != 0;
+}
+
+// Wait on an mbarrier phase from the 256 softmax threads. The group meets at named barriers, so
 // whether the wait timed out is decided for the whole group: if any thread gave up, all do.
 __device__ __forceinline__ bool softmax_wait(uint64_t* bar, uint32_t parity, int* status) {
   return !bar_any_softmax(!tc::mbar_wait(bar, parity, status));
 }
 
-// Global address of key c of tile j (keys past the tile's count reuse a valid row: masked).
-__device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const Row& w, int j,
-                                                        int c) {
+// Row of key c of tile j in the flat [rows, 512] view of its cache (the TMA coordinate). Keys past
+// the tile's count reuse a valid row (the softmax masks them); an unallocated page maps to row 0.
+__device__ __forceinline__ int32_t key_row(const AttnArgs& a, const Row& w, int j, int c) {
   if (j < w.twin) {
     int x = j * kNK + c;
     if (x >= w.nwin) x = 0;
-    const __nv_bfloat16* p = a.win.row<__nv_bfloat16>(w.seq, w.lo + x);
-    return p ? p : a.win.row<__nv_bfloat16>(w.seq, w.lo);
+    return (int32_t)a.win.row_index(w.seq, w.lo + x);
   }
   int i = (j - w.twin) * kNK + c;
   if (i >= w.npool) i = 0;
   int64_t e = a.pool_mode == 2 ? (int64_t)__ldg(a.sel + w.r * a.k + i) : i;
-  const __nv_bfloat16* p = a.pool.row<__nv_bfloat16>(w.seq, e < 0 ? 0 : e);
-  return p ? p : reinterpret_cast<const __nv_bfloat16*>(a.pool.base);
+  return (int32_t)a.pool.row_index(w.seq, e < 0 ? 0 : e);
 }
 
-template <bool kSplit, int kNThreads>
-__global__ void __launch_bounds__(kNThreads, 1)
+template <bool kSplit>
+__global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_win_box,
-                        const __grid_constant__ CUtensorMap tm_pool_box, AttnArgs a) {
+                        const __grid_constant__ CUtensorMap tm_pool_box,
+                        const __grid_constant__ CUtensorMap tm_win_row,
+                        const __grid_constant__ CUtensorMap tm_pool_row, AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
@@ -197,27 +251,23 @@ __global__ void __launch_bounds__(kNThreads, 1)
   const bool win_contig = a.win.block_table == nullptr;
   const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
   const bool any_gather = !win_contig || (a.pool_mode != 0 && !pool_contig);
-  if (any_gather && kNThreads < kThreads) {  // the launcher sizes the block from the same rule
-    if (threadIdx.x == 0 && status) atomicExch(status, tc::kStatusConfig);
-    return;
-  }
   const int64_t n_items = kSplit ? a.nrows * a.splits : a.nrows;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bar[kQFull], 1);
     tc::mbar_init(&bar[kQReady], 32);
-    tc::mbar_init(&bar[kQEmpty], kIssuers);
+    tc::mbar_init(&bar[kQEmpty], kQkChains);
     for (int b = 0; b < kPairs; ++b) {
-      // TMA thread (+ the gather group when some tiles are gathered)
-      tc::mbar_init(&bar[kPairFull0 + b], any_gather ? 1 + kGroupThreads : 1);
+      // the TMA thread's arrival, and with gathered tiles also the gather group's (one of the
+      // two posts the tile's bytes)
+      tc::mbar_init(&bar[kPairFull0 + b], any_gather ? 2 : 1);
       tc::mbar_init(&bar[kPairEmpty0 + b], 1);
     }
-    tc::mbar_init(&bar[kSFull], kIssuers);
-    tc::mbar_init(&bar[kSEmpty], 128);
-    tc::mbar_init(&bar[kPFull], 128);
-    tc::mbar_init(&bar[kPEmpty], kIssuers);
+    tc::mbar_init(&bar[kSFull], kQkChains);
+    tc::mbar_init(&bar[kSEmpty], kSoftmaxThreads);
+    tc::mbar_init(&bar[kPFull], kSoftmaxThreads);
     tc::mbar_init(&bar[kOFull], kIssuers);
-    tc::mbar_init(&bar[kOEmpty], 128);
+    tc::mbar_init(&bar[kOEmpty], kSoftmaxThreads);
     tc::fence_barrier_init();
   }
   if (warp == 1) tc::tmem_alloc(tmem_ptr, 512);
@@ -225,6 +275,10 @@ __global__ void __launch_bounds__(kNThreads, 1)
     tc::tma_prefetch_desc(&tm_q);
     tc::tma_prefetch_desc(&tm_win_box);
     tc::tma_prefetch_desc(&tm_pool_box);
+    if (any_gather) {
+      tc::tma_prefetch_desc(&tm_win_row);
+      tc::tma_prefetch_desc(&tm_pool_row);
+    }
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -256,14 +310,14 @@ __global__ void __launch_bounds__(kNThreads, 1)
           for (int b = 0; b < kPairs && ok; ++b) {
             if (g > 0) ok = tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status);
             if (!ok) break;
-            if (contig) {
-              uint8_t* dst = smem + kOffPair + b * kPairBytes;
-              tc::mbar_arrive_expect_tx(&bar[kPairFull0 + b], kPairBytes);
-              tc::tma_load_2d(dst, map, &bar[kPairFull0 + b], 128 * b, (int32_t)y0);
-              tc::tma_load_2d(dst + kRegion, map, &bar[kPairFull0 + b], 128 * b + 64, (int32_t)y0);
-            } else {
+            if (!contig) {  // the gather group fills this block and posts its bytes
               tc::mbar_arrive(&bar[kPairFull0 + b]);
+              continue;
             }
+            uint8_t* dst = smem + kOffPair + b * kPairBytes;
+            tc::mbar_arrive_expect_tx(&bar[kPairFull0 + b], kPairBytes);
+            tc::tma_load_2d(dst, map, &bar[kPairFull0 + b], 128 * b, (int32_t)y0);
+            tc::tma_load_2d(dst + kRegion, map, &bar[kPairFull0 + b], 128 * b + 64, (int32_t)y0);
           }
         }
         ++qi;
@@ -272,54 +326,67 @@ __global__ void __launch_bounds__(kNThreads, 1)
     __syncwarp();
   } else if (warp >= 1 && warp <= kIssuers) {
     // ------------------------------------------------------------------ MMA issuers
-    // Issuer i: S_i = K[:, block i] Q[:, block i]^T (8 K-steps), then O^T block i += V^T P^T
-    // (8 steps of 16 keys); each chain stays on one accumulator.
+    // Issuers 0 and 1: S^T partial c = K[:, blocks 2c, 2c+1] Q[:, same channels]^T (16 K-steps,
+    // each block as soon as it has arrived). Every issuer i then adds V^T P^T of dimension block i
+    // to O^T block i (8 steps of 16 keys). Each chain stays on one accumulator.
     const int bi = warp - 1;
     if (lane == 0) {
       uint32_t g = 0, qi = 0;
       bool ok = true;
-      const uint32_t q_base = tc::smem_u32(smem + kOffQ) + bi * 2 * kQRegion;
-      const uint32_t pair = tc::smem_u32(smem + kOffPair) + bi * kPairBytes;
+      const uint32_t q_base = tc::smem_u32(smem + kOffQ);
+      const uint32_t pairs = tc::smem_u32(smem + kOffPair);
       const uint64_t p_desc = tc::desc_sw128(tc::smem_u32(smem + kOffP), 0, 1024);
       const uint32_t s_acc = tmem + kColS + 64 * bi, o_acc = tmem + kColO + 64 * bi;
+      const bool qk = bi < kQkChains;
       for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const Row w = locate_item<kSplit>(a, it);
         if (w.j0 == w.j1) continue;
-        ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
+        if (qk) ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
         for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
           const bool first = j == w.j0, last = j == w.j1 - 1;
-          if (g > 0) ok = tc::mbar_wait(&bar[kSEmpty], (g - 1) & 1, status);
-          if (ok) ok = tc::mbar_wait(&bar[kPairFull0 + bi], g & 1, status);
-          if (!ok) break;
-          tc::tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // K-steps 8 bi + kk; the last block holds the rope slice of Q (K-steps 28..31),
-            // rotated in place before the row's first tile reads it
-            if (bi == kPairs - 1 && first && kk == kRopeStep - 8 * (kPairs - 1)) {
-              ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
+          if (qk) {
+            // ---- S^T partial bi over dimension blocks 2 bi and 2 bi + 1
+            if (g > 0) ok = tc::mbar_wait(&bar[kSEmpty], (g - 1) & 1, status);
+            for (int h = 0; h < 2 && ok; ++h) {
+              const int pb = 2 * bi + h;
+              ok = tc::mbar_wait(&bar[kPairFull0 + pb], g & 1, status);
               if (!ok) break;
               tc::tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                // the rope slice of Q (K-steps 28..31, the last block) is rotated in place before
+                // the row's first tile reads it
+                if (first && 8 * pb + kk == kRopeStep) {
+                  ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
+                  if (!ok) break;
+                  tc::tc_fence_after();
+                }
+                const uint32_t off =
+                    (uint32_t)(pb * kPairBytes + (kk >> 2) * kRegion + (kk & 3) * 32);
+                const uint32_t qoff = (uint32_t)((2 * pb + (kk >> 2)) * kQRegion + (kk & 3) * 32);
+                tc::mma_bf16_ss(s_acc, tc::desc_sw128(pairs + off, 0, 1024),
+                                tc::desc_sw128(q_base + qoff, 0, 1024), kIdescQK,
+                                (h > 0 || kk > 0) ? 1u : 0u);
+              }
             }
-            const uint32_t off = (uint32_t)((kk >> 2) * kRegion + (kk & 3) * 32);
-            const uint32_t qoff = (uint32_t)((kk >> 2) * kQRegion + (kk & 3) * 32);
-            tc::mma_bf16_ss(s_acc, tc::desc_sw128(pair + off, 0, 1024),
-                            tc::desc_sw128(q_base + qoff, 0, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+            if (!ok) break;
+            tc::mma_commit(&bar[kSFull]);
+            if (last) tc::mma_commit(&bar[kQEmpty]);
           }
-          if (!ok) break;
-          tc::mma_commit(&bar[kSFull]);
-          if (last) tc::mma_commit(&bar[kQEmpty]);
+          // ---- O^T block bi += V^T P^T once the softmax has written P (block bi has arrived:
+          // this wait names the phase the S chains already saw complete)
           ok = tc::mbar_wait(&bar[kPFull], g & 1, status);
+          if (ok) ok = tc::mbar_wait(&bar[kPairFull0 + bi], g & 1, status);
           if (ok && first && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
           if (!ok) break;
           tc::tc_fence_after();
+          const uint32_t pair = pairs + bi * kPairBytes;
 #pragma unroll
           for (int kk = 0; kk < kNK / 16; ++kk)
             tc::mma_bf16_ss(o_acc, tc::desc_sw128(pair + kk * 2048, kRegion, 1024),
                             p_desc + (uint64_t)(kk * 2048 >> 4), kIdescPV,
                             (first && kk == 0) ? 0u : 1u);
           tc::mma_commit(&bar[kPairEmpty0 + bi]);
-          tc::mma_commit(&bar[kPEmpty]);
           if (last) tc::mma_commit(&bar[kOFull]);
         }
         ++qi;
@@ -397,64 +464,64 @@ __global__ void __launch_bounds__(kNThreads, 1)
       tc::mbar_arrive(&bar[kQReady]);
       ++qi;
     }
-  } else if (warp >= kSoftmaxWarp0 + 4) {
+  } else if (warp >= kGatherWarp0 && warp < kSoftmaxWarp0) {
     if (!any_gather) goto done;  // every tile arrives by TMA
     // ------------------------------------------------------------------ gather group
-    // Thread t copies 16-byte slot t % 8 of key rows t / 8 + 16 i of both 64-channel regions of a
-    // dimension block, so a warp instruction reads four whole 128-byte row segments. Blocks are
-    // issued in order as soon as each is free; a block is handed over (wait_group) once the next
-    // block's copies are in flight. The pair barriers count this group's threads for every tile,
-    // so it also arrives for tiles that TMA fills (after the same wait for the block to be free,
-    // which keeps the barrier phases in tile order).
-    const int gt = (warp - kSoftmaxWarp0 - 4) * 32 + lane;
-    const int row0 = gt >> 3, slot = gt & 7;
-    constexpr int kRowsPer = kNK / 16;
+    // Tiles whose rows are not consecutive arrive by TMA row gathers: thread t takes keys
+    // 4(t % 32) .. 4(t % 32) + 3 and 64-channel region t / 32 of each dimension block, one
+    // four-row gather per block (4 x 128 B into rows 4(t % 32).. of the region; the 128-byte
+    // swizzle follows the shared-memory address, so the rows land as a box load would put them).
+    // Thread 0 waits for the block to be free and posts the tile's bytes on its barrier before the
+    // group issues. The TMA thread and thread 0 both wait for every block to be free and both
+    // arrive on every tile's barrier (the one that does not fill it without bytes), so neither can
+    // fall a phase behind and every parity wait names the phase it means. Whether a wait gave up
+    // is shared with the group at its named barrier, so the 64 threads leave together.
+    const int gt = (warp - kGatherWarp0) * 32 + lane;
+    const int kg = gt & 31, half = gt >> 5;
     uint32_t g = 0;
     bool ok = true;
     for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const Row w = locate_item<kSplit>(a, it);
       if (w.j0 == w.j1) continue;
       for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
-        const bool gath = !(j < w.twin ? win_contig : pool_contig);
-        const __nv_bfloat16* src[kRowsPer];
-        if (gath) {
-#pragma unroll
-          for (int i = 0; i < kRowsPer; ++i) src[i] = key_ptr(a, w, j, row0 + 16 * i);
+        const bool is_win = j < w.twin;
+        if (is_win ? win_contig : pool_contig) {  // filled by the TMA thread
+          bool mine = true;
+          if (gt == 0) {
+            for (int b = 0; b < kPairs && mine; ++b) {
+              if (g > 0) mine = tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status);
+              if (mine) tc::mbar_arrive(&bar[kPairFull0 + b]);
+            }
+          }
+          ok = !bar_any_gather(!mine);
+          continue;
         }
+        int32_t y[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) y[i] = key_row(a, w, j, 4 * kg + i);
+        const CUtensorMap* map = is_win ? &tm_win_row : &tm_pool_row;
 #pragma unroll
         for (int b = 0; b < kPairs; ++b) {
-          if (g > 0) ok = __all_sync(~0u, tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status));
+          bool mine = true;
+          if (gt == 0) {
+            if (g > 0) mine = tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status);
+            if (mine) tc::mbar_arrive_expect_tx(&bar[kPairFull0 + b], kPairBytes);
+          }
+          ok = !bar_any_gather(!mine);
           if (!ok) break;
-          if (!gath) {
-            tc::mbar_arrive(&bar[kPairFull0 + b]);
-            continue;
-          }
-          uint8_t* pr = smem + kOffPair + b * kPairBytes;
-#pragma unroll
-          for (int i = 0; i < kRowsPer; ++i) {
-            const int row = row0 + 16 * i;
-            uint8_t* d = pr + row * 128 + ((slot ^ (row & 7)) << 4);
-            tc::cp_async16(d, src[i] + 128 * b + slot * 8);
-            tc::cp_async16(d + kRegion, src[i] + 128 * b + 64 + slot * 8);
-          }
-          asm volatile("cp.async.commit_group;" ::: "memory");
-          if (b > 0) {  // the previous block's copies have landed: hand it over
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&bar[kPairFull0 + b - 1]);
-          }
+          const int region = 2 * b + half;
+          tc::tma_gather4(smem + kOffPair + b * kPairBytes + half * kRegion + kg * 512, map,
+                          &bar[kPairFull0 + b], 64 * region, y[0], y[1], y[2], y[3]);
         }
-        if (!ok || !gath) continue;
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        tc::fence_proxy_async_smem();
-        tc::mbar_arrive(&bar[kPairFull0 + kPairs - 1]);
       }
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
   } else if (warp >= kSoftmaxWarp0) {
     // ------------------------------------------------------------------ softmax + output
+    // Warp 8 + 4 hh + sp: keys 32 sp .. 32 sp + 31 of the tile (its TMEM lanes) and heads
+    // 32 hh .. 32 hh + 31, so each sub-partition has two softmax warps.
     const int sp = warp & 3;                  // TMEM sub-partition of this warp
-    const int tid = threadIdx.x - 32 * kSoftmaxWarp0;  // 0..127
+    const int h0 = 32 * ((warp - kSoftmaxWarp0) >> 2);  // first head of this warp
+    const int tid = threadIdx.x - 32 * kSoftmaxWarp0;  // 0..255
     const int key = 32 * sp + lane;           // key of the tile (TMEM lane) / channel in a block
     const uint32_t t_lane = tmem + ((uint32_t)(32 * sp) << 16);
     float* m_sm = reinterpret_cast<float*>(smem + kOffM);
@@ -463,10 +530,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
     float* wred_sm = reinterpret_cast<float*>(smem + kOffWmax);
     uint8_t* prow = smem + kOffP + key * 128;
     const float scale_log2 = a.scale * kLog2e;
-    // the two heads whose normaliser this lane keeps after the warp's reduce-scatter: bit 4 of
-    // the lane picks the half of the 64 heads, bit 3 the quarter, ... bit 0 the pair
-    const int h_mine = ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
-                       ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+    const int h_mine = h0 + lane;  // the head whose sums this lane keeps after a reduce-scatter
     uint32_t g = 0, qi = 0;
     bool ok = true;
     for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
@@ -475,7 +539,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
       // running max per head: starts at the sink logit (unsplit rows) or -inf (splits, whose
       // combine adds the sink); O^T starts fresh with the item's first PV
       if (tid < kHeads) m_sm[tid] = kSplit ? -INFINITY : __ldg(a.sinks + tid) * kLog2e;
-      float l0 = 0.f, l1 = 0.f;  // this warp's sums of p for heads h_mine, h_mine + 1
+      float l_acc = 0.f;  // this warp's sum of p for head h_mine
       bar_sync_softmax();
       for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
         const bool first = j == w.j0;
@@ -483,132 +547,94 @@ __global__ void __launch_bounds__(kNThreads, 1)
         if (!ok) break;
         tc::tc_fence_after();
         const bool valid = key < tile_keys(w, j);
-        float x[kHeads];
-#pragma unroll
-        for (int c = 0; c < kHeads; c += 16) {
-          uint32_t v0[16], v1[16], v2[16], v3[16];
-          tc::tmem_ld16(t_lane + kColS + c, v0);
-          tc::tmem_ld16(t_lane + kColS + 64 + c, v1);
-          tc::tmem_ld16(t_lane + kColS + 128 + c, v2);
-          tc::tmem_ld16(t_lane + kColS + 192 + c, v3);
+        float x[32];
+        {
+          uint32_t va[32], vb[32];
+          tc::tmem_ld32(t_lane + kColS + h0, va);
+          tc::tmem_ld32(t_lane + kColS + 64 + h0, vb);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            x[c + e] = valid ? ((__uint_as_float(v0[e]) + __uint_as_float(v1[e])) +
-                                (__uint_as_float(v2[e]) + __uint_as_float(v3[e]))) * scale_log2
-                             : -INFINITY;
+          for (int e = 0; e < 32; ++e)
+            x[e] = valid ? (__uint_as_float(va[e]) + __uint_as_float(vb[e])) * scale_log2
+                         : -INFINITY;
         }
         tc::tc_fence_before();
         tc::mbar_arrive(&bar[kSEmpty]);
-        // does any logit exceed its head's running max by more than the lazy margin?
-        bool exceed = false;
+        // The running max: on a row's first tile it is set from the exact per-head tile max (the
+        // sink as the floor); later it moves only for heads whose logits exceed it by the lazy
+        // margin, which a vote of the softmax threads detects first.
+        bool exceed = first;
+        if (!first) {
 #pragma unroll
-        for (int c = 0; c < kHeads; c += 4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(m_sm + c);
-          exceed |= (x[c] > m4.x + kLazy) | (x[c + 1] > m4.y + kLazy) |
-                    (x[c + 2] > m4.z + kLazy) | (x[c + 3] > m4.w + kLazy);
-        }
-        if (bar_any_softmax(exceed)) {
-          // exact per-head maximum of this tile, then move the heads that exceed by the margin
-#pragma unroll
-          for (int h = 0; h < kHeads; ++h) {
-            const float v = warp_max(x[h]);
-            if (lane == 0) wred_sm[sp * kHeads + h] = v;
+          for (int c = 0; c < 32; c += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(m_sm + h0 + c);
+            exceed |= (x[c] > m4.x + kLazy) | (x[c + 1] > m4.y + kLazy) |
+                      (x[c + 2] > m4.z + kLazy) | (x[c + 3] > m4.w + kLazy);
           }
+        }
+        if (first || bar_any_softmax(exceed)) {
+          // per-head maximum over this warp's 32 keys by reduce-scatter (lane i keeps head
+          // h0 + i), then over the four sub-partitions
+          wred_sm[sp * kHeads + h_mine] = reduce_scatter32<true>(x, lane);
           bar_sync_softmax();
           if (tid < kHeads) {
             const float tm = fmaxf(fmaxf(wred_sm[tid], wred_sm[kHeads + tid]),
                                    fmaxf(wred_sm[2 * kHeads + tid], wred_sm[3 * kHeads + tid]));
             const float old = m_sm[tid];
-            const float nm = tm > old + kLazy ? tm : old;
-            alpha_sm[tid] = exp2f(old - nm);
+            const float nm = first ? fmaxf(old, tm) : (tm > old + kLazy ? tm : old);
+            alpha_sm[tid] = first ? 1.f : tc::exp2_approx(old - nm);
             m_sm[tid] = nm;
           }
           bar_sync_softmax();
-          l0 *= alpha_sm[h_mine];
-          l1 *= alpha_sm[h_mine + 1];
           if (!first) {
-            // rescale this thread's channel row of every O^T block by alpha per head; PV of the
-            // previous tile has completed: its commit preceded this tile's S commits
+            l_acc *= alpha_sm[h_mine];
+            // rescale this thread's channel row of every O^T block by alpha per head (this
+            // warp's 32 heads); PV of the previous tile has completed: its commit preceded this
+            // tile's S commits
 #pragma unroll 1
             for (int blk = 0; blk < kPairs; ++blk) {
-#pragma unroll 1
-              for (int c = 0; c < kHeads; c += 16) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 16) {
                 uint32_t v[16];
-                tc::tmem_ld16(t_lane + kColO + 64 * blk + c, v);
+                tc::tmem_ld16(t_lane + kColO + 64 * blk + h0 + c, v);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                  v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha_sm[c + e]);
-                tc::tmem_st16(t_lane + kColO + 64 * blk + c, v);
+                  v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha_sm[h0 + c + e]);
+                tc::tmem_st16(t_lane + kColO + 64 * blk + h0 + c, v);
               }
             }
             tc::tmem_wait_st();
           }
         }
-        // P^T row of this key: 64 heads of bf16 in one 128-byte swizzled row
-        if (g > 0) ok = softmax_wait(&bar[kPEmpty], (g - 1) & 1, status);
-        if (!ok) break;
+        // P^T row of this key: 64 heads of bf16 in one 128-byte swizzled row, of which this warp
+        // writes 16-byte chunks 4 hh .. 4 hh + 3. The buffer is free: this tile's S came from keys
+        // that refilled every dimension block after the previous tile's PV of that block had
+        // completed (the pair barriers), so every PV MMA that read the previous P has finished;
+        // the same ordering covers the rescale of O^T above.
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const float4 ma = *reinterpret_cast<const float4*>(m_sm + 8 * ch);
-          const float4 mb = *reinterpret_cast<const float4*>(m_sm + 8 * ch + 4);
+        for (int ch = 0; ch < 4; ++ch) {
+          const float4 ma = *reinterpret_cast<const float4*>(m_sm + h0 + 8 * ch);
+          const float4 mb = *reinterpret_cast<const float4*>(m_sm + h0 + 8 * ch + 4);
           float* xs = x + 8 * ch;
-          xs[0] = exp2f(xs[0] - ma.x); xs[1] = exp2f(xs[1] - ma.y);
-          xs[2] = exp2f(xs[2] - ma.z); xs[3] = exp2f(xs[3] - ma.w);
-          xs[4] = exp2f(xs[4] - mb.x); xs[5] = exp2f(xs[5] - mb.y);
-          xs[6] = exp2f(xs[6] - mb.z); xs[7] = exp2f(xs[7] - mb.w);
+          xs[0] = tc::exp2_approx(xs[0] - ma.x); xs[1] = tc::exp2_approx(xs[1] - ma.y);
+          xs[2] = tc::exp2_approx(xs[2] - ma.z); xs[3] = tc::exp2_approx(xs[3] - ma.w);
+          xs[4] = tc::exp2_approx(xs[4] - mb.x); xs[5] = tc::exp2_approx(xs[5] - mb.y);
+          xs[6] = tc::exp2_approx(xs[6] - mb.z); xs[7] = tc::exp2_approx(xs[7] - mb.w);
           const uint4 pk = make_uint4(pack_bf16(xs[0], xs[1]), pack_bf16(xs[2], xs[3]),
                                       pack_bf16(xs[4], xs[5]), pack_bf16(xs[6], xs[7]));
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (key & 7)) << 4)) = pk;
+          const int chunk = (h0 >> 3) + ch;
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ (key & 7)) << 4)) = pk;
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         tc::mbar_arrive(&bar[kPFull]);
-        // reduce-scatter the 64 per-head probabilities over the warp's 32 keys: each step keeps
-        // half of the heads (chosen by one lane bit) and adds the partner's copy of that half
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool up = lane & 16;
-          const float send = up ? x[e] : x[e + 32];
-          const float keep = up ? x[e + 32] : x[e];
-          x[e] = keep + __shfl_xor_sync(~0u, send, 16);
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const bool up = lane & 8;
-          const float send = up ? x[e] : x[e + 16];
-          const float keep = up ? x[e + 16] : x[e];
-          x[e] = keep + __shfl_xor_sync(~0u, send, 8);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const bool up = lane & 4;
-          const float send = up ? x[e] : x[e + 8];
-          const float keep = up ? x[e + 8] : x[e];
-          x[e] = keep + __shfl_xor_sync(~0u, send, 4);
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool up = lane & 2;
-          const float send = up ? x[e] : x[e + 4];
-          const float keep = up ? x[e + 4] : x[e];
-          x[e] = keep + __shfl_xor_sync(~0u, send, 2);
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool up = lane & 1;
-          const float send = up ? x[e] : x[e + 2];
-          const float keep = up ? x[e + 2] : x[e];
-          x[e] = keep + __shfl_xor_sync(~0u, send, 1);
-        }
-        l0 += x[0];
-        l1 += x[1];
+        // per-head sums of p over this warp's 32 keys (reduce-scatter: lane i keeps head h0 + i)
+        l_acc += reduce_scatter32<false>(x, lane);
       }
       if (!ok) break;
-      // ---- output of the item: the normaliser per head from the four warps' sums
-      wred_sm[sp * kHeads + h_mine] = l0;
-      wred_sm[sp * kHeads + h_mine + 1] = l1;
+      // ---- output of the item: the normaliser per head from the four sub-partitions' sums
+      wred_sm[sp * kHeads + h_mine] = l_acc;
       bar_sync_softmax();
       if (tid < kHeads)
         l_sm[tid] = (wred_sm[tid] + wred_sm[kHeads + tid]) +
@@ -618,23 +644,24 @@ __global__ void __launch_bounds__(kNThreads, 1)
       tc::tc_fence_after();
       if (kSplit) {
         // this item's O (relative to its running max), max and normaliser in fp32 for the
-        // combine kernel: thread = channel of each block, 64 heads
-        float* po = a.part_o + (int64_t)it * kHeads * kDim;
+        // combine kernel: thread = channel of each block, this warp's 32 heads; the four blocks'
+        // columns of one group of 16 heads are loaded together (one TMEM round trip per group)
+        float* po = a.part_o + (int64_t)it * kHeads * kDim + key;
 #pragma unroll 1
-        for (int blk = 0; blk < kPairs; ++blk) {
-          const int d = 128 * blk + key;
-#pragma unroll 1
-          for (int c = 0; c < kHeads; c += 16) {
-            uint32_t v[16];
-            tc::tmem_ld16(t_lane + kColO + 64 * blk + c, v);
-            tc::tmem_wait_ld();
-            if (blk == kPairs - 1 && c + 16 == kHeads) {
-              tc::tc_fence_before();
-              tc::mbar_arrive(&bar[kOEmpty]);
-            }
+        for (int c = h0; c < h0 + 32; c += 16) {
+          uint32_t v[kPairs][16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) __stcg(po + (int64_t)(c + e) * kDim + d, __uint_as_float(v[e]));
+          for (int blk = 0; blk < kPairs; ++blk) tc::tmem_ld16(t_lane + kColO + 64 * blk + c, v[blk]);
+          tc::tmem_wait_ld();
+          if (c + 16 == h0 + 32) {
+            tc::tc_fence_before();
+            tc::mbar_arrive(&bar[kOEmpty]);
           }
+#pragma unroll
+          for (int blk = 0; blk < kPairs; ++blk)
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              __stcg(po + (int64_t)(c + e) * kDim + 128 * blk, __uint_as_float(v[blk][e]));
         }
         if (tid < kHeads)
           *reinterpret_cast<float2*>(a.part_ml + ((int64_t)it * kHeads + tid) * 2) =
@@ -646,51 +673,59 @@ __global__ void __launch_bounds__(kNThreads, 1)
       // O / (l + sink term), the rope slice turned by -P_t, bf16. A lane pair (2i, 2i+1) holds
       // channels d, d+1: after exchanging halves the even lane stores heads c..c+7 and the odd
       // lane heads c+8..c+15 of each group of 16, as bf16 pairs (64 contiguous bytes per warp and
-      // head).
-      if (tid < kHeads) l_sm[tid] = 1.f / (l_sm[tid] + exp2f(__ldg(a.sinks + tid) * kLog2e - m_sm[tid]));
+      // head). The four blocks' columns of one group of 16 heads are loaded together.
+      if (tid < kHeads)
+        l_sm[tid] = 1.f / (l_sm[tid] + tc::exp2_approx(__ldg(a.sinks + tid) * kLog2e - m_sm[tid]));
       bar_sync_softmax();
       const int64_t P = a.pos0 + w.t;
       const int rope_lo = kDim - a.rf.R;  // first rotated channel
       __nv_bfloat16* obase = reinterpret_cast<__nv_bfloat16*>(a.o) + w.r * kHeads * kDim;
       const int odd = lane & 1;
+      // only the last block can hold rope channels (R <= 64 < 128)
+      const int d3 = 128 * (kPairs - 1) + key - odd;  // even channel of the pair in the last block
+      const bool rot = d3 >= rope_lo;                 // the same for both lanes of a pair
+      float cc = 1.f, ss = 0.f;
+      if (rot) rope_cos_sin(a.rf, (d3 - rope_lo) >> 1, -P, cc, ss);
 #pragma unroll 1
-      for (int blk = 0; blk < kPairs; ++blk) {
-        const int d = 128 * blk + key;   // this thread's channel
-        const int d0 = d - odd;          // even channel of the lane pair
-        float cc = 1.f, ss = 0.f;
-        const bool rot = d0 >= rope_lo;  // the same for both lanes of a pair
-        if (rot) rope_cos_sin(a.rf, (d0 - rope_lo) >> 1, -P, cc, ss);
-#pragma unroll 1
-        for (int c = 0; c < kHeads; c += 16) {
-          uint32_t v[16];
-          tc::tmem_ld16(t_lane + kColO + 64 * blk + c, v);
-          tc::tmem_wait_ld();
-          if (blk == kPairs - 1 && c + 16 == kHeads) {
-            tc::tc_fence_before();
-            tc::mbar_arrive(&bar[kOEmpty]);
-          }
+      for (int c = h0; c < h0 + 32; c += 16) {
+        uint32_t v[kPairs][16];
+#pragma unroll
+        for (int blk = 0; blk < kPairs; ++blk) tc::tmem_ld16(t_lane + kColO + 64 * blk + c, v[blk]);
+        tc::tmem_wait_ld();
+        if (c + 16 == h0 + 32) {
+          tc::tc_fence_before();
+          tc::mbar_arrive(&bar[kOEmpty]);
+        }
+#pragma unroll
+        for (int blk = 0; blk < kPairs; ++blk) {
           float y[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(v[e]) * l_sm[c + e];
-          // partner's channel values for the same heads; on rope channels (the same decision for
-          // both lanes of a pair) each lane turns its own coordinate of (x0, x1) = (even, odd)
-          float z[16];
+          for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(v[blk][e]) * l_sm[c + e];
+          if (blk == kPairs - 1) {
+            // rope channels: each lane turns its own coordinate of (x0, x1) = (even, odd), with the
+            // partner lane's value of the pair (the same decision for both lanes of a pair)
+            float z[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) z[e] = __shfl_xor_sync(~0u, y[e], 1);
-          if (rot) {
+            for (int e = 0; e < 16; ++e) z[e] = __shfl_xor_sync(~0u, y[e], 1);
+            if (rot) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float x0 = odd ? z[e] : y[e], x1 = odd ? y[e] : z[e];
-              y[e] = odd ? x0 * ss + x1 * cc : x0 * cc - x1 * ss;
+              for (int e = 0; e < 16; ++e) {
+                const float x0 = odd ? z[e] : y[e], x1 = odd ? y[e] : z[e];
+                y[e] = odd ? x0 * ss + x1 * cc : x0 * cc - x1 * ss;
+              }
             }
           }
+          // pack heads (h, h+1) of this channel into one bf16 pair, swap packed words with the
+          // partner lane: the even lane then holds head h of channels (d0, d0+1), the odd lane head
+          // h+1 of them, each one 4-byte store
+          const int d0 = 128 * blk + key - odd;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) z[e] = __shfl_xor_sync(~0u, y[e], 1);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float lo = odd ? z[e + 8] : y[e], hi = odd ? y[e + 8] : z[e];
-            *reinterpret_cast<uint32_t*>(obase + (int64_t)(c + e + 8 * odd) * kDim + d0) =
-                pack_bf16(lo, hi);
+          for (int e = 0; e < 16; e += 2) {
+            const uint32_t mine = pack_bf16(y[e], y[e + 1]);
+            const uint32_t theirs = __shfl_xor_sync(~0u, mine, 1);
+            const uint32_t word = odd ? __byte_perm(theirs, mine, 0x7632)
+                                      : __byte_perm(mine, theirs, 0x5410);
+            *reinterpret_cast<uint32_t*>(obase + (int64_t)(c + e + odd) * kDim + d0) = word;
           }
         }
       }
@@ -794,7 +829,12 @@ bool attention_tc_supported(const AttnArgs& a, int dtype) {
 cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t pool_rows,
                                 cudaStream_t st) {
   if (a.nrows == 0) return cudaSuccess;
-  CUtensorMap tq, twb, tpb;
+  // a paged cache's block table addresses its page buffer, whose extent the call does not carry:
+  // its maps span every 32-bit row coordinate (the gathers read only the rows the table names)
+  constexpr int64_t kPagedRows = (int64_t(1) << 31) - 1;
+  if (a.win.block_table) win_rows = kPagedRows;
+  if (a.pool_mode != 0 && a.pool.block_table) pool_rows = kPagedRows;
+  CUtensorMap tq, twb, tpb, twr, tpr;
   cudaError_t e = make_tmap_bf16_2d(&tq, a.q, (uint64_t)a.nrows * kHeads, kDim, kDim * 2, 64, 64);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16_2d(&twb, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, kNK, 64);
@@ -803,14 +843,16 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
   e = make_tmap_bf16_2d(&tpb, has_pool ? a.pool.base : a.win.base,
                         (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
-  // the same rule as the kernel's any_gather: paged rows or CSA selections are gathered
-  const bool win_contig = a.win.block_table == nullptr;
-  const bool pool_contig = a.pool_mode == 1 && a.pool.block_table == nullptr;
-  const bool any_gather = !win_contig || (a.pool_mode != 0 && !pool_contig);
-  const void* kern = a.splits > 1 ? (any_gather ? (const void*)attention_tc_kernel<true, kThreads>
-                                                : (const void*)attention_tc_kernel<true, kThreadsTma>)
-                                  : (any_gather ? (const void*)attention_tc_kernel<false, kThreads>
-                                                : (const void*)attention_tc_kernel<false, kThreadsTma>);
+  // one-row boxes for the four-row gathers (row coordinates are 32-bit)
+  if (win_rows >= (int64_t(1) << 31) || pool_rows >= (int64_t(1) << 31))
+    return cudaErrorInvalidValue;
+  e = make_tmap_bf16_2d(&twr, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, 1, 64);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16_2d(&tpr, has_pool ? a.pool.base : a.win.base,
+                        (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, 1, 64);
+  if (e != cudaSuccess) return e;
+  const void* kern = a.splits > 1 ? (const void*)attention_tc_kernel<true>
+                                  : (const void*)attention_tc_kernel<false>;
   e = ensure_smem_limit(kern, kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -820,18 +862,10 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
     return cudaErrorInvalidValue;
   const int64_t items = a.nrows * a.splits;
   const int grid = (int)(items < sms ? items : sms);
-  if (a.splits > 1) {
-    if (any_gather)
-      attention_tc_kernel<true, kThreads><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
-    else
-      attention_tc_kernel<true, kThreadsTma><<<grid, kThreadsTma, kSmemBytes, st>>>(tq, twb, tpb, a);
-  } else {
-    if (any_gather)
-      attention_tc_kernel<false, kThreads><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
-    else
-      attention_tc_kernel<false, kThreadsTma><<<grid, kThreadsTma, kSmemBytes, st>>>(tq, twb, tpb,
-                                                                                    a);
-  }
+  if (a.splits > 1)
+    attention_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, twr, tpr, a);
+  else
+    attention_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, twr, tpr, a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.splits == 1) return e;
   attention_combine_kernel<<<dim3((unsigned)a.nrows, kHeads / kCombineHeads), 256, 0, st>>>(a);

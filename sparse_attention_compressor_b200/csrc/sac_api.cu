@@ -710,7 +710,7 @@ static int paged_attention(const sac_params* p, const PagedCall& c) {
   }
   a.status = status;
   decode_attach_splits(p, rows, c.ws, c.ws_bytes, used, a);
-  cudaError_t e = run_attention(p, a, 1, 1, st, c.timer);
+  cudaError_t e = run_attention(p, a, 0, 0, st, c.timer);  // paged: extents from the tables
   if (e != cudaSuccess) return cuda_fail(e, "attention");
   return SAC_OK;
 }

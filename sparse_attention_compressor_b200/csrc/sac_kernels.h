@@ -142,7 +142,8 @@ cudaError_t launch_attention_simt(int dtype, const AttnArgs& a, cudaStream_t st)
 
 // ---- attention on tcgen05 (attention_tc.cu): bf16, 64 heads, head_dim 512 ------------------
 // a.q: [nrows, 64, 512] un-rotated (rotated in the kernel); win/pool bases are [rows, 512]
-// buffers whose row counts (win_rows, pool_rows) bound the TMA coordinates.
+// buffers whose row counts (win_rows, pool_rows) bound the TMA coordinates; a paged cache's
+// count is ignored (its block table names the rows read).
 bool attention_tc_supported(const AttnArgs& a, int dtype);
 int attention_tc_max_splits();
 cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t pool_rows,

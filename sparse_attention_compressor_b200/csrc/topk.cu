@@ -27,6 +27,7 @@ constexpr int kBins = 4096;          // 12-bit digits
 constexpr int kCandCap = 2048;       // compacted keys of the threshold bin
 constexpr int kSmemKeyRows = 4096;   // rows up to this length keep their keys in shared memory
 constexpr int kSmemKeyLimit = 49152; // longest row whose keys fit in shared memory (192 KB)
+constexpr int kBatch = 8;            // loads a thread has in flight in the passes over a row
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t u = __float_as_uint(s + 0.0f);  // -0 and +0 compare equal
@@ -127,14 +128,27 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
     return kSmemKeys ? keys[i] : order_key(__ldcg(srow + i));
   };
 
-  // ---- digit 1: bits 31..20
+  // ---- digit 1: bits 31..20. The passes over the row issue kBatch loads before using any, so a
+  // thread waits for one memory latency per kBatch keys rather than per key.
   for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0;
   if (tid == 0) sh.n_cand = 0;
   __syncthreads();
-  for (int i = tid; i < n; i += NT) {
-    const uint32_t key = order_key(__ldcg(srow + i));
-    if (kSmemKeys) keys[i] = key;
-    atomicAdd(&sh.hist[key >> 20], 1);
+  for (int i0 = tid; i0 < n; i0 += NT * kBatch) {
+    float v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * NT;
+      v[u] = i < n ? __ldcg(srow + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * NT;
+      if (i < n) {
+        const uint32_t key = order_key(v[u]);
+        if (kSmemKeys) keys[i] = key;
+        atomicAdd(&sh.hist[key >> 20], 1);
+      }
+    }
   }
   __syncthreads();
   find_digit<NT>(sh, kBins, k);
@@ -146,16 +160,24 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
   // ---- compact the keys of digit d1 when they fit; otherwise scan the whole row with a mask
   const bool compact = c1 <= kCandCap;
   if (compact) {
-    for (int i0 = warp * 32; i0 < n; i0 += NT) {
-      const int i = i0 + lane;
-      const uint32_t key = i < n ? key_at(i) : 0u;
-      const bool hit = i < n && (key >> 20) == d1;
-      const uint32_t mask = __ballot_sync(~0u, hit);
-      if (mask) {
-        int base = 0;
-        if (lane == 0) base = atomicAdd(&sh.n_cand, __popc(mask));
-        base = __shfl_sync(~0u, base, 0);
-        if (hit) sh.cand[base + __popc(mask & ((1u << lane) - 1u))] = key;
+    for (int b0 = warp * 32; b0 < n; b0 += NT * kBatch) {
+      uint32_t kb[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = b0 + u * NT + lane;
+        kb[u] = i < n ? key_at(i) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = b0 + u * NT + lane;
+        const bool hit = i < n && (kb[u] >> 20) == d1;
+        const uint32_t mask = __ballot_sync(~0u, hit);
+        if (mask) {
+          int base = 0;
+          if (lane == 0) base = atomicAdd(&sh.n_cand, __popc(mask));
+          base = __shfl_sync(~0u, base, 0);
+          if (hit) sh.cand[base + __popc(mask & ((1u << lane) - 1u))] = kb[u];
+        }
       }
     }
   }
@@ -192,11 +214,19 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
   const int seg = ((n + (NT / 32) * 32 - 1) / ((NT / 32) * 32)) * 32;
   const int s0 = warp * seg, s1 = min(n, s0 + seg);
   int gt = 0, eq = 0;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
-    const int i = i0 + lane;
-    const uint32_t key = i < s1 ? key_at(i) : 0u;
-    gt += __popc(__ballot_sync(~0u, i < s1 && key > T));
-    eq += __popc(__ballot_sync(~0u, i < s1 && key == T));
+  for (int b0 = s0; b0 < s1; b0 += 32 * kBatch) {
+    uint32_t kb[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = b0 + 32 * u + lane;
+      kb[u] = i < s1 ? key_at(i) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const bool in = b0 + 32 * u + lane < s1;
+      gt += __popc(__ballot_sync(~0u, in && kb[u] > T));
+      eq += __popc(__ballot_sync(~0u, in && kb[u] == T));
+    }
   }
   if (lane == 0) {
     sh.warp_gt[warp] = gt;
@@ -211,17 +241,25 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
     eq_before += e;
   }
   const uint32_t lt = (1u << lane) - 1u;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
-    const int i = i0 + lane;
-    const uint32_t key = i < s1 ? key_at(i) : 0u;
-    const bool is_gt = i < s1 && key > T;
-    const bool is_eq = i < s1 && key == T;
-    const uint32_t eq_mask = __ballot_sync(~0u, is_eq);
-    const bool sel = is_gt || (is_eq && eq_before + __popc(eq_mask & lt) < take_eq);
-    const uint32_t sel_mask = __ballot_sync(~0u, sel);
-    if (sel) orow[sel_before + __popc(sel_mask & lt)] = i;
-    eq_before += __popc(eq_mask);
-    sel_before += __popc(sel_mask);
+  for (int b0 = s0; b0 < s1; b0 += 32 * kBatch) {
+    uint32_t kb[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = b0 + 32 * u + lane;
+      kb[u] = i < s1 ? key_at(i) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = b0 + 32 * u + lane;
+      const bool is_gt = i < s1 && kb[u] > T;
+      const bool is_eq = i < s1 && kb[u] == T;
+      const uint32_t eq_mask = __ballot_sync(~0u, is_eq);
+      const bool sel = is_gt || (is_eq && eq_before + __popc(eq_mask & lt) < take_eq);
+      const uint32_t sel_mask = __ballot_sync(~0u, sel);
+      if (sel) orow[sel_before + __popc(sel_mask & lt)] = i;
+      eq_before += __popc(eq_mask);
+      sel_before += __popc(sel_mask);
+    }
   }
 }
 

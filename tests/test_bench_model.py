@@ -79,3 +79,25 @@ def test_chunk_inputs_shapes_and_reproducibility():
     assert torch.equal(d["q"], d2["q"]) and torch.equal(d["kv_pages"], d2["kv_pages"])
     dec = W.decode_inputs(replace(wl, chunk=1), "csa")
     assert dec["q"].shape == (2, 4, 64) and dec["q_idx"].shape == (2, 3, 32)
+
+
+def test_traffic_record_reads_ncu_csv_and_goes_stale(tmp_path, monkeypatch):
+    """A traffic record is the mean DRAM bytes of the matching captured launches (units taken from
+    the CSV's unit row), scaled to the workload, and is dropped once the kernel's sources change."""
+    raw = tmp_path / "raw.csv"
+    raw.write_text('==PROF== log line\n'
+                   '"ID","Kernel Name","dram__bytes_read.sum","dram__bytes_write.sum"\n'
+                   '"","","Mbyte","Gbyte"\n'
+                   '"0","void attention_tc_kernel<0>(...)","500","1.5"\n'
+                   '"1","void other_kernel(...)","7","7"\n'
+                   '"2","void attention_tc_kernel<0>(...)","1,500","0.5"\n')
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "traffic.json"))
+    rec = bench.record_traffic(str(raw), "csa_8k_bf16", "attention", r"attention_tc_kernel",
+                               "attention.md", scale=2.0, scaled_from="x2")
+    assert rec["launches_captured"] == 2
+    assert rec["dram_bytes_per_launch"] == ((0.5e9 + 1.5e9) + (1.5e9 + 0.5e9)) / 2 * 2.0
+    t, r = bench.ncu_traffic("csa_8k_bf16", "attention")
+    assert t == rec["dram_bytes_per_launch"] and r["scaled_from"] == "x2"
+    assert bench.ncu_traffic("csa_8k_bf16", "topk") == (None, None)
+    monkeypatch.setattr(bench, "source_hash", lambda k: "changed")
+    assert bench.ncu_traffic("csa_8k_bf16", "attention") == (None, None)
