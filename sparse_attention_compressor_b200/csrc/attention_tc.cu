@@ -32,8 +32,9 @@
 // four sub-partitions at the end of the row.
 //
 // Warps: 0 = TMA producer (query, contiguous key tiles), 1-4 = MMA issuers (warp 1 owns TMEM),
-// 5 = query rotation, 6-7 = gather group for tiles whose rows are not consecutive (CSA
-// selections, paged caches; idle when every tile arrives by TMA), 8-15 = softmax and output.
+// 5 = query rotation, 6-7 and 16-19 = gather group for tiles whose rows are not consecutive (CSA
+// selections, paged caches; idle when every tile arrives by TMA), 8-15 = softmax and output. The
+// softmax warpgroups take registers from the others (setmaxnreg).
 #include <cuda_bf16.h>
 
 #include "launch_util.h"
@@ -53,9 +54,16 @@ constexpr int kPairBytes = 2 * kRegion;          // 32 KB: one dimension block
 constexpr int kQRegion = kHeads * 128;           // 8 KB: 64 heads x 64 channels
 constexpr int kQBytes = 8 * kQRegion;            // 64 KB
 constexpr int kPBytes = kNK * 128;               // 16 KB: P^T, 128 keys x 64 heads
-constexpr int kGatherWarp0 = 6;                  // warps 6-7: the gather group
-constexpr int kGroupThreads = 64;
-constexpr int kThreads = 512;                    // 16 warps: 128 registers a thread
+constexpr int kThreads = 640;                    // 20 warps (five warpgroups)
+constexpr int kGroupThreads = 192;               // the gather group: warps 6-7 and 16-19
+// Registers: the block launches with 96 a thread; the two softmax warpgroups (8-15) raise theirs
+// to 128, warpgroups 0-1 (producer, issuers, rotation, two gather warps) lower theirs to 80 and
+// warpgroup 4 (gather only) to 64 (setmaxnreg), which the launch's total covers exactly:
+// 2 x 128 x 128 + 2 x 128 x 80 + 128 x 64 = 61440 = 640 x 96.
+constexpr int kRegsLaunch = 96, kRegsSoftmax = 128, kRegsOther = 80, kRegsGather = 64;
+static_assert(2 * 128 * kRegsSoftmax + 2 * 128 * kRegsOther + 128 * kRegsGather <=
+                  kThreads * kRegsLaunch,
+              "register split above the launch's registers");
 constexpr int kIssuers = kPairs;                 // MMA issuer threads, one per dimension block
 constexpr int kSoftmaxWarp0 = 8;                 // warps 8-15: softmax and output
 constexpr int kSoftmaxThreads = 256;
@@ -84,7 +92,6 @@ constexpr int kRopeStep = 28;  // K-steps 28..31 read the last region of Q (the 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;  // move the running max only when a tile exceeds it by 2^8
 constexpr int kSoftmaxBar = 1; // named barrier of the 128 softmax threads
-constexpr int kGatherBar = 2;  // named barrier of the gather group
 
 struct Row {
   int seq;
@@ -195,47 +202,97 @@ __device__ __forceinline__ float reduce_scatter32(const float (&v)[32], int lane
   return kMax ? fmaxf(keep, recv) : keep + recv;
 }
 
-// true on every gather thread when v is true on any of them
-__device__ __forceinline__ bool bar_any_gather(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(kGatherBar), "r"(kGroupThreads)
-      : "memory");
-  return r != 0;
-}
-
 // Wait on an mbarrier phase from the 256 softmax threads. The group meets at named barriers, so
 // whether the wait timed out is decided for the whole group: if any thread gave up, all do.
 __device__ __forceinline__ bool softmax_wait(uint64_t* bar, uint32_t parity, int* status) {
   return !bar_any_softmax(!tc::mbar_wait(bar, parity, status));
 }
 
-// Row of key c of tile j in the flat [rows, 512] view of its cache (the TMA coordinate). Keys past
-// the tile's count reuse a valid row (the softmax masks them); an unallocated page maps to row 0.
-__device__ __forceinline__ int32_t key_row(const AttnArgs& a, const Row& w, int j, int c) {
+// Global address of key c of tile j (keys past the tile's count reuse a valid row: masked).
+__device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const Row& w, int j,
+                                                        int c) {
   if (j < w.twin) {
     int x = j * kNK + c;
     if (x >= w.nwin) x = 0;
-    return (int32_t)a.win.row_index(w.seq, w.lo + x);
+    const __nv_bfloat16* p = a.win.row<__nv_bfloat16>(w.seq, w.lo + x);
+    return p ? p : a.win.row<__nv_bfloat16>(w.seq, w.lo);
   }
   int i = (j - w.twin) * kNK + c;
   if (i >= w.npool) i = 0;
   int64_t e = a.pool_mode == 2 ? (int64_t)__ldg(a.sel + w.r * a.k + i) : i;
-  return (int32_t)a.pool.row_index(w.seq, e < 0 ? 0 : e);
+  const __nv_bfloat16* p = a.pool.row<__nv_bfloat16>(w.seq, e < 0 ? 0 : e);
+  return p ? p : reinterpret_cast<const __nv_bfloat16*>(a.pool.base);
+}
+
+// The gather group: 192 threads (warps 6-7 and 16-19; gt = the thread's index in the group) fill
+// the tiles whose rows are not consecutive. Thread gt copies 16-byte slot gt % 8 of key rows
+// gt / 8 + 24 i of both 64-channel regions of a dimension block, so a warp instruction reads four
+// whole 128-byte row segments. Blocks are issued in order as soon as each is free; a block is
+// handed over (wait_group) once the next block's copies are in flight. The pair barriers count
+// this group's threads for every tile, so it also arrives for tiles that TMA fills (after the same
+// wait for the block to be free): each party waits for every phase, so no parity wait can name a
+// phase other than the one it means.
+template <bool kSplit>
+__device__ __forceinline__ void gather_tiles(const AttnArgs& a, uint8_t* smem, uint64_t* bar,
+                                             int64_t n_items, bool win_contig, bool pool_contig,
+                                             int gt, int* status) {
+    const int row0 = gt >> 3, slot = gt & 7;
+  constexpr int kRowStride = kGroupThreads / 8;                     // 24
+  constexpr int kRowsPer = (kNK + kRowStride - 1) / kRowStride;     // 6 (the last only row0 < 8)
+  uint32_t g = 0;
+  bool ok = true;
+  for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    const Row w = locate_item<kSplit>(a, it);
+    if (w.j0 == w.j1) continue;
+    for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
+      const bool gath = !(j < w.twin ? win_contig : pool_contig);
+      const __nv_bfloat16* src[kRowsPer];
+      if (gath) {
+  #pragma unroll
+        for (int i = 0; i < kRowsPer; ++i) {
+          const int row = row0 + kRowStride * i;
+          src[i] = key_ptr(a, w, j, row < kNK ? row : 0);
+        }
+      }
+  #pragma unroll
+      for (int b = 0; b < kPairs; ++b) {
+        if (g > 0) ok = __all_sync(~0u, tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status));
+        if (!ok) break;
+        if (!gath) {
+          tc::mbar_arrive(&bar[kPairFull0 + b]);
+          continue;
+        }
+        uint8_t* pr = smem + kOffPair + b * kPairBytes;
+  #pragma unroll
+        for (int i = 0; i < kRowsPer; ++i) {
+          const int row = row0 + kRowStride * i;
+          if (row < kNK) {
+            uint8_t* d = pr + row * 128 + ((slot ^ (row & 7)) << 4);
+            tc::cp_async16(d, src[i] + 128 * b + slot * 8);
+            tc::cp_async16(d + kRegion, src[i] + 128 * b + 64 + slot * 8);
+          }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (b > 0) {  // the previous block's copies have landed: hand it over
+          asm volatile("cp.async.wait_group 1;" ::: "memory");
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(&bar[kPairFull0 + b - 1]);
+        }
+      }
+      if (!ok || !gath) continue;
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[kPairFull0 + kPairs - 1]);
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 template <bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_win_box,
-                        const __grid_constant__ CUtensorMap tm_pool_box,
-                        const __grid_constant__ CUtensorMap tm_win_row,
-                        const __grid_constant__ CUtensorMap tm_pool_row, AttnArgs a) {
+                        const __grid_constant__ CUtensorMap tm_pool_box, AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + kOffTmemPtr);
@@ -258,9 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bar[kQReady], 32);
     tc::mbar_init(&bar[kQEmpty], kQkChains);
     for (int b = 0; b < kPairs; ++b) {
-      // the TMA thread's arrival, and with gathered tiles also the gather group's (one of the
-      // two posts the tile's bytes)
-      tc::mbar_init(&bar[kPairFull0 + b], any_gather ? 2 : 1);
+      // the TMA thread's arrival (with the bytes of a box load), and with gathered tiles also
+      // every gather thread's
+      tc::mbar_init(&bar[kPairFull0 + b], any_gather ? 1 + kGroupThreads : 1);
       tc::mbar_init(&bar[kPairEmpty0 + b], 1);
     }
     tc::mbar_init(&bar[kSFull], kQkChains);
@@ -275,247 +332,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tma_prefetch_desc(&tm_q);
     tc::tma_prefetch_desc(&tm_win_box);
     tc::tma_prefetch_desc(&tm_pool_box);
-    if (any_gather) {
-      tc::tma_prefetch_desc(&tm_win_row);
-      tc::tma_prefetch_desc(&tm_pool_row);
-    }
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t g = 0, qi = 0;
-      bool ok = true;
-      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const Row w = locate_item<kSplit>(a, it);
-        if (w.bad && status) atomicExch(status, tc::kStatusBadInput);
-        if (w.j0 == w.j1) continue;
-        if (qi > 0) ok = tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status);
-        if (!ok) break;
-        tc::mbar_arrive_expect_tx(&bar[kQFull], kQBytes);
-        for (int c = 0; c < 8; ++c)
-          tc::tma_load_2d(smem + kOffQ + c * kQRegion, &tm_q, &bar[kQFull], 64 * c,
-                          (int32_t)(w.r * kHeads));
-        for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
-          const bool is_win = j < w.twin;
-          const bool contig = is_win ? win_contig : pool_contig;
-          const int64_t y0 = contig ? (is_win ? a.win.row_index(w.seq, w.lo + (int64_t)j * kNK)
-                                              : a.pool.row_index(w.seq, (int64_t)(j - w.twin) * kNK))
-                                    : 0;
-          const CUtensorMap* map = is_win ? &tm_win_box : &tm_pool_box;
-          for (int b = 0; b < kPairs && ok; ++b) {
-            if (g > 0) ok = tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status);
-            if (!ok) break;
-            if (!contig) {  // the gather group fills this block and posts its bytes
-              tc::mbar_arrive(&bar[kPairFull0 + b]);
-              continue;
-            }
-            uint8_t* dst = smem + kOffPair + b * kPairBytes;
-            tc::mbar_arrive_expect_tx(&bar[kPairFull0 + b], kPairBytes);
-            tc::tma_load_2d(dst, map, &bar[kPairFull0 + b], 128 * b, (int32_t)y0);
-            tc::tma_load_2d(dst + kRegion, map, &bar[kPairFull0 + b], 128 * b + 64, (int32_t)y0);
-          }
-        }
-        ++qi;
-      }
-    }
-    __syncwarp();
-  } else if (warp >= 1 && warp <= kIssuers) {
-    // ------------------------------------------------------------------ MMA issuers
-    // Issuers 0 and 1: S^T partial c = K[:, blocks 2c, 2c+1] Q[:, same channels]^T (16 K-steps,
-    // each block as soon as it has arrived). Every issuer i then adds V^T P^T of dimension block i
-    // to O^T block i (8 steps of 16 keys). Each chain stays on one accumulator.
-    const int bi = warp - 1;
-    if (lane == 0) {
-      uint32_t g = 0, qi = 0;
-      bool ok = true;
-      const uint32_t q_base = tc::smem_u32(smem + kOffQ);
-      const uint32_t pairs = tc::smem_u32(smem + kOffPair);
-      const uint64_t p_desc = tc::desc_sw128(tc::smem_u32(smem + kOffP), 0, 1024);
-      const uint32_t s_acc = tmem + kColS + 64 * bi, o_acc = tmem + kColO + 64 * bi;
-      const bool qk = bi < kQkChains;
-      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const Row w = locate_item<kSplit>(a, it);
-        if (w.j0 == w.j1) continue;
-        if (qk) ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
-        for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
-          const bool first = j == w.j0, last = j == w.j1 - 1;
-          if (qk) {
-            // ---- S^T partial bi over dimension blocks 2 bi and 2 bi + 1
-            if (g > 0) ok = tc::mbar_wait(&bar[kSEmpty], (g - 1) & 1, status);
-            for (int h = 0; h < 2 && ok; ++h) {
-              const int pb = 2 * bi + h;
-              ok = tc::mbar_wait(&bar[kPairFull0 + pb], g & 1, status);
-              if (!ok) break;
-              tc::tc_fence_after();
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                // the rope slice of Q (K-steps 28..31, the last block) is rotated in place before
-                // the row's first tile reads it
-                if (first && 8 * pb + kk == kRopeStep) {
-                  ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
-                  if (!ok) break;
-                  tc::tc_fence_after();
-                }
-                const uint32_t off =
-                    (uint32_t)(pb * kPairBytes + (kk >> 2) * kRegion + (kk & 3) * 32);
-                const uint32_t qoff = (uint32_t)((2 * pb + (kk >> 2)) * kQRegion + (kk & 3) * 32);
-                tc::mma_bf16_ss(s_acc, tc::desc_sw128(pairs + off, 0, 1024),
-                                tc::desc_sw128(q_base + qoff, 0, 1024), kIdescQK,
-                                (h > 0 || kk > 0) ? 1u : 0u);
-              }
-            }
-            if (!ok) break;
-            tc::mma_commit(&bar[kSFull]);
-            if (last) tc::mma_commit(&bar[kQEmpty]);
-          }
-          // ---- O^T block bi += V^T P^T once the softmax has written P (block bi has arrived:
-          // this wait names the phase the S chains already saw complete)
-          ok = tc::mbar_wait(&bar[kPFull], g & 1, status);
-          if (ok) ok = tc::mbar_wait(&bar[kPairFull0 + bi], g & 1, status);
-          if (ok && first && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
-          if (!ok) break;
-          tc::tc_fence_after();
-          const uint32_t pair = pairs + bi * kPairBytes;
-#pragma unroll
-          for (int kk = 0; kk < kNK / 16; ++kk)
-            tc::mma_bf16_ss(o_acc, tc::desc_sw128(pair + kk * 2048, kRegion, 1024),
-                            p_desc + (uint64_t)(kk * 2048 >> 4), kIdescPV,
-                            (first && kk == 0) ? 0u : 1u);
-          tc::mma_commit(&bar[kPairEmpty0 + bi]);
-          if (last) tc::mma_commit(&bar[kOFull]);
-        }
-        ++qi;
-      }
-    }
-    __syncwarp();
-  } else if (warp == kIssuers + 1) {
-    // ------------------------------------------------------------------ query rotation
-    // Lane p first writes (cos, sin) of rope pair p at the query's position to a shared table.
-    // Then thread i turns the rope pairs of head rows i and i+32 of the staged query tile (row h's
-    // 16-byte chunk c of a 128-byte region sits at chunk c ^ (h & 7)).
-    const int R = a.rf.R;
-    const int p0 = (kDim - R) >> 1;  // first rotated pair among the 256 channel pairs
-    float2* cs_tab = reinterpret_cast<float2*>(smem + kOffCs);
-    uint32_t qi = 0;
-    bool ok = true;
-    for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const Row w = locate_item<kSplit>(a, it);
-      if (w.j0 == w.j1) continue;
-      if (lane < R / 2) {
-        float c, sn;
-        rope_cos_sin(a.rf, lane, a.pos0 + w.t, c, sn);
-        cs_tab[lane] = make_float2(c, sn);
-      }
-      __syncwarp();
-      ok = __all_sync(~0u, tc::mbar_wait(&bar[kQFull], qi & 1, status));
-      if (!ok) break;
-      if ((R & 7) == 0) {
-        constexpr int kMaxChunks = 8;  // R <= 64: at most 8 chunks of 4 pairs
-        const int nch = R >> 3;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int h = hh * 32 + lane;
-          uint8_t* row = smem + kOffQ + h * 128;
-          uint4 v[kMaxChunks];
-#pragma unroll
-          for (int c = 0; c < kMaxChunks; ++c) {
-            const int pp = p0 + 4 * c;
-            if (c < nch)
-              v[c] = *reinterpret_cast<const uint4*>(row + (pp >> 5) * kQRegion +
-                                                     ((((pp & 31) >> 2) ^ (h & 7)) << 4));
-          }
-#pragma unroll
-          for (int c = 0; c < kMaxChunks; ++c) {
-            if (c >= nch) break;
-            const int pp = p0 + 4 * c;
-            const float4 cs01 = *reinterpret_cast<const float4*>(cs_tab + 4 * c);
-            const float4 cs23 = *reinterpret_cast<const float4*>(cs_tab + 4 * c + 2);
-            const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
-            const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
-            uint32_t* w4 = reinterpret_cast<uint32_t*>(&v[c]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 x = unpack_bf16(w4[u]);
-              w4[u] = pack_bf16(x.x * cc[u] - x.y * ss[u], x.x * ss[u] + x.y * cc[u]);
-            }
-            *reinterpret_cast<uint4*>(row + (pp >> 5) * kQRegion +
-                                      ((((pp & 31) >> 2) ^ (h & 7)) << 4)) = v[c];
-          }
-        }
-      } else {
-        for (int hh = 0; hh < 2; ++hh) {
-          const int h = hh * 32 + lane;
-          uint8_t* row = smem + kOffQ + h * 128;
-          for (int q = p0; q < kDim / 2; ++q) {
-            uint32_t* word = reinterpret_cast<uint32_t*>(
-                row + (q >> 5) * kQRegion + ((((q & 31) >> 2) ^ (h & 7)) << 4) + (q & 3) * 4);
-            const float2 cs = cs_tab[q - p0];
-            const float2 x = unpack_bf16(*word);
-            *word = pack_bf16(x.x * cs.x - x.y * cs.y, x.x * cs.y + x.y * cs.x);
-          }
-        }
-      }
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bar[kQReady]);
-      ++qi;
-    }
-  } else if (warp >= kGatherWarp0 && warp < kSoftmaxWarp0) {
-    if (!any_gather) goto done;  // every tile arrives by TMA
-    // ------------------------------------------------------------------ gather group
-    // Tiles whose rows are not consecutive arrive by TMA row gathers: thread t takes keys
-    // 4(t % 32) .. 4(t % 32) + 3 and 64-channel region t / 32 of each dimension block, one
-    // four-row gather per block (4 x 128 B into rows 4(t % 32).. of the region; the 128-byte
-    // swizzle follows the shared-memory address, so the rows land as a box load would put them).
-    // Thread 0 waits for the block to be free and posts the tile's bytes on its barrier before the
-    // group issues. The TMA thread and thread 0 both wait for every block to be free and both
-    // arrive on every tile's barrier (the one that does not fill it without bytes), so neither can
-    // fall a phase behind and every parity wait names the phase it means. Whether a wait gave up
-    // is shared with the group at its named barrier, so the 64 threads leave together.
-    const int gt = (warp - kGatherWarp0) * 32 + lane;
-    const int kg = gt & 31, half = gt >> 5;
-    uint32_t g = 0;
-    bool ok = true;
-    for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const Row w = locate_item<kSplit>(a, it);
-      if (w.j0 == w.j1) continue;
-      for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
-        const bool is_win = j < w.twin;
-        if (is_win ? win_contig : pool_contig) {  // filled by the TMA thread
-          bool mine = true;
-          if (gt == 0) {
-            for (int b = 0; b < kPairs && mine; ++b) {
-              if (g > 0) mine = tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status);
-              if (mine) tc::mbar_arrive(&bar[kPairFull0 + b]);
-            }
-          }
-          ok = !bar_any_gather(!mine);
-          continue;
-        }
-        int32_t y[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) y[i] = key_row(a, w, j, 4 * kg + i);
-        const CUtensorMap* map = is_win ? &tm_win_row : &tm_pool_row;
-#pragma unroll
-        for (int b = 0; b < kPairs; ++b) {
-          bool mine = true;
-          if (gt == 0) {
-            if (g > 0) mine = tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status);
-            if (mine) tc::mbar_arrive_expect_tx(&bar[kPairFull0 + b], kPairBytes);
-          }
-          ok = !bar_any_gather(!mine);
-          if (!ok) break;
-          const int region = 2 * b + half;
-          tc::tma_gather4(smem + kOffPair + b * kPairBytes + half * kRegion + kg * 512, map,
-                          &bar[kPairFull0 + b], 64 * region, y[0], y[1], y[2], y[3]);
-        }
-      }
-    }
-  } else if (warp >= kSoftmaxWarp0) {
+  // Register split by warpgroup: the two softmax warpgroups raise theirs, the other three lower
+  // theirs, each warpgroup at one instruction before its warps take their roles.
+  if (warp >= kSoftmaxWarp0 && warp < kSoftmaxWarp0 + 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------------ softmax + output
     // Warp 8 + 4 hh + sp: keys 32 sp .. 32 sp + 31 of the tile (its TMEM lanes) and heads
     // 32 hh .. 32 hh + 31, so each sub-partition has two softmax warps.
@@ -732,8 +558,198 @@ __global__ void __launch_bounds__(kThreads, 1)
       bar_sync_softmax();  // m_sm, l_sm and the warp sums are rewritten by the next item
       ++qi;
     }
+  } else if (warp >= kSoftmaxWarp0 + 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsGather));
+    if (any_gather)
+      gather_tiles<kSplit>(a, smem, bar, n_items, win_contig, pool_contig,
+                           64 + (warp - kSoftmaxWarp0 - 8) * 32 + lane, status);
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        uint32_t g = 0, qi = 0;
+        bool ok = true;
+        for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+          const Row w = locate_item<kSplit>(a, it);
+          if (w.bad && status) atomicExch(status, tc::kStatusBadInput);
+          if (w.j0 == w.j1) continue;
+          if (qi > 0) ok = tc::mbar_wait(&bar[kQEmpty], (qi - 1) & 1, status);
+          if (!ok) break;
+          tc::mbar_arrive_expect_tx(&bar[kQFull], kQBytes);
+          for (int c = 0; c < 8; ++c)
+            tc::tma_load_2d(smem + kOffQ + c * kQRegion, &tm_q, &bar[kQFull], 64 * c,
+                            (int32_t)(w.r * kHeads));
+          for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
+            const bool is_win = j < w.twin;
+            const bool contig = is_win ? win_contig : pool_contig;
+            const int64_t y0 = contig ? (is_win ? a.win.row_index(w.seq, w.lo + (int64_t)j * kNK)
+                                                : a.pool.row_index(w.seq, (int64_t)(j - w.twin) * kNK))
+                                      : 0;
+            const CUtensorMap* map = is_win ? &tm_win_box : &tm_pool_box;
+            for (int b = 0; b < kPairs && ok; ++b) {
+              if (g > 0) ok = tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status);
+              if (!ok) break;
+              if (!contig) {  // the gather group fills this block
+                tc::mbar_arrive(&bar[kPairFull0 + b]);
+                continue;
+              }
+              uint8_t* dst = smem + kOffPair + b * kPairBytes;
+              tc::mbar_arrive_expect_tx(&bar[kPairFull0 + b], kPairBytes);
+              tc::tma_load_2d(dst, map, &bar[kPairFull0 + b], 128 * b, (int32_t)y0);
+              tc::tma_load_2d(dst + kRegion, map, &bar[kPairFull0 + b], 128 * b + 64, (int32_t)y0);
+            }
+          }
+          ++qi;
+        }
+      }
+      __syncwarp();
+    } else if (warp >= 1 && warp <= kIssuers) {
+      // ------------------------------------------------------------------ MMA issuers
+      // Issuers 0 and 1: S^T partial c = K[:, blocks 2c, 2c+1] Q[:, same channels]^T (16 K-steps,
+      // each block as soon as it has arrived). Every issuer i then adds V^T P^T of dimension block i
+      // to O^T block i (8 steps of 16 keys). Each chain stays on one accumulator.
+      const int bi = warp - 1;
+      if (lane == 0) {
+        uint32_t g = 0, qi = 0;
+        bool ok = true;
+        const uint32_t q_base = tc::smem_u32(smem + kOffQ);
+        const uint32_t pairs = tc::smem_u32(smem + kOffPair);
+        const uint64_t p_desc = tc::desc_sw128(tc::smem_u32(smem + kOffP), 0, 1024);
+        const uint32_t s_acc = tmem + kColS + 64 * bi, o_acc = tmem + kColO + 64 * bi;
+        const bool qk = bi < kQkChains;
+        for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+          const Row w = locate_item<kSplit>(a, it);
+          if (w.j0 == w.j1) continue;
+          if (qk) ok = tc::mbar_wait(&bar[kQFull], qi & 1, status);
+          for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
+            const bool first = j == w.j0, last = j == w.j1 - 1;
+            if (qk) {
+              // ---- S^T partial bi over dimension blocks 2 bi and 2 bi + 1
+              if (g > 0) ok = tc::mbar_wait(&bar[kSEmpty], (g - 1) & 1, status);
+              for (int h = 0; h < 2 && ok; ++h) {
+                const int pb = 2 * bi + h;
+                ok = tc::mbar_wait(&bar[kPairFull0 + pb], g & 1, status);
+                if (!ok) break;
+                tc::tc_fence_after();
+  #pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  // the rope slice of Q (K-steps 28..31, the last block) is rotated in place before
+                  // the row's first tile reads it
+                  if (first && 8 * pb + kk == kRopeStep) {
+                    ok = tc::mbar_wait(&bar[kQReady], qi & 1, status);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                  }
+                  const uint32_t off =
+                      (uint32_t)(pb * kPairBytes + (kk >> 2) * kRegion + (kk & 3) * 32);
+                  const uint32_t qoff = (uint32_t)((2 * pb + (kk >> 2)) * kQRegion + (kk & 3) * 32);
+                  tc::mma_bf16_ss(s_acc, tc::desc_sw128(pairs + off, 0, 1024),
+                                  tc::desc_sw128(q_base + qoff, 0, 1024), kIdescQK,
+                                  (h > 0 || kk > 0) ? 1u : 0u);
+                }
+              }
+              if (!ok) break;
+              tc::mma_commit(&bar[kSFull]);
+              if (last) tc::mma_commit(&bar[kQEmpty]);
+            }
+            // ---- O^T block bi += V^T P^T once the softmax has written P (block bi has arrived:
+            // this wait names the phase the S chains already saw complete)
+            ok = tc::mbar_wait(&bar[kPFull], g & 1, status);
+            if (ok) ok = tc::mbar_wait(&bar[kPairFull0 + bi], g & 1, status);
+            if (ok && first && qi > 0) ok = tc::mbar_wait(&bar[kOEmpty], (qi - 1) & 1, status);
+            if (!ok) break;
+            tc::tc_fence_after();
+            const uint32_t pair = pairs + bi * kPairBytes;
+  #pragma unroll
+            for (int kk = 0; kk < kNK / 16; ++kk)
+              tc::mma_bf16_ss(o_acc, tc::desc_sw128(pair + kk * 2048, kRegion, 1024),
+                              p_desc + (uint64_t)(kk * 2048 >> 4), kIdescPV,
+                              (first && kk == 0) ? 0u : 1u);
+            tc::mma_commit(&bar[kPairEmpty0 + bi]);
+            if (last) tc::mma_commit(&bar[kOFull]);
+          }
+          ++qi;
+        }
+      }
+      __syncwarp();
+    } else if (warp == kIssuers + 1) {
+      // ------------------------------------------------------------------ query rotation
+      // Lane p first writes (cos, sin) of rope pair p at the query's position to a shared table.
+      // Then thread i turns the rope pairs of head rows i and i+32 of the staged query tile (row h's
+      // 16-byte chunk c of a 128-byte region sits at chunk c ^ (h & 7)).
+      const int R = a.rf.R;
+      const int p0 = (kDim - R) >> 1;  // first rotated pair among the 256 channel pairs
+      float2* cs_tab = reinterpret_cast<float2*>(smem + kOffCs);
+      uint32_t qi = 0;
+      bool ok = true;
+      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Row w = locate_item<kSplit>(a, it);
+        if (w.j0 == w.j1) continue;
+        if (lane < R / 2) {
+          float c, sn;
+          rope_cos_sin(a.rf, lane, a.pos0 + w.t, c, sn);
+          cs_tab[lane] = make_float2(c, sn);
+        }
+        __syncwarp();
+        ok = __all_sync(~0u, tc::mbar_wait(&bar[kQFull], qi & 1, status));
+        if (!ok) break;
+        if ((R & 7) == 0) {
+          constexpr int kMaxChunks = 8;  // R <= 64: at most 8 chunks of 4 pairs
+          const int nch = R >> 3;
+  #pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int h = hh * 32 + lane;
+            uint8_t* row = smem + kOffQ + h * 128;
+            uint4 v[kMaxChunks];
+  #pragma unroll
+            for (int c = 0; c < kMaxChunks; ++c) {
+              const int pp = p0 + 4 * c;
+              if (c < nch)
+                v[c] = *reinterpret_cast<const uint4*>(row + (pp >> 5) * kQRegion +
+                                                       ((((pp & 31) >> 2) ^ (h & 7)) << 4));
+            }
+  #pragma unroll
+            for (int c = 0; c < kMaxChunks; ++c) {
+              if (c >= nch) break;
+              const int pp = p0 + 4 * c;
+              const float4 cs01 = *reinterpret_cast<const float4*>(cs_tab + 4 * c);
+              const float4 cs23 = *reinterpret_cast<const float4*>(cs_tab + 4 * c + 2);
+              const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+              const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+              uint32_t* w4 = reinterpret_cast<uint32_t*>(&v[c]);
+  #pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 x = unpack_bf16(w4[u]);
+                w4[u] = pack_bf16(x.x * cc[u] - x.y * ss[u], x.x * ss[u] + x.y * cc[u]);
+              }
+              *reinterpret_cast<uint4*>(row + (pp >> 5) * kQRegion +
+                                        ((((pp & 31) >> 2) ^ (h & 7)) << 4)) = v[c];
+            }
+          }
+        } else {
+          for (int hh = 0; hh < 2; ++hh) {
+            const int h = hh * 32 + lane;
+            uint8_t* row = smem + kOffQ + h * 128;
+            for (int q = p0; q < kDim / 2; ++q) {
+              uint32_t* word = reinterpret_cast<uint32_t*>(
+                  row + (q >> 5) * kQRegion + ((((q & 31) >> 2) ^ (h & 7)) << 4) + (q & 3) * 4);
+              const float2 cs = cs_tab[q - p0];
+              const float2 x = unpack_bf16(*word);
+              *word = pack_bf16(x.x * cs.x - x.y * cs.y, x.x * cs.y + x.y * cs.x);
+            }
+          }
+        }
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(&bar[kQReady]);
+        ++qi;
+      }
+    } else if (warp == 6 || warp == 7) {
+      if (any_gather)
+        gather_tiles<kSplit>(a, smem, bar, n_items, win_contig, pool_contig, (warp - 6) * 32 + lane,
+                             status);
+    }
   }
-done:
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -834,7 +850,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
   constexpr int64_t kPagedRows = (int64_t(1) << 31) - 1;
   if (a.win.block_table) win_rows = kPagedRows;
   if (a.pool_mode != 0 && a.pool.block_table) pool_rows = kPagedRows;
-  CUtensorMap tq, twb, tpb, twr, tpr;
+  CUtensorMap tq, twb, tpb;
   cudaError_t e = make_tmap_bf16_2d(&tq, a.q, (uint64_t)a.nrows * kHeads, kDim, kDim * 2, 64, 64);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16_2d(&twb, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, kNK, 64);
@@ -843,18 +859,16 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
   e = make_tmap_bf16_2d(&tpb, has_pool ? a.pool.base : a.win.base,
                         (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, kNK, 64);
   if (e != cudaSuccess) return e;
-  // one-row boxes for the four-row gathers (row coordinates are 32-bit)
-  if (win_rows >= (int64_t(1) << 31) || pool_rows >= (int64_t(1) << 31))
-    return cudaErrorInvalidValue;
-  e = make_tmap_bf16_2d(&twr, a.win.base, (uint64_t)win_rows, kDim, kDim * 2, 1, 64);
-  if (e != cudaSuccess) return e;
-  e = make_tmap_bf16_2d(&tpr, has_pool ? a.pool.base : a.win.base,
-                        (uint64_t)(has_pool ? pool_rows : win_rows), kDim, kDim * 2, 1, 64);
-  if (e != cudaSuccess) return e;
   const void* kern = a.splits > 1 ? (const void*)attention_tc_kernel<true>
                                   : (const void*)attention_tc_kernel<false>;
   e = ensure_smem_limit(kern, kSmemBytes);
   if (e != cudaSuccess) return e;
+  // the register split needs the block launched with kRegsLaunch registers a thread: with fewer,
+  // the softmax warpgroups' raise would wait for registers that never come
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -863,9 +877,9 @@ cudaError_t launch_attention_tc(const AttnArgs& a, int64_t win_rows, int64_t poo
   const int64_t items = a.nrows * a.splits;
   const int grid = (int)(items < sms ? items : sms);
   if (a.splits > 1)
-    attention_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, twr, tpr, a);
+    attention_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
   else
-    attention_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, twr, tpr, a);
+    attention_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(tq, twb, tpb, a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.splits == 1) return e;
   attention_combine_kernel<<<dim3((unsigned)a.nrows, kHeads / kCombineHeads), 256, 0, st>>>(a);
