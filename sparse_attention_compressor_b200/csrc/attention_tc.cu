@@ -49,6 +49,7 @@ constexpr int kHeads = 64;
 constexpr int kDim = 512;
 constexpr int kNK = 128;                         // keys per tile (MMA M of S^T)
 constexpr int kPairs = kDim / 128;               // dimension blocks of a key tile
+static_assert(kPairs == 4, "the gather hands over four commit groups");
 constexpr int kRegion = kNK * 128;               // 16 KB: 128 keys x 64 channels, 128-B rows
 constexpr int kPairBytes = 2 * kRegion;          // 32 KB: one dimension block
 constexpr int kQRegion = kHeads * 128;           // 8 KB: 64 heads x 64 channels
@@ -67,7 +68,8 @@ static_assert(2 * 128 * kRegsSoftmax + 2 * 128 * kRegsOther + 128 * kRegsGather 
 constexpr int kIssuers = kPairs;                 // MMA issuer threads, one per dimension block
 constexpr int kSoftmaxWarp0 = 8;                 // warps 8-15: softmax and output
 constexpr int kSoftmaxThreads = 256;
-constexpr int kQkChains = 2;                     // S^T partial accumulators
+constexpr int kQkChains = 2;                     // S^T partial accumulators (2 or 4)
+static_assert(kQkChains == 2 || kQkChains == 4, "S^T partials: two or four chains");
 
 constexpr int kOffQ = 0;
 constexpr int kOffPair = kOffQ + kQBytes;
@@ -227,8 +229,8 @@ __device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const
 // The gather group: 192 threads (warps 6-7 and 16-19; gt = the thread's index in the group) fill
 // the tiles whose rows are not consecutive. Thread gt copies 16-byte slot gt % 8 of key rows
 // gt / 8 + 24 i of both 64-channel regions of a dimension block, so a warp instruction reads four
-// whole 128-byte row segments. Blocks are issued in order as soon as each is free; a block is
-// handed over (wait_group) once the next block's copies are in flight. The pair barriers count
+// whole 128-byte row segments. Blocks are issued in order as soon as each is free and handed over
+// in order as their copies land. The pair barriers count
 // this group's threads for every tile, so it also arrives for tiles that TMA fills (after the same
 // wait for the block to be free): each party waits for every phase, so no parity wait can name a
 // phase other than the one it means.
@@ -236,7 +238,7 @@ template <bool kSplit>
 __device__ __forceinline__ void gather_tiles(const AttnArgs& a, uint8_t* smem, uint64_t* bar,
                                              int64_t n_items, bool win_contig, bool pool_contig,
                                              int gt, int* status) {
-    const int row0 = gt >> 3, slot = gt & 7;
+  const int row0 = gt >> 3, slot = gt & 7;
   constexpr int kRowStride = kGroupThreads / 8;                     // 24
   constexpr int kRowsPer = (kNK + kRowStride - 1) / kRowStride;     // 6 (the last only row0 < 8)
   uint32_t g = 0;
@@ -248,13 +250,13 @@ __device__ __forceinline__ void gather_tiles(const AttnArgs& a, uint8_t* smem, u
       const bool gath = !(j < w.twin ? win_contig : pool_contig);
       const __nv_bfloat16* src[kRowsPer];
       if (gath) {
-  #pragma unroll
+#pragma unroll
         for (int i = 0; i < kRowsPer; ++i) {
           const int row = row0 + kRowStride * i;
           src[i] = key_ptr(a, w, j, row < kNK ? row : 0);
         }
       }
-  #pragma unroll
+#pragma unroll
       for (int b = 0; b < kPairs; ++b) {
         if (g > 0) ok = __all_sync(~0u, tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status));
         if (!ok) break;
@@ -263,7 +265,7 @@ __device__ __forceinline__ void gather_tiles(const AttnArgs& a, uint8_t* smem, u
           continue;
         }
         uint8_t* pr = smem + kOffPair + b * kPairBytes;
-  #pragma unroll
+#pragma unroll
         for (int i = 0; i < kRowsPer; ++i) {
           const int row = row0 + kRowStride * i;
           if (row < kNK) {
@@ -273,16 +275,22 @@ __device__ __forceinline__ void gather_tiles(const AttnArgs& a, uint8_t* smem, u
           }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
-        if (b > 0) {  // the previous block's copies have landed: hand it over
-          asm volatile("cp.async.wait_group 1;" ::: "memory");
-          tc::fence_proxy_async_smem();
-          tc::mbar_arrive(&bar[kPairFull0 + b - 1]);
-        }
       }
       if (!ok || !gath) continue;
+      // the four blocks' copies are all in flight (one commit group each, so the latency of the
+      // loads is paid once per tile): hand each block over as its group lands, in order
+      asm volatile("cp.async.wait_group 3;" ::: "memory");
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[kPairFull0 + 0]);
+      asm volatile("cp.async.wait_group 2;" ::: "memory");
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[kPairFull0 + 1]);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[kPairFull0 + 2]);
       asm volatile("cp.async.wait_group 0;" ::: "memory");
       tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bar[kPairFull0 + kPairs - 1]);
+      tc::mbar_arrive(&bar[kPairFull0 + 3]);
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -374,16 +382,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         const bool valid = key < tile_keys(w, j);
         float x[32];
-        {
+#pragma unroll
+        for (int c = 0; c < kQkChains; c += 2) {  // the partials of S^T, two per TMEM round trip
           uint32_t va[32], vb[32];
-          tc::tmem_ld32(t_lane + kColS + h0, va);
-          tc::tmem_ld32(t_lane + kColS + 64 + h0, vb);
+          tc::tmem_ld32(t_lane + kColS + 64 * c + h0, va);
+          tc::tmem_ld32(t_lane + kColS + 64 * (c + 1) + h0, vb);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            x[e] = valid ? (__uint_as_float(va[e]) + __uint_as_float(vb[e])) * scale_log2
-                         : -INFINITY;
+          for (int e = 0; e < 32; ++e) {
+            const float v = __uint_as_float(va[e]) + __uint_as_float(vb[e]);
+            x[e] = c == 0 ? v : x[e] + v;
+          }
         }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = valid ? x[e] * scale_log2 : -INFINITY;
         tc::tc_fence_before();
         tc::mbar_arrive(&bar[kSEmpty]);
         // The running max: on a row's first tile it is set from the exact per-head tile max (the
@@ -627,8 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (qk) {
               // ---- S^T partial bi over dimension blocks 2 bi and 2 bi + 1
               if (g > 0) ok = tc::mbar_wait(&bar[kSEmpty], (g - 1) & 1, status);
-              for (int h = 0; h < 2 && ok; ++h) {
-                const int pb = 2 * bi + h;
+              for (int h = 0; h < kPairs / kQkChains && ok; ++h) {
+                const int pb = (kPairs / kQkChains) * bi + h;
                 ok = tc::mbar_wait(&bar[kPairFull0 + pb], g & 1, status);
                 if (!ok) break;
                 tc::tc_fence_after();
