@@ -297,6 +297,7 @@ KERNEL_SOURCES = {
     "topk": ["topk.cu", "sac_common.cuh"],
     "compress": ["compress.cu", "pool_window.cuh", "tc_ptx.cuh", "sac_common.cuh"],
     "compress_index": ["compress.cu", "pool_window.cuh", "tc_ptx.cuh", "sac_common.cuh"],
+    "rotate_kv": ["compress.cu", "pool_window.cuh", "tc_ptx.cuh", "sac_common.cuh"],
     "decode_append": ["decode_append.cu", "pool_window.cuh", "sac_common.cuh"],
     "o_proj": ["oproj.cu", "tc_ptx.cuh"],
 }
@@ -343,17 +344,32 @@ def record_traffic(raw_csv: str, workload: str, kernel: str, name_regex: str, su
         rows = [r for r in csv.reader(f)]
     # ncu prints its own log lines before the table: the header row names the kernel column
     start = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
-    head, units, data = rows[start], rows[start + 1], rows[start + 2:]
+    head = rows[start]
     ik = head.index("Kernel Name")
     per = []
-    for r in data:
-        if len(r) != len(head) or not re.search(name_regex, r[ik]):
-            continue
-        tot = 0.0
-        for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
-            i = head.index(m)
-            tot += float(r[i].replace(",", "")) * to_bytes[units[i]]
-        per.append(tot)
+    if "Metric Name" in head:
+        # `--metrics ... --csv` launch list: one row per (launch ID, metric)
+        iid, im = head.index("ID"), head.index("Metric Name")
+        iu, iv = head.index("Metric Unit"), head.index("Metric Value")
+        by_launch = {}
+        for r in rows[start + 1:]:
+            if len(r) != len(head) or not re.search(name_regex, r[ik]):
+                continue
+            if r[im] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+                by_launch.setdefault(r[iid], 0.0)
+                by_launch[r[iid]] += float(r[iv].replace(",", "")) * to_bytes[r[iu]]
+        per = list(by_launch.values())
+    else:
+        # raw page: one row per launch, one column per metric, units in the second row
+        units, data = rows[start + 1], rows[start + 2:]
+        for r in data:
+            if len(r) != len(head) or not re.search(name_regex, r[ik]):
+                continue
+            tot = 0.0
+            for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+                i = head.index(m)
+                tot += float(r[i].replace(",", "")) * to_bytes[units[i]]
+            per.append(tot)
     if not per:
         raise SystemExit(f"no launch of {name_regex!r} in {raw_csv}")
     rec = {"workload": workload, "kernel": kernel,

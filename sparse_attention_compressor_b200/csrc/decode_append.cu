@@ -85,7 +85,8 @@ __device__ __forceinline__ void append_warp(const AppendPart& a, int seq, int la
   float u[V], acc[V];
   load_lane<T, V>(reinterpret_cast<const T*>(a.gate), lane, u);
   const int L = a.L;
-  pool_window<T, V, 1, 4>([&](int64_t j) { return j == t ? x_new : ring + (j % L) * C; }, u,
+  pool_window<T, V, 1, rows_in_flight<T, V>(64)>(
+      [&](int64_t j) { return j == t ? x_new : ring + (j % L) * C; }, u,
                           a.bias, lo, hi, L, true, 0, lane, sh, acc);
   T* dst = page_row<T>(a.pool_pages, a.pool_bt, a.pool_max_pages, a.page_size, C, seq, w);
   if (dst == nullptr) return;
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendPart a) {
   float u[V], acc[V];
   load_lane<T, V>(reinterpret_cast<const T*>(a.gate), lane, u);
   const int L = a.L;
-  pool_window<T, V, WPE, 4>(
+  pool_window<T, V, WPE, rows_in_flight<T, V>(64)>(
       [&](int64_t j) { return j == t ? x_new : ring + (j % L) * C; }, u, a.bias, lo, hi, L,
       WPE > 1 || warp == 0, warp, lane, sh, acc);
   if (warp != 0) return;

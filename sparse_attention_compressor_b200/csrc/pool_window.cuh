@@ -63,6 +63,55 @@ __device__ __forceinline__ void rotate_lane(float (&v)[V], int lane, int C, cons
   }
 }
 
+// A lane's V elements of a row kept as loaded (packed), so a batch of rows in flight costs
+// V * sizeof(T) / 4 registers a row instead of V.
+template <typename T, int V>
+struct RawLane {
+  static constexpr int kBytes = V * (int)sizeof(T);
+  static constexpr int kWords = (kBytes + 3) / 4;
+  uint32_t w[kWords];
+};
+// Rows a lane can keep in flight within about `regs` registers (1 to 16).
+template <typename T, int V>
+__host__ __device__ constexpr int rows_in_flight(int regs) {
+  const int n = regs / RawLane<T, V>::kWords;
+  return n < 1 ? 1 : (n > 16 ? 16 : n);
+}
+template <typename T, int V>
+__device__ __forceinline__ void load_lane_raw(const T* row, int lane, RawLane<T, V>& r) {
+  constexpr int kBytes = RawLane<T, V>::kBytes;
+  const T* src = row + lane * V;
+  if constexpr (kBytes % 16 == 0) {
+    const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int i = 0; i < kBytes / 16; ++i) {
+      const uint4 u = __ldg(p + i);
+      r.w[4 * i] = u.x;
+      r.w[4 * i + 1] = u.y;
+      r.w[4 * i + 2] = u.z;
+      r.w[4 * i + 3] = u.w;
+    }
+  } else if constexpr (kBytes % 8 == 0) {
+    const uint2* p = reinterpret_cast<const uint2*>(src);
+#pragma unroll
+    for (int i = 0; i < kBytes / 8; ++i) {
+      const uint2 u = __ldg(p + i);
+      r.w[2 * i] = u.x;
+      r.w[2 * i + 1] = u.y;
+    }
+  } else {
+    T* e = reinterpret_cast<T*>(r.w);
+#pragma unroll
+    for (int i = 0; i < V; ++i) e[i] = src[i];
+  }
+}
+template <typename T, int V>
+__device__ __forceinline__ void unpack_lane(const RawLane<T, V>& r, float (&v)[V]) {
+  const T* e = reinterpret_cast<const T*>(r.w);
+#pragma unroll
+  for (int i = 0; i < V; ++i) v[i] = to_f<T>(e[i]);
+}
+
 // Shared memory of pool_window for a block of 8 warps.
 template <int V, int WPE>
 struct PoolShared {
@@ -86,22 +135,24 @@ __device__ __forceinline__ void pool_window(RowFn row, const float (&u)[V], cons
     // rows in batches of kBatch: all loads of a batch are issued before any is used, so a
     // window costs ceil(rows / kBatch) memory latencies instead of one per row
     for (int64_t j0 = lo + sub; j0 < hi; j0 += kBatch * WPE) {
-      float xv[kBatch][V];
+      RawLane<T, V> raw[kBatch];
       float bb[kBatch];
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {
         const int64_t j = j0 + (int64_t)k * WPE;
         if (j < hi) {
-          load_lane<T, V>(row(j), lane, xv[k]);
+          load_lane_raw<T, V>(row(j), lane, raw[k]);
           bb[k] = __ldg(bias + (j - hi + L));
         }
       }
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {
         if (j0 + (int64_t)k * WPE >= hi) break;
+        float xk[V];
+        unpack_lane<T, V>(raw[k], xk);
         float d = 0.f;
 #pragma unroll
-        for (int i = 0; i < V; ++i) d = fmaf(xv[k][i], u[i], d);
+        for (int i = 0; i < V; ++i) d = fmaf(xk[i], u[i], d);
         const float g = warp_sum(d) + bb[k];
         if (g == -INFINITY) continue;
         if (g > M) {
@@ -114,7 +165,7 @@ __device__ __forceinline__ void pool_window(RowFn row, const float (&u)[V], cons
         const float p = __expf(g - M);
         Z += p;
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = fmaf(p, xv[k][i], acc[i]);
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(p, xk[i], acc[i]);
       }
     }
   }

@@ -22,6 +22,7 @@ constexpr int kThreads = 512;       // rows re-read from L2, and long rows with 
 // rows of at most kSmemKeyRows scores: more rows side by side per SM (measured at CSA-8k: 112 us
 // with 512 threads, 87 us with 256, 108 us with 128)
 constexpr int kShortThreads = 256;
+constexpr int kWideThreads = 1024;  // rows with keys in shared memory when there are few of them
 constexpr int kMaxEntries = 1 << 22;  // longest row (pool entries per sequence) accepted
 constexpr int kBins = 4096;          // 12-bit digits
 constexpr int kCandCap = 2048;       // compacted keys of the threshold bin
@@ -37,6 +38,7 @@ __device__ __forceinline__ uint32_t order_key(float s) {
 struct Shared {
   int hist[kBins];
   uint32_t cand[kCandCap];
+  int cand_idx[kCandCap];  // entry index of each compacted key
   int warp_tot[32];  // up to 1024 threads
   int warp_gt[32], warp_eq[32];
   int n_cand;
@@ -157,26 +159,40 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
   const int c1 = sh.hist[d1];
   __syncthreads();  // everyone has read hist before it is cleared
 
-  // ---- compact the keys of digit d1 when they fit; otherwise scan the whole row with a mask
+  // Warp w owns the contiguous segment [w*seg, (w+1)*seg) of the row in the passes below.
+  const int seg = ((n + (NT / 32) * 32 - 1) / ((NT / 32) * 32)) * 32;
+  const int s0 = warp * seg, s1 = min(n, s0 + seg);
+
+  // ---- one pass when the keys of digit d1 fit the candidate list: keys of a higher digit are
+  // all selected (each warp counts its own), those of digit d1 are compacted with their entry
+  // index, the rest are dropped. Then the finer digits and the per-segment counts of the output
+  // need only the candidates, not the row. Otherwise the finer digits scan the whole row.
   const bool compact = c1 <= kCandCap;
+  int above_d1 = 0;
   if (compact) {
-    for (int b0 = warp * 32; b0 < n; b0 += NT * kBatch) {
+    for (int b0 = s0; b0 < s1; b0 += 32 * kBatch) {
       uint32_t kb[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
-        const int i = b0 + u * NT + lane;
-        kb[u] = i < n ? key_at(i) : 0u;
+        const int i = b0 + 32 * u + lane;
+        kb[u] = i < s1 ? key_at(i) : 0u;
       }
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
-        const int i = b0 + u * NT + lane;
-        const bool hit = i < n && (kb[u] >> 20) == d1;
+        const int i = b0 + 32 * u + lane;
+        const uint32_t dg = kb[u] >> 20;
+        above_d1 += __popc(__ballot_sync(~0u, i < s1 && dg > d1));
+        const bool hit = i < s1 && dg == d1;
         const uint32_t mask = __ballot_sync(~0u, hit);
         if (mask) {
           int base = 0;
           if (lane == 0) base = atomicAdd(&sh.n_cand, __popc(mask));
           base = __shfl_sync(~0u, base, 0);
-          if (hit) sh.cand[base + __popc(mask & ((1u << lane) - 1u))] = kb[u];
+          if (hit) {
+            const int slot = base + __popc(mask & ((1u << lane) - 1u));
+            sh.cand[slot] = kb[u];
+            sh.cand_idx[slot] = i;
+          }
         }
       }
     }
@@ -210,27 +226,40 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
   const uint32_t T = (hi24 << 8) | (uint32_t)sh.digit;
   const int take_eq = sh.rem;  // keys equal to T to keep, lowest indices first
 
-  // ---- selection: warp w owns the contiguous segment [w*seg, (w+1)*seg)
-  const int seg = ((n + (NT / 32) * 32 - 1) / ((NT / 32) * 32)) * 32;
-  const int s0 = warp * seg, s1 = min(n, s0 + seg);
-  int gt = 0, eq = 0;
-  for (int b0 = s0; b0 < s1; b0 += 32 * kBatch) {
-    uint32_t kb[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int i = b0 + 32 * u + lane;
-      kb[u] = i < s1 ? key_at(i) : 0u;
+  // ---- selection: per-segment counts of keys > T and == T, then the output in entry order
+  if (compact) {
+    // keys above digit d1 were counted in the pass; the candidates add theirs
+    if (lane == 0) {
+      sh.warp_gt[warp] = above_d1;
+      sh.warp_eq[warp] = 0;
     }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const bool in = b0 + 32 * u + lane < s1;
-      gt += __popc(__ballot_sync(~0u, in && kb[u] > T));
-      eq += __popc(__ballot_sync(~0u, in && kb[u] == T));
+    __syncthreads();
+    for (int c = tid; c < nc; c += NT) {
+      const uint32_t key = sh.cand[c];
+      const int w = sh.cand_idx[c] / seg;
+      if (key > T) atomicAdd(&sh.warp_gt[w], 1);
+      else if (key == T) atomicAdd(&sh.warp_eq[w], 1);
     }
-  }
-  if (lane == 0) {
-    sh.warp_gt[warp] = gt;
-    sh.warp_eq[warp] = eq;
+  } else {
+    int gt = 0, eq = 0;
+    for (int b0 = s0; b0 < s1; b0 += 32 * kBatch) {
+      uint32_t kb[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = b0 + 32 * u + lane;
+        kb[u] = i < s1 ? key_at(i) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const bool in = b0 + 32 * u + lane < s1;
+        gt += __popc(__ballot_sync(~0u, in && kb[u] > T));
+        eq += __popc(__ballot_sync(~0u, in && kb[u] == T));
+      }
+    }
+    if (lane == 0) {
+      sh.warp_gt[warp] = gt;
+      sh.warp_eq[warp] = eq;
+    }
   }
   __syncthreads();
   int eq_before = 0, sel_before = 0;
@@ -284,6 +313,14 @@ cudaError_t launch_topk(const float* scores, int n_stride, QueryRows qr, int m, 
       cudaError_t err = ensure_smem_limit((const void*)topk_kernel<true, kShortThreads>, (int)smem);
       if (err != cudaSuccess) return err;
       topk_kernel<true, kShortThreads><<<(unsigned)nrows, kShortThreads, smem, st>>>(
+          scores, n_stride, qr, m, k, out);
+      return cudaGetLastError();
+    }
+    if (nrows <= sms) {
+      // fewer rows than SMs (decode): 1024 threads a row halve each pass's per-row time
+      cudaError_t err = ensure_smem_limit((const void*)topk_kernel<true, kWideThreads>, (int)smem);
+      if (err != cudaSuccess) return err;
+      topk_kernel<true, kWideThreads><<<(unsigned)nrows, kWideThreads, smem, st>>>(
           scores, n_stride, qr, m, k, out);
       return cudaGetLastError();
     }

@@ -101,3 +101,17 @@ def test_traffic_record_reads_ncu_csv_and_goes_stale(tmp_path, monkeypatch):
     assert bench.ncu_traffic("csa_8k_bf16", "topk") == (None, None)
     monkeypatch.setattr(bench, "source_hash", lambda k: "changed")
     assert bench.ncu_traffic("csa_8k_bf16", "attention") == (None, None)
+
+
+def test_traffic_record_reads_the_metrics_launch_list(tmp_path, monkeypatch):
+    """The `--metrics ... --csv` launch list (one row per launch and metric) gives the same sums."""
+    raw = tmp_path / "list.csv"
+    hdr = '"ID","Kernel Name","Metric Name","Metric Unit","Metric Value"\n'
+    raw.write_text('==PROF== x\n' + hdr +
+                   '"0","attention_tc_kernel<0>","dram__bytes_read.sum","Gbyte","2.5"\n'
+                   '"0","attention_tc_kernel<0>","dram__bytes_write.sum","Mbyte","500"\n'
+                   '"0","attention_tc_kernel<0>","gpu__time_duration.sum","ms","30"\n'
+                   '"1","topk_kernel","dram__bytes_read.sum","Gbyte","9"\n')
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "traffic.json"))
+    rec = bench.record_traffic(str(raw), "csa_128k_bf16", "attention", r"attention_tc", "x.md")
+    assert rec["launches_captured"] == 1 and rec["dram_bytes_per_launch"] == 3.0e9
