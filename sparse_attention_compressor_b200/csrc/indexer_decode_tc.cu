@@ -226,11 +226,15 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
 #pragma unroll
       for (int qi = 0; qi < Q; ++qi) {
         float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+        // the row's 64 head sums in two loads and one wait (one TMEM round trip)
+        uint32_t vv[kNI];
+        tc::tmem_ld32(t_lane + acc * K::kN + qi * kNI, *reinterpret_cast<uint32_t(*)[32]>(vv));
+        tc::tmem_ld32(t_lane + acc * K::kN + qi * kNI + 32,
+                      *reinterpret_cast<uint32_t(*)[32]>(vv + 32));
+        tc::tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < kNI; c += 16) {
-          uint32_t v[16];
-          tc::tmem_ld16(t_lane + acc * K::kN + qi * kNI + c, v);
-          tc::tmem_wait_ld();
+          const uint32_t* v = vv + c;
 #pragma unroll
           for (int u = 0; u < 16; u += 4) {
             const float4 wv = w4[(qi * kNI + c + u) / 4];
