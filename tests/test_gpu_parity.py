@@ -126,6 +126,25 @@ def test_topk_all_scores_equal():
         assert np.array_equal(g["topk"][0, t].numpy(), expect), t
 
 
+@pytest.mark.parametrize("S", [8448, 33024])
+def test_topk_ties_beyond_candidate_capacity(S):
+    # All scores equal (q_idx = 0), on rows long enough that the threshold digit holds more keys
+    # than the candidate list (2048): the top-k takes its whole-row fallback. S = 8448 keeps each
+    # row's keys in shared memory (2112 entries), S = 33024 re-reads them from L2 (8256 entries).
+    # Each row must keep its k lowest visible entries, in order.
+    wl = wl_small("csa", "bf16", S=S, H=8, D=128, R=32, nI=64, cI=128, k=512, W=128,
+                  theta=160000.0, seed=21)
+    x = W.prefill_inputs(wl)
+    x["q_idx"] = torch.zeros_like(x["q_idx"])
+    g = gpu_prefill(wl, x, with_aux=False)
+    sel = g["topk"][0].numpy()
+    for t in list(range(0, S, 97)) + list(range(S - 64, S)):
+        nvis = (t + 1) // wl.m
+        expect = np.arange(wl.k) if nvis >= wl.k else np.concatenate(
+            [np.arange(nvis), -np.ones(wl.k - nvis, dtype=np.int64)])
+        assert np.array_equal(sel[t], expect), t
+
+
 def test_relative_position_invariance_on_gpu():
     wl = SMALL[1][1]
     x = W.prefill_inputs(wl)
