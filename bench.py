@@ -861,6 +861,8 @@ def run_decode(args, wl0):
         "roofline": roof_of(wl.name, dom, d, peaks),
         "kernels": krows,
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = inline_cpu_baseline(run_reference_paged, wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -929,6 +931,8 @@ def run_oproj(args, wl0):
                                                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                                  "frac": ach / peaks["bf16_tflops"]}, peaks),
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = inline_cpu_baseline(run_reference_oproj, wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -1047,6 +1051,16 @@ def run_reference_oproj(args, wl):
     s = sum(times) / len(times)
     return ("grouped output projection tokens/s", per / s, "tokens/s", True, s * 1e3,
             oracle.max_threads(), f"each step: {per} random token rows of {T}")
+
+
+def inline_cpu_baseline(fn, wl) -> dict:
+    """The oracle arm of a decode, chunked-prefill or projection workload on a small sample (one
+    warm-up and two timed steps), as the bench line's cpu_baseline."""
+    class _A:
+        warmup, steps = 1, 2
+    _, value, unit, _, _, threads, sample = fn(_A, wl)
+    return {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample,
+            "cpu_model": cpu_model()}
 
 
 def run_reference(args, wl):
