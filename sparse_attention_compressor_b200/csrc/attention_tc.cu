@@ -210,20 +210,48 @@ __device__ __forceinline__ bool softmax_wait(uint64_t* bar, uint32_t parity, int
   return !bar_any_softmax(!tc::mbar_wait(bar, parity, status));
 }
 
-// Global address of key c of tile j (keys past the tile's count reuse a valid row: masked).
-__device__ __forceinline__ const __nv_bfloat16* key_ptr(const AttnArgs& a, const Row& w, int j,
-                                                        int c) {
-  if (j < w.twin) {
-    int x = j * kNK + c;
-    if (x >= w.nwin) x = 0;
-    const __nv_bfloat16* p = a.win.row<__nv_bfloat16>(w.seq, w.lo + x);
-    return p ? p : a.win.row<__nv_bfloat16>(w.seq, w.lo);
+// Global addresses of keys c0 + stride * i (i < N) of tile j. Keys past the tile's count reuse a
+// valid row (the softmax masks them); an unallocated page reads its buffer's first row. Each level
+// of index loads (the CSA selection, then the block table) is issued for all N keys before any is
+// used, so a tile's addresses cost two memory latencies at most, not two per key.
+template <int N>
+__device__ __forceinline__ void key_ptrs(const AttnArgs& a, const Row& w, int j, int c0,
+                                         int stride, const __nv_bfloat16* (&src)[N]) {
+  const bool is_win = j < w.twin;
+  uint32_t lr[N];  // row of the key in its sequence's stream (window row or pool entry)
+  if (is_win) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      int x = j * kNK + min(c0 + stride * i, kNK - 1);
+      if (x >= w.nwin) x = 0;
+      lr[i] = (uint32_t)(w.lo + x);
+    }
+  } else {
+    int e[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      int x = (j - w.twin) * kNK + min(c0 + stride * i, kNK - 1);
+      if (x >= w.npool) x = 0;
+      e[i] = a.pool_mode == 2 ? __ldg(a.sel + w.r * a.k + x) : x;
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) lr[i] = (uint32_t)(e[i] < 0 ? 0 : e[i]);
   }
-  int i = (j - w.twin) * kNK + c;
-  if (i >= w.npool) i = 0;
-  int64_t e = a.pool_mode == 2 ? (int64_t)__ldg(a.sel + w.r * a.k + i) : i;
-  const __nv_bfloat16* p = a.pool.row<__nv_bfloat16>(w.seq, e < 0 ? 0 : e);
-  return p ? p : reinterpret_cast<const __nv_bfloat16*>(a.pool.base);
+  const RowAddr& ra = is_win ? a.win : a.pool;
+  const __nv_bfloat16* base = reinterpret_cast<const __nv_bfloat16*>(ra.base);
+  if (ra.block_table == nullptr) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) src[i] = base + ((int64_t)w.seq * ra.seq_stride + lr[i]) * kDim;
+    return;
+  }
+  const uint32_t ps = (uint32_t)ra.page_size;
+  const int32_t* bt = ra.block_table + (int64_t)w.seq * ra.max_pages;
+  int pg[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) pg[i] = __ldg(bt + lr[i] / ps);
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    src[i] = pg[i] < 0 ? base : base + ((int64_t)pg[i] * ps + lr[i] % ps) * kDim;
 }
 
 // The gather group: 192 threads (warps 6-7 and 16-19; gt = the thread's index in the group) fill
@@ -249,13 +277,7 @@ __device__ __forceinline__ void gather_tiles(const AttnArgs& a, uint8_t* smem, u
     for (int j = w.j0; j < w.j1 && ok; ++j, ++g) {
       const bool gath = !(j < w.twin ? win_contig : pool_contig);
       const __nv_bfloat16* src[kRowsPer];
-      if (gath) {
-#pragma unroll
-        for (int i = 0; i < kRowsPer; ++i) {
-          const int row = row0 + kRowStride * i;
-          src[i] = key_ptr(a, w, j, row < kNK ? row : 0);
-        }
-      }
+      if (gath) key_ptrs<kRowsPer>(a, w, j, row0, kRowStride, src);
 #pragma unroll
       for (int b = 0; b < kPairs; ++b) {
         if (g > 0) ok = __all_sync(~0u, tc::mbar_wait(&bar[kPairEmpty0 + b], (g - 1) & 1, status));

@@ -123,10 +123,11 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
   const int gc = g & 15, gr = g >> 4;
   auto row_ptr = [&](int64_t e) -> const __nv_bfloat16* {
     if (e >= e_end) return nullptr;
-    const int64_t page = __ldg(a.kpool.block_table + (int64_t)seq * a.kpool.max_pages +
-                               e / a.kpool.page_size);
+    // entry numbers fit 32 bits: 32-bit division by the page size
+    const uint32_t ue = (uint32_t)e, ps = (uint32_t)a.kpool.page_size;
+    const int64_t page = __ldg(a.kpool.block_table + (int64_t)seq * a.kpool.max_pages + ue / ps);
     if (page < 0) return nullptr;
-    return pool + (page * a.kpool.page_size + e % a.kpool.page_size) * kCI;
+    return pool + (page * ps + ue % ps) * kCI;
   };
   auto issue_block = [&](int kb, const __nv_bfloat16* my_row) {
     uint8_t* dst = smem + kOffKv + (kb % kStages) * kBlockBytes;
