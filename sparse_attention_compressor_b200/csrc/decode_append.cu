@@ -53,9 +53,10 @@ __device__ __forceinline__ int64_t checked_ctx(const AppendPart& a, int seq) {
 template <typename T>
 __device__ __forceinline__ T* page_row(void* base, const int32_t* bt, int max_pages, int page_size,
                                        int C, int seq, int64_t j) {
-  const int page = __ldg(bt + (int64_t)seq * max_pages + j / page_size);
+  const uint32_t uj = (uint32_t)j, ps = (uint32_t)page_size;  // rows of a sequence fit 32 bits
+  const int page = __ldg(bt + (int64_t)seq * max_pages + uj / ps);
   if (page < 0) return nullptr;
-  return reinterpret_cast<T*>(base) + ((int64_t)page * page_size + j % page_size) * C;
+  return reinterpret_cast<T*>(base) + ((int64_t)page * ps + uj % ps) * C;
 }
 
 // One warp's append of sequence seq when a single warp pools a window (L < 64): the new row to
@@ -64,12 +65,13 @@ template <typename T, int V>
 __device__ __forceinline__ void append_warp(const AppendPart& a, int seq, int lane,
                                             PoolShared<V, 1>& sh) {
   constexpr int C = 32 * V;
-  const int64_t t = checked_ctx(a, seq) - 1;
-  if (t < 0) return;
+  // the new row does not depend on the context length: its load goes out with ctx's
   const T* x_new = reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * C;
-  T* ring = a.m > 0 ? reinterpret_cast<T*>(a.ring) + (int64_t)seq * a.L * C : nullptr;
   float v[V];
   load_lane<T, V>(x_new, lane, v);
+  const int64_t t = checked_ctx(a, seq) - 1;
+  if (t < 0) return;
+  T* ring = a.m > 0 ? reinterpret_cast<T*>(a.ring) + (int64_t)seq * a.L * C : nullptr;
   if (ring) store_lane<T, V>(ring + (t % a.L) * C, lane, v);
   if (a.kv_pages) {
     T* dst = page_row<T>(a.kv_pages, a.kv_bt, a.kv_max_pages, a.page_size, C, seq, t);
@@ -84,11 +86,12 @@ __device__ __forceinline__ void append_warp(const AppendPart& a, int seq, int la
   const int64_t lo = hi - a.L < 0 ? 0 : hi - a.L;
   float u[V], acc[V];
   load_lane<T, V>(reinterpret_cast<const T*>(a.gate), lane, u);
+  // the entry's page is looked up before the pooling, so its load overlaps the rows'
+  T* dst = page_row<T>(a.pool_pages, a.pool_bt, a.pool_max_pages, a.page_size, C, seq, w);
   const int L = a.L;
   pool_window<T, V, 1, rows_in_flight<T, V>(64)>(
       [&](int64_t j) { return j == t ? x_new : ring + (j % L) * C; }, u,
                           a.bias, lo, hi, L, true, 0, lane, sh, acc);
-  T* dst = page_row<T>(a.pool_pages, a.pool_bt, a.pool_max_pages, a.page_size, C, seq, w);
   if (dst == nullptr) return;
   if (a.rotate) rotate_lane<V>(acc, lane, C, a.rf, a.pos0 + w * a.m);
   store_lane<T, V>(dst, lane, acc);
@@ -114,14 +117,15 @@ __global__ void __launch_bounds__(256) append_kernel(AppendPart a) {
   __shared__ PoolShared<V, WPE> sh;
   const int seq = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the new row does not depend on the context length: its load goes out with ctx's
+  const T* x_new = reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * C;
+  float v[V];
+  if (warp == 0) load_lane<T, V>(x_new, lane, v);
   const int64_t t = checked_ctx(a, seq) - 1;
   if (t < 0) return;
-  const T* x_new = reinterpret_cast<const T*>(a.x_new) + (int64_t)seq * C;
   T* ring = a.m > 0 ? reinterpret_cast<T*>(a.ring) + (int64_t)seq * a.L * C : nullptr;
   const bool closing = a.m > 0 && (t + 1) % a.m == 0;
   if (warp == 0) {
-    float v[V];
-    load_lane<T, V>(x_new, lane, v);
     if (ring) store_lane<T, V>(ring + (t % a.L) * C, lane, v);
     if (a.kv_pages) {
       T* dst = page_row<T>(a.kv_pages, a.kv_bt, a.kv_max_pages, a.page_size, C, seq, t);
@@ -141,12 +145,15 @@ __global__ void __launch_bounds__(256) append_kernel(AppendPart a) {
   const int64_t lo = hi - a.L < 0 ? 0 : hi - a.L;
   float u[V], acc[V];
   load_lane<T, V>(reinterpret_cast<const T*>(a.gate), lane, u);
+  // the entry's page is looked up before the pooling, so its load overlaps the rows'
+  T* dst = warp == 0 ? page_row<T>(a.pool_pages, a.pool_bt, a.pool_max_pages, a.page_size, C,
+                                   seq, w)
+                     : nullptr;
   const int L = a.L;
   pool_window<T, V, WPE, rows_in_flight<T, V>(64)>(
       [&](int64_t j) { return j == t ? x_new : ring + (j % L) * C; }, u, a.bias, lo, hi, L,
       WPE > 1 || warp == 0, warp, lane, sh, acc);
   if (warp != 0) return;
-  T* dst = page_row<T>(a.pool_pages, a.pool_bt, a.pool_max_pages, a.page_size, C, seq, w);
   if (dst == nullptr) return;
   if (a.rotate) rotate_lane<V>(acc, lane, C, a.rf, a.pos0 + w * a.m);
   store_lane<T, V>(dst, lane, acc);
