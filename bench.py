@@ -293,7 +293,8 @@ KERNEL_SOURCES = {
     "attention": ["attention_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
     "csa_decode_attention": ["attention_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
     "hca_decode_attention": ["attention_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
-    "indexer_score": ["indexer_tc.cu", "indexer_decode_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
+    # the prefill indexer; decode and chunked prefill run indexer_decode_tc.cu (below)
+    "indexer_score": ["indexer_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
     "topk": ["topk.cu", "sac_common.cuh"],
     "compress": ["compress.cu", "pool_window.cuh", "tc_ptx.cuh", "sac_common.cuh"],
     "compress_index": ["compress.cu", "pool_window.cuh", "tc_ptx.cuh", "sac_common.cuh"],
@@ -301,13 +302,20 @@ KERNEL_SOURCES = {
     "decode_append": ["decode_append.cu", "pool_window.cuh", "sac_common.cuh"],
     "o_proj": ["oproj.cu", "tc_ptx.cuh"],
 }
+# kernels whose source differs for the paged (decode / chunked-prefill) workloads
+PAGED_SOURCES = {
+    "indexer_score": ["indexer_decode_tc.cu", "tc_ptx.cuh", "sac_common.cuh"],
+}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 
 
-def source_hash(kernel: str) -> str:
+def source_hash(kernel: str, workload: str = "") -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES.get(kernel, []):
+    paged = workload in W.WORKLOADS and W.WORKLOADS[workload].kind == "decode"
+    files = PAGED_SOURCES.get(kernel) if paged and kernel in PAGED_SOURCES else \
+        KERNEL_SOURCES.get(kernel, [])
+    for f in files:
         path = os.path.join(CSRC, f)
         if os.path.exists(path):
             with open(path, "rb") as fh:
@@ -324,7 +332,7 @@ def ncu_traffic(workload: str, kernel: str):
         recs = json.load(f)
     for r in recs:
         if r["workload"] == workload and r["kernel"] == kernel and \
-                r["source_sha256"] == source_hash(kernel):
+                r["source_sha256"] == source_hash(kernel, workload):
             return float(r["dram_bytes_per_launch"]), r
     return None, None
 
@@ -374,7 +382,7 @@ def record_traffic(raw_csv: str, workload: str, kernel: str, name_regex: str, su
         raise SystemExit(f"no launch of {name_regex!r} in {raw_csv}")
     rec = {"workload": workload, "kernel": kernel,
            "dram_bytes_per_launch": sum(per) / len(per) * scale,
-           "launches_captured": len(per), "source_sha256": source_hash(kernel),
+           "launches_captured": len(per), "source_sha256": source_hash(kernel, workload),
            "summary": summary}
     if scaled_from:
         rec["scaled_from"] = scaled_from

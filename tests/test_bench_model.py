@@ -99,7 +99,7 @@ def test_traffic_record_reads_ncu_csv_and_goes_stale(tmp_path, monkeypatch):
     t, r = bench.ncu_traffic("csa_8k_bf16", "attention")
     assert t == rec["dram_bytes_per_launch"] and r["scaled_from"] == "x2"
     assert bench.ncu_traffic("csa_8k_bf16", "topk") == (None, None)
-    monkeypatch.setattr(bench, "source_hash", lambda k: "changed")
+    monkeypatch.setattr(bench, "source_hash", lambda k, w="": "changed")
     assert bench.ncu_traffic("csa_8k_bf16", "attention") == (None, None)
 
 
