@@ -157,8 +157,14 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_decode_tc_kernel(IndexerA
       tc::cp_async16(smem + kOffQ + sw_off(r, gc, kQRegion), q + r * kCI + gc * 8);
     }
     const int res_row = 2 * warp + (lane & 1) + 8 * (lane >> 1);
-    for (int kb = 0; kb < kStages && kb < nkb; ++kb)
-      issue_block(kb, row_ptr(e_begin + (int64_t)kb * kBE + res_row));
+    // the first blocks' block-table loads all go out before any copy is issued
+    const __nv_bfloat16* rp0[kStages];
+#pragma unroll
+    for (int kb = 0; kb < kStages; ++kb)
+      rp0[kb] = kb < nkb ? row_ptr(e_begin + (int64_t)kb * kBE + res_row) : nullptr;
+#pragma unroll
+    for (int kb = 0; kb < kStages; ++kb)
+      if (kb < nkb) issue_block(kb, rp0[kb]);
   }
   tc::tc_fence_before();
   __syncthreads();
