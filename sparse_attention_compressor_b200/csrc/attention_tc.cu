@@ -257,11 +257,12 @@ __device__ __forceinline__ void key_ptrs(const AttnArgs& a, const Row& w, int j,
 // The gather group: 192 threads (warps 6-7 and 16-19; gt = the thread's index in the group) fill
 // the tiles whose rows are not consecutive. Thread gt copies 16-byte slot gt % 8 of key rows
 // gt / 8 + 24 i of both 64-channel regions of a dimension block, so a warp instruction reads four
-// whole 128-byte row segments. Blocks are issued in order as soon as each is free and handed over
-// in order as their copies land. The pair barriers count
-// this group's threads for every tile, so it also arrives for tiles that TMA fills (after the same
-// wait for the block to be free): each party waits for every phase, so no parity wait can name a
-// phase other than the one it means.
+// whole 128-byte row segments. A tile's row addresses are resolved before the wait for its first
+// block (they overlap the previous tile's work); its four blocks are issued in order as soon as
+// each is free, all four in flight at once, and handed over in order as their copies land. The
+// pair barriers count this group's threads for every tile, so it also arrives for tiles that TMA
+// fills (after the same wait for the block to be free): each party waits for every phase, so no
+// parity wait can name a phase other than the one it means.
 template <bool kSplit>
 __device__ __forceinline__ void gather_tiles(const AttnArgs& a, uint8_t* smem, uint64_t* bar,
                                              int64_t n_items, bool win_contig, bool pool_contig,
