@@ -18,9 +18,10 @@
 namespace sac {
 namespace {
 
-constexpr int kThreads = 512;       // rows re-read from L2, and long rows with keys in smem
-// rows of at most kSmemKeyRows scores: more rows side by side per SM (measured at CSA-8k: 112 us
-// with 512 threads, 87 us with 256, 108 us with 128)
+constexpr int kThreads = 512;       // long rows with keys in shared memory
+// rows of at most kSmemKeyRows scores, and rows re-read from L2: more rows side by side per SM
+// (measured at CSA-8k: 112 us with 512 threads, 87 us with 256, 108 us with 128; CSA-128k rows
+// re-read from L2: 0.56 ms a launch with 512 threads, 0.50 ms with 256)
 constexpr int kShortThreads = 256;
 constexpr int kWideThreads = 1024;  // rows with keys in shared memory when there are few of them
 constexpr int kMaxEntries = 1 << 22;  // longest row (pool entries per sequence) accepted
@@ -329,7 +330,7 @@ cudaError_t launch_topk(const float* scores, int n_stride, QueryRows qr, int m, 
     topk_kernel<true, kThreads><<<(unsigned)nrows, kThreads, smem, st>>>(scores, n_stride, qr, m,
                                                                          k, out);
   } else {
-    topk_kernel<false, kThreads><<<(unsigned)nrows, kThreads, sizeof(Shared), st>>>(
+    topk_kernel<false, kShortThreads><<<(unsigned)nrows, kShortThreads, sizeof(Shared), st>>>(
         scores, n_stride, qr, m, k, out);
   }
   return cudaGetLastError();
