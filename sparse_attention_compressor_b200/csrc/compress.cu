@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) compress_bulk_kernel(BulkArgs
 }
 
 // WPE warps cooperate on one entry (rows strided by WPE), merging their online-softmax partials.
-template <typename T, int V, int WPE>
+template <typename T, int V, int WPE, int kRows>
 __global__ void __launch_bounds__(256) compress_kernel(const T* __restrict__ x,
                                                        const T* __restrict__ gate,
                                                        const float* __restrict__ bias, int B,
@@ -341,8 +341,8 @@ __global__ void __launch_bounds__(256) compress_kernel(const T* __restrict__ x,
   float u[V], acc[V];
   load_lane<T, V>(gate, lane, u);
   const T* xb = x + (int64_t)b * S * C;
-  pool_window<T, V, WPE>([&](int64_t j) { return xb + j * C; }, u, bias, lo, hi, L, active, warp,
-                         lane, sh, acc);
+  pool_window<T, V, WPE, kRows>([&](int64_t j) { return xb + j * C; }, u, bias, lo, hi, L, active,
+                                warp, lane, sh, acc);
   if (!active || warp % WPE != 0) return;
   if (rotate) rotate_lane<V>(acc, lane, C, rf, pos0 + w * m);
   store_lane<T, V>(out + e * C, lane, acc);
@@ -394,12 +394,14 @@ cudaError_t compress_t(const void* x, const void* gate, const float* bias, int B
     return cudaGetLastError();
   }
   if (L >= 64) {
+    // rows each warp keeps in flight (8 at 16 bf16 channels a lane)
+    constexpr int kHcaRows = rows_in_flight<T, V>(64);
     int64_t blocks = entries;
-    compress_kernel<T, V, 8><<<(unsigned)blocks, 256, 0, st>>>(
+    compress_kernel<T, V, 8, kHcaRows><<<(unsigned)blocks, 256, 0, st>>>(
         (const T*)x, (const T*)gate, bias, B, S, m, L, rotate, rf, pos0, (T*)out);
   } else {
     int64_t blocks = (entries + 7) / 8;
-    compress_kernel<T, V, 1><<<(unsigned)blocks, 256, 0, st>>>(
+    compress_kernel<T, V, 1, 4><<<(unsigned)blocks, 256, 0, st>>>(
         (const T*)x, (const T*)gate, bias, B, S, m, L, rotate, rf, pos0, (T*)out);
   }
   return cudaGetLastError();

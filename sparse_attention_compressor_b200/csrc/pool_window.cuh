@@ -105,6 +105,19 @@ __device__ __forceinline__ void load_lane_raw(const T* row, int lane, RawLane<T,
     for (int i = 0; i < V; ++i) e[i] = src[i];
   }
 }
+// Elements (2i, 2i+1) of a raw lane (V odd: the last pair's second element is 0).
+template <typename T, int V>
+__device__ __forceinline__ float2 lane_pair(const RawLane<T, V>& r, int i) {
+  if constexpr (sizeof(T) == 4) {
+    return make_float2(__uint_as_float(r.w[2 * i]),
+                       2 * i + 1 < V ? __uint_as_float(r.w[2 * i + 1]) : 0.f);
+  } else {
+    const uint32_t w = r.w[i];
+    return make_float2(__uint_as_float(w << 16),
+                       2 * i + 1 < V ? __uint_as_float(w & 0xFFFF0000u) : 0.f);
+  }
+}
+
 template <typename T, int V>
 __device__ __forceinline__ void unpack_lane(const RawLane<T, V>& r, float (&v)[V]) {
   const T* e = reinterpret_cast<const T*>(r.w);
@@ -133,7 +146,8 @@ __device__ __forceinline__ void pool_window(RowFn row, const float (&u)[V], cons
   float M = -INFINITY, Z = 0.f;
   if (active) {
     // rows in batches of kBatch: all loads of a batch are issued before any is used, so a
-    // window costs ceil(rows / kBatch) memory latencies instead of one per row
+    // window costs ceil(rows / kBatch) memory latencies instead of one per row; the batch's dot
+    // reductions run interleaved and the running max is raised once per batch
     for (int64_t j0 = lo + sub; j0 < hi; j0 += kBatch * WPE) {
       RawLane<T, V> raw[kBatch];
       float bb[kBatch];
@@ -143,29 +157,50 @@ __device__ __forceinline__ void pool_window(RowFn row, const float (&u)[V], cons
         if (j < hi) {
           load_lane_raw<T, V>(row(j), lane, raw[k]);
           bb[k] = __ldg(bias + (j - hi + L));
+        } else {
+#pragma unroll
+          for (int i = 0; i < RawLane<T, V>::kWords; ++i) raw[k].w[i] = 0u;
+          bb[k] = 0.f;
         }
+      }
+      float g[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        float2 d = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < (V + 1) / 2; ++i)
+          d = __ffma2_rn(lane_pair<T, V>(raw[k], i),
+                         make_float2(u[2 * i], 2 * i + 1 < V ? u[2 * i + 1] : 0.f), d);
+        g[k] = d.x + d.y;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) g[k] += __shfl_xor_sync(~0u, g[k], o);
+      float bm = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        g[k] = j0 + (int64_t)k * WPE < hi ? g[k] + bb[k] : -INFINITY;
+        bm = fmaxf(bm, g[k]);
+      }
+      if (bm > M) {
+        const float sc = __expf(M - bm);  // 0 when M = -inf
+        Z *= sc;
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] *= sc;
+        M = bm;
       }
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {
-        if (j0 + (int64_t)k * WPE >= hi) break;
-        float xk[V];
-        unpack_lane<T, V>(raw[k], xk);
-        float d = 0.f;
-#pragma unroll
-        for (int i = 0; i < V; ++i) d = fmaf(xk[i], u[i], d);
-        const float g = warp_sum(d) + bb[k];
-        if (g == -INFINITY) continue;
-        if (g > M) {
-          const float sc = __expf(M - g);  // 0 when M = -inf
-          Z *= sc;
-#pragma unroll
-          for (int i = 0; i < V; ++i) acc[i] *= sc;
-          M = g;
-        }
-        const float p = __expf(g - M);
+        if (g[k] == -INFINITY) continue;  // rows past the window, and -inf logits
+        const float p = __expf(g[k] - M);
         Z += p;
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = fmaf(p, xk[i], acc[i]);
+        for (int i = 0; i < (V + 1) / 2; ++i) {
+          const float2 x = lane_pair<T, V>(raw[k], i);
+          acc[2 * i] = fmaf(p, x.x, acc[2 * i]);
+          if (2 * i + 1 < V) acc[2 * i + 1] = fmaf(p, x.y, acc[2 * i + 1]);
+        }
       }
     }
   }

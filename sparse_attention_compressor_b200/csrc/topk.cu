@@ -8,10 +8,13 @@
 // first digit (sign, exponent and 3 mantissa bits) spreads real score distributions over many
 // bins, so the histogram atomics rarely collide; the keys in the bin that holds T (usually a few
 // hundred) are compacted and the two finer digits only visit them. Every digit is located with a
-// block-wide scan of the histogram rather than a serial walk. The final pass gives each warp a
-// contiguous segment of the row and keeps every key > T plus the first (k - #{key > T}) keys == T in
-// index order, using ballots for the in-warp order and per-warp counts for the rest, so the chosen
-// entries come out in ascending order with conflict-free shared-memory reads.
+// block-wide scan of the histogram rather than a serial walk. Each warp owns a contiguous segment
+// of the row; the output keeps every key > T plus the first (k - #{key > T}) keys == T in index
+// order. For rows of at most kMapEntries scores the compaction pass also records, one ballot word
+// per 32 entries, which keys lie above the threshold bin; the candidates then add theirs (> T, and
+// == T in a second map), and the ordered output walks these bit maps (one word per 32 entries)
+// instead of the row. Longer rows, and rows whose threshold bin overflows the candidate list, take
+// a last pass over the row with ballots for the in-warp order and per-warp counts for the rest.
 #include "launch_util.h"
 #include "sac_kernels.h"
 
@@ -30,10 +33,25 @@ constexpr int kCandCap = 2048;       // compacted keys of the threshold bin
 constexpr int kSmemKeyRows = 4096;   // rows up to this length keep their keys in shared memory
 constexpr int kSmemKeyLimit = 49152; // longest row whose keys fit in shared memory (192 KB)
 constexpr int kBatch = 8;            // loads a thread has in flight in the passes over a row
+constexpr int kMapWords = 1024;      // selection bit map: one bit per entry
+constexpr int kMapEntries = 32 * kMapWords;  // longest row selected through the bit maps
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t u = __float_as_uint(s + 0.0f);  // -0 and +0 compare equal
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix sum over the lanes of a warp; *total gets the warp's sum.
+__device__ __forceinline__ int warp_exclusive_sum(int v, int& total) {
+  const int lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(~0u, x, o);
+    if (lane >= o) x += y;
+  }
+  total = __shfl_sync(~0u, x, 31);
+  return x - v;
 }
 
 struct Shared {
@@ -42,6 +60,7 @@ struct Shared {
   int cand_idx[kCandCap];  // entry index of each compacted key
   int warp_tot[32];  // up to 1024 threads
   int warp_gt[32], warp_eq[32];
+  uint32_t gt_map[kMapWords];  // bit i: entry i is selected (key > T)
   int n_cand;
   int digit, rem;
 };
@@ -169,6 +188,8 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
   // index, the rest are dropped. Then the finer digits and the per-segment counts of the output
   // need only the candidates, not the row. Otherwise the finer digits scan the whole row.
   const bool compact = c1 <= kCandCap;
+  // (rows whose keys sit in shared memory and are short re-read them faster than the maps cost)
+  const bool use_map = compact && n <= kMapEntries && (!kSmemKeys || n > kSmemKeyRows);
   int above_d1 = 0;
   if (compact) {
     for (int b0 = s0; b0 < s1; b0 += 32 * kBatch) {
@@ -182,7 +203,11 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
       for (int u = 0; u < kBatch; ++u) {
         const int i = b0 + 32 * u + lane;
         const uint32_t dg = kb[u] >> 20;
-        above_d1 += __popc(__ballot_sync(~0u, i < s1 && dg > d1));
+        const uint32_t gt_mask = __ballot_sync(~0u, i < s1 && dg > d1);
+        above_d1 += __popc(gt_mask);
+        // the warp's 32 entries of this step are one word of the map (segments start at
+        // multiples of 32)
+        if (use_map && lane == 0 && b0 + 32 * u < s1) sh.gt_map[(b0 + 32 * u) >> 5] = gt_mask;
         const bool hit = i < s1 && dg == d1;
         const uint32_t mask = __ballot_sync(~0u, hit);
         if (mask) {
@@ -226,6 +251,75 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
   find_digit<NT>(sh, 256, rem);
   const uint32_t T = (hi24 << 8) | (uint32_t)sh.digit;
   const int take_eq = sh.rem;  // keys equal to T to keep, lowest indices first
+
+  if (use_map) {
+    // ---- selection through the bit maps: the candidates above T join the keys above digit d1
+    // in gt_map, those equal to T go to eq_map (the histogram's storage, free now)
+    uint32_t* eq_map = reinterpret_cast<uint32_t*>(sh.hist);
+    const int nwords = (n + 31) >> 5;
+    for (int i = tid; i < nwords; i += NT) eq_map[i] = 0u;
+    __syncthreads();
+    for (int c = tid; c < nc; c += NT) {
+      const uint32_t key = sh.cand[c];
+      const int e = sh.cand_idx[c];
+      if (key > T) atomicOr(&sh.gt_map[e >> 5], 1u << (e & 31));
+      else if (key == T) atomicOr(&eq_map[e >> 5], 1u << (e & 31));
+    }
+    __syncthreads();
+    // warp w's words cover its segment [s0, s1); an empty segment (s0 >= n) has none
+    const int w0 = s0 >> 5, w1 = (s1 + 31) >> 5;
+    int gt = 0, eq = 0;
+    for (int wd = w0 + lane; wd < w1; wd += 32) {
+      gt += __popc(sh.gt_map[wd]);
+      eq += __popc(eq_map[wd]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gt += __shfl_xor_sync(~0u, gt, o);
+      eq += __shfl_xor_sync(~0u, eq, o);
+    }
+    if (lane == 0) {
+      sh.warp_gt[warp] = gt;
+      sh.warp_eq[warp] = eq;
+    }
+    __syncthreads();
+    int eq_before = 0, sel_before = 0;
+    for (int w = 0; w < warp; ++w) {
+      const int e = sh.warp_eq[w];
+      sel_before += sh.warp_gt[w] + min(max(take_eq - eq_before, 0), e);
+      eq_before += e;
+    }
+    // 32 words (1024 entries) per step, lane l on word wb + l; the keys == T are taken in entry
+    // order while the count taken before them stays below take_eq
+    for (int wb = w0; wb < w1; wb += 32) {
+      const int wd = wb + lane;
+      const uint32_t g = wd < w1 ? sh.gt_map[wd] : 0u;
+      const uint32_t e = wd < w1 ? eq_map[wd] : 0u;
+      const int ne = __popc(e);
+      int ne_tot;
+      const int ne_before = warp_exclusive_sum(ne, ne_tot);
+      int q = take_eq - (eq_before + ne_before);
+      uint32_t taken = 0u;
+      if (q >= ne) {
+        taken = e;
+      } else {
+        for (uint32_t rest = e; q > 0; --q) {  // the lowest q bits of e
+          taken |= rest & (0u - rest);
+          rest &= rest - 1u;
+        }
+      }
+      uint32_t sel = g | taken;
+      int ns_tot;
+      int pos = sel_before + warp_exclusive_sum(__popc(sel), ns_tot);
+      while (sel) {
+        orow[pos++] = (wd << 5) + (__ffs(sel) - 1);
+        sel &= sel - 1u;
+      }
+      eq_before += ne_tot;
+      sel_before += ns_tot;
+    }
+    return;
+  }
 
   // ---- selection: per-segment counts of keys > T and == T, then the output in entry order
   if (compact) {

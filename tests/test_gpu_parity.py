@@ -287,13 +287,20 @@ def small_decode_workload():
 
 
 @pytest.mark.parametrize("layer", ["csa", "hca"])
-@pytest.mark.parametrize("which", ["small", "full"])
+@pytest.mark.parametrize("which", ["small", "full", "ps24", "ps12"])
 def test_decode_parity(layer, which):
-    wl = small_decode_workload() if which == "small" else W.WORKLOADS["decode_bf16"]
+    """Decode of both layers against the oracle. The page sizes: 64 (the workload's), 24 (the
+    paged indexer's box loads in runs of 8 rows) and 12 (not a multiple of 8: its row gathers)."""
+    if which == "full":
+        wl = W.WORKLOADS["decode_bf16"]
+    elif which.startswith("ps"):
+        wl = replace(small_decode_workload(), page_size=int(which[2:]))
+    else:
+        wl = small_decode_workload()
     d = W.decode_inputs(wl, layer)
     o, tk = gpu_decode(wl, d, layer, int(d["ctx_lens"].max()))
     nseq = wl.nseq
-    seqs = np.arange(nseq) if which == "small" else np.arange(0, nseq, 8)
+    seqs = np.arange(0, nseq, 8) if which == "full" else np.arange(nseq)
     gsel = None
     if layer == "csa":
         # oracle's own selections (via its decode) and the tie-band comparison on its scores
