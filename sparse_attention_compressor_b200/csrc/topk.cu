@@ -150,12 +150,44 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
     return kSmemKeys ? keys[i] : order_key(__ldcg(srow + i));
   };
 
-  // ---- digit 1: bits 31..20. The passes over the row issue kBatch loads before using any, so a
-  // thread waits for one memory latency per kBatch keys rather than per key.
+  // ---- digit 1: bits 31..20. The passes over the row issue all of a batch's loads before using
+  // any, so a thread waits for one memory latency per batch rather than per key.
   for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0;
   if (tid == 0) sh.n_cand = 0;
   __syncthreads();
-  for (int i0 = tid; i0 < n; i0 += NT * kBatch) {
+  auto count_key = [&](int i, float v) {
+    const uint32_t key = order_key(v);
+    if (kSmemKeys) keys[i] = key;
+    atomicAdd(&sh.hist[key >> 20], 1);
+  };
+  // rows on 16-byte boundaries are read as float4 (kBatch / 2 of them in flight a thread: twice
+  // the bytes of kBatch scalars, a quarter of the load instructions), the rest key by key
+  int i_scalar = 0;
+  if ((reinterpret_cast<uintptr_t>(srow) & 15) == 0) {
+    constexpr int kVec = kBatch / 2;
+    const float4* s4 = reinterpret_cast<const float4*>(srow);
+    const int n4 = n >> 2;
+    for (int i0 = tid; i0 < n4; i0 += NT * kVec) {
+      float4 v[kVec];
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int i = i0 + u * NT;
+        v[u] = i < n4 ? __ldcg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int i = i0 + u * NT;
+        if (i < n4) {
+          count_key(4 * i, v[u].x);
+          count_key(4 * i + 1, v[u].y);
+          count_key(4 * i + 2, v[u].z);
+          count_key(4 * i + 3, v[u].w);
+        }
+      }
+    }
+    i_scalar = 4 * n4;
+  }
+  for (int i0 = i_scalar + tid; i0 < n; i0 += NT * kBatch) {
     float v[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -165,11 +197,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(const float* __restrict__ scor
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = i0 + u * NT;
-      if (i < n) {
-        const uint32_t key = order_key(v[u]);
-        if (kSmemKeys) keys[i] = key;
-        atomicAdd(&sh.hist[key >> 20], 1);
-      }
+      if (i < n) count_key(i, v[u]);
     }
   }
   __syncthreads();
